@@ -1,0 +1,16 @@
+"""Fused causal scaled-dot-product attention for B200 (sm_100a).
+
+The compute lives in ``libattn_b200.so`` (hand-written CUDA, C ABI declared in ``include/attn.h``).
+``causal_attention_attn_b200.attn`` is the thin ctypes binding; importing this package does not
+load the library, so the seeded-input module can be used on machines without the build.
+"""
+
+__version__ = "0.1.0"
+
+
+def __getattr__(name):
+    if name in ("attn_fwd", "attn_fwd_host", "AttnError", "library_path", "load_library"):
+        from . import attn as _attn
+
+        return getattr(_attn, name)
+    raise AttributeError(name)

@@ -1,0 +1,155 @@
+/*
+ * Plain CPU oracle for causal scaled-dot-product attention, in fp64.
+ *
+ * TEST INFRASTRUCTURE. Only the tests, the smoke check and the bench's CPU-baseline leg load this
+ * file's library; the CUDA product path never calls it, links it or shares code with it.
+ *
+ * What it computes is the plain definition, with no blocking, fusion or online rescaling:
+ *
+ *   for every batch b, query head h and query row i (kv head = h / (Hq / Hkv)):
+ *     visible keys  V_i = { j : 0 <= j < Skv and (!causal or j <= i + (Skv - Sq)) }
+ *     s_j   = scale * sum_d q[i,d] * k[j,d]                                  (step 1)
+ *     m     = max_{j in V_i} s_j                                              (pass 1)
+ *     l     = sum_{j in V_i} exp(s_j - m)                                     (pass 2)
+ *     o[i,:]= sum_{j in V_i} exp(s_j - m) * v[j,:] / l ;  lse_i = m + ln(l)   (pass 3)
+ *
+ * Sources (page title, section):
+ *  - "05 · Tích vô hướng, Softmax và toán của Attention", §1 (dot product as the relevance score;
+ *    worked example (2,-1,0.5).(3,4,2) = 3), "Vì sao chia cho √128" (divide scores by sqrt(d)),
+ *    §2 (softmax = exp then divide by the sum; subtract the row max first), §3 (one query against
+ *    all keys -> scale -> softmax -> weighted sum of values).
+ *  - "AI Infra 入门：RMSNorm、Softmax、Causal Mask、Sampling 的数学与底层优化", §2 (safe softmax:
+ *    subtract the max M), §3 (causal mask adds -inf for j > i; softmax as three passes: max, then
+ *    denominator, then result; LSE = m + ln(l) so that softmax(z_i) = exp(z_i - LSE)).
+ *  - "Bộ 06 · Bên trong model", Q1 (softmax(x - c) = softmax(x)), Q2 (the mask adds -inf, whose
+ *    exponential is exactly 0, so a masked key gets weight exactly 0).
+ *  - "第11节：Attention 实现（Flash vs Fallback）", §3 (with a KV cache the triangular -inf mask is
+ *    added to the LAST seq_len key columns only: key j is hidden from query i iff
+ *    j - (Skv - Sq) > i), §4 (scores have shape [B, H, Q_len, K_len], heads-major), §5 (softmax
+ *    in float, i.e. in a precision above the bf16 inputs).
+ *
+ * Readings where the pages leave a step open:
+ *  - A masked key is left out of the max and of both sums. That is what adding -inf does, since
+ *    exp(-inf) = 0; no finite stand-in such as -65504 is used.
+ *  - GQA grouping is consecutive: query head h reads kv head h / (Hq / Hkv).
+ *  - LSE is the natural logarithm of the sum over the SCALED scores.
+ *  - Inputs are bf16 bit patterns widened exactly to double; `scale` is the fp32 value the GPU
+ *    receives, widened exactly to double. All arithmetic is fp64.
+ *  - causal with Sq > Skv is rejected (the cache-aligned mask leaves early rows with no key).
+ */
+#include <math.h>
+#include <omp.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_OK 0
+#define ORACLE_ERR_ARGS (-1)
+#define ORACLE_ERR_NOMEM (-2)
+
+/* bf16 -> double: a bf16 value is the upper 16 bits of an IEEE fp32 value, so the widening is exact. */
+static double bf16_to_double(uint16_t bits)
+{
+    uint32_t u = ((uint32_t)bits) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* One query row: fills out[0..D) and *lse_out. `scores` is scratch of length Skv. */
+static void oracle_row(const uint16_t *q_row, const uint16_t *k_head, const uint16_t *v_head,
+                       int Skv, int D, int last_visible, double scale,
+                       double *scores, double *out, double *lse_out)
+{
+    /* step 1: scaled dot products for the visible keys 0..last_visible */
+    for (int j = 0; j <= last_visible; ++j) {
+        const uint16_t *k_row = k_head + (size_t)j * D;
+        double dot = 0.0;
+        for (int d = 0; d < D; ++d)
+            dot += bf16_to_double(q_row[d]) * bf16_to_double(k_row[d]);
+        scores[j] = scale * dot;
+    }
+    (void)Skv;
+
+    /* pass 1: row maximum over the visible keys */
+    double m = -INFINITY;
+    for (int j = 0; j <= last_visible; ++j)
+        if (scores[j] > m)
+            m = scores[j];
+
+    /* pass 2: denominator */
+    double l = 0.0;
+    for (int j = 0; j <= last_visible; ++j)
+        l += exp(scores[j] - m);
+
+    /* pass 3: normalised weighted sum of the value rows, and the log-sum-exp */
+    for (int d = 0; d < D; ++d)
+        out[d] = 0.0;
+    for (int j = 0; j <= last_visible; ++j) {
+        double w = exp(scores[j] - m) / l;
+        const uint16_t *v_row = v_head + (size_t)j * D;
+        for (int d = 0; d < D; ++d)
+            out[d] += w * bf16_to_double(v_row[d]);
+    }
+    *lse_out = m + log(l);
+}
+
+/*
+ * q: [B, Hq, Sq, D], k/v: [B, Hkv, Skv, D], all bf16 bit patterns, contiguous.
+ * rows: optional list of n_rows flat row ids r = (b * Hq + h) * Sq + i; NULL means every row in order.
+ * o: [n_rows, D] fp64, lse: [n_rows] fp64.
+ * n_threads <= 0 uses the OpenMP default.
+ */
+int oracle_attn(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                double *o, double *lse,
+                int B, int Hq, int Hkv, int Sq, int Skv, int D,
+                float scale, int causal,
+                const int64_t *rows, int64_t n_rows, int n_threads)
+{
+    if (!q || !k || !v || !o || !lse)
+        return ORACLE_ERR_ARGS;
+    if (B < 1 || Hq < 1 || Hkv < 1 || Sq < 1 || Skv < 1 || D < 1 || Hq % Hkv != 0)
+        return ORACLE_ERR_ARGS;
+    if (causal && Sq > Skv)
+        return ORACLE_ERR_ARGS;
+    const int64_t total_rows = (int64_t)B * Hq * Sq;
+    if (rows == NULL)
+        n_rows = total_rows;
+    if (n_rows < 0)
+        return ORACLE_ERR_ARGS;
+    for (int64_t r = 0; rows && r < n_rows; ++r)
+        if (rows[r] < 0 || rows[r] >= total_rows)
+            return ORACLE_ERR_ARGS;
+
+    const int group = Hq / Hkv;
+    const int offset = Skv - Sq; /* the mask covers the last Sq key columns */
+    const double scale_d = (double)scale;
+    int failed = 0;
+
+#pragma omp parallel num_threads(n_threads > 0 ? n_threads : omp_get_max_threads())
+    {
+        double *scores = (double *)malloc(sizeof(double) * (size_t)Skv);
+        if (!scores) {
+#pragma omp atomic write
+            failed = 1;
+        }
+#pragma omp for schedule(dynamic, 8)
+        for (int64_t r = 0; r < n_rows; ++r) {
+            if (!scores)
+                continue;
+            const int64_t row = rows ? rows[r] : r;
+            const int i = (int)(row % Sq);
+            const int64_t bh = row / Sq;
+            const int h = (int)(bh % Hq);
+            const int b = (int)(bh / Hq);
+            const int kvh = h / group;
+            const int last_visible = causal ? i + offset : Skv - 1;
+            const uint16_t *q_row = q + (size_t)row * D;
+            const size_t kv_off = ((size_t)b * Hkv + kvh) * (size_t)Skv * D;
+            oracle_row(q_row, k + kv_off, v + kv_off, Skv, D, last_visible, scale_d, scores,
+                       o + (size_t)r * D, lse + r);
+        }
+        free(scores);
+    }
+    return failed ? ORACLE_ERR_NOMEM : ORACLE_OK;
+}
