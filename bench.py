@@ -1,0 +1,372 @@
+"""Benchmark: fused causal attention on B200, prefill TFLOP/s and decode KV-read GB/s.
+
+One step = one pass of the whole hot path over one batch of synthetic input: the causal prefill of
+an 8B-shaped layer (B=1, Hq=32, Hkv=8, S=4096, D=128) through the prefill kernel, then the GQA
+decode over a 16 x 4096-token KV cache through the split-KV decode kernel. Inputs are resident in
+HBM before timing; L2 is flushed (a 256 MiB write) before every step, outside the kernel events.
+
+``python bench.py --gpus N --steps K --warmup W`` prints one JSON line (rank 0). For N > 1 it is
+launched with torchrun, one rank per GPU; every rank processes its own copy of the workload (the
+(batch, head) problems are independent, so there is no data-path collective) and the time is the
+max over ranks. ``--impl reference`` times the CPU oracle instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from causal_attention_attn_b200 import inputs  # noqa: E402
+
+METRIC = "prefill attn TFLOP/s & decode KV-read GB/s, as fraction of B200 roofline"
+PREFILL = inputs.PREFILL_8B
+DECODE = inputs.DECODE_GQA
+L2_FLUSH_BYTES = 256 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples taken every 100 ms while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.device_index = device_index
+        self.proc = None
+        self.out = None
+
+    def __enter__(self):
+        try:
+            self.out = open(os.devnull, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.device_index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=self.out, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+        if self.out:
+            self.out.close()
+
+    def summary(self):
+        sm, smax, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = max(smax, float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax or None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def prefill_sample_flops(w, rows):
+    i = rows % w.Sq
+    visible = (i + w.offset + 1) if w.causal else torch.full_like(i, w.Skv)
+    return int(4 * w.D * int(visible.sum()))
+
+
+def cpu_baseline(w, every: int, offset: int = 0, threads=None):
+    """Time the oracle on every `every`-th row of workload `w` (rows offset, offset+every, ...)."""
+    import oracle  # the CPU baseline is the oracle as it stands
+
+    q, k, v = inputs.generate(w)
+    total = w.B * w.Hq * w.Sq
+    rows = torch.arange(offset % every, total, every, dtype=torch.int64)
+    cores = len(os.sched_getaffinity(0))
+    t0 = time.perf_counter()
+    oracle.attention(q, k, v, w.scale, w.causal, rows=rows.numpy(), threads=threads or cores)
+    dt = time.perf_counter() - t0
+    flops = prefill_sample_flops(w, rows)
+    return flops / dt / 1e12, dt, cores, rows.numel()
+
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    w = PREFILL
+    every = 32
+    times, flops = [], []
+    for s in range(args.warmup + args.steps):
+        tf, dt, cores, n = cpu_baseline(w, every, offset=s)
+        if s >= args.warmup:
+            times.append(dt)
+            flops.append(tf * dt * 1e12)
+    value = sum(flops) / sum(times) / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sum(times) / len(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) bf16 inputs)", "config": PREFILL.config(),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"every {every}th query row of the workload per step (rows offset by the step "
+                                   f"index), {n} rows; fp64 three-pass oracle"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    from causal_attention_attn_b200 import attn
+
+    attn.load_library()
+    peaks, peak_kind = load_peaks()
+
+    qp, kp, vp = inputs.generate(PREFILL)
+    qd, kd, vd = inputs.generate(DECODE)
+    pq, pk, pv = (t.to(dev) for t in (qp, kp, vp))
+    dq, dk, dv = (t.to(dev) for t in (qd, kd, vd))
+    po = torch.empty_like(pq)
+    pl = torch.empty(pq.shape[:3], dtype=torch.float32, device=dev)
+    do = torch.empty_like(dq)
+    dl = torch.empty(dq.shape[:3], dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(evs=None):
+        flush.zero_()
+        if evs:
+            evs[0].record(stream)
+        attn.attn_fwd(pq, pk, pv, scale=PREFILL.scale, causal=True, out=po, lse=pl, stream=stream)
+        if evs:
+            evs[1].record(stream)
+        attn.attn_fwd(dq, dk, dv, scale=DECODE.scale, causal=True, out=do, lse=dl, stream=stream)
+        if evs:
+            evs[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t_all0 = torch.cuda.Event(enable_timing=True)
+    t_all1 = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clocks:
+        t_all0.record(stream)
+        for s in range(args.steps):
+            step(events[s])
+        t_all1.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    pre_ms = sum(e[0].elapsed_time(e[1]) for e in events)
+    dec_ms = sum(e[1].elapsed_time(e[2]) for e in events)
+    region_ms = t_all0.elapsed_time(t_all1)
+    if world > 1:
+        t = torch.tensor([pre_ms, dec_ms, region_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        pre_ms, dec_ms, region_ms = t.tolist()
+
+    prefill_tflops = world * args.steps * PREFILL.flops() / (pre_ms * 1e-3) / 1e12
+    decode_bytes = DECODE.io_bytes()  # K and V read once, plus q, o and lse
+    decode_gbs = world * args.steps * decode_bytes / (dec_ms * 1e-3) / 1e9
+    pre_launch_s = pre_ms * 1e-3 / args.steps
+    dec_launch_s = dec_ms * 1e-3 / args.steps
+    tensor_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+
+    # End to end through the public call on HOST buffers: pinned H2D of q, k, v, the kernel, D2H of o, lse.
+    hq, hk, hv = (t.pin_memory() for t in (qp, kp, vp))
+    ho = torch.empty(qp.shape, dtype=torch.bfloat16, pin_memory=True)
+    hl = torch.empty(qp.shape[:3], dtype=torch.float32, pin_memory=True)
+    bufs = (pq, pk, pv, po, pl)
+    for _ in range(2):
+        attn.attn_fwd_host(hq, hk, hv, scale=PREFILL.scale, causal=True, stream=stream, out_host=ho, lse_host=hl,
+                           dev_bufs=bufs)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(3, min(args.steps, 10))
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        attn.attn_fwd_host(hq, hk, hv, scale=PREFILL.scale, causal=True, stream=stream, out_host=ho, lse_host=hl,
+                           dev_bufs=bufs)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = t.item()
+        torch.distributed.barrier()
+    e2e_tflops = world * e2e_steps * PREFILL.flops() / (e2e_ms * 1e-3) / 1e12
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+    d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+
+    if rank == 0:
+        base_tf, base_dt, cores, n_rows = cpu_baseline(PREFILL, every=1) if world == 1 else (None, None, None, None)
+        traffic = read_traffic("prefill_kernel", PREFILL.name)
+        line = {
+            "metric": METRIC, "value": prefill_tflops, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": (pre_ms + dec_ms) / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16 inputs)",
+            "config": dict(PREFILL.config(), l2="flushed before every step (256 MiB write)",
+                           parallelism=f"replicas x{world}"),
+            "roofline": {"bound": "tensor", "achieved": PREFILL.flops() / pre_launch_s / 1e12, "peak": tensor_peak,
+                         "unit": "TFLOP/s", "frac": PREFILL.flops() / pre_launch_s / 1e12 / tensor_peak,
+                         "traffic": traffic, "peak_kind": f"{peak_kind} bf16 dense (burst)",
+                         "kernel": "prefill_kernel<128>"},
+            "decode": {
+                "metric": "decode KV-read GB/s", "value": decode_gbs, "unit": "GB/s", "config": DECODE.config(),
+                "roofline": {"bound": "hbm", "achieved": decode_bytes / dec_launch_s / 1e9, "peak": hbm_peak,
+                             "unit": "GB/s", "frac": decode_bytes / dec_launch_s / 1e9 / hbm_peak,
+                             "traffic": read_traffic("decode_kernel", DECODE.name),
+                             "peak_kind": f"{peak_kind} HBM copy", "kernel": "decode_kernel<128,4>"},
+                "us_per_launch": dec_launch_s * 1e6,
+                "splits": attn.decode_splits(DECODE.B, DECODE.Hq, DECODE.Hkv, DECODE.Skv, DECODE.D),
+            },
+            "prefill_us_per_launch": pre_launch_s * 1e6,
+            "timed_region_ms": region_ms,
+            "e2e": {"value": e2e_tflops, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "steps": e2e_steps, "what": "prefill through attn_fwd on pinned host buffers, copies included"},
+            "gpu_launches": 2 * args.steps,
+            "clocks": clocks.summary(),
+        }
+        if base_tf is not None:
+            line["cpu_baseline"] = {"value": base_tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                                    "sample": f"every query row of the prefill workload ({n_rows} rows, "
+                                              f"{base_dt:.1f} s); fp64 three-pass oracle"}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+KERNEL_SOURCES = {
+    "prefill_kernel": ["prefill_sm100.cu", "sm100_ptx.cuh"],
+    "decode_kernel": ["decode_sm100.cu", "sm100_ptx.cuh"],
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
+    import hashlib
+
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "causal_attention_attn_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def read_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch for `kernel` from the committed ncu summary (profiles/traffic.json),
+    or None when there is none for this workload or the kernel's source changed since the capture."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    try:
+        with open(path) as f:
+            entry = json.load(f).get(kernel, {})
+        if entry.get("workload") != workload or entry.get("source_hash") != kernel_source_hash(kernel):
+            return None
+        return entry.get("dram_bytes_per_launch")
+    except (OSError, ValueError):
+        return None
+
+
+def run_case(args):
+    """Run one named workload `--repeat` times through attn_fwd (no L2 flush, no JSON line): the
+    command the committed ncu summaries were captured with."""
+    from causal_attention_attn_b200 import attn
+
+    w = inputs.SHORT_NAMES[args.case]
+    q, k, v = (t.cuda() for t in inputs.generate(w))
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ev[0].record()
+    for _ in range(args.repeat):
+        attn.attn_fwd(q, k, v, scale=w.scale, causal=w.causal, out=o, lse=lse)
+    ev[1].record()
+    torch.cuda.synchronize()
+    ms = ev[0].elapsed_time(ev[1]) / args.repeat
+    print(json.dumps({"case": w.name, "repeat": args.repeat, "us_per_launch": ms * 1e3,
+                      "tflops": w.flops() / (ms * 1e-3) / 1e12, "io_gbs": w.io_bytes() / (ms * 1e-3) / 1e9,
+                      "device_status": attn.device_status()}), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--case", choices=sorted(inputs.SHORT_NAMES), default=None,
+                    help="only run this workload --repeat times (for profiling); prints no bench line")
+    ap.add_argument("--repeat", type=int, default=3)
+    args = ap.parse_args()
+    if args.case:
+        return run_case(args)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

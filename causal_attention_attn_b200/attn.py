@@ -1,0 +1,188 @@
+"""Thin ctypes binding over ``libattn_b200.so`` (C ABI in ``include/attn.h``).
+
+Argument marshalling only: tensors are checked for dtype/device/contiguity, their data pointers and
+the current CUDA stream are passed to the C entry points, and a non-zero status becomes an
+``AttnError``. PyTorch supplies device memory and streams; every step of the attention itself runs
+in the library's kernels. There is no fallback: if the library is missing the call fails.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_NAME = "libattn_b200.so"
+library_path = os.path.join(_PKG, LIB_NAME)
+
+ATTN_OK = 0
+STATUS_NAMES = {
+    0: "ATTN_OK", -1: "ATTN_ERR_NULL", -2: "ATTN_ERR_SHAPE", -3: "ATTN_ERR_GQA", -4: "ATTN_ERR_HEADDIM",
+    -5: "ATTN_ERR_ALIGN", -6: "ATTN_ERR_CAUSAL_SQ_GT_SKV", -7: "ATTN_ERR_ARCH", -8: "ATTN_ERR_WORKSPACE",
+    -9: "ATTN_ERR_LAUNCH", -10: "ATTN_ERR_DEVICE_TIMEOUT", -11: "ATTN_ERR_SCALE", -12: "ATTN_ERR_CUDA",
+}
+EXPORTED = ("attn_fwd", "attn_fwd_ex", "attn_decode_splits", "attn_status_string", "attn_version",
+            "attn_device_status")
+
+_lock = threading.Lock()
+_lib = None
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+def load_library(path: str | None = None):
+    """Load the library once. Raises if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is not None and path is None:
+            return _lib
+        p = path or library_path
+        if not os.path.exists(p):
+            raise RuntimeError(f"{LIB_NAME} is not built (expected at {p}); "
+                               "run `python -m causal_attention_attn_b200.build`")
+        lib = ctypes.CDLL(p)
+        i, f, vp = ctypes.c_int, ctypes.c_float, ctypes.c_void_p
+        lib.attn_fwd.restype = i
+        lib.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp]
+        lib.attn_fwd_ex.restype = i
+        lib.attn_fwd_ex.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, vp]
+        lib.attn_decode_splits.restype = i
+        lib.attn_decode_splits.argtypes = [i, i, i, i, i]
+        lib.attn_status_string.restype = ctypes.c_char_p
+        lib.attn_status_string.argtypes = [i]
+        lib.attn_version.restype = i
+        lib.attn_version.argtypes = []
+        lib.attn_device_status.restype = i
+        lib.attn_device_status.argtypes = [vp]
+        if path is None:
+            _lib = lib
+        return lib
+
+
+def status_string(status: int) -> str:
+    return load_library().attn_status_string(int(status)).decode()
+
+
+def _check(status: int):
+    if status != ATTN_OK:
+        raise AttnError(status, status_string(status))
+
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _check_tensor(name, t, dtype, ndim):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must live on a CUDA device")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def attn_fwd_raw(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, lse_ptr: int, B: int, Hq: int, Hkv: int,
+                 Sq: int, Skv: int, D: int, scale: float, causal: bool, stream: int = 0,
+                 decode_splits: int = 0) -> int:
+    """Call the C entry point with raw pointers; returns the status code (no exception)."""
+    lib = load_library()
+    if decode_splits:
+        return lib.attn_fwd_ex(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, Hq, Hkv, Sq, Skv, D, float(scale),
+                               int(causal), int(decode_splits), stream)
+    return lib.attn_fwd(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, Hq, Hkv, Sq, Skv, D, float(scale), int(causal),
+                        stream)
+
+
+def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: float | None = None, causal: bool = True,
+             out: torch.Tensor | None = None, lse: torch.Tensor | None = None, stream=None,
+             decode_splits: int = 0):
+    """Fused causal attention forward on the GPU.
+
+    q: [B, Hq, Sq, D], k/v: [B, Hkv, Skv, D], bf16, contiguous, on one CUDA device.
+    Returns (o [B, Hq, Sq, D] bf16, lse [B, Hq, Sq] fp32). ``scale`` defaults to 1/sqrt(D).
+    """
+    _check_tensor("q", q, torch.bfloat16, 4)
+    _check_tensor("k", k, torch.bfloat16, 4)
+    _check_tensor("v", v, torch.bfloat16, 4)
+    B, Hq, Sq, D = q.shape
+    Bk, Hkv, Skv, Dk = k.shape
+    if tuple(v.shape) != tuple(k.shape) or Bk != B or Dk != D:
+        raise ValueError(f"shape mismatch: q {tuple(q.shape)}, k {tuple(k.shape)}, v {tuple(v.shape)}")
+    if scale is None:
+        scale = D ** -0.5
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _check_tensor("out", out, torch.bfloat16, 4)
+        if out.shape != q.shape:
+            raise ValueError("out must have the shape of q")
+    if lse is None:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    else:
+        _check_tensor("lse", lse, torch.float32, 3)
+        if tuple(lse.shape) != (B, Hq, Sq):
+            raise ValueError("lse must be [B, Hq, Sq]")
+    with torch.cuda.device(q.device):
+        rc = attn_fwd_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, Hq, Hkv,
+                          Sq, Skv, D, scale, causal, _stream_handle(stream), decode_splits)
+    _check(rc)
+    return out, lse
+
+
+def attn_fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: float | None = None,
+                  causal: bool = True, device="cuda", stream=None, out_host=None, lse_host=None, dev_bufs=None):
+    """End-to-end call on HOST tensors: copy q, k, v to the device, run attn_fwd, copy o and lse back.
+
+    Inputs should be pinned for asynchronous copies. ``dev_bufs`` optionally supplies reusable
+    device tensors (q, k, v, o, lse) so that a loop of calls does not allocate. Returns host
+    (o, lse); the call synchronises on the stream before returning.
+    """
+    stream = stream or torch.cuda.current_stream(device)
+    with torch.cuda.stream(stream):
+        if dev_bufs is None:
+            qd = q.to(device, non_blocking=True)
+            kd = k.to(device, non_blocking=True)
+            vd = v.to(device, non_blocking=True)
+            od, ld = None, None
+        else:
+            qd, kd, vd, od, ld = dev_bufs
+            qd.copy_(q, non_blocking=True)
+            kd.copy_(k, non_blocking=True)
+            vd.copy_(v, non_blocking=True)
+        od, ld = attn_fwd(qd, kd, vd, scale=scale, causal=causal, out=od, lse=ld, stream=stream)
+        if out_host is None:
+            out_host = torch.empty(od.shape, dtype=od.dtype, pin_memory=True)
+        if lse_host is None:
+            lse_host = torch.empty(ld.shape, dtype=ld.dtype, pin_memory=True)
+        out_host.copy_(od, non_blocking=True)
+        lse_host.copy_(ld, non_blocking=True)
+    stream.synchronize()
+    return out_host, lse_host
+
+
+def decode_splits(B: int, Hq: int, Hkv: int, Skv: int, D: int) -> int:
+    rc = load_library().attn_decode_splits(B, Hq, Hkv, Skv, D)
+    if rc < 0:
+        _check(rc)
+    return rc
+
+
+def device_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device status word: 0 or ATTN_ERR_DEVICE_TIMEOUT."""
+    return load_library().attn_device_status(_stream_handle(stream))
+
+
+def version() -> int:
+    return load_library().attn_version()

@@ -1,0 +1,340 @@
+/*
+ * attn_api.cu — the C ABI declared in include/attn.h: argument validation, dispatch between the
+ * prefill and decode kernels, the per-device workspace, and status reporting. No arithmetic of the
+ * method happens here; every step runs in the two kernels.
+ */
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "attn.h"
+#include "kernels.h"
+
+namespace attn_b200 {
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+    bool probed = false;
+    bool supported = false;
+    int sm_count = 0;
+    void *block = nullptr;  // status word + counters + partials, one allocation
+    size_t bytes = 0;
+    int *status = nullptr;
+    int *counters = nullptr;
+    size_t counter_count = 0;
+    float *partials = nullptr;
+    size_t partial_floats = 0;
+};
+
+std::mutex g_mutex;
+DeviceState g_dev[kMaxDevices];
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int validate(const void *q, const void *k, const void *v, const void *o, const float *lse, int B, int Hq, int Hkv,
+             int Sq, int Skv, int D, float scale, int causal)
+{
+    if (!q || !k || !v || !o || !lse)
+        return ATTN_ERR_NULL;
+    if (B < 1 || Hq < 1 || Hkv < 1 || Sq < 1 || Skv < 1 || D < 1)
+        return ATTN_ERR_SHAPE;
+    if (Hq % Hkv != 0)
+        return ATTN_ERR_GQA;
+    if (D != 32 && D != 64 && D != 128)
+        return ATTN_ERR_HEADDIM;
+    // Flat row indices (b*H + h)*S + i must fit in a 32-bit int.
+    if (static_cast<long long>(B) * Hq * Sq > INT_MAX || static_cast<long long>(B) * Hkv * Skv > INT_MAX)
+        return ATTN_ERR_SHAPE;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+        return ATTN_ERR_ALIGN;
+    if (causal != 0 && causal != 1)
+        return ATTN_ERR_SHAPE;
+    if (causal && Sq > Skv)
+        return ATTN_ERR_CAUSAL_SQ_GT_SKV;
+    if (!(scale > 0.f) || !std::isfinite(scale))
+        return ATTN_ERR_SCALE;
+    return ATTN_OK;
+}
+
+// Probe the current device once; returns the state or nullptr with *err set.
+DeviceState *device_state(int *err)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        *err = ATTN_ERR_CUDA;
+        return nullptr;
+    }
+    DeviceState &s = g_dev[dev];
+    if (!s.probed) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+            cudaGetLastError();
+            *err = ATTN_ERR_CUDA;
+            return nullptr;
+        }
+        s.supported = (major == 10 && minor == 0);
+        s.sm_count = sms;
+        s.probed = true;
+    }
+    if (!s.supported) {
+        *err = ATTN_ERR_ARCH;
+        return nullptr;
+    }
+    return &s;
+}
+
+// Make sure the workspace holds `counters` ints and `partials` floats (plus the status word).
+int ensure_workspace(DeviceState &s, size_t counters, size_t partials, cudaStream_t stream)
+{
+    if (s.block && counters <= s.counter_count && partials <= s.partial_floats)
+        return ATTN_OK;
+    size_t nc = counters > s.counter_count ? counters : s.counter_count;
+    size_t np = partials > s.partial_floats ? partials : s.partial_floats;
+    if (nc < 1024)
+        nc = 1024;
+    const size_t head = 256;  // status word, padded
+    const size_t cbytes = ((nc * sizeof(int) + 255) / 256) * 256;
+    const size_t bytes = head + cbytes + np * sizeof(float);
+    void *block = nullptr;
+    if (cudaMalloc(&block, bytes) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_WORKSPACE;
+    }
+    // The old block may still be read by queued kernels: wait for the device before freeing it.
+    if (s.block) {
+        if (cudaDeviceSynchronize() != cudaSuccess) {
+            cudaGetLastError();
+            cudaFree(block);
+            return ATTN_ERR_WORKSPACE;
+        }
+        cudaFree(s.block);
+    }
+    if (cudaMemsetAsync(block, 0, head + cbytes, stream) != cudaSuccess) {
+        cudaGetLastError();
+        cudaFree(block);
+        s.block = nullptr;
+        s.bytes = s.counter_count = s.partial_floats = 0;
+        return ATTN_ERR_WORKSPACE;
+    }
+    s.block = block;
+    s.bytes = bytes;
+    s.status = static_cast<int *>(block);
+    s.counters = reinterpret_cast<int *>(static_cast<char *>(block) + head);
+    s.counter_count = nc;
+    s.partials = reinterpret_cast<float *>(static_cast<char *>(block) + head + cbytes);
+    s.partial_floats = np;
+    return ATTN_OK;
+}
+
+int choose_splits(const DeviceState &s, int B, int Hq, int Hkv, int Skv, int D)
+{
+    const int group = Hq / Hkv;
+    const int G = decode_heads_per_cta(group);
+    const long long pairs = static_cast<long long>(B) * Hkv * (group / G);
+    const int per_sm = decode_ctas_per_sm(D, group);
+    const long long slots = static_cast<long long>(s.sm_count) * per_sm;
+    const int ck = decode_keys_per_chunk(group);
+    const int max_splits = (Skv + ck - 1) / ck;
+    // Pick the split count whose waves of resident CTAs waste the least, preferring fewer splits
+    // (less merge work) when two choices are within 3% of each other.
+    int best = 1;
+    double best_cost = 1e30;
+    for (int sp = 1; sp <= max_splits && sp <= 64; ++sp) {
+        const int eff = decode_effective_splits(Skv, group, sp);
+        if (eff != sp)
+            continue;
+        const long long ctas = pairs * sp;
+        const long long waves = (ctas + slots - 1) / slots;
+        const double cost = static_cast<double>(waves) / sp + 0.002 * sp;  // + merge overhead per split
+        if (cost < best_cost * 0.97) {
+            best_cost = cost;
+            best = sp;
+        }
+    }
+    return best;
+}
+
+int run(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq, int Hkv, int Sq, int Skv,
+        int D, float scale, int causal, int decode_splits, void *stream_ptr)
+{
+    int rc = validate(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, D, scale, causal);
+    if (rc != ATTN_OK)
+        return rc;
+    if (decode_splits < 0)
+        return ATTN_ERR_SHAPE;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+    std::lock_guard<std::mutex> lock(g_mutex);
+    int err = ATTN_OK;
+    DeviceState *s = device_state(&err);
+    if (!s)
+        return err;
+
+    if (Sq == 1) {
+        const int group = Hq / Hkv;
+        const int G = decode_heads_per_cta(group);
+        const long long pairs = static_cast<long long>(B) * Hkv * (group / G);
+        int splits = decode_splits > 0 ? decode_splits : choose_splits(*s, B, Hq, Hkv, Skv, D);
+        splits = decode_effective_splits(Skv, group, splits);
+        if (pairs * splits > INT_MAX)
+            return ATTN_ERR_SHAPE;
+        const size_t n_partials =
+            splits > 1 ? static_cast<size_t>(B) * Hq * splits * (static_cast<size_t>(D) + 1) : 0;
+        rc = ensure_workspace(*s, static_cast<size_t>(pairs), n_partials, stream);
+        if (rc != ATTN_OK)
+            return rc;
+        DecodeArgs a;
+        a.q = q;
+        a.k = k;
+        a.v = v;
+        a.o = o;
+        a.lse = lse;
+        a.B = B;
+        a.Hq = Hq;
+        a.Hkv = Hkv;
+        a.Skv = Skv;
+        a.D = D;
+        a.scale = scale;
+        a.splits = splits;
+        a.ws_o = s->partials;
+        a.ws_lse = s->partials + static_cast<size_t>(B) * Hq * splits * D;
+        a.counters = s->counters;
+        a.status = s->status;
+        if (launch_decode(a, stream) != cudaSuccess) {
+            cudaGetLastError();
+            return ATTN_ERR_LAUNCH;
+        }
+        return ATTN_OK;
+    }
+
+    rc = ensure_workspace(*s, 0, 0, stream);
+    if (rc != ATTN_OK)
+        return rc;
+    PrefillArgs a;
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.o = o;
+    a.lse = lse;
+    a.B = B;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.Sq = Sq;
+    a.Skv = Skv;
+    a.D = D;
+    a.scale = scale;
+    a.causal = causal;
+    a.status = s->status;
+    int encode_error = 0;
+    const cudaError_t e = launch_prefill(a, stream, &encode_error);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return encode_error != 0 ? ATTN_ERR_CUDA : ATTN_ERR_LAUNCH;
+    }
+    return ATTN_OK;
+}
+
+}  // namespace
+}  // namespace attn_b200
+
+using namespace attn_b200;
+
+extern "C" int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq, int Hkv,
+                        int Sq, int Skv, int D, float scale, int causal, void *stream)
+{
+    return run(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, D, scale, causal, 0, stream);
+}
+
+extern "C" int attn_fwd_ex(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
+                           int Hkv, int Sq, int Skv, int D, float scale, int causal, int decode_splits, void *stream)
+{
+    return run(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, D, scale, causal, decode_splits, stream);
+}
+
+extern "C" int attn_decode_splits(int B, int Hq, int Hkv, int Skv, int D)
+{
+    if (B < 1 || Hq < 1 || Hkv < 1 || Skv < 1)
+        return ATTN_ERR_SHAPE;
+    if (Hq % Hkv != 0)
+        return ATTN_ERR_GQA;
+    if (D != 32 && D != 64 && D != 128)
+        return ATTN_ERR_HEADDIM;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    int err = ATTN_OK;
+    DeviceState *s = device_state(&err);
+    if (!s)
+        return err;
+    return decode_effective_splits(Skv, Hq / Hkv, choose_splits(*s, B, Hq, Hkv, Skv, D));
+}
+
+extern "C" const char *attn_status_string(int status)
+{
+    switch (status) {
+    case ATTN_OK:
+        return "ok";
+    case ATTN_ERR_NULL:
+        return "a required pointer is NULL";
+    case ATTN_ERR_SHAPE:
+        return "invalid size: every size must be >= 1, causal must be 0 or 1, and flat row indices must fit in int32";
+    case ATTN_ERR_GQA:
+        return "Hq must be a multiple of Hkv";
+    case ATTN_ERR_HEADDIM:
+        return "unsupported head dim: D must be 32, 64 or 128";
+    case ATTN_ERR_ALIGN:
+        return "every pointer must be 16-byte aligned";
+    case ATTN_ERR_CAUSAL_SQ_GT_SKV:
+        return "causal attention needs Sq <= Skv (the mask covers the last Sq keys)";
+    case ATTN_ERR_ARCH:
+        return "the current device is not an sm_100 (B200-class) GPU";
+    case ATTN_ERR_WORKSPACE:
+        return "could not allocate the library workspace";
+    case ATTN_ERR_LAUNCH:
+        return "kernel launch failed";
+    case ATTN_ERR_DEVICE_TIMEOUT:
+        return "a kernel-side wait ran out of time; the results of that call are invalid";
+    case ATTN_ERR_SCALE:
+        return "scale must be finite and > 0";
+    case ATTN_ERR_CUDA:
+        return "a CUDA runtime call failed";
+    default:
+        return "unknown status";
+    }
+}
+
+extern "C" int attn_version(void) { return kVersion; }
+
+extern "C" int attn_device_status(void *stream_ptr)
+{
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+    std::lock_guard<std::mutex> lock(g_mutex);
+    int err = ATTN_OK;
+    DeviceState *s = device_state(&err);
+    if (!s)
+        return err;
+    if (!s->block)
+        return ATTN_OK;
+    int value = 0;
+    if (cudaMemcpyAsync(&value, s->status, sizeof(int), cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+        cudaStreamSynchronize(stream) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_CUDA;
+    }
+    if (value != 0) {
+        const int zero = 0;
+        if (cudaMemcpyAsync(s->status, &zero, sizeof(int), cudaMemcpyHostToDevice, stream) != cudaSuccess ||
+            cudaStreamSynchronize(stream) != cudaSuccess) {
+            cudaGetLastError();
+            return ATTN_ERR_CUDA;
+        }
+        return ATTN_ERR_DEVICE_TIMEOUT;
+    }
+    return ATTN_OK;
+}

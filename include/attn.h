@@ -1,0 +1,109 @@
+/*
+ * attn.h — C ABI of libattn_b200.so: fused causal scaled-dot-product attention on B200 (sm_100a).
+ *
+ * The operation (per batch b, query head h, query row i; kv head = h / (Hq / Hkv)):
+ *
+ *   key j is visible to query i  iff  j < Skv  and  (!causal or j <= i + (Skv - Sq))
+ *   s_j    = scale * (q_i . k_j)
+ *   o_i    = sum_j softmax(s)_j * v_j          over the visible keys
+ *   lse_i  = ln( sum_j exp(s_j) )              over the visible keys (natural log, scaled scores)
+ *
+ * Sources (page title, section):
+ *   scores and the 1/sqrt(d) scale ... "05 · Tích vô hướng, Softmax và toán của Attention", §1 and
+ *                                      "Vì sao chia cho √128";
+ *   safe / online softmax, LSE ....... "AI Infra 入门：RMSNorm、Softmax、Causal Mask、Sampling 的数学与
+ *                                      底层优化", §2-§3 (running max and sum rescaled by
+ *                                      exp(m_old - m_new); LSE compresses (m, l) into one scalar and
+ *                                      is the merge key of split-KV decoding);
+ *   mask aligned to the last Sq keys . "第11节：Attention 实现（Flash vs Fallback）", §3 (the -inf upper
+ *                                      triangle is added to the last seq_len key columns of a KV cache);
+ *   decode needs no mask ............. "AI Infra 入门…", §3 (a single new query sees every cached key);
+ *   grouped K/V heads ................ "05 · Tích vô hướng…", §4 (32 query heads share 8 K/V heads).
+ *
+ * Layout (all contiguous, row-major): q [B, Hq, Sq, D], k and v [B, Hkv, Skv, D], o [B, Hq, Sq, D],
+ * all bf16; lse [B, Hq, Sq] fp32.
+ *
+ * Ownership: every pointer is a DEVICE pointer owned by the caller. The library keeps no pointer
+ * after the work completes on `stream`. The library owns one small per-device workspace (the
+ * split-KV partials of the decode kernel and a status word); it grows on the first call that needs
+ * more, with cudaMalloc (so that first call is not stream-ordered and cannot be graph-captured).
+ * Concurrent decode calls on different streams of one device share that workspace and must be
+ * serialised by the caller.
+ *
+ * Errors: argument errors are detected on the host before any launch and returned as a negative
+ * attn_status; nothing is launched then. Launch failures return ATTN_ERR_LAUNCH. The call never
+ * synchronises the stream, never aborts the process and never traps on the device. Kernel-side
+ * waits are bounded: a wait that runs out sets the device status word, which attn_device_status()
+ * reads.
+ */
+#ifndef ATTN_B200_ATTN_H
+#define ATTN_B200_ATTN_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum attn_status {
+    ATTN_OK = 0,
+    ATTN_ERR_NULL = -1,             /* a required pointer is NULL */
+    ATTN_ERR_SHAPE = -2,            /* a size is < 1 or the problem exceeds the supported index range */
+    ATTN_ERR_GQA = -3,              /* Hq is not a multiple of Hkv */
+    ATTN_ERR_HEADDIM = -4,          /* D is not 32, 64 or 128 */
+    ATTN_ERR_ALIGN = -5,            /* a pointer is not 16-byte aligned */
+    ATTN_ERR_CAUSAL_SQ_GT_SKV = -6, /* causal with Sq > Skv: early rows would see no key */
+    ATTN_ERR_ARCH = -7,             /* the current device is not compute capability 10.0 (sm_100a) */
+    ATTN_ERR_WORKSPACE = -8,        /* the library workspace could not be allocated */
+    ATTN_ERR_LAUNCH = -9,           /* a kernel launch failed */
+    ATTN_ERR_DEVICE_TIMEOUT = -10,  /* a kernel-side wait ran out (reported by attn_device_status) */
+    ATTN_ERR_SCALE = -11,           /* scale is not finite and > 0 */
+    ATTN_ERR_CUDA = -12             /* a CUDA runtime call failed (device query, tensor map, copy) */
+} attn_status;
+
+/*
+ * attn_fwd — the whole forward pass: o and lse for every (b, h, i).
+ *   q, k, v   device pointers, bf16, layouts above, 16-byte aligned.
+ *   o         device pointer, bf16 [B, Hq, Sq, D], written entirely.
+ *   lse       device pointer, fp32 [B, Hq, Sq], written entirely.
+ *   B, Hq, Hkv, Sq, Skv, D   sizes; Hq % Hkv == 0; D in {32, 64, 128}.
+ *   scale     multiplies q . k (normally 1/sqrt(D)); must be finite and > 0.
+ *   causal    0 or 1. With Sq == 1 the mask hides nothing and both values give the same result.
+ *   stream    a cudaStream_t (NULL = the legacy default stream).
+ * Sq == 1 runs the split-KV decode kernel; every other shape runs the prefill kernel.
+ * Returns ATTN_OK or a negative attn_status.
+ */
+int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+             int B, int Hq, int Hkv, int Sq, int Skv, int D,
+             float scale, int causal, void *stream);
+
+/*
+ * attn_fwd_ex — attn_fwd with the decode split count fixed by the caller (decode_splits >= 1),
+ * or chosen by the library (decode_splits == 0). The split count is a performance parameter:
+ * results agree with attn_fwd within rounding. Ignored when Sq > 1.
+ */
+int attn_fwd_ex(const void *q, const void *k, const void *v, void *o, float *lse,
+                int B, int Hq, int Hkv, int Sq, int Skv, int D,
+                float scale, int causal, int decode_splits, void *stream);
+
+/* attn_decode_splits — the split count attn_fwd would use for a decode of this shape on the
+ * current device (>= 1), or a negative attn_status. */
+int attn_decode_splits(int B, int Hq, int Hkv, int Skv, int D);
+
+/* attn_status_string — a static, human-readable description of a status code. Never NULL. */
+const char *attn_status_string(int status);
+
+/* attn_version — library version as major * 10000 + minor * 100 + patch. */
+int attn_version(void);
+
+/*
+ * attn_device_status — synchronises `stream`, then reads and clears the current device's status
+ * word. Returns ATTN_OK if no kernel-side wait has run out since the last call,
+ * ATTN_ERR_DEVICE_TIMEOUT if one has, or ATTN_ERR_CUDA if the stream could not be synchronised.
+ * This is a diagnostic call: it blocks the host, so it does not belong on a hot path.
+ */
+int attn_device_status(void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_B200_ATTN_H */
