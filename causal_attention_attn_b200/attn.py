@@ -22,9 +22,10 @@ STATUS_NAMES = {
     0: "ATTN_OK", -1: "ATTN_ERR_NULL", -2: "ATTN_ERR_SHAPE", -3: "ATTN_ERR_GQA", -4: "ATTN_ERR_HEADDIM",
     -5: "ATTN_ERR_ALIGN", -6: "ATTN_ERR_CAUSAL_SQ_GT_SKV", -7: "ATTN_ERR_ARCH", -8: "ATTN_ERR_WORKSPACE",
     -9: "ATTN_ERR_LAUNCH", -10: "ATTN_ERR_DEVICE_TIMEOUT", -11: "ATTN_ERR_SCALE", -12: "ATTN_ERR_CUDA",
+    -13: "ATTN_ERR_SCRATCH_LIMIT",
 }
 EXPORTED = ("attn_fwd", "attn_fwd_ex", "attn_decode_splits", "attn_status_string", "attn_version",
-            "attn_device_status")
+            "attn_device_status", "attn_decode_noalloc")
 
 _lock = threading.Lock()
 _lib = None
@@ -60,6 +61,8 @@ def load_library(path: str | None = None):
         lib.attn_version.argtypes = []
         lib.attn_device_status.restype = i
         lib.attn_device_status.argtypes = [vp]
+        lib.attn_decode_noalloc.restype = i
+        lib.attn_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, vp]
         if path is None:
             _lib = lib
         return lib
@@ -170,6 +173,33 @@ def attn_fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: floa
         lse_host.copy_(ld, non_blocking=True)
     stream.synchronize()
     return out_host, lse_host
+
+
+def attn_decode_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: float | None = None,
+                        out: torch.Tensor | None = None, lse: torch.Tensor | None = None, stream=None):
+    """Single-token decode through ``attn_decode_noalloc``: the library allocates nothing (its
+    scratch is a fixed device array). For callers that must not have the library call cudaMalloc.
+    ``out`` and ``lse`` should be passed by such callers; when omitted they are created here with
+    torch. q: [B, Hq, 1, D]; k/v: [B, Hkv, Skv, D]. Returns (o, lse)."""
+    _check_tensor("q", q, torch.bfloat16, 4)
+    _check_tensor("k", k, torch.bfloat16, 4)
+    _check_tensor("v", v, torch.bfloat16, 4)
+    B, Hq, Sq, D = q.shape
+    Bk, Hkv, Skv, Dk = k.shape
+    if Sq != 1 or tuple(v.shape) != tuple(k.shape) or Bk != B or Dk != D:
+        raise ValueError(f"expected q [B,Hq,1,D] and k, v [B,Hkv,Skv,D]; got {tuple(q.shape)}, {tuple(k.shape)}")
+    if scale is None:
+        scale = D ** -0.5
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, Hq, 1), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check_tensor("out", out, torch.bfloat16, 4)
+    _check_tensor("lse", lse, torch.float32, 3)
+    with torch.cuda.device(q.device):
+        rc = load_library().attn_decode_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                                lse.data_ptr(), B, Hq, Hkv, Skv, D, float(scale),
+                                                _stream_handle(stream))
+    _check(rc)
+    return out, lse
 
 
 def decode_splits(B: int, Hq: int, Hkv: int, Skv: int, D: int) -> int:

@@ -304,6 +304,9 @@ extern "C" const char *attn_status_string(int status)
         return "scale must be finite and > 0";
     case ATTN_ERR_CUDA:
         return "a CUDA runtime call failed";
+    case ATTN_ERR_SCRATCH_LIMIT:
+        return "the decode needs more scratch than the fixed no-allocation buffer holds "
+               "(too many (batch, kv head) pairs for attn_decode_noalloc)";
     default:
         return "unknown status";
     }

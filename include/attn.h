@@ -56,7 +56,8 @@ typedef enum attn_status {
     ATTN_ERR_LAUNCH = -9,           /* a kernel launch failed */
     ATTN_ERR_DEVICE_TIMEOUT = -10,  /* a kernel-side wait ran out (reported by attn_device_status) */
     ATTN_ERR_SCALE = -11,           /* scale is not finite and > 0 */
-    ATTN_ERR_CUDA = -12             /* a CUDA runtime call failed (device query, tensor map, copy) */
+    ATTN_ERR_CUDA = -12,            /* a CUDA runtime call failed (device query, tensor map, copy) */
+    ATTN_ERR_SCRATCH_LIMIT = -13    /* attn_decode_noalloc: the problem needs more scratch than its fixed buffer */
 } attn_status;
 
 /*
@@ -101,6 +102,37 @@ int attn_version(void);
  * This is a diagnostic call: it blocks the host, so it does not belong on a hot path.
  */
 int attn_device_status(void *stream);
+
+/*
+ * attn_decode_noalloc — single-token decode (Sq == 1) that allocates no memory.
+ *
+ * The pages have no counterpart to this entry point: it is an interface addition for callers that
+ * must not have a library allocate device memory — a serving loop that cannot absorb the device
+ * synchronisation and latency of cudaMalloc in the middle of a request, or a process whose device
+ * memory is owned by one allocator or a budget fixed at start-up, where an allocation behind that
+ * allocator's back fails or breaks its accounting. attn_fwd grows a workspace with cudaMalloc on
+ * first use; this call instead uses a fixed array of ATTN_DECODE_NOALLOC_SCRATCH_BYTES in the
+ * library's own device memory, reserved on every GPU that loads the library until the process
+ * exits. It calls no cudaMalloc, cudaFree or other allocating routine.
+ *
+ * Arguments are those of attn_fwd with Sq = 1 and no causal flag (a single new query sees every
+ * cached key): q [B, Hq, 1, D], k and v [B, Hkv, Skv, D], o [B, Hq, 1, D] bf16; lse [B, Hq, 1] fp32;
+ * all device pointers owned by the caller, 16-byte aligned. Results agree with attn_fwd within
+ * rounding (the split count may be lowered so that the partials fit).
+ *
+ * The first call on a device looks up that device's address of the array (cudaGetSymbolAddress,
+ * with the device current); make that first call before any stream capture. Every call on a device
+ * shares the array and it keeps the last call's contents; the counters that must start at zero are
+ * cleared on `stream` before each launch. Calls that overlap on the GPU (different streams with no
+ * ordering between them) race on the array: serialise them.
+ *
+ * Returns ATTN_OK, an argument error as attn_fwd does, or ATTN_ERR_SCRATCH_LIMIT when the
+ * arrival counters alone (one int per (batch, kv head, group of up to 8 query heads)) do not fit in
+ * the array, i.e. beyond about two million such triples; nothing is launched then.
+ */
+#define ATTN_DECODE_NOALLOC_SCRATCH_BYTES (8u << 20) /* 8 MiB */
+int attn_decode_noalloc(const void *q, const void *k, const void *v, void *o, float *lse,
+                        int B, int Hq, int Hkv, int Skv, int D, float scale, void *stream);
 
 #ifdef __cplusplus
 }
