@@ -1,18 +1,25 @@
 /*
  * prefill_sm100.cu — fused causal attention forward for Sq > 1 on sm_100a.
  *
- * One CTA computes one tile of 128 query rows of one (batch, query head). Per KV tile of 128 keys:
+ * One CTA computes two consecutive 128-row query tiles (A and B) of one (batch, query head). Both
+ * tiles stream the same K/V tiles of 128 keys, so each K/V tile is brought into shared memory once
+ * for 256 query rows. Per KV tile j and per query tile X in {A, B}:
  *
- *   S = Q K^T          tcgen05.mma, bf16 operands in shared memory (TMA-loaded, 128B swizzle),
- *                      fp32 accumulator in tensor memory (TMEM), double-buffered so the next
- *                      tile's S is computed while this tile's softmax runs;
- *   online softmax     one query row per thread (TMEM lane = row): scale, cache-aligned causal
- *                      mask on diagonal tiles only, running max m and running sum l, rescale of the
- *                      O accumulator by exp(m_old - m_new);
- *   O += P V           P rounded to bf16 into shared memory, tcgen05.mma with V read MN-major
- *                      (O is divided by the sum of these rounded weights; the LSE uses the sum of
- *                      the exact fp32 weights);
- *   epilogue           O / l to bf16, LSE = (m + log2 l) * ln 2.
+ *   S_X = Q_X K_j^T    tcgen05.mma, bf16 Q and K in shared memory (TMA-loaded, 128B swizzle),
+ *                      fp32 accumulator in tensor memory (TMEM);
+ *   online softmax     one query row per thread (TMEM lane = row): scale to log2 units, the
+ *                      cache-aligned causal mask on diagonal tiles only, running max and sum, and
+ *                      the exp(m_old - m_new) rescale of the O_X accumulator in TMEM;
+ *   O_X += P_X V_j     P_X rounded to bf16 and written back into TMEM over the first half of
+ *                      S_X's columns, then tcgen05.mma with A = P_X read from TMEM and B = V_j read
+ *                      MN-major from shared memory;
+ *   epilogue           O_X / l_X to bf16, LSE = (m + log2 l) * ln 2.
+ *
+ * The two tiles ping-pong: while the softmax warps of A work on S_A(j), the tensor core runs
+ * S_B(j) and the PV product and next S of B, and the other way round. Because the MMAs of one
+ * thread execute in issue order, the commit that announces S_X(j) also proves that PV_X(j-1) has
+ * finished, so the softmax may rescale O_X right away, and S_X(j+1) — issued after PV_X(j) — never
+ * overwrites P_X(j) before it has been read.
  *
  * Sources (page title, section): the fused single sweep over K/V per Q tile with S and P never
  * written to HBM — "AI Infra 入门：RMSNorm、Softmax、Causal Mask、Sampling 的数学与底层优化", §3
@@ -21,16 +28,21 @@
  * and sum with the exp(m_old - m_new) rescale, which must also be applied to the output
  * accumulator — same page §3 and "Bộ 06 · Bên trong model", Q1; the mask aligned to the last Sq
  * key columns — "第11节：Attention 实现（Flash vs Fallback）", §3; bf16 storage with fp32
- * accumulation — "MLA 矩阵乘法吸收的数值稳定性治理", §二.2 and §五.
+ * accumulation — "MLA 矩阵乘法吸收的数值稳定性治理", §二.2 and §五; the tcgen05/TMEM design space
+ * (two query tiles, P kept on chip, softmax warps separate from the MMA issuer) — "AI Infra 入门",
+ * §3 (FA4 paragraph), taken as prior art.
  *
  * Rescale threshold: the running max used for the exponentials is only moved when the new row
  * max exceeds it by more than 8 (in log2 units). The exponentials are then at most 2^8, which bf16
  * P and the fp32 sums hold without loss, and O and l stay consistent because both are accumulated
  * against the same reference max; the final O / l and LSE = m_ref + log2 l are the same quantities
- * as with an exact running max.
+ * as with an exact running max. O is divided by the sum of the bf16-rounded weights it was built
+ * from; the LSE uses the sum of the exact fp32 weights.
  *
- * Warp roles (192 threads): warps 0-3 softmax + correction + epilogue (warp w owns TMEM lanes
- * 32w..32w+31), warp 4 TMA producer, warp 5 TMEM allocator and MMA issuer (one thread issues).
+ * Warp roles (384 threads): warps 0-3 softmax / correction / epilogue of tile A, warps 4-7 the
+ * same for tile B (warp w owns TMEM lanes 32(w%4)..+31), warp 8 TMA producer, warp 9 TMEM
+ * allocator and MMA issuer (one thread issues), warps 10-11 idle. setmaxnreg moves registers from
+ * the third warpgroup to the two softmax warpgroups.
  */
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -49,11 +61,19 @@ namespace {
 constexpr int kBM = 128;  // query rows per tile = TMEM lanes = MMA M
 constexpr int kBN = 128;  // keys per KV tile = MMA N of S and K of PV
 constexpr int kRing = 4;  // K/V tile slots
-constexpr int kSoftmaxWarps = 4;
-constexpr int kWarpTma = 4;
-constexpr int kWarpMma = 5;
-constexpr int kThreads = 192;
-constexpr uint32_t kTmemCols = 512;  // S0 [0,128), S1 [128,256), O [256, 256+D)
+constexpr int kWarpTma = 8;
+constexpr int kWarpMma = 9;
+constexpr int kThreads = 384;  // three warpgroups: softmax A, softmax B, producer + MMA (+ 2 spare warps)
+// Register split: the block is launched with kLaunchRegs per thread (the host checks the compiled
+// count before every first launch); the producer/MMA warpgroup gives registers back and the two
+// softmax warpgroups take them, so the three shares add up to exactly the launch allocation.
+constexpr int kLaunchRegs = 168;
+constexpr int kRegsSoftmax = 232;
+constexpr int kRegsOther = 40;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther == kThreads * kLaunchRegs, "register split");
+constexpr uint32_t kTmemCols = 512;  // S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512)
+__host__ __device__ constexpr uint32_t col_s(int x) { return static_cast<uint32_t>(x) * 128u; }        // S_X
+__host__ __device__ constexpr uint32_t col_o(int x) { return 256u + static_cast<uint32_t>(x) * 128u; }  // O_X
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;
@@ -66,11 +86,9 @@ struct Cfg {
     static constexpr int kChunks = D / kChunkElems;
     static constexpr int kChunkBytes = 128 * kSwizzleBytes;  // 128 rows of one column block
     static constexpr int kTileBytes = 128 * D * 2;
-    static constexpr int kPBytes = kBM * kBN * 2;
-    static constexpr int kOffQ = 0;
-    static constexpr int kOffRing = kOffQ + kTileBytes;
-    static constexpr int kOffP = kOffRing + kRing * kTileBytes;
-    static constexpr int kOffBar = kOffP + kPBytes;
+    static constexpr int kOffQ = 0;  // Q_A, then Q_B
+    static constexpr int kOffRing = kOffQ + 2 * kTileBytes;
+    static constexpr int kOffBar = kOffRing + kRing * kTileBytes;
     static constexpr int kUsed = kOffBar + 256;
     // >= 118 KB so that two CTAs never share an SM: each one allocates all 512 TMEM columns.
     static constexpr int kSmem = (kUsed + 1024 > 118 * 1024) ? kUsed + 1024 : 118 * 1024;
@@ -82,11 +100,10 @@ enum Bar : int {
     kBarQ = 0,
     kBarFull0 = 1,
     kBarEmpty0 = kBarFull0 + kRing,
-    kBarSFull0 = kBarEmpty0 + kRing,
-    kBarSFree0 = kBarSFull0 + 2,
-    kBarPFull = kBarSFree0 + 2,
-    kBarODone = kBarPFull + 1,
-    kBarDrain = kBarODone + 1,
+    kBarSFull0 = kBarEmpty0 + kRing,  // [A, B]
+    kBarPFull0 = kBarSFull0 + 2,      // [A, B]
+    kBarOFinal0 = kBarPFull0 + 2,     // [A, B]
+    kBarDrain = kBarOFinal0 + 2,
     kNumBars = kBarDrain + 1,
 };
 static_assert(kNumBars * 8 <= 128, "barrier area");
@@ -95,7 +112,7 @@ struct Params {
     __nv_bfloat16 *o;
     float *lse;
     int *status;
-    int B, Hq, Hkv, Sq, Skv, group, offset, causal, n_qtiles;
+    int B, Hq, Hkv, Sq, Skv, group, offset, causal, n_pairs;
     float scale_log2;
 };
 
@@ -112,12 +129,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
-{
-    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
-                 : "memory");
-}
-
 // Wait that ignores the abort flag (used to drain in-flight async work before exit).
 __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, uint64_t limit_ns)
 {
@@ -129,23 +140,15 @@ __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, u
     return true;
 }
 
-// Order in which K and V tiles are loaded and consumed: K0, K1, V0, K2, V1, ..., K(n-1), V(n-2), V(n-1).
-__device__ __forceinline__ void kv_item(int it, int n_kv, int &tile, bool &is_v)
+// Number of KV tiles a 128-row query tile starting at q0 needs (0 if the tile lies past Sq).
+__device__ __forceinline__ int kv_tiles_for(const Params &p, int q0)
 {
-    if (it == 0) {
-        tile = 0;
-        is_v = false;
-        return;
-    }
-    const int u = it - 1;
-    const int j = u >> 1;
-    if ((u & 1) == 0 && j + 1 < n_kv) {
-        tile = j + 1;
-        is_v = false;
-    } else {
-        tile = j;
-        is_v = true;
-    }
+    if (q0 >= p.Sq)
+        return 0;
+    int kv_end = p.Skv;
+    if (p.causal)
+        kv_end = min(p.Skv, q0 + kBM + p.offset);  // last visible key of the tile's last row, + 1
+    return (kv_end + kBN - 1) / kBN;
 }
 
 template <int D>
@@ -159,7 +162,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t s_base = smem_u32(smem);
     const uint32_t sQ = s_base + C::kOffQ;
     const uint32_t sRing = s_base + C::kOffRing;
-    const uint32_t sP = s_base + C::kOffP;
     const uint32_t bar0 = s_base + C::kOffBar;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kOffBar + 128);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::kOffBar + 132);
@@ -168,22 +170,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // Tile decode: heads fastest, then batch, then query tiles from the last (heaviest) one.
+    // Work decode: heads fastest, then batch, then pairs of query tiles from the last (heaviest).
     int t = blockIdx.x;
     const int h = t % p.Hq;
     t /= p.Hq;
     const int b = t % p.B;
     t /= p.B;
-    const int qt = p.n_qtiles - 1 - t;
-    const int q0 = qt * kBM;
+    const int pair = p.n_pairs - 1 - t;
+    const int q0_a = pair * 2 * kBM;  // tile A rows [q0_a, q0_a + 128), tile B the next 128
+    const int n_a = kv_tiles_for(p, q0_a);
+    const int n_b = kv_tiles_for(p, q0_a + kBM);
+    const int n_max = max(n_a, n_b);
+    auto q0_of = [&](int x) { return q0_a + x * kBM; };
+    auto n_of = [&](int x) { return x ? n_b : n_a; };
     const int bh_q = b * p.Hq + h;
     const int bh_kv = b * p.Hkv + h / p.group;
-
-    // Keys visible to any row of this tile: [0, kv_end). Tiles past it are skipped entirely.
-    int kv_end = p.Skv;
-    if (p.causal)
-        kv_end = min(p.Skv, q0 + kBM + p.offset);
-    const int n_kv = (kv_end + kBN - 1) / kBN;
 
     if (threadIdx.x == 0) {
         mbar_init(BAR(kBarQ), 1);
@@ -191,12 +192,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(BAR(kBarFull0 + r), 1);
             mbar_init(BAR(kBarEmpty0 + r), 1);
         }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(BAR(kBarSFull0 + i), 1);
-            mbar_init(BAR(kBarSFree0 + i), kSoftmaxWarps * 32);
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(BAR(kBarSFull0 + x), 1);
+            mbar_init(BAR(kBarPFull0 + x), 128);
+            mbar_init(BAR(kBarOFinal0 + x), 1);
         }
-        mbar_init(BAR(kBarPFull), kSoftmaxWarps * 32);
-        mbar_init(BAR(kBarODone), 1);
         mbar_init(BAR(kBarDrain), 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -215,31 +215,35 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == kWarpTma) {
+    if (warp >= 8) {
+      // Third warpgroup: gives registers back, then splits into the producer and the MMA issuer.
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
+      if (warp == kWarpTma) {
         // ---------------------------------------------------------------- TMA producer
         if (lane == 0) {
             const uint64_t pol = l2_policy_evict_last();  // K/V tiles are re-read by sibling CTAs
-            mbar_arrive_expect_tx(BAR(kBarQ), C::kTileBytes);
+            const int n_q = (n_b > 0) ? 2 : 1;
+            mbar_arrive_expect_tx(BAR(kBarQ), n_q * C::kTileBytes);
+            for (int x = 0; x < n_q; ++x)
 #pragma unroll
-            for (int c = 0; c < C::kChunks; ++c)
-                tma_load_3d(sQ + c * C::kChunkBytes, &tm_q, BAR(kBarQ), c * C::kChunkElems, q0, bh_q);
-            const int n_items = 2 * n_kv;
+                for (int c = 0; c < C::kChunks; ++c)
+                    tma_load_3d(sQ + x * C::kTileBytes + c * C::kChunkBytes, &tm_q, BAR(kBarQ), c * C::kChunkElems,
+                                q0_of(x), bh_q);
+            // Items in consumption order: K0, V0, K1, V1, ...
+            const int n_items = 2 * n_max;
             int issued = 0;
             for (int it = 0; it < n_items; ++it) {
-                int tile;
-                bool is_v;
-                kv_item(it, n_kv, tile, is_v);
                 const int slot = it % kRing;
                 const uint32_t round = static_cast<uint32_t>(it / kRing);
                 if (!mbar_wait(BAR(kBarEmpty0 + slot), (round & 1u) ^ 1u, abort_flag, p.status, kSitePrefillTmaEmpty))
                     break;
                 mbar_arrive_expect_tx(BAR(kBarFull0 + slot), C::kTileBytes);
-                const CUtensorMap *map = is_v ? &tm_v : &tm_k;
+                const CUtensorMap *map = (it & 1) ? &tm_v : &tm_k;
                 const uint32_t dst = sRing + slot * C::kTileBytes;
 #pragma unroll
                 for (int c = 0; c < C::kChunks; ++c)
                     tma_load_3d_hint(dst + c * C::kChunkBytes, map, BAR(kBarFull0 + slot), c * C::kChunkElems,
-                                     tile * kBN, bh_kv, pol);
+                                     (it >> 1) * kBN, bh_kv, pol);
                 ++issued;
             }
             if (*abort_flag) {
@@ -256,73 +260,73 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr uint32_t kIdS = idesc_bf16_f32(kBM, kBN, false);
             constexpr uint32_t kIdO = idesc_bf16_f32(kBM, D, true);
             constexpr uint32_t kSbo = 8 * C::kSwizzleBytes;  // 8 rows of one swizzled column block
-            const uint32_t tS0 = tmem;
-            const uint32_t tO = tmem + 2 * kBN;
-            int it = 0;
 
-            auto issue_s = [&](uint32_t d_tmem, uint32_t sK) {
+            auto issue_s = [&](int x, uint32_t sK) {
+                const uint32_t sQx = sQ + x * C::kTileBytes;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const int c = kk / (C::kChunkElems / 16);
                     const int w = kk % (C::kChunkElems / 16);
                     const uint32_t off = c * C::kChunkBytes + w * 32;
-                    tc_mma_ss(d_tmem, smem_desc(sQ + off, 16, kSbo, C::kSwizzleMode),
+                    tc_mma_ss(tmem + col_s(x), smem_desc(sQx + off, 16, kSbo, C::kSwizzleMode),
                               smem_desc(sK + off, 16, kSbo, C::kSwizzleMode), kIdS, kk > 0 ? 1u : 0u);
                 }
             };
-            auto issue_pv = [&](uint32_t sV, bool accumulate) {
+            auto issue_pv = [&](int x, uint32_t sV, bool accumulate) {
 #pragma unroll
                 for (int kk = 0; kk < kBN / 16; ++kk) {
-                    const uint32_t a_addr = sP + (kk >> 2) * (kBM * 128) + (kk & 3) * 32;
-                    const uint32_t b_addr = sV + kk * 16 * C::kSwizzleBytes;
-                    tc_mma_ss(tO, smem_desc(a_addr, 16, 1024, kSwizzle128B),
-                              smem_desc(b_addr, C::kChunkBytes, kSbo, C::kSwizzleMode), kIdO,
+                    // P_X: 16 keys = 8 packed columns per step, in the first half of S_X's columns.
+                    tc_mma_ts(tmem + col_o(x), tmem + col_s(x) + kk * 8,
+                              smem_desc(sV + kk * 16 * C::kSwizzleBytes, C::kChunkBytes, kSbo, C::kSwizzleMode), kIdO,
                               (accumulate || kk > 0) ? 1u : 0u);
                 }
             };
+            auto wait_item = [&](int item) -> bool {
+                return mbar_wait(BAR(kBarFull0 + item % kRing), static_cast<uint32_t>(item / kRing) & 1u, abort_flag,
+                                 p.status, kSitePrefillMmaFull);
+            };
+            auto slot_of = [&](int item) { return sRing + (item % kRing) * C::kTileBytes; };
 
             bool ok = mbar_wait(BAR(kBarQ), 0, abort_flag, p.status, kSitePrefillMmaQ);
-            if (ok) {
-                const int slot = it % kRing;
-                ok = mbar_wait(BAR(kBarFull0 + slot), static_cast<uint32_t>(it / kRing) & 1u, abort_flag, p.status,
-                               kSitePrefillMmaFull);
+            if (ok && n_max > 0) {
+                ok = wait_item(0);
                 if (ok) {
                     tc_fence_after_sync();
-                    issue_s(tS0, sRing + slot * C::kTileBytes);
-                    tc_commit(BAR(kBarSFull0));
-                    tc_commit(BAR(kBarEmpty0 + slot));
-                    ++it;
+                    for (int x = 0; x < 2; ++x)
+                        if (n_of(x) > 0) {
+                            issue_s(x, slot_of(0));
+                            tc_commit(BAR(kBarSFull0 + x));
+                        }
+                    tc_commit(BAR(kBarEmpty0 + 0));
                 }
             }
-            for (int j = 0; ok && j < n_kv; ++j) {
-                if (j + 1 < n_kv) {
-                    const int sb = (j + 1) & 1;
-                    const uint32_t use = static_cast<uint32_t>((j + 1) >> 1);
-                    if (!(ok = mbar_wait(BAR(kBarSFree0 + sb), (use & 1u) ^ 1u, abort_flag, p.status,
-                                         kSitePrefillMmaSFree)))
+            for (int j = 0; ok && j < n_max; ++j) {
+                const int item_v = 2 * j + 1, item_k = 2 * j + 2;
+                for (int x = 0; ok && x < 2; ++x) {
+                    if (j >= n_of(x))
+                        continue;
+                    if (!(ok = mbar_wait(BAR(kBarPFull0 + x), static_cast<uint32_t>(j) & 1u, abort_flag, p.status,
+                                         kSitePrefillMmaPFull)))
                         break;
-                    const int slot = it % kRing;
-                    if (!(ok = mbar_wait(BAR(kBarFull0 + slot), static_cast<uint32_t>(it / kRing) & 1u, abort_flag,
-                                         p.status, kSitePrefillMmaFull)))
+                    if (!(ok = wait_item(item_v)))
                         break;
                     tc_fence_after_sync();
-                    issue_s(tS0 + sb * kBN, sRing + slot * C::kTileBytes);
-                    tc_commit(BAR(kBarSFull0 + sb));
-                    tc_commit(BAR(kBarEmpty0 + slot));
-                    ++it;
+                    issue_pv(x, slot_of(item_v), j > 0);
+                    if (j + 1 < n_of(x)) {
+                        if (!(ok = wait_item(item_k)))
+                            break;
+                        tc_fence_after_sync();
+                        issue_s(x, slot_of(item_k));
+                        tc_commit(BAR(kBarSFull0 + x));
+                    } else {
+                        tc_commit(BAR(kBarOFinal0 + x));
+                    }
                 }
-                if (!(ok = mbar_wait(BAR(kBarPFull), static_cast<uint32_t>(j) & 1u, abort_flag, p.status,
-                                     kSitePrefillMmaPFull)))
+                if (!ok)
                     break;
-                const int slot = it % kRing;
-                if (!(ok = mbar_wait(BAR(kBarFull0 + slot), static_cast<uint32_t>(it / kRing) & 1u, abort_flag,
-                                     p.status, kSitePrefillMmaFull)))
-                    break;
-                tc_fence_after_sync();
-                issue_pv(sRing + slot * C::kTileBytes, j > 0);
-                tc_commit(BAR(kBarODone));
-                tc_commit(BAR(kBarEmpty0 + slot));
-                ++it;
+                tc_commit(BAR(kBarEmpty0 + item_v % kRing));
+                if (j + 1 < n_max)
+                    tc_commit(BAR(kBarEmpty0 + item_k % kRing));
             }
             // Every MMA issued above has completed once this barrier flips.
             tc_commit(BAR(kBarDrain));
@@ -332,36 +336,37 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         __syncwarp();
+      }
     } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
         // ---------------------------------------------------------------- softmax / correction / epilogue
-        const int r = threadIdx.x;  // row within the tile == TMEM lane
-        const int row = q0 + r;
-        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-        const uint32_t tO = tmem + lane_base + 2 * kBN;
+        const int x = warp >> 2;        // query tile: 0 = A, 1 = B
+        const int r = threadIdx.x & 127;  // row within the tile == TMEM lane
+        const int row = q0_of(x) + r;
+        const int n = n_of(x);
+        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t tS = tmem + lane_base + col_s(x);
+        const uint32_t tO = tmem + lane_base + col_o(x);
         const float sl2 = p.scale_log2;
         float m = -INFINITY;  // reference max, log2-scaled units
         float l = 0.f;        // running sum of the exact fp32 weights (gives the LSE)
         float l_pv = 0.f;     // running sum of the bf16-rounded weights the PV product uses (normalises O)
         bool ok = true;
 
-        for (int j = 0; j < n_kv; ++j) {
-            const int sb = j & 1;
-            if (!(ok = mbar_wait(BAR(kBarSFull0 + sb), static_cast<uint32_t>(j >> 1) & 1u, abort_flag, p.status,
+        for (int j = 0; j < n; ++j) {
+            if (!(ok = mbar_wait(BAR(kBarSFull0 + x), static_cast<uint32_t>(j) & 1u, abort_flag, p.status,
                                  kSitePrefillSoftmaxSFull)))
                 break;
             tc_fence_after_sync();
             uint32_t s_raw[kBN];
-            tmem_ld128_wait(tmem + lane_base + sb * kBN, s_raw);
-            tc_fence_before_sync();
-            mbar_arrive(BAR(kBarSFree0 + sb));
-
-            float x[kBN];
+            tmem_ld128_wait(tS, s_raw);
+            float s[kBN];
 #pragma unroll
             for (int c = 0; c < kBN; ++c)
-                x[c] = __uint_as_float(s_raw[c]);
+                s[c] = __uint_as_float(s_raw[c]);
 
             const int k0 = j * kBN;
-            const bool need_mask = (k0 + kBN > p.Skv) || (p.causal && k0 + kBN - 1 > q0 + p.offset);
+            const bool need_mask = (k0 + kBN > p.Skv) || (p.causal && k0 + kBN - 1 > q0_of(x) + p.offset);
             if (need_mask) {
                 int limit = p.Skv - 1 - k0;  // last visible column of this tile for this row
                 if (p.causal)
@@ -369,12 +374,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int c = 0; c < kBN; ++c)
                     if (c > limit)
-                        x[c] = -INFINITY;
+                        s[c] = -INFINITY;
             }
-            float mx = x[0];
+            // Row max with eight independent chains.
+            float mx8[8];
 #pragma unroll
-            for (int c = 1; c < kBN; ++c)
-                mx = fmaxf(mx, x[c]);
+            for (int i = 0; i < 8; ++i)
+                mx8[i] = s[i];
+#pragma unroll
+            for (int c = 8; c < kBN; ++c)
+                mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
+            const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
             const float mx2 = mx * sl2;  // scale > 0, so the max commutes with scaling
 
             float alpha = 1.f;
@@ -389,58 +400,57 @@ __global__ void __launch_bounds__(kThreads, 1)
                     m = m_new;
                 }
             }
-            const float neg_m = -m;
-            float rowsum = 0.f, rowsum_pv = 0.f;
-            uint32_t pk[kBN / 2];
+            // Exponentials, packed bf16 weights, and both running sums; then P_X -> TMEM.
+            const float2 sl2x2 = make_float2(sl2, sl2);
+            const float2 negm2 = make_float2(-m, -m);
+            float2 sum[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                             make_float2(0.f, 0.f)};
+            float2 sum_pv[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                                make_float2(0.f, 0.f)};
 #pragma unroll
-            for (int c = 0; c < kBN / 2; ++c) {
-                const float p0 = ex2(fmaf(x[2 * c], sl2, neg_m));
-                const float p1 = ex2(fmaf(x[2 * c + 1], sl2, neg_m));
-                pk[c] = pack_bf16x2(p0, p1);
-                rowsum += p0 + p1;
-                // The bf16-rounded weights that the PV product uses are summed as well, so that
-                // O is divided by exactly the weight it was built from (a key that dominates a row
-                // then contributes its V row without the rounding error of its weight).
-                rowsum_pv += __uint_as_float(pk[c] << 16) + __uint_as_float(pk[c] & 0xffff0000u);
+            for (int half = 0; half < 2; ++half) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    const int col = half * 64 + 2 * c;
+                    const float2 e = __ffma2_rn(make_float2(s[col], s[col + 1]), sl2x2, negm2);
+                    const float2 pe = make_float2(ex2(e.x), ex2(e.y));
+                    pk[c] = pack_bf16x2(pe.x, pe.y);
+                    sum[c & 3] = __fadd2_rn(sum[c & 3], pe);
+                    sum_pv[c & 3] = __fadd2_rn(
+                        sum_pv[c & 3], make_float2(__uint_as_float(pk[c] << 16), __uint_as_float(pk[c] & 0xffff0000u)));
+                }
+                tmem_st32_wait(tS + half * 32, pk);
             }
-            l = l * alpha + rowsum;
-            l_pv = l_pv * alpha + rowsum_pv;
-
-            if (j > 0) {
-                // O and the P buffer belong to the previous PV product until it completes.
-                if (!(ok = mbar_wait(BAR(kBarODone), static_cast<uint32_t>(j - 1) & 1u, abort_flag, p.status,
-                                     kSitePrefillSoftmaxODone)))
-                    break;
-                tc_fence_after_sync();
-                if (rescale) {
+            const float2 s01 = __fadd2_rn(__fadd2_rn(sum[0], sum[1]), __fadd2_rn(sum[2], sum[3]));
+            const float2 q01 = __fadd2_rn(__fadd2_rn(sum_pv[0], sum_pv[1]), __fadd2_rn(sum_pv[2], sum_pv[3]));
+            l = l * alpha + (s01.x + s01.y);
+            l_pv = l_pv * alpha + (q01.x + q01.y);
+            // O_X is stable here (the commit announcing S_X(j) came after PV_X(j-1)), and PV_X(j) is
+            // not issued before the arrival below, so the rescale fits in between.
+            if (rescale) {
 #pragma unroll 1
-                    for (int cc = 0; cc < D / 32; ++cc) {
-                        uint32_t ov[32];
-                        tmem_ld32_wait(tO + cc * 32, ov);
+                for (int cc = 0; cc < D / 32; ++cc) {
+                    uint32_t ov[32];
+                    tmem_ld32_wait(tO + cc * 32, ov);
 #pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-                        tmem_st32_wait(tO + cc * 32, ov);
+                    for (int i = 0; i < 32; i += 2) {
+                        const float2 v2 = __fmul2_rn(make_float2(__uint_as_float(ov[i]), __uint_as_float(ov[i + 1])),
+                                                     make_float2(alpha, alpha));
+                        ov[i] = __float_as_uint(v2.x);
+                        ov[i + 1] = __float_as_uint(v2.y);
                     }
+                    tmem_st32_wait(tO + cc * 32, ov);
                 }
             }
-            // P row -> K-major 128B-swizzled tile: 16-byte unit u of row r lands at unit u ^ (r & 7).
-#pragma unroll
-            for (int u = 0; u < kBN / 8; ++u) {
-                const int chunk = u >> 3;
-                const int uu = u & 7;
-                const uint32_t addr = sP + chunk * (kBM * 128) + r * 128 + ((uu ^ (r & 7)) << 4);
-                st_shared_v4(addr, pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-            }
-            fence_proxy_async_smem();
+
             tc_fence_before_sync();
-            mbar_arrive(BAR(kBarPFull));
+            mbar_arrive(BAR(kBarPFull0 + x));
         }
 
-        if (ok)
-            ok = mbar_wait(BAR(kBarODone), static_cast<uint32_t>(n_kv - 1) & 1u, abort_flag, p.status,
-                           kSitePrefillEpilogue);
-        if (ok) {
+        if (ok && n > 0)
+            ok = mbar_wait(BAR(kBarOFinal0 + x), 0, abort_flag, p.status, kSitePrefillEpilogue);
+        if (ok && n > 0) {
             tc_fence_after_sync();
             const float inv_l = 1.f / l_pv;
             const bool store = row < p.Sq;
@@ -525,7 +535,15 @@ cudaError_t launch(const PrefillArgs &a, cudaStream_t stream, int *encode_error)
 
     static bool attr_set = false;  // benign race: every caller sets the same value
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+        // The setmaxnreg split inside the kernel is only valid for the register count it was
+        // written for; refuse to launch a build that was compiled to anything else.
+        cudaFuncAttributes fa;
+        cudaError_t e = cudaFuncGetAttributes(&fa, prefill_kernel<D>);
+        if (e != cudaSuccess)
+            return e;
+        if (fa.numRegs != kLaunchRegs)
+            return cudaErrorInvalidConfiguration;
+        e = cudaFuncSetAttribute(prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
         if (e != cudaSuccess)
             return e;
         attr_set = true;
@@ -542,9 +560,10 @@ cudaError_t launch(const PrefillArgs &a, cudaStream_t stream, int *encode_error)
     p.group = a.Hq / a.Hkv;
     p.offset = a.Skv - a.Sq;
     p.causal = a.causal;
-    p.n_qtiles = (a.Sq + kBM - 1) / kBM;
+    const int n_qtiles = (a.Sq + kBM - 1) / kBM;
+    p.n_pairs = (n_qtiles + 1) / 2;
     p.scale_log2 = a.scale * kLog2e;
-    const long long grid = static_cast<long long>(p.n_qtiles) * a.B * a.Hq;
+    const long long grid = static_cast<long long>(p.n_pairs) * a.B * a.Hq;
     prefill_kernel<D><<<static_cast<unsigned>(grid), kThreads, C::kSmem, stream>>>(tq, tk, tv, p);
     return cudaGetLastError();
 }

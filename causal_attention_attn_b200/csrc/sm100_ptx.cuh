@@ -194,6 +194,17 @@ __device__ __forceinline__ void tc_mma_ss(uint32_t d_tmem, uint64_t a_desc, uint
                  : "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B[smem]: the A operand (M x K, K-major) is read from tensor memory, row i
+// in lane i, two 16-bit elements per 32-bit column (element 2c in the low half of column c).
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate)
+{
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+                 "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+                 : "memory");
+}
+
 // Shared-memory matrix descriptor (tcgen05 "matrix descriptor"):
 //   bits  0-13 start address >> 4, 16-29 leading-dimension byte offset >> 4,
 //   bits 32-45 stride-dimension byte offset >> 4, bits 46-47 version (1 on sm_100),
