@@ -24,7 +24,7 @@ STATUS_NAMES = {
     -9: "ATTN_ERR_LAUNCH", -10: "ATTN_ERR_DEVICE_TIMEOUT", -11: "ATTN_ERR_SCALE", -12: "ATTN_ERR_CUDA",
     -13: "ATTN_ERR_SCRATCH_LIMIT",
 }
-EXPORTED = ("attn_fwd", "attn_fwd_ex", "attn_decode_splits", "attn_status_string", "attn_version",
+EXPORTED = ("attn_fwd", "attn_fwd_ex", "attn_decode_ctas", "attn_status_string", "attn_version",
             "attn_device_status", "attn_decode_noalloc")
 
 _lock = threading.Lock()
@@ -53,8 +53,8 @@ def load_library(path: str | None = None):
         lib.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp]
         lib.attn_fwd_ex.restype = i
         lib.attn_fwd_ex.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, vp]
-        lib.attn_decode_splits.restype = i
-        lib.attn_decode_splits.argtypes = [i, i, i, i, i]
+        lib.attn_decode_ctas.restype = i
+        lib.attn_decode_ctas.argtypes = [i, i, i, i, i]
         lib.attn_status_string.restype = ctypes.c_char_p
         lib.attn_status_string.argtypes = [i]
         lib.attn_version.restype = i
@@ -98,19 +98,19 @@ def _check_tensor(name, t, dtype, ndim):
 
 def attn_fwd_raw(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, lse_ptr: int, B: int, Hq: int, Hkv: int,
                  Sq: int, Skv: int, D: int, scale: float, causal: bool, stream: int = 0,
-                 decode_splits: int = 0) -> int:
+                 decode_ctas: int = 0) -> int:
     """Call the C entry point with raw pointers; returns the status code (no exception)."""
     lib = load_library()
-    if decode_splits:
+    if decode_ctas:
         return lib.attn_fwd_ex(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, Hq, Hkv, Sq, Skv, D, float(scale),
-                               int(causal), int(decode_splits), stream)
+                               int(causal), int(decode_ctas), stream)
     return lib.attn_fwd(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, Hq, Hkv, Sq, Skv, D, float(scale), int(causal),
                         stream)
 
 
 def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: float | None = None, causal: bool = True,
              out: torch.Tensor | None = None, lse: torch.Tensor | None = None, stream=None,
-             decode_splits: int = 0):
+             decode_ctas: int = 0):
     """Fused causal attention forward on the GPU.
 
     q: [B, Hq, Sq, D], k/v: [B, Hkv, Skv, D], bf16, contiguous, on one CUDA device.
@@ -139,7 +139,7 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: float | N
             raise ValueError("lse must be [B, Hq, Sq]")
     with torch.cuda.device(q.device):
         rc = attn_fwd_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, Hq, Hkv,
-                          Sq, Skv, D, scale, causal, _stream_handle(stream), decode_splits)
+                          Sq, Skv, D, scale, causal, _stream_handle(stream), decode_ctas)
     _check(rc)
     return out, lse
 
@@ -202,8 +202,9 @@ def attn_decode_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale
     return out, lse
 
 
-def decode_splits(B: int, Hq: int, Hkv: int, Skv: int, D: int) -> int:
-    rc = load_library().attn_decode_splits(B, Hq, Hkv, Skv, D)
+def decode_ctas(B: int, Hq: int, Hkv: int, Skv: int, D: int) -> int:
+    """Number of CTAs attn_fwd launches for a decode of this shape on the current device."""
+    rc = load_library().attn_decode_ctas(B, Hq, Hkv, Skv, D)
     if rc < 0:
         _check(rc)
     return rc

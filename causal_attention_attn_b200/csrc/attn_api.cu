@@ -135,41 +135,13 @@ int ensure_workspace(DeviceState &s, size_t counters, size_t partials, cudaStrea
     return ATTN_OK;
 }
 
-int choose_splits(const DeviceState &s, int B, int Hq, int Hkv, int Skv, int D)
-{
-    const int group = Hq / Hkv;
-    const int G = decode_heads_per_cta(group);
-    const long long pairs = static_cast<long long>(B) * Hkv * (group / G);
-    const int per_sm = decode_ctas_per_sm(D, group);
-    const long long slots = static_cast<long long>(s.sm_count) * per_sm;
-    const int ck = decode_keys_per_chunk(group);
-    const int max_splits = (Skv + ck - 1) / ck;
-    // Pick the split count whose waves of resident CTAs waste the least, preferring fewer splits
-    // (less merge work) when two choices are within 3% of each other.
-    int best = 1;
-    double best_cost = 1e30;
-    for (int sp = 1; sp <= max_splits && sp <= 64; ++sp) {
-        const int eff = decode_effective_splits(Skv, group, sp);
-        if (eff != sp)
-            continue;
-        const long long ctas = pairs * sp;
-        const long long waves = (ctas + slots - 1) / slots;
-        const double cost = static_cast<double>(waves) / sp + 0.002 * sp;  // + merge overhead per split
-        if (cost < best_cost * 0.97) {
-            best_cost = cost;
-            best = sp;
-        }
-    }
-    return best;
-}
-
 int run(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq, int Hkv, int Sq, int Skv,
-        int D, float scale, int causal, int decode_splits, void *stream_ptr)
+        int D, float scale, int causal, int decode_ctas, void *stream_ptr)
 {
     int rc = validate(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, D, scale, causal);
     if (rc != ATTN_OK)
         return rc;
-    if (decode_splits < 0)
+    if (decode_ctas < 0)
         return ATTN_ERR_SHAPE;
     cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
     std::lock_guard<std::mutex> lock(g_mutex);
@@ -179,16 +151,12 @@ int run(const void *q, const void *k, const void *v, void *o, float *lse, int B,
         return err;
 
     if (Sq == 1) {
-        const int group = Hq / Hkv;
-        const int G = decode_heads_per_cta(group);
-        const long long pairs = static_cast<long long>(B) * Hkv * (group / G);
-        int splits = decode_splits > 0 ? decode_splits : choose_splits(*s, B, Hq, Hkv, Skv, D);
-        splits = decode_effective_splits(Skv, group, splits);
-        if (pairs * splits > INT_MAX)
+        DecodePlan plan;
+        if (decode_plan(B, Hq, Hkv, Skv, D, decode_ctas, s->sm_count, &plan) != cudaSuccess) {
+            cudaGetLastError();
             return ATTN_ERR_SHAPE;
-        const size_t n_partials =
-            splits > 1 ? static_cast<size_t>(B) * Hq * splits * (static_cast<size_t>(D) + 1) : 0;
-        rc = ensure_workspace(*s, static_cast<size_t>(pairs), n_partials, stream);
+        }
+        rc = ensure_workspace(*s, static_cast<size_t>(plan.pairs), plan.partial_floats, stream);
         if (rc != ATTN_OK)
             return rc;
         DecodeArgs a;
@@ -203,9 +171,8 @@ int run(const void *q, const void *k, const void *v, void *o, float *lse, int B,
         a.Skv = Skv;
         a.D = D;
         a.scale = scale;
-        a.splits = splits;
-        a.ws_o = s->partials;
-        a.ws_lse = s->partials + static_cast<size_t>(B) * Hq * splits * D;
+        a.plan = plan;
+        a.ws = s->partials;
         a.counters = s->counters;
         a.status = s->status;
         if (launch_decode(a, stream) != cudaSuccess) {
@@ -254,12 +221,12 @@ extern "C" int attn_fwd(const void *q, const void *k, const void *v, void *o, fl
 }
 
 extern "C" int attn_fwd_ex(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
-                           int Hkv, int Sq, int Skv, int D, float scale, int causal, int decode_splits, void *stream)
+                           int Hkv, int Sq, int Skv, int D, float scale, int causal, int decode_ctas, void *stream)
 {
-    return run(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, D, scale, causal, decode_splits, stream);
+    return run(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, D, scale, causal, decode_ctas, stream);
 }
 
-extern "C" int attn_decode_splits(int B, int Hq, int Hkv, int Skv, int D)
+extern "C" int attn_decode_ctas(int B, int Hq, int Hkv, int Skv, int D)
 {
     if (B < 1 || Hq < 1 || Hkv < 1 || Skv < 1)
         return ATTN_ERR_SHAPE;
@@ -272,7 +239,12 @@ extern "C" int attn_decode_splits(int B, int Hq, int Hkv, int Skv, int D)
     DeviceState *s = device_state(&err);
     if (!s)
         return err;
-    return decode_effective_splits(Skv, Hq / Hkv, choose_splits(*s, B, Hq, Hkv, Skv, D));
+    DecodePlan plan;
+    if (decode_plan(B, Hq, Hkv, Skv, D, 0, s->sm_count, &plan) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_SHAPE;
+    }
+    return plan.ctas;
 }
 
 extern "C" const char *attn_status_string(int status)
@@ -306,7 +278,7 @@ extern "C" const char *attn_status_string(int status)
         return "a CUDA runtime call failed";
     case ATTN_ERR_SCRATCH_LIMIT:
         return "the decode needs more scratch than the fixed no-allocation buffer holds "
-               "(too many (batch, kv head) pairs for attn_decode_noalloc)";
+               "(too many (batch, kv head, head group) work units for attn_decode_noalloc)";
     default:
         return "unknown status";
     }

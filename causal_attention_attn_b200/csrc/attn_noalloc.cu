@@ -86,21 +86,33 @@ extern "C" int attn_decode_noalloc(const void *q, const void *k, const void *v, 
     if (!(scale > 0.f) || !std::isfinite(scale))
         return ATTN_ERR_SCALE;
 
-    // Same split choice as attn_fwd (this also checks that the device is an sm_100 part).
-    int splits = attn_decode_splits(B, Hq, Hkv, Skv, D);
-    if (splits < 0)
-        return splits;
-
-    const int group = Hq / Hkv;
-    const long long pairs = static_cast<long long>(B) * Hkv * (group / decode_heads_per_cta(group));
-    const size_t counter_bytes = ((static_cast<size_t>(pairs) * sizeof(int) + 255) / 256) * 256;
+    // Same work split as attn_fwd (this also checks that the device is an sm_100 part); if the
+    // shared-pair partials do not fit, one CTA per pair needs none.
+    const int ctas = attn_decode_ctas(B, Hq, Hkv, Skv, D);
+    if (ctas < 0)
+        return ctas;
+    int sm_count = 0, dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_CUDA;
+    }
+    DecodePlan plan;
+    if (decode_plan(B, Hq, Hkv, Skv, D, ctas, sm_count, &plan) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_SHAPE;
+    }
+    const size_t counter_bytes = ((static_cast<size_t>(plan.pairs) * sizeof(int) + 255) / 256) * 256;
     if (kStatusBytes + counter_bytes > kScratchBytes)
         return ATTN_ERR_SCRATCH_LIMIT;
     const size_t partial_room = (kScratchBytes - kStatusBytes - counter_bytes) / sizeof(float);
-    // Fewer splits need fewer partials; one split needs none.
-    while (splits > 1 &&
-           static_cast<size_t>(B) * Hq * static_cast<size_t>(splits) * (static_cast<size_t>(D) + 1) > partial_room)
-        splits = decode_effective_splits(Skv, group, splits - 1);
+    if (plan.partial_floats > partial_room) {
+        if (decode_plan(B, Hq, Hkv, Skv, D, static_cast<int>(plan.pairs), sm_count, &plan) != cudaSuccess ||
+            plan.partial_floats > partial_room) {
+            cudaGetLastError();
+            return ATTN_ERR_SCRATCH_LIMIT;
+        }
+    }
 
     unsigned char *scratch = nullptr;
     const int rc = scratch_for_current_device(&scratch);
@@ -109,7 +121,7 @@ extern "C" int attn_decode_noalloc(const void *q, const void *k, const void *v, 
     cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
     int *counters = reinterpret_cast<int *>(scratch + kStatusBytes);
     float *partials = reinterpret_cast<float *>(scratch + kStatusBytes + counter_bytes);
-    if (cudaMemsetAsync(counters, 0, static_cast<size_t>(pairs) * sizeof(int), stream) != cudaSuccess) {
+    if (cudaMemsetAsync(counters, 0, static_cast<size_t>(plan.pairs) * sizeof(int), stream) != cudaSuccess) {
         cudaGetLastError();
         return ATTN_ERR_CUDA;
     }
@@ -126,9 +138,8 @@ extern "C" int attn_decode_noalloc(const void *q, const void *k, const void *v, 
     a.Skv = Skv;
     a.D = D;
     a.scale = scale;
-    a.splits = splits;
-    a.ws_o = partials;
-    a.ws_lse = partials + static_cast<size_t>(B) * Hq * splits * D;
+    a.plan = plan;
+    a.ws = partials;
     a.counters = counters;
     a.status = reinterpret_cast<int *>(scratch);
     if (launch_decode(a, stream) != cudaSuccess) {

@@ -34,27 +34,39 @@ struct PrefillArgs {
     int *status;  // device status word
 };
 
+// How a decode (Sq == 1) is spread over persistent CTAs. A "pair" is one (batch, kv head, group of
+// G query heads); its keys are cut into `cpp` chunks of `ck` keys; CTA c of `ctas` takes units
+// [c*total/ctas, (c+1)*total/ctas) of the pairs' chunks laid end to end.
+struct DecodePlan {
+    int G;                  // query heads per pair
+    int head_groups;        // (Hq / Hkv) / G
+    long long pairs;        // B * Hkv * head_groups
+    int ck;                 // keys per chunk
+    int cpp;                // chunks per pair
+    long long total;        // pairs * cpp
+    int ctas;               // CTAs launched
+    int max_contrib;        // most CTAs that can share one pair
+    size_t partial_floats;  // workspace floats for shared pairs' partials (0 if no pair is shared)
+};
+
 struct DecodeArgs {
     const void *q, *k, *v;
     void *o;
     float *lse;
     int B, Hq, Hkv, Skv, D;
     float scale;
-    int splits;         // >= 1, already clamped so that every split is non-empty
-    float *ws_o;        // [B*Hq*splits*D] partial outputs (only when splits > 1)
-    float *ws_lse;      // [B*Hq*splits] partial log2-sum-exp (only when splits > 1)
-    int *counters;      // [B*Hkv*head_groups] arrival counters, zero between calls
+    DecodePlan plan;
+    float *ws;          // plan.partial_floats floats (may be null when that is 0)
+    int *counters;      // plan.pairs arrival counters, zero between calls
     int *status;        // device status word
 };
 
 // Returns a cudaError_t value (cudaSuccess on success); never synchronises.
 cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t stream, int *encode_error);
 
-// Decode geometry shared by the host planner and the launcher.
-int decode_heads_per_cta(int group);           // G: 1, 2, 4 or 8
-int decode_keys_per_chunk(int group);          // keys per pipeline stage
-int decode_effective_splits(int Skv, int group, int requested);  // clamp so that no split is empty
+// Decode planning and launch. requested_ctas <= 0 means one CTA per resident slot on the device.
+int decode_heads_per_cta(int group, int D);  // G: 1, 2, 4 or 8 (at most 4 for D = 128)
+cudaError_t decode_plan(int B, int Hq, int Hkv, int Skv, int D, int requested_ctas, int sm_count, DecodePlan *plan);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream);
-int decode_ctas_per_sm(int D, int group);      // occupancy of the decode kernel (>= 1)
 
 }  // namespace attn_b200

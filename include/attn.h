@@ -77,17 +77,19 @@ int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
              float scale, int causal, void *stream);
 
 /*
- * attn_fwd_ex — attn_fwd with the decode split count fixed by the caller (decode_splits >= 1),
- * or chosen by the library (decode_splits == 0). The split count is a performance parameter:
- * results agree with attn_fwd within rounding. Ignored when Sq > 1.
+ * attn_fwd_ex — attn_fwd with the number of CTAs of the decode kernel fixed by the caller
+ * (decode_ctas >= 1), or chosen by the library (decode_ctas == 0: one CTA per slot the GPU can keep
+ * resident). The decode spreads the chunks of every (batch, kv head) key range evenly over those
+ * CTAs, so this is a performance parameter: results agree with attn_fwd within rounding. Ignored
+ * when Sq > 1.
  */
 int attn_fwd_ex(const void *q, const void *k, const void *v, void *o, float *lse,
                 int B, int Hq, int Hkv, int Sq, int Skv, int D,
-                float scale, int causal, int decode_splits, void *stream);
+                float scale, int causal, int decode_ctas, void *stream);
 
-/* attn_decode_splits — the split count attn_fwd would use for a decode of this shape on the
+/* attn_decode_ctas — the number of CTAs attn_fwd would launch for a decode of this shape on the
  * current device (>= 1), or a negative attn_status. */
-int attn_decode_splits(int B, int Hq, int Hkv, int Skv, int D);
+int attn_decode_ctas(int B, int Hq, int Hkv, int Skv, int D);
 
 /* attn_status_string — a static, human-readable description of a status code. Never NULL. */
 const char *attn_status_string(int status);
@@ -118,7 +120,8 @@ int attn_device_status(void *stream);
  * Arguments are those of attn_fwd with Sq = 1 and no causal flag (a single new query sees every
  * cached key): q [B, Hq, 1, D], k and v [B, Hkv, Skv, D], o [B, Hq, 1, D] bf16; lse [B, Hq, 1] fp32;
  * all device pointers owned by the caller, 16-byte aligned. Results agree with attn_fwd within
- * rounding (the split count may be lowered so that the partials fit).
+ * rounding (when the partials of the usual work split would not fit, each CTA takes whole
+ * (batch, kv head) key ranges instead, which needs none).
  *
  * The first call on a device looks up that device's address of the array (cudaGetSymbolAddress,
  * with the device current); make that first call before any stream capture. Every call on a device

@@ -87,7 +87,7 @@ def test_argument_errors(lib, name, override, expected):
     assert rc == expected, (name, rc)
 
 
-def test_negative_split_request_rejected(lib):
+def test_negative_cta_request_rejected(lib):
     rc = lib.attn_fwd_ex(*A, 1, 4, 2, 1, 8, 64, 0.125, 1, -1, None)
     assert rc == -2
 

@@ -30,14 +30,14 @@ def gpu():
     assert attn.device_status() == 0, "a kernel-side wait ran out during the parity tests"
 
 
-def run_gpu(q, k, v, scale, causal, decode_splits=0):
-    o, lse = attn.attn_fwd(q.cuda(), k.cuda(), v.cuda(), scale=scale, causal=causal, decode_splits=decode_splits)
+def run_gpu(q, k, v, scale, causal, decode_ctas=0):
+    o, lse = attn.attn_fwd(q.cuda(), k.cuda(), v.cuda(), scale=scale, causal=causal, decode_ctas=decode_ctas)
     torch.cuda.synchronize()
     return o.cpu(), lse.cpu()
 
 
-def check(q, k, v, scale, causal, rows=None, decode_splits=0):
-    o, lse = run_gpu(q, k, v, scale, causal, decode_splits)
+def check(q, k, v, scale, causal, rows=None, decode_ctas=0):
+    o, lse = run_gpu(q, k, v, scale, causal, decode_ctas)
     if rows is None:
         o_ref, lse_ref = oracle.attention(q, k, v, scale, causal)
         rep = compare(o, lse, o_ref, lse_ref)
@@ -98,14 +98,24 @@ def test_decode_matches_oracle(shape):
     check(q, k, v, w.scale, True)
 
 
-@pytest.mark.parametrize("splits", [1, 2, 3, 7, 16, 64])
-def test_decode_split_count_does_not_matter(splits):
+@pytest.mark.parametrize("ctas", [1, 2, 3, 7, 16, 61, 64, 97, 500])
+def test_decode_cta_count_does_not_matter(ctas):
+    """The decode spreads the pairs' key chunks over any number of CTAs (shared pairs are merged
+    through their LSEs): the result does not depend on that number beyond rounding."""
     w = inputs.custom(2, 8, 2, 1, 4000, 128, True, seed=99)
     q, k, v = inputs.generate(w)
-    o, lse, _ = check(q, k, v, w.scale, True, decode_splits=splits)
-    o1, lse1 = run_gpu(q, k, v, w.scale, True, decode_splits=1)
+    o, lse, _ = check(q, k, v, w.scale, True, decode_ctas=ctas)
+    o1, lse1 = run_gpu(q, k, v, w.scale, True, decode_ctas=4)  # one CTA per (batch, kv head)
     assert (o.float() - o1.float()).abs().max().item() <= 2 ** -7
     assert (lse - lse1).abs().max().item() <= 1e-4
+
+
+def test_decode_many_short_caches_share_ctas():
+    """More (batch, kv head) pairs than CTAs, each with a short cache: CTAs cover several pairs."""
+    w = inputs.custom(64, 16, 4, 1, 37, 64, True, seed=98)
+    q, k, v = inputs.generate(w)
+    check(q, k, v, w.scale, True)
+    check(q, k, v, w.scale, True, decode_ctas=5)
 
 
 # ------------------------------------------------------------------------------ the five workloads
