@@ -23,8 +23,9 @@
  *   scores   G*(8/G) = 8 partial dot products per lane (packed f32x2 FMAs), reduced across the
  *            group by a transposing butterfly (7 shuffles for 8 sums) that leaves lane t with
  *            score (head t/(8/G), key t%(8/G));
- *   softmax  running max and running sum per head and group, with the exp(m_old - m_new) rescale
- *            of the sum and of the fp32 accumulator;
+ *   softmax  running (reference) max and running sum per head and group, with the
+ *            exp(m_old - m_new) rescale of the sum and of the fp32 accumulator when the max grows
+ *            by more than 2^8;
  *   PV       each lane accumulates its dims of sum_j p_j v_j for all G heads (f32x2 FMAs).
  *
  * At the end of a segment the groups merge by shuffles, the warps through shared memory.
@@ -57,6 +58,7 @@ namespace {
 constexpr int kMaxStages = ATTN_DECODE_STAGES;  // K/V chunks in flight per CTA, when they fit
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleThreshold = 8.0f;
 
 #ifndef ATTN_DECODE_LANES
 #define ATTN_DECODE_LANES 8
@@ -377,6 +379,13 @@ __global__ void __launch_bounds__(DecCfg<D, G>::kThreads, 1) decode_kernel(const
                         for (int i = 0; i < NW2; ++i)
                             kw[kk][i] = 0u;
                 }
+                // Widen each K element once; the G heads then share it.
+                float2 kf[KB][NW2];
+#pragma unroll
+                for (int kk = 0; kk < KB; ++kk)
+#pragma unroll
+                    for (int i = 0; i < NW2; ++i)
+                        kf[kk][i] = bf16x2_to_float2(kw[kk][i]);
                 float part[LG];
 #pragma unroll
                 for (int gg = 0; gg < G; ++gg) {
@@ -388,7 +397,7 @@ __global__ void __launch_bounds__(DecCfg<D, G>::kThreads, 1) decode_kernel(const
                     for (int i = 0; i < NW2; ++i) {
 #pragma unroll
                         for (int kk = 0; kk < KB; ++kk)
-                            s2[kk] = __ffma2_rn(q2[gg][i], bf16x2_to_float2(kw[kk][i]), s2[kk]);
+                            s2[kk] = __ffma2_rn(q2[gg][i], kf[kk][i], s2[kk]);
                     }
 #pragma unroll
                     for (int kk = 0; kk < KB; ++kk)
@@ -411,13 +420,17 @@ __global__ void __launch_bounds__(DecCfg<D, G>::kThreads, 1) decode_kernel(const
 #pragma unroll
                 for (int o = 1; o < KB; o <<= 1)
                     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-                // In a ragged chunk a group batch may lie wholly past `rows`: state unchanged.
-                const float m_new = fmaxf(m_run, mx);
-                const float alpha = (!kFull && m_new == -INFINITY) ? 1.f : ex2(m_run - m_new);
+                // The reference max m_run only moves when the batch max exceeds it by more than 8
+                // (log2 units): weights stay below 2^8 and the accumulators are rescaled rarely;
+                // O and the sum are both relative to m_run, so O / sum is unchanged. In a ragged
+                // chunk a group batch may lie wholly past `rows`: its state is then unchanged.
+                const bool move = mx > m_run + kRescaleThreshold;
+                const float m_new = move ? mx : m_run;
+                const float alpha = move ? ex2(m_run - m_new) : 1.f;
                 const float pv = (!kFull && m_new == -INFINITY) ? 0.f : ex2(s2 - m_new);
                 lsum = lsum * alpha + pv;
                 m_run = m_new;
-                if (__any_sync(0xffffffffu, alpha != 1.f)) {
+                if (__any_sync(0xffffffffu, move)) {
 #pragma unroll
                     for (int gg = 0; gg < G; ++gg) {
                         const float a = __shfl_sync(0xffffffffu, alpha, obase + gg * KB);
@@ -435,13 +448,17 @@ __global__ void __launch_bounds__(DecCfg<D, G>::kThreads, 1) decode_kernel(const
 #pragma unroll
                         for (int i = 0; i < NW2; ++i)
                             vw[i] = 0u;
+                    float2 vf[NW2];
+#pragma unroll
+                    for (int i = 0; i < NW2; ++i)
+                        vf[i] = bf16x2_to_float2(vw[i]);
 #pragma unroll
                     for (int gg = 0; gg < G; ++gg) {
                         const float w = __shfl_sync(0xffffffffu, pv, obase + gg * KB + kk);
                         const float2 w2 = make_float2(w, w);
 #pragma unroll
                         for (int i = 0; i < NW2; ++i)
-                            acc[gg][i] = __ffma2_rn(w2, bf16x2_to_float2(vw[i]), acc[gg][i]);
+                            acc[gg][i] = __ffma2_rn(w2, vf[i], acc[gg][i]);
                     }
                 }
             };
