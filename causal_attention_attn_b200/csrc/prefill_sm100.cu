@@ -123,6 +123,25 @@ __device__ __forceinline__ float ex2(float x)
     return y;
 }
 
+// Three-input maximum (one instruction on sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// acc + lo + hi for the two bf16 values packed in w, each added with fp32 accumulation (mixed-
+// precision adds: no separate widening of the bf16 halves).
+__device__ __forceinline__ float add_bf16x2(float acc, uint32_t w)
+{
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\t"
+        "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %0, hi, %0;\n\t}"
+        : "+f"(acc)
+        : "r"(w));
+    return acc;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -376,16 +395,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (c > limit)
                         s[c] = -INFINITY;
             }
-            // Row max with eight independent chains.
+            // Row max: eight independent chains of three-input maxima.
+            static_assert(kBN % 16 == 0, "row max walks the tile 16 columns at a time");
             float mx8[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i)
-                mx8[i] = s[i];
+                mx8[i] = fmaxf(s[2 * i], s[2 * i + 1]);
 #pragma unroll
-            for (int c = 8; c < kBN; ++c)
-                mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
-            const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+            for (int c = 16; c < kBN; c += 16)
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    mx8[i] = fmax3(mx8[i], s[c + 2 * i], s[c + 2 * i + 1]);
+            const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
             const float mx2 = mx * sl2;  // scale > 0, so the max commutes with scaling
 
             float alpha = 1.f;
@@ -405,8 +426,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float2 negm2 = make_float2(-m, -m);
             float2 sum[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                              make_float2(0.f, 0.f)};
-            float2 sum_pv[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                                make_float2(0.f, 0.f)};
+            float sum_pv[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t pk[32];
@@ -417,15 +437,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const float2 pe = make_float2(ex2(e.x), ex2(e.y));
                     pk[c] = pack_bf16x2(pe.x, pe.y);
                     sum[c & 3] = __fadd2_rn(sum[c & 3], pe);
-                    sum_pv[c & 3] = __fadd2_rn(
-                        sum_pv[c & 3], make_float2(__uint_as_float(pk[c] << 16), __uint_as_float(pk[c] & 0xffff0000u)));
+                    sum_pv[c & 3] = add_bf16x2(sum_pv[c & 3], pk[c]);
                 }
                 tmem_st32_wait(tS + half * 32, pk);
             }
             const float2 s01 = __fadd2_rn(__fadd2_rn(sum[0], sum[1]), __fadd2_rn(sum[2], sum[3]));
-            const float2 q01 = __fadd2_rn(__fadd2_rn(sum_pv[0], sum_pv[1]), __fadd2_rn(sum_pv[2], sum_pv[3]));
+            const float q01 = (sum_pv[0] + sum_pv[1]) + (sum_pv[2] + sum_pv[3]);
             l = l * alpha + (s01.x + s01.y);
-            l_pv = l_pv * alpha + (q01.x + q01.y);
+            l_pv = l_pv * alpha + q01;
             // O_X is stable here (the commit announcing S_X(j) came after PV_X(j-1)), and PV_X(j) is
             // not issued before the arrival below, so the rescale fits in between.
             if (rescale) {
