@@ -68,8 +68,8 @@ constexpr int kThreads = 384;  // three warpgroups: softmax A, softmax B, produc
 // count before every first launch); the producer/MMA warpgroup gives registers back and the two
 // softmax warpgroups take them, so the three shares add up to exactly the launch allocation.
 constexpr int kLaunchRegs = 168;
-constexpr int kRegsSoftmax = 232;
-constexpr int kRegsOther = 40;
+constexpr int kRegsSoftmax = 200;
+constexpr int kRegsOther = 104;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther == kThreads * kLaunchRegs, "register split");
 constexpr uint32_t kTmemCols = 512;  // S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512)
 __host__ __device__ constexpr uint32_t col_s(int x) { return static_cast<uint32_t>(x) * 128u; }        // S_X
@@ -101,12 +101,13 @@ enum Bar : int {
     kBarFull0 = 1,
     kBarEmpty0 = kBarFull0 + kRing,
     kBarSFull0 = kBarEmpty0 + kRing,  // [A, B]
-    kBarPFull0 = kBarSFull0 + 2,      // [A, B]
+    kBarPHalf0 = kBarSFull0 + 2,      // [A, B] first half of P_X stored
+    kBarPFull0 = kBarPHalf0 + 2,      // [A, B] all of P_X stored
     kBarOFinal0 = kBarPFull0 + 2,     // [A, B]
     kBarDrain = kBarOFinal0 + 2,
     kNumBars = kBarDrain + 1,
 };
-static_assert(kNumBars * 8 <= 128, "barrier area");
+static_assert(kNumBars * 8 <= 192, "barrier area");
 
 struct Params {
     __nv_bfloat16 *o;
@@ -182,8 +183,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t sQ = s_base + C::kOffQ;
     const uint32_t sRing = s_base + C::kOffRing;
     const uint32_t bar0 = s_base + C::kOffBar;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kOffBar + 128);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::kOffBar + 132);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kOffBar + 192);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::kOffBar + 196);
 #define BAR(i) (bar0 + 8u * static_cast<uint32_t>(i))
 
     const int warp = threadIdx.x >> 5;
@@ -213,6 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int x = 0; x < 2; ++x) {
             mbar_init(BAR(kBarSFull0 + x), 1);
+            mbar_init(BAR(kBarPHalf0 + x), 128);
             mbar_init(BAR(kBarPFull0 + x), 128);
             mbar_init(BAR(kBarOFinal0 + x), 1);
         }
@@ -275,36 +277,54 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == kWarpMma) {
         // ---------------------------------------------------------------- MMA issuer
-        if (lane == 0) {
+        // The whole warp walks the schedule, so every descriptor and wait is warp-uniform; the
+        // elected lane (the same one throughout) issues the MMAs and the commits that track them.
+        {
             constexpr uint32_t kIdS = idesc_bf16_f32(kBM, kBN, false);
             constexpr uint32_t kIdO = idesc_bf16_f32(kBM, D, true);
             constexpr uint32_t kSbo = 8 * C::kSwizzleBytes;  // 8 rows of one swizzled column block
+            const bool leader = elect_one();
+            // Descriptors of the tile bases; a K step moves the start address, which is the low
+            // field (address >> 4, 14 bits) of the descriptor: every address here is below 2^18.
+            const uint64_t desc_q0 = smem_desc(sQ, 16, kSbo, C::kSwizzleMode);
+            const uint64_t desc_k0 = smem_desc(sRing, 16, kSbo, C::kSwizzleMode);
+            const uint64_t desc_v0 = smem_desc(sRing, C::kChunkBytes, kSbo, C::kSwizzleMode);
+            constexpr uint64_t kSlotStep = static_cast<uint64_t>(C::kTileBytes >> 4);  // one tile, in descriptor units
 
-            auto issue_s = [&](int x, uint32_t sK) {
-                const uint32_t sQx = sQ + x * C::kTileBytes;
+            auto issue_s = [&](int x, int item) {
+                const uint64_t dq = desc_q0 + static_cast<uint64_t>(x) * kSlotStep;  // Q_B follows Q_A
+                const uint64_t dk = desc_k0 + static_cast<uint64_t>(item % kRing) * kSlotStep;
+                if (leader) {
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const int c = kk / (C::kChunkElems / 16);
-                    const int w = kk % (C::kChunkElems / 16);
-                    const uint32_t off = c * C::kChunkBytes + w * 32;
-                    tc_mma_ss(tmem + col_s(x), smem_desc(sQx + off, 16, kSbo, C::kSwizzleMode),
-                              smem_desc(sK + off, 16, kSbo, C::kSwizzleMode), kIdS, kk > 0 ? 1u : 0u);
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const int c = kk / (C::kChunkElems / 16);
+                        const int w = kk % (C::kChunkElems / 16);
+                        const uint64_t off = static_cast<uint64_t>((c * C::kChunkBytes + w * 32) >> 4);
+                        tc_mma_ss(tmem + col_s(x), dq + off, dk + off, kIdS, kk > 0 ? 1u : 0u);
+                    }
                 }
             };
-            auto issue_pv = [&](int x, uint32_t sV, bool accumulate) {
+            // PV for the keys of one half of the tile: kk in [half * kBN / 32, (half + 1) * kBN / 32).
+            auto issue_pv = [&](int x, int item, bool accumulate, int half) {
+                const uint64_t dv = desc_v0 + static_cast<uint64_t>(item % kRing) * kSlotStep;
+                if (leader) {
 #pragma unroll
-                for (int kk = 0; kk < kBN / 16; ++kk) {
-                    // P_X: 16 keys = 8 packed columns per step, in the first half of S_X's columns.
-                    tc_mma_ts(tmem + col_o(x), tmem + col_s(x) + kk * 8,
-                              smem_desc(sV + kk * 16 * C::kSwizzleBytes, C::kChunkBytes, kSbo, C::kSwizzleMode), kIdO,
-                              (accumulate || kk > 0) ? 1u : 0u);
+                    for (int kk = half * (kBN / 32); kk < (half + 1) * (kBN / 32); ++kk) {
+                        // P_X: 16 keys = 8 packed columns per step, in the first half of S_X's columns.
+                        const uint64_t off = static_cast<uint64_t>((kk * 16 * C::kSwizzleBytes) >> 4);
+                        tc_mma_ts(tmem + col_o(x), tmem + col_s(x) + kk * 8, dv + off, kIdO,
+                                  (accumulate || kk > 0) ? 1u : 0u);
+                    }
                 }
+            };
+            auto commit = [&](int bar) {
+                if (leader)
+                    tc_commit(BAR(bar));
             };
             auto wait_item = [&](int item) -> bool {
                 return mbar_wait(BAR(kBarFull0 + item % kRing), static_cast<uint32_t>(item / kRing) & 1u, abort_flag,
                                  p.status, kSitePrefillMmaFull);
             };
-            auto slot_of = [&](int item) { return sRing + (item % kRing) * C::kTileBytes; };
 
             bool ok = mbar_wait(BAR(kBarQ), 0, abort_flag, p.status, kSitePrefillMmaQ);
             if (ok && n_max > 0) {
@@ -313,10 +333,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_fence_after_sync();
                     for (int x = 0; x < 2; ++x)
                         if (n_of(x) > 0) {
-                            issue_s(x, slot_of(0));
-                            tc_commit(BAR(kBarSFull0 + x));
+                            issue_s(x, 0);
+                            commit(kBarSFull0 + x);
                         }
-                    tc_commit(BAR(kBarEmpty0 + 0));
+                    commit(kBarEmpty0 + 0);
                 }
             }
             for (int j = 0; ok && j < n_max; ++j) {
@@ -324,32 +344,38 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int x = 0; ok && x < 2; ++x) {
                     if (j >= n_of(x))
                         continue;
-                    if (!(ok = mbar_wait(BAR(kBarPFull0 + x), static_cast<uint32_t>(j) & 1u, abort_flag, p.status,
+                    // The first half of PV_X(j) runs while the softmax finishes the second half of P_X(j).
+                    if (!(ok = mbar_wait(BAR(kBarPHalf0 + x), static_cast<uint32_t>(j) & 1u, abort_flag, p.status,
                                          kSitePrefillMmaPFull)))
                         break;
                     if (!(ok = wait_item(item_v)))
                         break;
                     tc_fence_after_sync();
-                    issue_pv(x, slot_of(item_v), j > 0);
+                    issue_pv(x, item_v, j > 0, 0);
+                    if (!(ok = mbar_wait(BAR(kBarPFull0 + x), static_cast<uint32_t>(j) & 1u, abort_flag, p.status,
+                                         kSitePrefillMmaPFull)))
+                        break;
+                    tc_fence_after_sync();
+                    issue_pv(x, item_v, true, 1);
                     if (j + 1 < n_of(x)) {
                         if (!(ok = wait_item(item_k)))
                             break;
                         tc_fence_after_sync();
-                        issue_s(x, slot_of(item_k));
-                        tc_commit(BAR(kBarSFull0 + x));
+                        issue_s(x, item_k);
+                        commit(kBarSFull0 + x);
                     } else {
-                        tc_commit(BAR(kBarOFinal0 + x));
+                        commit(kBarOFinal0 + x);
                     }
                 }
                 if (!ok)
                     break;
-                tc_commit(BAR(kBarEmpty0 + item_v % kRing));
+                commit(kBarEmpty0 + item_v % kRing);
                 if (j + 1 < n_max)
-                    tc_commit(BAR(kBarEmpty0 + item_k % kRing));
+                    commit(kBarEmpty0 + item_k % kRing);
             }
             // Every MMA issued above has completed once this barrier flips.
-            tc_commit(BAR(kBarDrain));
-            if (!mbar_wait_drain(BAR(kBarDrain), 0, kWaitLimitNs)) {
+            commit(kBarDrain);
+            if (!mbar_wait_drain(BAR(kBarDrain), 0, kWaitLimitNs) && leader) {
                 *abort_flag = 1;
                 atomicExch(p.status, kSitePrefillDrain);
             }
@@ -421,7 +447,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                     m = m_new;
                 }
             }
-            // Exponentials, packed bf16 weights, and both running sums; then P_X -> TMEM.
+            // O_X is stable here (the commit announcing S_X(j) came after PV_X(j-1)), and PV_X(j) is
+            // not issued before the first arrival below, so the (rare) rescale fits in between.
+            if (rescale) {
+#pragma unroll 1
+                for (int cc = 0; cc < D / 32; ++cc) {
+                    uint32_t ov[32];
+                    tmem_ld32_wait(tO + cc * 32, ov);
+#pragma unroll
+                    for (int i = 0; i < 32; i += 2) {
+                        const float2 v2 = __fmul2_rn(make_float2(__uint_as_float(ov[i]), __uint_as_float(ov[i + 1])),
+                                                     make_float2(alpha, alpha));
+                        ov[i] = __float_as_uint(v2.x);
+                        ov[i + 1] = __float_as_uint(v2.y);
+                    }
+                    tmem_st32_wait(tO + cc * 32, ov);
+                }
+            }
+            // Exponentials, packed bf16 weights, and both running sums; P_X -> TMEM in two halves,
+            // each announced as soon as it is stored so that the tensor core can start on it.
             const float2 sl2x2 = make_float2(sl2, sl2);
             const float2 negm2 = make_float2(-m, -m);
             float2 sum[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
@@ -439,32 +483,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     sum[c & 3] = __fadd2_rn(sum[c & 3], pe);
                     sum_pv[c & 3] = add_bf16x2(sum_pv[c & 3], pk[c]);
                 }
-                tmem_st32_wait(tS + half * 32, pk);
+                tmem_st32(tS + half * 32, pk);
+                tmem_wait_st();
+                tc_fence_before_sync();
+                mbar_arrive(BAR((half == 0 ? kBarPHalf0 : kBarPFull0) + x));
             }
             const float2 s01 = __fadd2_rn(__fadd2_rn(sum[0], sum[1]), __fadd2_rn(sum[2], sum[3]));
             const float q01 = (sum_pv[0] + sum_pv[1]) + (sum_pv[2] + sum_pv[3]);
             l = l * alpha + (s01.x + s01.y);
             l_pv = l_pv * alpha + q01;
-            // O_X is stable here (the commit announcing S_X(j) came after PV_X(j-1)), and PV_X(j) is
-            // not issued before the arrival below, so the rescale fits in between.
-            if (rescale) {
-#pragma unroll 1
-                for (int cc = 0; cc < D / 32; ++cc) {
-                    uint32_t ov[32];
-                    tmem_ld32_wait(tO + cc * 32, ov);
-#pragma unroll
-                    for (int i = 0; i < 32; i += 2) {
-                        const float2 v2 = __fmul2_rn(make_float2(__uint_as_float(ov[i]), __uint_as_float(ov[i + 1])),
-                                                     make_float2(alpha, alpha));
-                        ov[i] = __float_as_uint(v2.x);
-                        ov[i + 1] = __float_as_uint(v2.y);
-                    }
-                    tmem_st32_wait(tO + cc * 32, ov);
-                }
-            }
-
-            tc_fence_before_sync();
-            mbar_arrive(BAR(kBarPFull0 + x));
         }
 
         if (ok && n > 0)
