@@ -679,10 +679,7 @@ cudaError_t dispatch_d(int G, const DecodeArgs *a, cudaStream_t stream, int *cta
     case 4:
         return a ? launch_dg<D, 4>(*a, stream) : prepare_dg<D, 4>(ctas_per_sm);
     default:
-        if constexpr (D == 128)
-            return cudaErrorInvalidValue;  // never chosen for D = 128
-        else
-            return a ? launch_dg<D, 8>(*a, stream) : prepare_dg<D, 8>(ctas_per_sm);
+        return a ? launch_dg<D, 8>(*a, stream) : prepare_dg<D, 8>(ctas_per_sm);
     }
 }
 
@@ -694,7 +691,9 @@ cudaError_t dispatch(int D, int G, const DecodeArgs *a, cudaStream_t stream, int
     case 64:
         return dispatch_d<64>(G, a, stream, ctas_per_sm);
     case 128:
-        return dispatch_d<128>(G, a, stream, ctas_per_sm);
+        if (a)
+            return launch_decode_tc(*a, stream);
+        return decode_tc_ctas_per_sm(G, ctas_per_sm);
     default:
         return cudaErrorInvalidValue;
     }
@@ -704,9 +703,10 @@ cudaError_t dispatch(int D, int G, const DecodeArgs *a, cudaStream_t stream, int
 
 int decode_heads_per_cta(int group, int D)
 {
-    // Largest power of two that divides the group size, at most 8 (at most 4 for D = 128, where q
-    // and the accumulators of eight heads would not fit in registers).
-    const int cap = (D == 128) ? 4 : 8;
+    if (D == 128)
+        return decode_tc_heads_per_pair(group);
+    // Largest power of two that divides the group size, at most 8.
+    const int cap = 8;
     int g = 1;
     while (g < cap && group % (2 * g) == 0)
         g *= 2;
@@ -720,7 +720,7 @@ cudaError_t decode_plan(int B, int Hq, int Hkv, int Skv, int D, int requested_ct
     pl.G = decode_heads_per_cta(group, D);
     pl.head_groups = group / pl.G;
     pl.pairs = static_cast<long long>(B) * Hkv * pl.head_groups;
-    pl.ck = keys_per_stage(pl.G);
+    pl.ck = (D == 128) ? decode_tc_chunk_keys() : keys_per_stage(pl.G);
     pl.cpp = (Skv + pl.ck - 1) / pl.ck;
     pl.total = pl.pairs * pl.cpp;
     long long ctas = requested_ctas;

@@ -1,0 +1,663 @@
+/*
+ * decode_tc_sm100.cu — attention of one new query token per (batch, query head) over a bf16 K/V
+ * cache (Sq == 1) with head dim 128, on the tensor core.
+ *
+ * Work split: as the CUDA-core decode kernel (decode_sm100.cu). A "pair" is one (batch, kv head,
+ * group of G query heads sharing that kv head), its keys are cut into chunks of 128, all pairs'
+ * chunks are laid end to end and CTA c of the launched CTAs streams the units
+ * [c*T/P, (c+1)*T/P); a CTA that holds a whole pair writes its output, the pieces of a shared pair
+ * are merged by whichever contributing CTA finishes last: M = max_s LSE_s,
+ * LSE = M + log2 sum_s 2^(LSE_s - M), O = sum_s 2^(LSE_s - LSE) O_s.
+ *
+ * Per chunk of 128 keys (K_c, V_c: 128 x 128 bf16 each, TMA-loaded with 128-byte swizzle):
+ *
+ *   S^T = K_c Q^T     tcgen05.mma, M = 128 keys, N = 16 (the G query heads, padded), K = 128 dims;
+ *                     fp32 scores in tensor memory, key i in TMEM lane i;
+ *   softmax           thread i owns key i: it scales its G scores to log2 units; the chunk's max
+ *                     per head comes from a warp butterfly and one exchange between the four
+ *                     warps; the reference max m moves only when a head's max exceeds it by more
+ *                     than 8 (then the O accumulator and the running sums are scaled by
+ *                     2^(m_old - m_new)); the weights 2^(s - m), rounded to bf16, go to shared
+ *                     memory as P^T (16 x 128, K-major, 128-byte swizzle);
+ *   O^T += V_c^T P^T  tcgen05.mma, M = 128 dims (A = V_c read MN-major), N = 16 heads, K = 128 keys.
+ *
+ * The tensor core takes the dot products, so each key costs the CUDA cores a handful of
+ * instructions per head and the kernel streams K/V at memory speed. S^T is double-buffered in
+ * TMEM and P^T in shared memory: S^T of chunk c+1 is computed while the softmax of chunk c runs.
+ * Each thread keeps two running sums per head over the keys it owned: of the fp32 weights (gives
+ * the LSE) and of the bf16-rounded weights the PV product used (normalises O).
+ *
+ * Warp roles (192 threads, one CTA per SM): warps 0-3 softmax and epilogue (thread i = TMEM lane
+ * i), warp 4 TMA producer, warp 5 TMEM allocator and MMA issuer (whole warp walks the schedule,
+ * one elected lane issues).
+ *
+ * Sources (page title, section): decode attends to every cached key, no mask needed — "AI Infra
+ * 入门：RMSNorm、Softmax、Causal Mask、Sampling 的数学与底层优化", §3; Flash-Decoding split-K merged by
+ * LSE — same page, §3 (LSE paragraph); grouped query heads sharing a K/V head and decode being
+ * bound by reading K/V — "05 · Tích vô hướng, Softmax và toán của Attention", §4; running max and
+ * sum with rescale — same page §6 and "Bộ 06 · Bên trong model", Q1.
+ */
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+
+#include "kernels.h"
+#include "sm100_ptx.cuh"
+#include "tma_host.h"
+
+namespace attn_b200 {
+namespace {
+
+constexpr int kD = 128;         // head dim (the only one this kernel serves)
+constexpr int kCK = 128;        // keys per chunk = M of S^T = K of O^T
+constexpr int kN = 16;          // MMA N: query heads of one pair, padded
+constexpr int kStages = 3;      // K/V chunks in flight
+constexpr int kWarpTma = 4;
+constexpr int kWarpMma = 5;
+constexpr int kSoftmaxThreads = 128;
+constexpr int kThreads = 192;
+constexpr int kBarSoftmax = 1;  // named barrier of the softmax warps
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleThreshold = 8.0f;
+
+constexpr int kHalfBytes = kCK * 128;          // 128 rows x 64 dims: one swizzled half of a K or V chunk
+constexpr int kTileBytes = 2 * kHalfBytes;     // one K or V chunk
+constexpr int kStageBytes = 2 * kTileBytes;    // K chunk, then V chunk
+constexpr int kSmallHalf = kN * 128;           // 16 rows x 128 bytes: half of Q^T or of P^T
+constexpr int kSmallBytes = 2 * kSmallHalf;
+constexpr int kOffRing = 0;
+constexpr int kOffQ = kOffRing + kStages * kStageBytes;  // two Q^T slots (one per segment parity)
+constexpr int kOffP = kOffQ + 2 * kSmallBytes;           // two P^T buffers (one per chunk parity)
+constexpr int kOffRedMax = kOffP + 2 * kSmallBytes;      // [chunk parity][warp][head] chunk maxima
+constexpr int kOffRedSum = kOffRedMax + 2 * 4 * kN * 4;  // [warp][head][2] running sums
+constexpr int kOffBar = kOffRedSum + 4 * kN * 2 * 4;
+enum TcBar : int {
+    kBarFull0 = 0,                      // [stage] K/V chunk landed
+    kBarEmpty0 = kBarFull0 + kStages,   // [stage] chunk consumed by both MMAs
+    kBarQFull0 = kBarEmpty0 + kStages,  // [segment parity] Q^T landed
+    kBarQEmpty0 = kBarQFull0 + 2,       // [segment parity] last S^T of the segment done
+    kBarSFull0 = kBarQEmpty0 + 2,       // [chunk parity] S^T ready
+    kBarPFull0 = kBarSFull0 + 2,        // [chunk parity] P^T written (128 arrivals)
+    kBarODone0 = kBarPFull0 + 2,        // [chunk parity] O^T += V^T P^T done
+    kBarOFree = kBarODone0 + 2,         // segment's O^T read out (128 arrivals)
+    kBarDrain = kBarOFree + 1,
+    kNumTcBars = kBarDrain + 1,
+};
+constexpr int kOffMisc = kOffBar + kNumTcBars * 8;  // tmem slot, abort flag, merge bookkeeping
+constexpr int kUsed = kOffMisc + 64;
+constexpr int kSmem = kUsed + 1024;  // + alignment of the base to the 1024-byte swizzle repeat
+static_assert(kSmem <= 227 * 1024, "shared memory budget");
+static_assert(kOffQ % 1024 == 0 && kOffP % 1024 == 0, "swizzled tiles sit on 1024-byte boundaries");
+constexpr uint32_t kTmemCols = 64;  // S^T [0,16) and [16,32), O^T [32,48)
+constexpr uint32_t kColO = 32;
+
+struct TcParams {
+    __nv_bfloat16 *o;
+    float *lse;
+    float *ws;  // partials: [pairs][max_contrib][G*D + G]
+    int *counters, *status;
+    int Hq, Hkv, Skv, group, head_groups, cpp, ctas, max_contrib;
+    long long total;
+    float scale_log2;
+};
+
+__device__ __forceinline__ float ex2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ long long range_start(long long c, long long total, int ctas) { return c * total / ctas; }
+
+// The CTA whose range holds unit g: the largest c with range_start(c) <= g (c0 or c0 + 1).
+__device__ __forceinline__ int cta_of_unit(long long g, long long total, int ctas)
+{
+    long long c0 = g * ctas / total;
+    if (c0 + 1 < ctas && range_start(c0 + 1, total, ctas) <= g)
+        ++c0;
+    return static_cast<int>(c0);
+}
+
+// Wait that ignores the abort flag (drains copies in flight before the CTA exits).
+__device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity, uint64_t limit_ns)
+{
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > limit_ns)
+            return false;
+    }
+    return true;
+}
+
+template <int G>
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v, const TcParams p)
+{
+    static_assert(G >= 1 && G <= kN, "one pair's heads fit the MMA's N");
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t s_base = smem_u32(smem);
+    const uint32_t sRing = s_base + kOffRing;
+    const uint32_t sQ = s_base + kOffQ;
+    const uint32_t sP = s_base + kOffP;
+    const uint32_t bar0 = s_base + kOffBar;
+#define BAR(i) (bar0 + 8u * static_cast<uint32_t>(i))
+    float *red_max = reinterpret_cast<float *>(smem + kOffRedMax);
+    float *red_sum = reinterpret_cast<float *>(smem + kOffRedSum);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffMisc);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffMisc + 4);
+    int *last_flag = reinterpret_cast<int *>(smem + kOffMisc + 8);                     // [3]
+    long long *deferred_pair = reinterpret_cast<long long *>(smem + kOffMisc + 24);    // [2]
+    int *deferred_first = reinterpret_cast<int *>(smem + kOffMisc + 40);              // [2]
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int cta = blockIdx.x;
+    const long long g_begin = range_start(cta, p.total, p.ctas);
+    const long long g_end = range_start(cta + 1, p.total, p.ctas);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(BAR(kBarFull0 + s), 1);
+            mbar_init(BAR(kBarEmpty0 + s), 1);
+        }
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(BAR(kBarQFull0 + x), 1);
+            mbar_init(BAR(kBarQEmpty0 + x), 1);
+            mbar_init(BAR(kBarSFull0 + x), 1);
+            mbar_init(BAR(kBarPFull0 + x), kSoftmaxThreads);
+            mbar_init(BAR(kBarODone0 + x), 1);
+        }
+        mbar_init(BAR(kBarOFree), kSoftmaxThreads);
+        mbar_init(BAR(kBarDrain), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    // P^T rows G..15 are never written by the softmax: keep them zero.
+    for (int i = threadIdx.x; i < 2 * kSmallBytes / 16; i += kThreads)
+        reinterpret_cast<uint4 *>(smem + kOffP)[i] = make_uint4(0u, 0u, 0u, 0u);
+    fence_proxy_async_smem();
+    if (warp == kWarpTma && lane == 0) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+    }
+    if (warp == kWarpMma) {
+        tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == kWarpTma) {
+        // ---------------------------------------------------------------- TMA producer
+        if (lane == 0) {
+            int issued = 0, seg = 0;
+            long long pair = g_begin / p.cpp;
+            int local = static_cast<int>(g_begin - pair * p.cpp);
+            int bk = 0;
+            for (long long g = g_begin; g < g_end; ++g) {
+                if (g == g_begin || local == 0) {
+                    // A new segment: Q^T of its pair (G heads, padded to 16 rows) into the segment's slot.
+                    const int qs = seg & 1;
+                    if (!mbar_wait(BAR(kBarQEmpty0 + qs), (static_cast<uint32_t>(seg >> 1) & 1u) ^ 1u, abort_flag,
+                                   p.status, kSiteDecodeProducer))
+                        break;
+                    const int hg = static_cast<int>(pair % p.head_groups);
+                    bk = static_cast<int>(pair / p.head_groups);  // b * Hkv + kv head
+                    const int b = bk / p.Hkv;
+                    const int h0 = (bk % p.Hkv) * p.group + hg * G;
+                    mbar_arrive_expect_tx(BAR(kBarQFull0 + qs), kSmallBytes);
+                    for (int hf = 0; hf < 2; ++hf)
+                        tma_load_3d(sQ + qs * kSmallBytes + hf * kSmallHalf, &tm_q, BAR(kBarQFull0 + qs), hf * 64,
+                                    b * p.Hq + h0, 0);
+                    ++seg;
+                }
+                const int slot = issued % kStages;
+                if (!mbar_wait(BAR(kBarEmpty0 + slot), (static_cast<uint32_t>(issued / kStages) & 1u) ^ 1u, abort_flag,
+                               p.status, kSiteDecodeProducer))
+                    break;
+                const uint32_t dst = sRing + slot * kStageBytes;
+                const int key0 = local * kCK;
+                mbar_arrive_expect_tx(BAR(kBarFull0 + slot), kStageBytes);
+                for (int hf = 0; hf < 2; ++hf) {
+                    tma_load_3d(dst + hf * kHalfBytes, &tm_k, BAR(kBarFull0 + slot), hf * 64, key0, bk);
+                    tma_load_3d(dst + kTileBytes + hf * kHalfBytes, &tm_v, BAR(kBarFull0 + slot), hf * 64, key0, bk);
+                }
+                ++issued;
+                if (++local == p.cpp) {
+                    local = 0;
+                    ++pair;
+                }
+            }
+            if (*abort_flag) {
+                // Let every copy already issued land before the CTA exits.
+                for (int c = (issued > kStages ? issued - kStages : 0); c < issued; ++c)
+                    wait_drain(BAR(kBarFull0 + c % kStages), static_cast<uint32_t>(c / kStages) & 1u, 100000000ull);
+                for (int s = (seg > 2 ? seg - 2 : 0); s < seg; ++s)
+                    wait_drain(BAR(kBarQFull0 + (s & 1)), static_cast<uint32_t>(s >> 1) & 1u, 100000000ull);
+            }
+        }
+    } else if (warp == kWarpMma) {
+        // ---------------------------------------------------------------- MMA issuer
+        constexpr uint32_t kIdS = idesc_bf16_f32_ab(kCK, kN, false, false);  // A = K chunk, B = Q^T
+        constexpr uint32_t kIdO = idesc_bf16_f32_ab(kD, kN, true, false);    // A = V chunk read MN-major, B = P^T
+        const bool leader = elect_one();
+        // A K step moves the start address, the low field of a descriptor (address >> 4): every
+        // address here is below 2^18, so the field never overflows.
+        const uint64_t desc_k0 = smem_desc(sRing, 16, 1024, kSwizzle128B);
+        const uint64_t desc_v0 = smem_desc(sRing + kTileBytes, kHalfBytes, 1024, kSwizzle128B);
+        const uint64_t desc_q0 = smem_desc(sQ, 16, 1024, kSwizzle128B);
+        const uint64_t desc_p0 = smem_desc(sP, 16, 1024, kSwizzle128B);
+        auto commit = [&](int bar) {
+            if (leader)
+                tc_commit(BAR(bar));
+        };
+        auto issue_s = [&](int c, int qs) {
+            const uint64_t dk = desc_k0 + static_cast<uint64_t>((c % kStages) * (kStageBytes >> 4));
+            const uint64_t dq = desc_q0 + static_cast<uint64_t>(qs * (kSmallBytes >> 4));
+            if (leader) {
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk) {
+                    const uint64_t oa = static_cast<uint64_t>(((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4);
+                    const uint64_t ob = static_cast<uint64_t>(((kk >> 2) * kSmallHalf + (kk & 3) * 32) >> 4);
+                    tc_mma_ss(tmem + 16u * static_cast<uint32_t>(c & 1), dk + oa, dq + ob, kIdS, kk > 0 ? 1u : 0u);
+                }
+            }
+        };
+        auto issue_o = [&](int c, bool accumulate) {
+            const uint64_t dv = desc_v0 + static_cast<uint64_t>((c % kStages) * (kStageBytes >> 4));
+            const uint64_t dp = desc_p0 + static_cast<uint64_t>((c & 1) * (kSmallBytes >> 4));
+            if (leader) {
+#pragma unroll
+                for (int kk = 0; kk < kCK / 16; ++kk) {
+                    const uint64_t oa = static_cast<uint64_t>((kk * 16 * 128) >> 4);  // 16 keys of 128-byte rows
+                    const uint64_t ob = static_cast<uint64_t>(((kk >> 2) * kSmallHalf + (kk & 3) * 32) >> 4);
+                    tc_mma_ss(tmem + kColO, dv + oa, dp + ob, kIdO, (accumulate || kk > 0) ? 1u : 0u);
+                }
+            }
+        };
+        // O^T += V_c^T P^T once chunk c's weights are written; a segment's first chunk overwrites
+        // O^T, after the previous segment's O^T has been read out.
+        auto finish_o = [&](int c, bool first, int sg) -> bool {
+            if (first && sg > 0 &&
+                !mbar_wait(BAR(kBarOFree), static_cast<uint32_t>(sg - 1) & 1u, abort_flag, p.status, kSiteDecodeConsumer))
+                return false;
+            if (!mbar_wait(BAR(kBarPFull0 + (c & 1)), static_cast<uint32_t>(c >> 1) & 1u, abort_flag, p.status,
+                           kSiteDecodeConsumer))
+                return false;
+            tc_fence_after_sync();
+            issue_o(c, !first);
+            commit(kBarODone0 + (c & 1));
+            commit(kBarEmpty0 + c % kStages);
+            return true;
+        };
+
+        bool ok = true;
+        int c = 0, seg = -1;
+        bool have_prev = false, prev_first = false;
+        int prev_seg = 0;
+        long long pair = g_begin / p.cpp;
+        int local = static_cast<int>(g_begin - pair * p.cpp);
+        for (long long g = g_begin; ok && g < g_end; ++g) {
+            const bool first = (g == g_begin) || (local == 0);
+            const bool last = (g + 1 == g_end) || (local + 1 == p.cpp);
+            if (first) {
+                ++seg;
+                if (!(ok = mbar_wait(BAR(kBarQFull0 + (seg & 1)), static_cast<uint32_t>(seg >> 1) & 1u, abort_flag,
+                                     p.status, kSiteDecodeConsumer)))
+                    break;
+            }
+            if (!(ok = mbar_wait(BAR(kBarFull0 + c % kStages), static_cast<uint32_t>(c / kStages) & 1u, abort_flag,
+                                 p.status, kSiteDecodeConsumer)))
+                break;
+            tc_fence_after_sync();
+            issue_s(c, seg & 1);
+            commit(kBarSFull0 + (c & 1));
+            if (last)
+                commit(kBarQEmpty0 + (seg & 1));
+            // S^T(c) is queued behind O^T(c-1)'s predecessor; now the PV product of the previous chunk.
+            if (have_prev && !(ok = finish_o(c - 1, prev_first, prev_seg)))
+                break;
+            have_prev = true;
+            prev_first = first;
+            prev_seg = seg;
+            ++c;
+            if (++local == p.cpp) {
+                local = 0;
+                ++pair;
+            }
+        }
+        if (ok && have_prev)
+            ok = finish_o(c - 1, prev_first, prev_seg);
+        commit(kBarDrain);
+        if (!wait_drain(BAR(kBarDrain), 0, kWaitLimitNs) && leader) {
+            *abort_flag = 1;
+            atomicExch(p.status, kSiteDecodeConsumer);
+        }
+        __syncwarp();
+    } else {
+        // ---------------------------------------------------------------- softmax and epilogue
+        const int i = threadIdx.x;  // TMEM lane: key i of a chunk in S^T, dim i in O^T
+        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+        const uint32_t tS = tmem + lane_base;
+        const uint32_t tO = tmem + lane_base + kColO;
+        constexpr int n_out = G * kD;
+        bool ok = true;
+        int c = 0, n_deferred = 0;
+        for (long long g = g_begin; g < g_end;) {
+            const long long pair = g / p.cpp;
+            const int local0 = static_cast<int>(g - pair * p.cpp);
+            const long long seg_end = min(g_end, (pair + 1) * p.cpp);
+            const int n_chunks = static_cast<int>(seg_end - g);
+            const bool whole_pair = (local0 == 0) && (seg_end == (pair + 1) * p.cpp);
+            const int bk = static_cast<int>(pair / p.head_groups);
+            const int b = bk / p.Hkv;
+            const int h0 = (bk % p.Hkv) * p.group + static_cast<int>(pair % p.head_groups) * G;
+
+            float m[G], l[G], lpv[G];
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                m[h] = -INFINITY;
+                l[h] = 0.f;
+                lpv[h] = 0.f;
+            }
+            for (int j = 0; j < n_chunks; ++j, ++c) {
+                const bool okw = mbar_wait(BAR(kBarSFull0 + (c & 1)), static_cast<uint32_t>(c >> 1) & 1u, abort_flag,
+                                           p.status, kSiteDecodeConsumer);
+                float x[G];
+                if (okw) {
+                    tc_fence_after_sync();
+                    uint32_t r[16];
+                    tmem_ld16_wait(tS + 16u * static_cast<uint32_t>(c & 1), r);
+                    const bool valid = (local0 + j) * kCK + i < p.Skv;
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        x[h] = valid ? __uint_as_float(r[h]) * p.scale_log2 : -INFINITY;
+                        float v = x[h];
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1)
+                            v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+                        if (lane == 0)
+                            red_max[((c & 1) * 4 + warp) * kN + h] = v;
+                    }
+                }
+                // One barrier per chunk both exchanges the warps' maxima and agrees on carrying on.
+                if (!(ok = bar_and(kBarSoftmax, kSoftmaxThreads, okw && ok)))
+                    break;
+                const float *rm = red_max + (c & 1) * 4 * kN;
+                bool rescale = false;
+                float cmax[G];
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    cmax[h] = fmaxf(fmaxf(rm[h], rm[kN + h]), fmaxf(rm[2 * kN + h], rm[3 * kN + h]));
+                    rescale = rescale || (cmax[h] > m[h] + kRescaleThreshold);
+                }
+                if (j == 0) {
+#pragma unroll
+                    for (int h = 0; h < G; ++h)
+                        m[h] = cmax[h];  // the chunk holds at least one key, so this is finite
+                } else if (rescale) {
+                    // The same values in every thread, so every thread takes this branch. O^T(c-1)
+                    // must be complete before it is scaled.
+                    float alpha[G];
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        const float mn = fmaxf(m[h], cmax[h]);
+                        alpha[h] = ex2(m[h] - mn);
+                        m[h] = mn;
+                        l[h] *= alpha[h];
+                        lpv[h] *= alpha[h];
+                    }
+                    if (mbar_wait(BAR(kBarODone0 + ((c - 1) & 1)), static_cast<uint32_t>((c - 1) >> 1) & 1u,
+                                  abort_flag, p.status, kSiteDecodeConsumer)) {
+                        tc_fence_after_sync();
+                        uint32_t ov[16];
+                        tmem_ld16_wait(tO, ov);
+#pragma unroll
+                        for (int h = 0; h < G; ++h)
+                            ov[h] = __float_as_uint(__uint_as_float(ov[h]) * alpha[h]);
+                        tmem_st16_wait(tO, ov);
+                    } else {
+                        ok = false;
+                    }
+                }
+                // Weights, both running sums, and P^T (row h, column i) for the PV product. P^T is
+                // K-major with the 128-byte swizzle: key i sits in half i / 64 of row h, in 16-byte
+                // unit ((i % 64) / 8) XOR (h % 8).
+                uint8_t *pbuf = smem + kOffP + (c & 1) * kSmallBytes + (i >> 6) * kSmallHalf;
+                const int kk = i & 63;
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    const float pe = ex2(x[h] - m[h]);
+                    l[h] += pe;
+                    const __nv_bfloat16 pb = __float2bfloat16_rn(pe);
+                    lpv[h] += __bfloat162float(pb);
+                    const int off = (h >> 3) * 1024 + (h & 7) * 128 + ((((kk >> 3) ^ (h & 7)) << 4) | ((kk & 7) << 1));
+                    *reinterpret_cast<__nv_bfloat16 *>(pbuf + off) = pb;
+                }
+                fence_proxy_async_smem();
+                tc_fence_before_sync();
+                mbar_arrive(BAR(kBarPFull0 + (c & 1)));
+            }
+            if (!ok)
+                break;
+
+            // ------------------------------------------------ end of segment
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                float a = l[h], q = lpv[h];
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    a += __shfl_xor_sync(0xffffffffu, a, o);
+                    q += __shfl_xor_sync(0xffffffffu, q, o);
+                }
+                if (lane == 0) {
+                    red_sum[(warp * kN + h) * 2] = a;
+                    red_sum[(warp * kN + h) * 2 + 1] = q;
+                }
+            }
+            const bool okw = mbar_wait(BAR(kBarODone0 + ((c - 1) & 1)), static_cast<uint32_t>((c - 1) >> 1) & 1u,
+                                       abort_flag, p.status, kSiteDecodeConsumer);
+            if (!(ok = bar_and(kBarSoftmax, kSoftmaxThreads, okw && ok)))
+                break;
+            tc_fence_after_sync();
+            uint32_t ov[16];
+            tmem_ld16_wait(tO, ov);
+            tc_fence_before_sync();
+            mbar_arrive(BAR(kBarOFree));  // the next segment may overwrite O^T
+
+            int contrib_first = 0;
+            if (!whole_pair)
+                contrib_first = cta_of_unit(pair * p.cpp, p.total, p.ctas);
+            float *slot_base = p.ws + (static_cast<size_t>(pair) * p.max_contrib + (cta - contrib_first)) * (n_out + G);
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                float L = 0.f, LPV = 0.f;
+#pragma unroll
+                for (int w = 0; w < 4; ++w) {
+                    L += red_sum[(w * kN + h) * 2];
+                    LPV += red_sum[(w * kN + h) * 2 + 1];
+                }
+                const float o = __uint_as_float(ov[h]) / LPV;
+                const size_t bh = static_cast<size_t>(b) * p.Hq + h0 + h;
+                if (whole_pair) {
+                    p.o[bh * kD + i] = __float2bfloat16_rn(o);
+                    if (i == h)
+                        p.lse[bh] = (m[h] + log2f(L)) * kLn2;
+                } else {
+                    slot_base[h * kD + i] = o;
+                    if (i == h)
+                        slot_base[n_out + h] = m[h] + log2f(L);
+                }
+            }
+            if (!whole_pair) {
+                // Signalled once the whole range is streamed (below): only the first and the last
+                // segment of a range can be a piece of a shared pair.
+                if (i == 0) {
+                    deferred_pair[n_deferred] = pair;
+                    deferred_first[n_deferred] = contrib_first;
+                }
+                ++n_deferred;
+            }
+            g = seg_end;
+        }
+
+        // ---------------------------------------------------------------- shared pairs: the last CTA merges
+        if (ok) {
+            int n_def = 0;
+            if (i == 0) {
+                n_def = n_deferred;
+                if (n_def > 0)
+                    __threadfence();  // publish this CTA's partials before the counters move
+                for (int k = 0; k < n_def; ++k) {
+                    const long long pr = deferred_pair[k];
+                    const int first = deferred_first[k];
+                    const int n_contrib = cta_of_unit((pr + 1) * p.cpp - 1, p.total, p.ctas) - first + 1;
+                    const int prev = atomicAdd(&p.counters[pr], 1);
+                    last_flag[k] = (prev == n_contrib - 1) ? n_contrib : 0;
+                }
+                last_flag[2] = n_def;
+            }
+            bar_and(kBarSoftmax, kSoftmaxThreads, true);
+            n_def = last_flag[2];
+            for (int k = 0; k < n_def; ++k) {
+                const int n_contrib = last_flag[k];
+                if (n_contrib == 0)
+                    continue;
+                __threadfence();
+                const long long pr = deferred_pair[k];
+                const int bk = static_cast<int>(pr / p.head_groups);
+                const int b = bk / p.Hkv;
+                const int h0 = (bk % p.Hkv) * p.group + static_cast<int>(pr % p.head_groups) * G;
+                const float *pbase = p.ws + static_cast<size_t>(pr) * p.max_contrib * (n_out + G);
+                for (int idx = i; idx < n_out; idx += kSoftmaxThreads) {
+                    const int h = idx / kD;
+                    const int d = idx % kD;
+                    float M = -INFINITY;
+                    for (int s = 0; s < n_contrib; ++s)
+                        M = fmaxf(M, __ldcg(pbase + s * (n_out + G) + n_out + h));
+                    float W = 0.f, O = 0.f;
+                    for (int s = 0; s < n_contrib; ++s) {
+                        const float w = ex2(__ldcg(pbase + s * (n_out + G) + n_out + h) - M);
+                        W += w;
+                        O = fmaf(w, __ldcg(pbase + s * (n_out + G) + idx), O);
+                    }
+                    const size_t bh = static_cast<size_t>(b) * p.Hq + h0 + h;
+                    p.o[bh * kD + d] = __float2bfloat16_rn(O / W);
+                    if (d == 0)
+                        p.lse[bh] = (M + log2f(W)) * kLn2;
+                }
+                if (i == 0)
+                    atomicExch(&p.counters[pr], 0);  // ready for the next call
+            }
+        }
+    }
+
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == kWarpMma) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+#undef BAR
+}
+
+template <int G>
+cudaError_t prepare_g(int *ctas_per_sm)
+{
+    static int cached = 0;
+    if (cached == 0) {
+        cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+        int n = 0;
+        if (e == cudaSuccess)
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_tc_kernel<G>, kThreads, kSmem);
+        if (e != cudaSuccess)
+            return e;
+        cached = n > 0 ? n : 1;
+    }
+    if (ctas_per_sm)
+        *ctas_per_sm = cached;
+    return cudaSuccess;
+}
+
+template <int G>
+cudaError_t launch_g(const DecodeArgs &a, cudaStream_t stream)
+{
+    cudaError_t e = prepare_g<G>(nullptr);
+    if (e != cudaSuccess)
+        return e;
+    auto encode = get_encode_fn();
+    if (!encode)
+        return cudaErrorInitializationError;
+    int err = 0;
+    CUtensorMap tq, tk, tv;
+    // q as [1][B*Hq][D] (one row per query head), k and v as [B*Hkv][Skv][D].
+    if (!make_map(encode, &tq, a.q, kD, a.B * a.Hq, 1, 64, kN, CU_TENSOR_MAP_SWIZZLE_128B, &err) ||
+        !make_map(encode, &tk, a.k, kD, a.Skv, a.B * a.Hkv, 64, kCK, CU_TENSOR_MAP_SWIZZLE_128B, &err) ||
+        !make_map(encode, &tv, a.v, kD, a.Skv, a.B * a.Hkv, 64, kCK, CU_TENSOR_MAP_SWIZZLE_128B, &err))
+        return cudaErrorInvalidValue;
+    const DecodePlan &pl = a.plan;
+    TcParams p;
+    p.o = static_cast<__nv_bfloat16 *>(a.o);
+    p.lse = a.lse;
+    p.ws = a.ws;
+    p.counters = a.counters;
+    p.status = a.status;
+    p.Hq = a.Hq;
+    p.Hkv = a.Hkv;
+    p.Skv = a.Skv;
+    p.group = a.Hq / a.Hkv;
+    p.head_groups = pl.head_groups;
+    p.cpp = pl.cpp;
+    p.ctas = pl.ctas;
+    p.max_contrib = pl.max_contrib;
+    p.total = pl.total;
+    p.scale_log2 = a.scale * kLog2e;
+    decode_tc_kernel<G><<<static_cast<unsigned>(pl.ctas), kThreads, kSmem, stream>>>(tq, tk, tv, p);
+    return cudaGetLastError();
+}
+
+cudaError_t dispatch_tc(int G, const DecodeArgs *a, cudaStream_t stream, int *ctas_per_sm)
+{
+    switch (G) {
+    case 1:
+        return a ? launch_g<1>(*a, stream) : prepare_g<1>(ctas_per_sm);
+    case 2:
+        return a ? launch_g<2>(*a, stream) : prepare_g<2>(ctas_per_sm);
+    case 4:
+        return a ? launch_g<4>(*a, stream) : prepare_g<4>(ctas_per_sm);
+    case 8:
+        return a ? launch_g<8>(*a, stream) : prepare_g<8>(ctas_per_sm);
+    case 16:
+        return a ? launch_g<16>(*a, stream) : prepare_g<16>(ctas_per_sm);
+    default:
+        return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace
+
+int decode_tc_heads_per_pair(int group)
+{
+    // Largest power of two that divides the group size, at most the MMA's N of 16.
+    int g = 1;
+    while (g < kN && group % (2 * g) == 0)
+        g *= 2;
+    return g;
+}
+
+int decode_tc_chunk_keys() { return kCK; }
+
+cudaError_t decode_tc_ctas_per_sm(int G, int *ctas_per_sm) { return dispatch_tc(G, nullptr, nullptr, ctas_per_sm); }
+
+cudaError_t launch_decode_tc(const DecodeArgs &a, cudaStream_t stream) { return dispatch_tc(a.plan.G, &a, stream, nullptr); }
+
+}  // namespace attn_b200

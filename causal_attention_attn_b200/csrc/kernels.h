@@ -65,8 +65,14 @@ struct DecodeArgs {
 cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t stream, int *encode_error);
 
 // Decode planning and launch. requested_ctas <= 0 means one CTA per resident slot on the device.
-int decode_heads_per_cta(int group, int D);  // G: 1, 2, 4 or 8 (at most 4 for D = 128)
+int decode_heads_per_cta(int group, int D);  // G: 1, 2, 4 or 8 (up to 16 for D = 128)
 cudaError_t decode_plan(int B, int Hq, int Hkv, int Skv, int D, int requested_ctas, int sm_count, DecodePlan *plan);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream);
+
+// Head dim 128 decodes on the tensor core (decode_tc_sm100.cu); launch_decode routes there.
+int decode_tc_heads_per_pair(int group);  // G: largest power of two dividing the group, at most 16
+int decode_tc_chunk_keys();               // keys per chunk (128)
+cudaError_t decode_tc_ctas_per_sm(int G, int *ctas_per_sm);
+cudaError_t launch_decode_tc(const DecodeArgs &a, cudaStream_t stream);
 
 }  // namespace attn_b200

@@ -54,6 +54,7 @@
 
 #include "kernels.h"
 #include "sm100_ptx.cuh"
+#include "tma_host.h"
 
 namespace attn_b200 {
 namespace {
@@ -530,38 +531,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 #undef BAR
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn()
-{
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult qres;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qres) == cudaSuccess &&
-            qres == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    });
-    return fn;
-}
-
-// 3-D map over [BH][S][D] bf16 with a box of (inner, 128 rows, 1).
-bool make_map(PFN_cuTensorMapEncodeTiled_v12000 encode, CUtensorMap *map, const void *base, int D, int S, int BH,
-              int box_inner, CUtensorMapSwizzle swizzle, int *err)
-{
-    cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(S), static_cast<cuuint64_t>(BH)};
-    cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(S) * D * 2};
-    cuuint32_t box[3] = {static_cast<cuuint32_t>(box_inner), 128u, 1u};
-    cuuint32_t estr[3] = {1u, 1u, 1u};
-    CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) {
-        *err = static_cast<int>(r);
-        return false;
-    }
-    return true;
-}
-
 template <int D>
 cudaError_t launch(const PrefillArgs &a, cudaStream_t stream, int *encode_error)
 {
@@ -574,9 +543,9 @@ cudaError_t launch(const PrefillArgs &a, cudaStream_t stream, int *encode_error)
     const CUtensorMapSwizzle swz =
         (C::kSwizzleBytes == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
     CUtensorMap tq, tk, tv;
-    if (!make_map(encode, &tq, a.q, D, a.Sq, a.B * a.Hq, C::kChunkElems, swz, encode_error) ||
-        !make_map(encode, &tk, a.k, D, a.Skv, a.B * a.Hkv, C::kChunkElems, swz, encode_error) ||
-        !make_map(encode, &tv, a.v, D, a.Skv, a.B * a.Hkv, C::kChunkElems, swz, encode_error))
+    if (!make_map(encode, &tq, a.q, D, a.Sq, a.B * a.Hq, C::kChunkElems, 128, swz, encode_error) ||
+        !make_map(encode, &tk, a.k, D, a.Skv, a.B * a.Hkv, C::kChunkElems, 128, swz, encode_error) ||
+        !make_map(encode, &tv, a.v, D, a.Skv, a.B * a.Hkv, C::kChunkElems, 128, swz, encode_error))
         return cudaErrorInvalidValue;
 
     static bool attr_set = false;  // benign race: every caller sets the same value

@@ -1,0 +1,53 @@
+/*
+ * tma_host.h — host-side construction of TMA tensor maps for bf16 [BH][S][D] tensors.
+ *
+ * The driver's cuTensorMapEncodeTiled is reached through cudaGetDriverEntryPoint, so the library
+ * does not link against libcuda. Internal to the library; not part of the public ABI.
+ */
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+namespace attn_b200 {
+
+// The driver's tensor-map encoder, looked up once; null when the driver does not provide it.
+inline PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult qres;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qres) == cudaSuccess &&
+            qres == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// 3-D map over a contiguous bf16 tensor [BH][S][D] with a box of (box_inner elements of D,
+// box_rows rows of S, 1). Reads outside the tensor fill with zeros. Returns false (and the driver's
+// code in *err) when the driver rejects the map: base not 16-byte aligned, a stride not a multiple
+// of 16 bytes, or a box the swizzle mode cannot hold.
+inline bool make_map(PFN_cuTensorMapEncodeTiled_v12000 encode, CUtensorMap *map, const void *base, int D, int S,
+                     int BH, int box_inner, int box_rows, CUtensorMapSwizzle swizzle, int *err)
+{
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(S), static_cast<cuuint64_t>(BH)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(S) * D * 2};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_rows), 1u};
+    cuuint32_t estr[3] = {1u, 1u, 1u};
+    CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        *err = static_cast<int>(r);
+        return false;
+    }
+    return true;
+}
+
+}  // namespace attn_b200
