@@ -2,7 +2,7 @@
 
 One step = one pass of the whole hot path over one batch of synthetic input: the causal prefill of
 an 8B-shaped layer (B=1, Hq=32, Hkv=8, S=4096, D=128) through the prefill kernel, then the GQA
-decode over a 16 x 4096-token KV cache through the split-KV decode kernel. Inputs are resident in
+decode over a 16 x 4096-token KV cache through the tensor-core split-KV decode kernel. Inputs are resident in
 HBM before timing; L2 is flushed before each of the two kernels (a 256 MiB write, then a 256 MiB read
 so that the written lines are cleaned before the kernel starts), outside the kernel events.
 
@@ -284,8 +284,8 @@ def run_ours(args):
                 "metric": "decode KV-read GB/s", "value": decode_gbs, "unit": "GB/s", "config": DECODE.config(),
                 "roofline": {"bound": "hbm", "achieved": decode_bytes / dec_launch_s / 1e9, "peak": hbm_peak,
                              "unit": "GB/s", "frac": decode_bytes / dec_launch_s / 1e9 / hbm_peak,
-                             "traffic": read_traffic("decode_kernel", DECODE.name),
-                             "peak_kind": f"{peak_kind} HBM copy", "kernel": "decode_kernel<128,4>"},
+                             "traffic": read_traffic("decode_tc_kernel", DECODE.name),
+                             "peak_kind": f"{peak_kind} HBM copy", "kernel": "decode_tc_kernel<4>"},
                 "us_per_launch": dec_launch_s * 1e6,
                 "ctas": attn.decode_ctas(DECODE.B, DECODE.Hq, DECODE.Hkv, DECODE.Skv, DECODE.D),
             },
@@ -309,7 +309,7 @@ def run_ours(args):
 
 KERNEL_SOURCES = {
     "prefill_kernel": ["prefill_sm100.cu", "sm100_ptx.cuh"],
-    "decode_kernel": ["decode_sm100.cu", "sm100_ptx.cuh"],
+    "decode_tc_kernel": ["decode_tc_sm100.cu", "sm100_ptx.cuh"],
 }
 
 
