@@ -1,6 +1,8 @@
 /*
  * decode_sm100.cu — attention of one new query token per (batch, query head) over a bf16 K/V cache
- * (Sq == 1) on sm_100a: a persistent split-KV kernel with the LSE merge fused into the same launch.
+ * (Sq == 1) on sm_100a for head dims 32 and 64 (head dim 128 runs on the tensor core,
+ * decode_tc_sm100.cu): a persistent split-KV kernel with the LSE merge fused into the same launch.
+ * This file also holds the decode plan both kernels share.
  *
  * Work: a "pair" is one (batch, kv head, group of G query heads sharing that kv head); its Skv keys
  * are cut into chunks of CK keys. All pairs' chunks form one sequence of T = pairs * chunks_per_pair

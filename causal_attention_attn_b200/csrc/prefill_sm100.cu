@@ -41,8 +41,10 @@
  *
  * Warp roles (384 threads): warps 0-3 softmax / correction / epilogue of tile A, warps 4-7 the
  * same for tile B (warp w owns TMEM lanes 32(w%4)..+31), warp 8 TMA producer, warp 9 TMEM
- * allocator and MMA issuer (one thread issues), warps 10-11 idle. setmaxnreg moves registers from
- * the third warpgroup to the two softmax warpgroups.
+ * allocator and MMA issuer (the whole warp walks the schedule, one elected lane issues), warps
+ * 10-11 idle. setmaxnreg moves registers from the third warpgroup to the two softmax warpgroups.
+ * P_X is handed to the tensor core in two halves: PV on the first 64 keys starts while the softmax
+ * computes the second half.
  */
 #include <cuda.h>
 #include <cuda_bf16.h>
