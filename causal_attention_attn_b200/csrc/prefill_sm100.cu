@@ -116,7 +116,9 @@ struct Params {
     __nv_bfloat16 *o;
     float *lse;
     int *status;
-    int B, Hq, Hkv, Sq, Skv, group, offset, causal, n_pairs;
+    int B, Hq, Hkv, Sq, Skv, group, offset, causal;
+    int n_items;      // work items along the query dimension (see the work decode)
+    int pair_heads;   // 1: tiles A and B are the same query tile of two heads sharing a kv head
     float scale_log2;
 };
 
@@ -193,21 +195,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // Work decode: heads fastest, then batch, then pairs of query tiles from the last (heaviest).
+    // Work decode, heaviest items first (query tiles from the last). With pair_heads (the GQA group
+    // is even), tiles A and B are the same 128 query rows of heads 2k and 2k+1, which share a kv head:
+    // both need the same number of KV tiles, so they ping-pong to the last one. Otherwise they are
+    // two consecutive query tiles of one head, and B needs one KV tile more than A.
     int t = blockIdx.x;
-    const int h = t % p.Hq;
-    t /= p.Hq;
+    const int heads_per_item = p.pair_heads ? 2 : 1;
+    const int hu = t % (p.Hq / heads_per_item);
+    t /= p.Hq / heads_per_item;
     const int b = t % p.B;
     t /= p.B;
-    const int pair = p.n_pairs - 1 - t;
-    const int q0_a = pair * 2 * kBM;  // tile A rows [q0_a, q0_a + 128), tile B the next 128
-    const int n_a = kv_tiles_for(p, q0_a);
-    const int n_b = kv_tiles_for(p, q0_a + kBM);
+    const int item = p.n_items - 1 - t;
+    const int h_a = hu * heads_per_item;                       // head of tile A
+    const int q0_a = p.pair_heads ? item * kBM : item * 2 * kBM;  // first query row of tile A
+    auto q0_of = [&](int x) { return p.pair_heads ? q0_a : q0_a + x * kBM; };
+    auto bh_q_of = [&](int x) { return b * p.Hq + h_a + (p.pair_heads ? x : 0); };
+    const int n_a = kv_tiles_for(p, q0_of(0));
+    const int n_b = kv_tiles_for(p, q0_of(1));
     const int n_max = max(n_a, n_b);
-    auto q0_of = [&](int x) { return q0_a + x * kBM; };
     auto n_of = [&](int x) { return x ? n_b : n_a; };
-    const int bh_q = b * p.Hq + h;
-    const int bh_kv = b * p.Hkv + h / p.group;
+    const int bh_kv = b * p.Hkv + h_a / p.group;
 
     if (threadIdx.x == 0) {
         mbar_init(BAR(kBarQ), 1);
@@ -252,7 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int c = 0; c < C::kChunks; ++c)
                     tma_load_3d(sQ + x * C::kTileBytes + c * C::kChunkBytes, &tm_q, BAR(kBarQ), c * C::kChunkElems,
-                                q0_of(x), bh_q);
+                                q0_of(x), bh_q_of(x));
             // Items in consumption order: K0, V0, K1, V1, ...
             const int n_items = 2 * n_max;
             int issued = 0;
@@ -503,7 +510,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after_sync();
             const float inv_l = 1.f / l_pv;
             const bool store = row < p.Sq;
-            __nv_bfloat16 *orow = p.o + (static_cast<size_t>(bh_q) * p.Sq + (store ? row : 0)) * D;
+            const size_t bh_q = static_cast<size_t>(bh_q_of(x));
+            __nv_bfloat16 *orow = p.o + (bh_q * p.Sq + (store ? row : 0)) * D;
 #pragma unroll 1
             for (int cc = 0; cc < D / 32; ++cc) {
                 uint32_t ov[32];
@@ -520,7 +528,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             if (store)
-                p.lse[static_cast<size_t>(bh_q) * p.Sq + row] = (m + log2f(l)) * kLn2;
+                p.lse[bh_q * p.Sq + row] = (m + log2f(l)) * kLn2;
         }
     }
 
@@ -578,9 +586,10 @@ cudaError_t launch(const PrefillArgs &a, cudaStream_t stream, int *encode_error)
     p.offset = a.Skv - a.Sq;
     p.causal = a.causal;
     const int n_qtiles = (a.Sq + kBM - 1) / kBM;
-    p.n_pairs = (n_qtiles + 1) / 2;
+    p.pair_heads = (p.group % 2 == 0) ? 1 : 0;
+    p.n_items = p.pair_heads ? n_qtiles : (n_qtiles + 1) / 2;
     p.scale_log2 = a.scale * kLog2e;
-    const long long grid = static_cast<long long>(p.n_pairs) * a.B * a.Hq;
+    const long long grid = static_cast<long long>(p.n_items) * a.B * (a.Hq / (p.pair_heads ? 2 : 1));
     prefill_kernel<D><<<static_cast<unsigned>(grid), kThreads, C::kSmem, stream>>>(tq, tk, tv, p);
     return cudaGetLastError();
 }
