@@ -66,6 +66,8 @@ PREFILL_SHAPES = [
     (1, 3, 3, 100, 300, 64, False),     # non-causal over a longer cache
     (1, 4, 1, 512, 512, 128, True),     # four diagonal tiles
     (1, 1, 1, 1000, 1200, 32, True),    # D 32, offset 200
+    (1, 6, 2, 300, 300, 64, True),      # odd GQA group 3: the two tiles of a CTA are consecutive rows
+    (2, 8, 4, 257, 257, 128, True),     # GQA 2: the two tiles of a CTA are two heads, one row past
 ]
 
 
@@ -87,6 +89,9 @@ DECODE_SHAPES = [
     (2, 12, 4, 5000, 128),   # group 3 -> 1 head per CTA
     (1, 32, 8, 64, 128),     # exactly one chunk
     (2, 32, 8, 65, 128),     # one key into the second chunk
+    (2, 4, 2, 257, 128),     # group 2 on the tensor core, ragged last chunk
+    (2, 32, 2, 700, 128),    # group 16: all sixteen MMA columns used
+    (1, 64, 2, 300, 128),    # group 32 -> two pairs of 16 heads per kv head
 ]
 
 
