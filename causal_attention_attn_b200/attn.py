@@ -25,7 +25,7 @@ STATUS_NAMES = {
     -13: "ATTN_ERR_SCRATCH_LIMIT",
 }
 EXPORTED = ("attn_fwd", "attn_fwd_ex", "attn_decode_ctas", "attn_status_string", "attn_version",
-            "attn_device_status", "attn_decode_noalloc")
+            "attn_device_status", "attn_decode_noalloc", "attn_decode_paged")
 
 _lock = threading.Lock()
 _lib = None
@@ -63,6 +63,8 @@ def load_library(path: str | None = None):
         lib.attn_device_status.argtypes = [vp]
         lib.attn_decode_noalloc.restype = i
         lib.attn_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, vp]
+        lib.attn_decode_paged.restype = i
+        lib.attn_decode_paged.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, vp]
         if path is None:
             _lib = lib
         return lib
@@ -198,6 +200,42 @@ def attn_decode_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale
         rc = load_library().attn_decode_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                                                 lse.data_ptr(), B, Hq, Hkv, Skv, D, float(scale),
                                                 _stream_handle(stream))
+    _check(rc)
+    return out, lse
+
+
+def attn_decode_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor, block_table: torch.Tensor,
+                      seq_lens: torch.Tensor, max_seq_len: int, scale: float | None = None,
+                      out: torch.Tensor | None = None, lse: torch.Tensor | None = None, stream=None,
+                      decode_ctas: int = 0):
+    """Single-token decode over a paged, variable-length KV cache through ``attn_decode_paged``.
+    q: [B, Hq, 1, 128] bf16; k_pages, v_pages: [num_pages, Hkv, page_size, 128] bf16;
+    block_table: int32 [B, pages_per_seq]; seq_lens: int32 [B] (all on the GPU); max_seq_len: a
+    host-side bound of the lengths. Returns (o [B, Hq, 1, 128], lse [B, Hq, 1])."""
+    _check_tensor("q", q, torch.bfloat16, 4)
+    _check_tensor("k_pages", k_pages, torch.bfloat16, 4)
+    _check_tensor("v_pages", v_pages, torch.bfloat16, 4)
+    _check_tensor("block_table", block_table, torch.int32, 2)
+    _check_tensor("seq_lens", seq_lens, torch.int32, 1)
+    B, Hq, Sq, D = q.shape
+    num_pages, Hkv, page_size, Dk = k_pages.shape
+    if Sq != 1 or tuple(v_pages.shape) != tuple(k_pages.shape) or Dk != D:
+        raise ValueError(f"expected q [B,Hq,1,D] and k, v pages [P,Hkv,page,D]; got {tuple(q.shape)}, "
+                         f"{tuple(k_pages.shape)}")
+    if block_table.shape[0] != B or seq_lens.shape[0] != B:
+        raise ValueError("block_table and seq_lens need one row / entry per batch element")
+    if scale is None:
+        scale = D ** -0.5
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, Hq, 1), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check_tensor("out", out, torch.bfloat16, 4)
+    _check_tensor("lse", lse, torch.float32, 3)
+    with torch.cuda.device(q.device):
+        rc = load_library().attn_decode_paged(q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(),
+                                              block_table.data_ptr(), seq_lens.data_ptr(), out.data_ptr(),
+                                              lse.data_ptr(), B, Hq, Hkv, num_pages, page_size,
+                                              int(block_table.shape[1]), int(max_seq_len), float(scale),
+                                              int(decode_ctas), _stream_handle(stream))
     _check(rc)
     return out, lse
 

@@ -16,7 +16,7 @@
 namespace attn_b200 {
 namespace {
 
-constexpr int kVersion = 100;  // 0.1.0
+constexpr int kVersion = 200;  // 0.2.0: adds attn_decode_paged
 constexpr int kMaxDevices = 64;
 
 struct DeviceState {
@@ -310,6 +310,75 @@ extern "C" int attn_device_status(void *stream_ptr)
             return ATTN_ERR_CUDA;
         }
         return ATTN_ERR_DEVICE_TIMEOUT;
+    }
+    return ATTN_OK;
+}
+
+extern "C" int attn_decode_paged(const void *q, const void *k_pages, const void *v_pages, const int *block_table,
+                                 const int *seq_lens, void *o, float *lse, int B, int Hq, int Hkv, int num_pages,
+                                 int page_size, int pages_per_seq, int max_seq_len, float scale, int decode_ctas,
+                                 void *stream_ptr)
+{
+    using namespace attn_b200;
+    if (!q || !k_pages || !v_pages || !block_table || !seq_lens || !o || !lse)
+        return ATTN_ERR_NULL;
+    if (B < 1 || B > kPagedMaxBatch || Hq < 1 || Hkv < 1 || num_pages < 1 || pages_per_seq < 1 || max_seq_len < 0 ||
+        decode_ctas < 0)
+        return ATTN_ERR_SHAPE;
+    const bool page_ok = page_size == 16 || page_size == 32 || page_size == 64 ||
+                         (page_size >= 128 && page_size % 128 == 0);
+    if (!page_ok)
+        return ATTN_ERR_SHAPE;
+    if (Hq % Hkv != 0)
+        return ATTN_ERR_GQA;
+    // Page coordinates (page * Hkv + h), block-table offsets and output rows must fit in 32 bits.
+    if (static_cast<long long>(num_pages) * Hkv > INT_MAX || static_cast<long long>(B) * pages_per_seq > INT_MAX ||
+        static_cast<long long>(pages_per_seq) * page_size > INT_MAX || static_cast<long long>(B) * Hq > INT_MAX)
+        return ATTN_ERR_SHAPE;
+    if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(o) || !aligned16(lse) ||
+        (reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
+        return ATTN_ERR_ALIGN;
+    if (!(scale > 0.f) || !std::isfinite(scale))
+        return ATTN_ERR_SCALE;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+    std::lock_guard<std::mutex> lock(g_mutex);
+    int err = ATTN_OK;
+    DeviceState *s = device_state(&err);
+    if (!s)
+        return err;
+    DecodePlan plan;
+    if (decode_plan_paged(B, Hq, Hkv, max_seq_len, decode_ctas, s->sm_count, &plan) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_SHAPE;
+    }
+    int rc = ensure_workspace(*s, static_cast<size_t>(plan.pairs), plan.partial_floats, stream);
+    if (rc != ATTN_OK)
+        return rc;
+    DecodeArgs a;
+    a.q = q;
+    a.k = k_pages;
+    a.v = v_pages;
+    a.o = o;
+    a.lse = lse;
+    a.B = B;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.Skv = 0;
+    a.D = 128;
+    a.scale = scale;
+    a.plan = plan;
+    a.ws = s->partials;
+    a.counters = s->counters;
+    a.status = s->status;
+    a.seq_lens = seq_lens;
+    a.block_table = block_table;
+    a.num_pages = num_pages;
+    a.page_size = page_size;
+    a.pages_per_seq = pages_per_seq;
+    a.max_seq_len = max_seq_len;
+    if (launch_decode_tc(a, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_LAUNCH;
     }
     return ATTN_OK;
 }

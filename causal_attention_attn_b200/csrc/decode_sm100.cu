@@ -749,8 +749,11 @@ cudaError_t decode_plan(int B, int Hq, int Hkv, int Skv, int D, int requested_ct
     if (mc > pl.ctas)
         mc = pl.ctas;
     pl.max_contrib = shared ? static_cast<int>(mc) : 1;
-    pl.partial_floats =
-        shared ? static_cast<size_t>(pl.pairs) * pl.max_contrib * (static_cast<size_t>(pl.G) * D + pl.G) : 0;
+    if (D == 128)  // the tensor-core kernel keeps at most two partials per CTA
+        pl.partial_floats = shared ? decode_tc_partial_floats(pl.G, pl.ctas) : 0;
+    else
+        pl.partial_floats =
+            shared ? static_cast<size_t>(pl.pairs) * pl.max_contrib * (static_cast<size_t>(pl.G) * D + pl.G) : 0;
     *plan = pl;
     return cudaSuccess;
 }

@@ -87,7 +87,10 @@ enum TcBar : int {
     kNumTcBars = kBarDrain + 1,
 };
 constexpr int kOffMisc = kOffBar + kNumTcBars * 8;  // tmem slot, abort flag, merge bookkeeping
-constexpr int kUsed = kOffMisc + 64;
+// Paged decode only: first unit of each batch entry (and the total), then the clamped lengths.
+constexpr int kOffBatchStart = kOffMisc + 64;
+constexpr int kOffBatchLen = kOffBatchStart + 8 * (kPagedMaxBatch + 1);
+constexpr int kUsed = kOffBatchLen + 4 * kPagedMaxBatch;
 constexpr int kSmem = kUsed + 1024;  // + alignment of the base to the 1024-byte swizzle repeat
 static_assert(kSmem <= 227 * 1024, "shared memory budget");
 static_assert(kOffQ % 1024 == 0 && kOffP % 1024 == 0, "swizzled tiles sit on 1024-byte boundaries");
@@ -97,11 +100,14 @@ constexpr uint32_t kColO = 32;
 struct TcParams {
     __nv_bfloat16 *o;
     float *lse;
-    float *ws;  // partials: [pairs][max_contrib][G*D + G]
+    float *ws;  // partials: [CTA][first or last segment][G*D + G]
     int *counters, *status;
-    int Hq, Hkv, Skv, group, head_groups, cpp, ctas, max_contrib;
+    int Hq, Hkv, Skv, group, head_groups, cpp, ctas;
     long long total;
     float scale_log2;
+    // paged, variable-length cache
+    const int *seq_lens, *block_table;
+    int B, num_pages, page_size, pages_per_seq, max_seq_len;
 };
 
 __device__ __forceinline__ float ex2(float x)
@@ -113,13 +119,12 @@ __device__ __forceinline__ float ex2(float x)
 
 __device__ __forceinline__ long long range_start(long long c, long long total, int ctas) { return c * total / ctas; }
 
-// The CTA whose range holds unit g: the largest c with range_start(c) <= g (c0 or c0 + 1).
+// The CTA whose range holds unit g (0 <= g < total): the largest c with range_start(c) <= g.
+// floor(c T / P) <= g  <=>  c < (g + 1) P / T, so c = ceil((g + 1) P / T) - 1. Exact also when
+// there are fewer units than CTAs and several CTAs have empty ranges starting at the same unit.
 __device__ __forceinline__ int cta_of_unit(long long g, long long total, int ctas)
 {
-    long long c0 = g * ctas / total;
-    if (c0 + 1 < ctas && range_start(c0 + 1, total, ctas) <= g)
-        ++c0;
-    return static_cast<int>(c0);
+    return static_cast<int>(((g + 1) * ctas - 1) / total);
 }
 
 // Wait that ignores the abort flag (drains copies in flight before the CTA exits).
@@ -133,7 +138,14 @@ __device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity, uint64
     return true;
 }
 
-template <int G>
+// Where unit g of the whole sequence of chunks falls: its pair, the chunk within the pair, the
+// pair's chunk count and the pair's first unit.
+struct UnitPos {
+    long long pair, pair_start;
+    int local, cpp;
+};
+
+template <int G, bool kPaged>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const TcParams p)
@@ -155,11 +167,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     long long *deferred_pair = reinterpret_cast<long long *>(smem + kOffMisc + 24);    // [2]
     int *deferred_first = reinterpret_cast<int *>(smem + kOffMisc + 40);              // [2]
 
+    long long *batch_start = reinterpret_cast<long long *>(smem + kOffBatchStart);  // [B + 1]
+    int *batch_len = reinterpret_cast<int *>(smem + kOffBatchLen);                   // [B]
+
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int cta = blockIdx.x;
-    const long long g_begin = range_start(cta, p.total, p.ctas);
-    const long long g_end = range_start(cta + 1, p.total, p.ctas);
+    const int pairs_per_b = p.Hkv * p.head_groups;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -191,59 +205,170 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_alloc(smem_u32(tmem_slot), kTmemCols);
         tmem_relinquish();
     }
+    if constexpr (kPaged) {
+        // Each batch entry's length, clamped to what its block-table row and the workspace (sized
+        // for max_seq_len) can hold, and the first unit of its chunks (an exclusive scan by warp 0).
+        const int cap = min(p.max_seq_len, p.pages_per_seq * p.page_size);
+        for (int b = threadIdx.x; b < p.B; b += kThreads)
+            batch_len[b] = min(max(p.seq_lens[b], 0), cap);
+        __syncthreads();
+        if (warp == 0) {
+            long long running = 0;
+            for (int base = 0; base < p.B; base += 32) {
+                const int b = base + lane;
+                const long long u = (b < p.B) ? static_cast<long long>(pairs_per_b) * ((batch_len[b] + kCK - 1) / kCK) : 0;
+                long long incl = u;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const long long y = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o)
+                        incl += y;
+                }
+                if (b < p.B)
+                    batch_start[b] = running + incl - u;
+                running += __shfl_sync(0xffffffffu, incl, 31);
+            }
+            if (lane == 0)
+                batch_start[p.B] = running;
+        }
+    }
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
+    const long long total = kPaged ? batch_start[p.B] : p.total;
+    const long long g_begin = range_start(cta, total, p.ctas);
+    const long long g_end = range_start(cta + 1, total, p.ctas);
+
+    auto locate = [&](long long g) -> UnitPos {
+        UnitPos u;
+        if constexpr (kPaged) {
+            // The batch entry holding unit g: the largest b with batch_start[b] <= g (an entry with
+            // no chunks never qualifies, because the next entry starts at the same unit).
+            int lo = 0, hi = p.B - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (batch_start[mid] <= g)
+                    lo = mid;
+                else
+                    hi = mid - 1;
+            }
+            u.cpp = (batch_len[lo] + kCK - 1) / kCK;
+            const long long w = g - batch_start[lo];
+            const long long in_b = w / u.cpp;
+            u.pair = static_cast<long long>(lo) * pairs_per_b + in_b;
+            u.local = static_cast<int>(w - in_b * u.cpp);
+            u.pair_start = batch_start[lo] + in_b * u.cpp;
+        } else {
+            u.cpp = p.cpp;
+            u.pair = g / p.cpp;
+            u.local = static_cast<int>(g - u.pair * p.cpp);
+            u.pair_start = u.pair * p.cpp;
+        }
+        return u;
+    };
+    auto pair_first_unit = [&](long long pair, int *cpp) -> long long {
+        if constexpr (kPaged) {
+            const int b = static_cast<int>(pair / pairs_per_b);
+            *cpp = (batch_len[b] + kCK - 1) / kCK;
+            return batch_start[b] + (pair - static_cast<long long>(b) * pairs_per_b) * *cpp;
+        } else {
+            *cpp = p.cpp;
+            return pair * p.cpp;
+        }
+    };
 
     if (warp == kWarpTma) {
         // ---------------------------------------------------------------- TMA producer
-        if (lane == 0) {
-            int issued = 0, seg = 0;
-            long long pair = g_begin / p.cpp;
-            int local = static_cast<int>(g_begin - pair * p.cpp);
-            int bk = 0;
-            for (long long g = g_begin; g < g_end; ++g) {
-                if (g == g_begin || local == 0) {
-                    // A new segment: Q^T of its pair (G heads, padded to 16 rows) into the segment's slot.
-                    const int qs = seg & 1;
-                    if (!mbar_wait(BAR(kBarQEmpty0 + qs), (static_cast<uint32_t>(seg >> 1) & 1u) ^ 1u, abort_flag,
-                                   p.status, kSiteDecodeProducer))
-                        break;
-                    const int hg = static_cast<int>(pair % p.head_groups);
-                    bk = static_cast<int>(pair / p.head_groups);  // b * Hkv + kv head
-                    const int b = bk / p.Hkv;
-                    const int h0 = (bk % p.Hkv) * p.group + hg * G;
+        // The whole warp walks the schedule (waits agreed with __all_sync); lane 0 issues the
+        // copies. For a paged cache each lane keeps one block-table entry of a 32-entry window, so
+        // the table costs one coalesced load per 32 pages instead of a dependent load per page.
+        const bool issuer = (lane == 0);
+        int issued = 0, seg = 0;
+        UnitPos pos = locate(g_begin);
+        long long pair = pos.pair;
+        int local = pos.local, cpp = pos.cpp;
+        int bk = 0;
+        int tab_row = -1, tab_base = 0, tab_val = 0;  // this lane holds entry tab_base + lane of row tab_row
+        for (long long g = g_begin; g < g_end; ++g) {
+            if (g == g_begin || local == 0) {
+                // A new segment: Q^T of its pair (G heads, padded to 16 rows) into the segment's slot.
+                const int qs = seg & 1;
+                if (!__all_sync(0xffffffffu, mbar_wait(BAR(kBarQEmpty0 + qs), (static_cast<uint32_t>(seg >> 1) & 1u) ^ 1u,
+                                                       abort_flag, p.status, kSiteDecodeProducer)))
+                    break;
+                const int hg = static_cast<int>(pair % p.head_groups);
+                bk = static_cast<int>(pair / p.head_groups);  // b * Hkv + kv head
+                const int b = bk / p.Hkv;
+                const int h0 = (bk % p.Hkv) * p.group + hg * G;
+                if (issuer) {
                     mbar_arrive_expect_tx(BAR(kBarQFull0 + qs), kSmallBytes);
                     for (int hf = 0; hf < 2; ++hf)
                         tma_load_3d(sQ + qs * kSmallBytes + hf * kSmallHalf, &tm_q, BAR(kBarQFull0 + qs), hf * 64,
                                     b * p.Hq + h0, 0);
-                    ++seg;
                 }
-                const int slot = issued % kStages;
-                if (!mbar_wait(BAR(kBarEmpty0 + slot), (static_cast<uint32_t>(issued / kStages) & 1u) ^ 1u, abort_flag,
-                               p.status, kSiteDecodeProducer))
-                    break;
-                const uint32_t dst = sRing + slot * kStageBytes;
-                const int key0 = local * kCK;
+                ++seg;
+            }
+            const int slot = issued % kStages;
+            if (!__all_sync(0xffffffffu, mbar_wait(BAR(kBarEmpty0 + slot), (static_cast<uint32_t>(issued / kStages) & 1u) ^ 1u,
+                                                   abort_flag, p.status, kSiteDecodeProducer)))
+                break;
+            const uint32_t dst = sRing + slot * kStageBytes;
+            const int key0 = local * kCK;
+            if (issuer)
                 mbar_arrive_expect_tx(BAR(kBarFull0 + slot), kStageBytes);
+            if constexpr (kPaged) {
+                // The chunk's keys come page by page: boxes of min(page_size, 128) rows, box l issued
+                // by lane l so that small pages do not queue behind one thread. A box past the
+                // sequence's length reads the page beyond the last one, which the map fills with
+                // zeros, and never touches the block table past its row.
+                const int b = bk / p.Hkv;
+                const int kvh = bk - b * p.Hkv;
+                const int rows = min(p.page_size, kCK);
+                const int n_box = kCK / rows;
+                const int e0 = key0 / p.page_size;  // block-table entry of the chunk's first key
+                if (b != tab_row || e0 < tab_base || e0 + n_box > tab_base + 32) {  // the same in every lane
+                    tab_row = b;
+                    tab_base = e0;
+                    const int idx = e0 + lane;
+                    tab_val = (idx < p.pages_per_seq) ? p.block_table[static_cast<size_t>(b) * p.pages_per_seq + idx]
+                                                      : p.num_pages;
+                }
+                const int key = key0 + lane * rows;
+                const int e = (lane < n_box) ? key / p.page_size : e0;
+                int page = __shfl_sync(0xffffffffu, tab_val, e - tab_base);
+                if (lane < n_box) {
+                    if (key >= batch_len[b])
+                        page = p.num_pages;
+                    const int coord = static_cast<int>(static_cast<long long>(page) * p.Hkv + kvh);
+                    const int in_page = key % p.page_size;
+                    for (int hf = 0; hf < 2; ++hf) {
+                        tma_load_3d(dst + hf * kHalfBytes + lane * rows * 128, &tm_k, BAR(kBarFull0 + slot), hf * 64,
+                                    in_page, coord);
+                        tma_load_3d(dst + kTileBytes + hf * kHalfBytes + lane * rows * 128, &tm_v, BAR(kBarFull0 + slot),
+                                    hf * 64, in_page, coord);
+                    }
+                }
+            } else if (issuer) {
                 for (int hf = 0; hf < 2; ++hf) {
                     tma_load_3d(dst + hf * kHalfBytes, &tm_k, BAR(kBarFull0 + slot), hf * 64, key0, bk);
                     tma_load_3d(dst + kTileBytes + hf * kHalfBytes, &tm_v, BAR(kBarFull0 + slot), hf * 64, key0, bk);
                 }
-                ++issued;
-                if (++local == p.cpp) {
-                    local = 0;
-                    ++pair;
-                }
             }
-            if (*abort_flag) {
-                // Let every copy already issued land before the CTA exits.
-                for (int c = (issued > kStages ? issued - kStages : 0); c < issued; ++c)
-                    wait_drain(BAR(kBarFull0 + c % kStages), static_cast<uint32_t>(c / kStages) & 1u, 100000000ull);
-                for (int s = (seg > 2 ? seg - 2 : 0); s < seg; ++s)
-                    wait_drain(BAR(kBarQFull0 + (s & 1)), static_cast<uint32_t>(s >> 1) & 1u, 100000000ull);
+            ++issued;
+            if (++local == cpp && g + 1 < g_end) {
+                pos = locate(g + 1);
+                pair = pos.pair;
+                local = pos.local;
+                cpp = pos.cpp;
             }
+        }
+        if (*abort_flag && issuer) {
+            // Let every copy already issued land before the CTA exits.
+            for (int c = (issued > kStages ? issued - kStages : 0); c < issued; ++c)
+                wait_drain(BAR(kBarFull0 + c % kStages), static_cast<uint32_t>(c / kStages) & 1u, 100000000ull);
+            for (int s = (seg > 2 ? seg - 2 : 0); s < seg; ++s)
+                wait_drain(BAR(kBarQFull0 + (s & 1)), static_cast<uint32_t>(s >> 1) & 1u, 100000000ull);
         }
     } else if (warp == kWarpMma) {
         // ---------------------------------------------------------------- MMA issuer
@@ -304,11 +429,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         int c = 0, seg = -1;
         bool have_prev = false, prev_first = false;
         int prev_seg = 0;
-        long long pair = g_begin / p.cpp;
-        int local = static_cast<int>(g_begin - pair * p.cpp);
+        UnitPos pos = locate(g_begin);
+        int local = pos.local, cpp = pos.cpp;
         for (long long g = g_begin; ok && g < g_end; ++g) {
             const bool first = (g == g_begin) || (local == 0);
-            const bool last = (g + 1 == g_end) || (local + 1 == p.cpp);
+            const bool last = (g + 1 == g_end) || (local + 1 == cpp);
             if (first) {
                 ++seg;
                 if (!(ok = mbar_wait(BAR(kBarQFull0 + (seg & 1)), static_cast<uint32_t>(seg >> 1) & 1u, abort_flag,
@@ -330,9 +455,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             prev_first = first;
             prev_seg = seg;
             ++c;
-            if (++local == p.cpp) {
-                local = 0;
-                ++pair;
+            if (++local == cpp && g + 1 < g_end) {
+                pos = locate(g + 1);
+                local = pos.local;
+                cpp = pos.cpp;
             }
         }
         if (ok && have_prev)
@@ -350,17 +476,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t tS = tmem + lane_base;
         const uint32_t tO = tmem + lane_base + kColO;
         constexpr int n_out = G * kD;
+        if constexpr (kPaged) {
+            // A sequence with no keys has nothing to attend to: O = 0 and LSE = -inf, written by
+            // CTA (b mod P) since no unit of work names it.
+            for (int b = cta; b < p.B; b += p.ctas) {
+                if (batch_len[b] != 0)
+                    continue;
+                for (int h = 0; h < p.Hq; ++h) {
+                    p.o[(static_cast<size_t>(b) * p.Hq + h) * kD + i] = __float2bfloat16_rn(0.f);
+                    if (i == 0)
+                        p.lse[static_cast<size_t>(b) * p.Hq + h] = -INFINITY;
+                }
+            }
+        }
         bool ok = true;
         int c = 0, n_deferred = 0;
         for (long long g = g_begin; g < g_end;) {
-            const long long pair = g / p.cpp;
-            const int local0 = static_cast<int>(g - pair * p.cpp);
-            const long long seg_end = min(g_end, (pair + 1) * p.cpp);
+            const UnitPos pos = locate(g);
+            const long long pair = pos.pair;
+            const int local0 = pos.local;
+            const long long seg_end = min(g_end, pos.pair_start + pos.cpp);
             const int n_chunks = static_cast<int>(seg_end - g);
-            const bool whole_pair = (local0 == 0) && (seg_end == (pair + 1) * p.cpp);
+            const bool whole_pair = (local0 == 0) && (seg_end == pos.pair_start + pos.cpp);
             const int bk = static_cast<int>(pair / p.head_groups);
             const int b = bk / p.Hkv;
             const int h0 = (bk % p.Hkv) * p.group + static_cast<int>(pair % p.head_groups) * G;
+            const int seq_len = kPaged ? batch_len[b] : p.Skv;
 
             float m[G], l[G], lpv[G];
 #pragma unroll
@@ -377,7 +518,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_fence_after_sync();
                     uint32_t r[16];
                     tmem_ld16_wait(tS + 16u * static_cast<uint32_t>(c & 1), r);
-                    const bool valid = (local0 + j) * kCK + i < p.Skv;
+                    const bool valid = (local0 + j) * kCK + i < seq_len;
 #pragma unroll
                     for (int h = 0; h < G; ++h) {
                         x[h] = valid ? __uint_as_float(r[h]) * p.scale_log2 : -INFINITY;
@@ -443,6 +584,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int off = (h >> 3) * 1024 + (h & 7) * 128 + ((((kk >> 3) ^ (h & 7)) << 4) | ((kk & 7) << 1));
                     *reinterpret_cast<__nv_bfloat16 *>(pbuf + off) = pb;
                 }
+                if constexpr (kPaged) {
+                    // Rows past the sequence's length in its last page hold whatever the cache holds
+                    // there; their weights are 0, but 0 * NaN is not, so zero them before the PV product.
+                    if ((local0 + j) * kCK + i >= seq_len) {
+                        uint4 *vrow = reinterpret_cast<uint4 *>(smem + kOffRing + (c % kStages) * kStageBytes + kTileBytes +
+                                                                i * 128);
+#pragma unroll
+                        for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+                            for (int u = 0; u < 8; ++u)
+                                vrow[hf * (kHalfBytes / 16) + u] = make_uint4(0u, 0u, 0u, 0u);
+                    }
+                }
                 fence_proxy_async_smem();
                 tc_fence_before_sync();
                 mbar_arrive(BAR(kBarPFull0 + (c & 1)));
@@ -474,10 +628,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before_sync();
             mbar_arrive(BAR(kBarOFree));  // the next segment may overwrite O^T
 
-            int contrib_first = 0;
-            if (!whole_pair)
-                contrib_first = cta_of_unit(pair * p.cpp, p.total, p.ctas);
-            float *slot_base = p.ws + (static_cast<size_t>(pair) * p.max_contrib + (cta - contrib_first)) * (n_out + G);
+            // A CTA writes at most two partials: of its first segment (slot 0) and of its last one
+            // (slot 1); the merging CTA finds them the same way (see below).
+            const int which = (g == g_begin) ? 0 : 1;
+            float *slot_base = p.ws + (static_cast<size_t>(cta) * 2 + which) * (n_out + G);
 #pragma unroll
             for (int h = 0; h < G; ++h) {
                 float L = 0.f, LPV = 0.f;
@@ -501,10 +655,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!whole_pair) {
                 // Signalled once the whole range is streamed (below): only the first and the last
                 // segment of a range can be a piece of a shared pair.
-                if (i == 0) {
+                if (i == 0)
                     deferred_pair[n_deferred] = pair;
-                    deferred_first[n_deferred] = contrib_first;
-                }
                 ++n_deferred;
             }
             g = seg_end;
@@ -518,11 +670,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (n_def > 0)
                     __threadfence();  // publish this CTA's partials before the counters move
                 for (int k = 0; k < n_def; ++k) {
+                    // The pair's contributors: the CTAs from the one holding its first unit to the
+                    // one holding its last, except those with an empty range (fewer units than CTAs).
                     const long long pr = deferred_pair[k];
-                    const int first = deferred_first[k];
-                    const int n_contrib = cta_of_unit((pr + 1) * p.cpp - 1, p.total, p.ctas) - first + 1;
+                    int pr_cpp = 0;
+                    const long long pr_start = pair_first_unit(pr, &pr_cpp);
+                    const int first = cta_of_unit(pr_start, total, p.ctas);
+                    const int last = cta_of_unit(pr_start + pr_cpp - 1, total, p.ctas);
+                    int n_contrib = 0;
+                    for (int cc = first; cc <= last; ++cc)
+                        n_contrib += (range_start(cc, total, p.ctas) < range_start(cc + 1, total, p.ctas)) ? 1 : 0;
+                    deferred_first[k] = first;
                     const int prev = atomicAdd(&p.counters[pr], 1);
-                    last_flag[k] = (prev == n_contrib - 1) ? n_contrib : 0;
+                    last_flag[k] = (prev == n_contrib - 1) ? last - first + 1 : 0;
                 }
                 last_flag[2] = n_def;
             }
@@ -537,18 +697,34 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int bk = static_cast<int>(pr / p.head_groups);
                 const int b = bk / p.Hkv;
                 const int h0 = (bk % p.Hkv) * p.group + static_cast<int>(pr % p.head_groups) * G;
-                const float *pbase = p.ws + static_cast<size_t>(pr) * p.max_contrib * (n_out + G);
+                // n_contrib here is the span of CTAs (first .. first + span - 1); a contributor whose
+                // range starts inside the pair wrote its first segment (slot 0), the one whose range
+                // started before it wrote its last segment (slot 1).
+                const int first = deferred_first[k];
+                int pr_cpp = 0;
+                const long long pr_start = pair_first_unit(pr, &pr_cpp);
+                auto slot_of = [&](int cc) -> const float * {
+                    const int which = (range_start(cc, total, p.ctas) >= pr_start) ? 0 : 1;
+                    return p.ws + (static_cast<size_t>(cc) * 2 + which) * (n_out + G);
+                };
+                auto contributes = [&](int cc) {
+                    return range_start(cc, total, p.ctas) < range_start(cc + 1, total, p.ctas);
+                };
                 for (int idx = i; idx < n_out; idx += kSoftmaxThreads) {
                     const int h = idx / kD;
                     const int d = idx % kD;
                     float M = -INFINITY;
-                    for (int s = 0; s < n_contrib; ++s)
-                        M = fmaxf(M, __ldcg(pbase + s * (n_out + G) + n_out + h));
+                    for (int cc = first; cc < first + n_contrib; ++cc)
+                        if (contributes(cc))
+                            M = fmaxf(M, __ldcg(slot_of(cc) + n_out + h));
                     float W = 0.f, O = 0.f;
-                    for (int s = 0; s < n_contrib; ++s) {
-                        const float w = ex2(__ldcg(pbase + s * (n_out + G) + n_out + h) - M);
+                    for (int cc = first; cc < first + n_contrib; ++cc) {
+                        if (!contributes(cc))
+                            continue;
+                        const float *sb = slot_of(cc);
+                        const float w = ex2(__ldcg(sb + n_out + h) - M);
                         W += w;
-                        O = fmaf(w, __ldcg(pbase + s * (n_out + G) + idx), O);
+                        O = fmaf(w, __ldcg(sb + idx), O);
                     }
                     const size_t bh = static_cast<size_t>(b) * p.Hq + h0 + h;
                     p.o[bh * kD + d] = __float2bfloat16_rn(O / W);
@@ -570,15 +746,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 #undef BAR
 }
 
-template <int G>
+template <int G, bool kPaged>
 cudaError_t prepare_g(int *ctas_per_sm)
 {
     static int cached = 0;
     if (cached == 0) {
-        cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+        cudaError_t e =
+            cudaFuncSetAttribute(decode_tc_kernel<G, kPaged>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
         int n = 0;
         if (e == cudaSuccess)
-            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_tc_kernel<G>, kThreads, kSmem);
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_tc_kernel<G, kPaged>, kThreads, kSmem);
         if (e != cudaSuccess)
             return e;
         cached = n > 0 ? n : 1;
@@ -588,10 +765,10 @@ cudaError_t prepare_g(int *ctas_per_sm)
     return cudaSuccess;
 }
 
-template <int G>
+template <int G, bool kPaged>
 cudaError_t launch_g(const DecodeArgs &a, cudaStream_t stream)
 {
-    cudaError_t e = prepare_g<G>(nullptr);
+    cudaError_t e = prepare_g<G, kPaged>(nullptr);
     if (e != cudaSuccess)
         return e;
     auto encode = get_encode_fn();
@@ -599,10 +776,14 @@ cudaError_t launch_g(const DecodeArgs &a, cudaStream_t stream)
         return cudaErrorInitializationError;
     int err = 0;
     CUtensorMap tq, tk, tv;
-    // q as [1][B*Hq][D] (one row per query head), k and v as [B*Hkv][Skv][D].
+    // q as [1][B*Hq][D] (one row per query head); k and v as [B*Hkv][Skv][D], or, paged, as
+    // [num_pages*Hkv][page_size][D] read in boxes of min(page_size, 128) rows.
+    const int kv_rows = kPaged ? a.page_size : a.Skv;
+    const int kv_bh = kPaged ? a.num_pages * a.Hkv : a.B * a.Hkv;
+    const int box_rows = kPaged ? (a.page_size < kCK ? a.page_size : kCK) : kCK;
     if (!make_map(encode, &tq, a.q, kD, a.B * a.Hq, 1, 64, kN, CU_TENSOR_MAP_SWIZZLE_128B, &err) ||
-        !make_map(encode, &tk, a.k, kD, a.Skv, a.B * a.Hkv, 64, kCK, CU_TENSOR_MAP_SWIZZLE_128B, &err) ||
-        !make_map(encode, &tv, a.v, kD, a.Skv, a.B * a.Hkv, 64, kCK, CU_TENSOR_MAP_SWIZZLE_128B, &err))
+        !make_map(encode, &tk, a.k, kD, kv_rows, kv_bh, 64, box_rows, CU_TENSOR_MAP_SWIZZLE_128B, &err) ||
+        !make_map(encode, &tv, a.v, kD, kv_rows, kv_bh, 64, box_rows, CU_TENSOR_MAP_SWIZZLE_128B, &err))
         return cudaErrorInvalidValue;
     const DecodePlan &pl = a.plan;
     TcParams p;
@@ -618,26 +799,40 @@ cudaError_t launch_g(const DecodeArgs &a, cudaStream_t stream)
     p.head_groups = pl.head_groups;
     p.cpp = pl.cpp;
     p.ctas = pl.ctas;
-    p.max_contrib = pl.max_contrib;
     p.total = pl.total;
     p.scale_log2 = a.scale * kLog2e;
-    decode_tc_kernel<G><<<static_cast<unsigned>(pl.ctas), kThreads, kSmem, stream>>>(tq, tk, tv, p);
+    p.seq_lens = a.seq_lens;
+    p.block_table = a.block_table;
+    p.B = a.B;
+    p.num_pages = a.num_pages;
+    p.page_size = a.page_size;
+    p.pages_per_seq = a.pages_per_seq;
+    p.max_seq_len = a.max_seq_len;
+    decode_tc_kernel<G, kPaged><<<static_cast<unsigned>(pl.ctas), kThreads, kSmem, stream>>>(tq, tk, tv, p);
     return cudaGetLastError();
+}
+
+template <int G>
+cudaError_t dispatch_g(const DecodeArgs *a, cudaStream_t stream, int *ctas_per_sm)
+{
+    if (!a)
+        return prepare_g<G, false>(ctas_per_sm);
+    return a->seq_lens ? launch_g<G, true>(*a, stream) : launch_g<G, false>(*a, stream);
 }
 
 cudaError_t dispatch_tc(int G, const DecodeArgs *a, cudaStream_t stream, int *ctas_per_sm)
 {
     switch (G) {
     case 1:
-        return a ? launch_g<1>(*a, stream) : prepare_g<1>(ctas_per_sm);
+        return dispatch_g<1>(a, stream, ctas_per_sm);
     case 2:
-        return a ? launch_g<2>(*a, stream) : prepare_g<2>(ctas_per_sm);
+        return dispatch_g<2>(a, stream, ctas_per_sm);
     case 4:
-        return a ? launch_g<4>(*a, stream) : prepare_g<4>(ctas_per_sm);
+        return dispatch_g<4>(a, stream, ctas_per_sm);
     case 8:
-        return a ? launch_g<8>(*a, stream) : prepare_g<8>(ctas_per_sm);
+        return dispatch_g<8>(a, stream, ctas_per_sm);
     case 16:
-        return a ? launch_g<16>(*a, stream) : prepare_g<16>(ctas_per_sm);
+        return dispatch_g<16>(a, stream, ctas_per_sm);
     default:
         return cudaErrorInvalidValue;
     }
@@ -659,5 +854,38 @@ int decode_tc_chunk_keys() { return kCK; }
 cudaError_t decode_tc_ctas_per_sm(int G, int *ctas_per_sm) { return dispatch_tc(G, nullptr, nullptr, ctas_per_sm); }
 
 cudaError_t launch_decode_tc(const DecodeArgs &a, cudaStream_t stream) { return dispatch_tc(a.plan.G, &a, stream, nullptr); }
+
+size_t decode_tc_partial_floats(int G, int ctas) { return static_cast<size_t>(2) * ctas * (static_cast<size_t>(G) * kD + G); }
+
+cudaError_t decode_plan_paged(int B, int Hq, int Hkv, int max_seq_len, int requested_ctas, int sm_count,
+                              DecodePlan *plan)
+{
+    DecodePlan pl;
+    const int group = Hq / Hkv;
+    pl.G = decode_tc_heads_per_pair(group);
+    pl.head_groups = group / pl.G;
+    pl.pairs = static_cast<long long>(B) * Hkv * pl.head_groups;
+    pl.ck = kCK;
+    pl.cpp = (max_seq_len + kCK - 1) / kCK;  // an upper bound: lengths are read on the device
+    pl.total = 0;                            // computed by each CTA from the lengths
+    long long ctas = requested_ctas;
+    if (ctas <= 0) {
+        int per_sm = 1;
+        const cudaError_t e = prepare_g<1, true>(&per_sm);
+        if (e != cudaSuccess)
+            return e;
+        // As for the dense cache: one CTA per pair when the pairs alone fill most of the GPU
+        // (measured faster than sharing pairs among all SMs), else one CTA per resident slot.
+        const long long slots = static_cast<long long>(sm_count) * per_sm;
+        ctas = (pl.pairs <= slots && 4 * pl.pairs >= 3 * slots) ? pl.pairs : slots;
+    }
+    if (ctas > (1LL << 22))
+        return cudaErrorInvalidValue;
+    pl.ctas = static_cast<int>(ctas);
+    pl.max_contrib = 0;  // unused by this kernel: partials are kept per CTA
+    pl.partial_floats = decode_tc_partial_floats(pl.G, pl.ctas);
+    *plan = pl;
+    return cudaSuccess;
+}
 
 }  // namespace attn_b200

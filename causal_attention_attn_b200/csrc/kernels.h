@@ -59,6 +59,12 @@ struct DecodeArgs {
     float *ws;          // plan.partial_floats floats (may be null when that is 0)
     int *counters;      // plan.pairs arrival counters, zero between calls
     int *status;        // device status word
+    // Paged, variable-length cache (tensor-core decode only; seq_lens == nullptr: the dense cache
+    // above). k, v are then [num_pages][Hkv][page_size][D]; block_table [B][pages_per_seq] and
+    // seq_lens [B] are device int32 arrays; lengths are clamped to [0, min(max_seq_len, capacity)].
+    const int *seq_lens = nullptr;
+    const int *block_table = nullptr;
+    int num_pages = 0, page_size = 0, pages_per_seq = 0, max_seq_len = 0;
 };
 
 // Returns a cudaError_t value (cudaSuccess on success); never synchronises.
@@ -73,6 +79,12 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream);
 int decode_tc_heads_per_pair(int group);  // G: largest power of two dividing the group, at most 16
 int decode_tc_chunk_keys();               // keys per chunk (128)
 cudaError_t decode_tc_ctas_per_sm(int G, int *ctas_per_sm);
+size_t decode_tc_partial_floats(int G, int ctas);  // workspace floats for shared pairs' partials
+constexpr int kPagedMaxBatch = 1024;  // batch entries a paged decode may have (per-CTA scan in shared memory)
+// Plan of a paged, variable-length decode: lengths are only known on the device, so the plan holds
+// upper bounds (cpp from max_seq_len; total is computed by each CTA); every pair may be shared.
+cudaError_t decode_plan_paged(int B, int Hq, int Hkv, int max_seq_len, int requested_ctas, int sm_count,
+                              DecodePlan *plan);
 cudaError_t launch_decode_tc(const DecodeArgs &a, cudaStream_t stream);
 
 }  // namespace attn_b200

@@ -137,6 +137,37 @@ int attn_device_status(void *stream);
 int attn_decode_noalloc(const void *q, const void *k, const void *v, void *o, float *lse,
                         int B, int Hq, int Hkv, int Skv, int D, float scale, void *stream);
 
+/*
+ * attn_decode_paged — single-token decode (Sq == 1) over a paged KV cache whose sequences have
+ * different lengths: each sequence attends only to the keys it has filled.
+ *
+ * Source (page title, section): a KV cache allocated for more tokens than it holds, of which only
+ * the filled part is attended to — "第11节：Attention 实现（Flash vs Fallback）", §3 and "Bộ 06 · Bên
+ * trong model", Q2 (the cache grows by one token per decode step); decode needs no mask — "AI Infra
+ * 入门…", §3. The page layout itself is this library's choice: the pages describe none.
+ *
+ * Layout (device pointers owned by the caller; bf16 unless noted):
+ *   q            [B, Hq, 1, 128]; o [B, Hq, 1, 128]; lse fp32 [B, Hq, 1].
+ *   k_pages      [num_pages, Hkv, page_size, 128]: page p of kv head h holds page_size consecutive
+ *   v_pages      keys' rows. 16-byte aligned.
+ *   block_table  int32 [B, pages_per_seq]: the n-th page_size keys of sequence b live in page
+ *                block_table[b * pages_per_seq + n].
+ *   seq_lens     int32 [B]: keys filled in sequence b. Each length is clamped to
+ *                [0, min(max_seq_len, pages_per_seq * page_size)]; a page index outside
+ *                [0, num_pages) reads as zeros. Sequence b attends to keys 0 .. len_b - 1; a
+ *                sequence with no keys gets o = 0 and lse = -inf.
+ *   max_seq_len  host-side upper bound of the lengths (sizes nothing larger than it needs).
+ *   page_size    16, 32, 64 or a multiple of 128.
+ *   decode_ctas  CTAs to launch (0: one per resident slot). A performance parameter only.
+ * Head dim 128 only; 1 <= B <= 1024; Hq % Hkv == 0. Lengths are read on the device: the call
+ * never synchronises, so block_table and seq_lens may be written by earlier work on `stream`.
+ * Returns ATTN_OK or a negative attn_status (argument errors before any launch).
+ */
+int attn_decode_paged(const void *q, const void *k_pages, const void *v_pages, const int *block_table,
+                      const int *seq_lens, void *o, float *lse, int B, int Hq, int Hkv, int num_pages,
+                      int page_size, int pages_per_seq, int max_seq_len, float scale, int decode_ctas,
+                      void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -37,7 +37,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.attn_version() == 100
+    assert lib.attn_version() == 200
     for code, name in attn.STATUS_NAMES.items():
         s = attn.status_string(code)
         assert s and s != "unknown status", (code, name)
@@ -101,3 +101,28 @@ def test_non_causal_allows_more_queries_than_keys_in_validation(lib):
         pytest.skip("would reach the device with fake pointers")
     rc = attn.attn_fwd_raw(*A, 1, 4, 2, 9, 8, 64, 0.125, 0, 0)
     assert rc in (-12, -7), rc
+
+
+PAGED_GOOD = dict(B=2, Hq=8, Hkv=2, num_pages=4, page_size=64, pages_per_seq=2, max_seq_len=128, scale=0.1, ctas=0)
+PAGED_CASES = [
+    ("null block table", dict(ptrs=[A[0], A[1], A[2], 0, A[4], A[3], A[4]]), -1),
+    ("page size 48", dict(page_size=48), -2),
+    ("page size 192", dict(page_size=192), -2),
+    ("batch 1025", dict(B=1025), -2),
+    ("negative max length", dict(max_seq_len=-1), -2),
+    ("negative cta count", dict(ctas=-1), -2),
+    ("gqa not divisible", dict(Hq=6, Hkv=4), -3),
+    ("misaligned seq_lens", dict(ptrs=[A[0], A[1], A[2], A[3], A[4] + 2, A[3], A[4]]), -5),
+    ("zero scale", dict(scale=0.0), -11),
+]
+
+
+@pytest.mark.parametrize("name,override,expected", PAGED_CASES, ids=[c[0] for c in PAGED_CASES])
+def test_paged_argument_errors(lib, name, override, expected):
+    a = dict(PAGED_GOOD)
+    a.update({k: v for k, v in override.items() if k != "ptrs"})
+    ptrs = override.get("ptrs", [A[0], A[1], A[2], A[3], A[4], A[3], A[4]])
+    rc = lib.attn_decode_paged(*ptrs, a["B"], a["Hq"], a["Hkv"], a["num_pages"], a["page_size"], a["pages_per_seq"],
+                               a["max_seq_len"], a["scale"], a["ctas"], None)
+    assert rc == expected, (name, rc)
+
