@@ -59,6 +59,14 @@ def _bind(path: str):
         ctypes.c_float, ctypes.c_int,
         ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
     ]
+    bwd = lib.oracle_attn_bwd
+    bwd.restype = ctypes.c_int
+    bwd.argtypes = [
+        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,  # q k v dout (bf16 bits)
+        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,  # dq dk dv (fp64)
+        ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+        ctypes.c_float, ctypes.c_int, ctypes.c_int,
+    ]
     return lib
 
 
@@ -121,3 +129,29 @@ def attention(q, k, v, scale: float, causal: bool, rows=None, threads: int | Non
     if rows is None:
         return o.reshape(B, Hq, Sq, D), lse.reshape(B, Hq, Sq)
     return o, lse
+
+
+def attention_bwd(q, k, v, dout, scale: float, causal: bool, threads: int | None = None, lib=None):
+    """Oracle backward pass: the gradients of a loss L with respect to q, k, v, given dO = dL/dO.
+
+    q, dout: [B, Hq, Sq, D]; k, v: [B, Hkv, Skv, D]; bf16 (torch) or bf16 bits (numpy uint16).
+    Returns ``(dq, dk, dv)`` as float64 numpy arrays of the input shapes.
+    """
+    qb, kb, vb, ob = _as_bf16_bits(q), _as_bf16_bits(k), _as_bf16_bits(v), _as_bf16_bits(dout)
+    if qb.ndim != 4 or kb.ndim != 4 or vb.shape != kb.shape or ob.shape != qb.shape:
+        raise ValueError("expected q, dout [B,Hq,Sq,D] and k, v [B,Hkv,Skv,D]")
+    B, Hq, Sq, D = qb.shape
+    Bk, Hkv, Skv, Dk = kb.shape
+    if Bk != B or Dk != D:
+        raise ValueError("q and k/v disagree on batch or head dim")
+    dq = np.empty((B, Hq, Sq, D), dtype=np.float64)
+    dk = np.empty((B, Hkv, Skv, D), dtype=np.float64)
+    dv = np.empty((B, Hkv, Skv, D), dtype=np.float64)
+    lib = lib if lib is not None else load()
+    rc = lib.oracle_attn_bwd(qb.ctypes.data, kb.ctypes.data, vb.ctypes.data, ob.ctypes.data, dq.ctypes.data,
+                             dk.ctypes.data, dv.ctypes.data, B, Hq, Hkv, Sq, Skv, D, ctypes.c_float(scale),
+                             int(bool(causal)), int(threads or 0))
+    if rc != 0:
+        raise ValueError(f"oracle_attn_bwd rejected its arguments (code {rc})")
+    return dq, dk, dv
+

@@ -153,3 +153,118 @@ int oracle_attn(const uint16_t *q, const uint16_t *k, const uint16_t *v,
     }
     return failed ? ORACLE_ERR_NOMEM : ORACLE_OK;
 }
+
+/*
+ * Backward pass of the same operation, in fp64: given dO (the gradient of a loss with respect to
+ * O), the gradients dQ, dK, dV.
+ *
+ * TEST INFRASTRUCTURE, like the forward above.
+ *
+ * The pages state only that the backward pass recomputes the softmax weights from the saved LSE
+ * instead of storing them ("AI Infra 入门…", §3, LSE paragraph); the gradients below are the
+ * textbook derivative of the forward definition above, written out with no blocking:
+ *
+ *   for every batch b, kv head g, every query head h of g's group and query row i:
+ *     P_ij  = exp(s_ij - lse_i)                 (visible j; lse_i as in the forward: m + ln l)
+ *     dP_ij = dO_i . v_j
+ *     D_i   = sum_j P_ij dP_ij                  (equal to dO_i . O_i)
+ *     dS_ij = P_ij (dP_ij - D_i)                (softmax derivative)
+ *     dQ_i  = scale * sum_j dS_ij k_j
+ *     dK_j += scale * dS_ij q_i                 (summed over rows and over the group's heads)
+ *     dV_j += P_ij dO_i
+ *
+ * q: [B, Hq, Sq, D], k/v: [B, Hkv, Skv, D], dout: [B, Hq, Sq, D], all bf16 bit patterns.
+ * dq: [B, Hq, Sq, D], dk/dv: [B, Hkv, Skv, D], fp64. Work is split over (b, kv head), so each
+ * thread owns the dK/dV rows it accumulates.
+ */
+int oracle_attn_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const uint16_t *dout,
+                    double *dq, double *dk, double *dv,
+                    int B, int Hq, int Hkv, int Sq, int Skv, int D,
+                    float scale, int causal, int n_threads)
+{
+    if (!q || !k || !v || !dout || !dq || !dk || !dv)
+        return ORACLE_ERR_ARGS;
+    if (B < 1 || Hq < 1 || Hkv < 1 || Sq < 1 || Skv < 1 || D < 1 || Hq % Hkv != 0)
+        return ORACLE_ERR_ARGS;
+    if (causal && Sq > Skv)
+        return ORACLE_ERR_ARGS;
+    const int group = Hq / Hkv;
+    const int offset = Skv - Sq;
+    const double scale_d = (double)scale;
+    int failed = 0;
+
+#pragma omp parallel num_threads(n_threads > 0 ? n_threads : omp_get_max_threads())
+    {
+        double *s = (double *)malloc(sizeof(double) * (size_t)Skv);
+        double *p = (double *)malloc(sizeof(double) * (size_t)Skv);
+        double *dp = (double *)malloc(sizeof(double) * (size_t)Skv);
+        if (!s || !p || !dp) {
+#pragma omp atomic write
+            failed = 1;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t bg = 0; bg < (int64_t)B * Hkv; ++bg) {
+            if (!s || !p || !dp)
+                continue;
+            const int b = (int)(bg / Hkv);
+            const int g = (int)(bg % Hkv);
+            const size_t kv_off = ((size_t)b * Hkv + g) * (size_t)Skv * D;
+            const uint16_t *k_head = k + kv_off;
+            const uint16_t *v_head = v + kv_off;
+            double *dk_head = dk + kv_off;
+            double *dv_head = dv + kv_off;
+            for (size_t e = 0; e < (size_t)Skv * D; ++e) {
+                dk_head[e] = 0.0;
+                dv_head[e] = 0.0;
+            }
+            for (int h = g * group; h < (g + 1) * group; ++h) {
+                for (int i = 0; i < Sq; ++i) {
+                    const size_t row = ((size_t)b * Hq + h) * Sq + i;
+                    const uint16_t *q_row = q + row * D;
+                    const uint16_t *do_row = dout + row * D;
+                    double *dq_row = dq + row * D;
+                    const int last = causal ? i + offset : Skv - 1;
+                    /* scores, then lse exactly as the forward computes it */
+                    double m = -INFINITY;
+                    for (int j = 0; j <= last; ++j) {
+                        double dot = 0.0;
+                        for (int d = 0; d < D; ++d)
+                            dot += bf16_to_double(q_row[d]) * bf16_to_double(k_head[(size_t)j * D + d]);
+                        s[j] = scale_d * dot;
+                        if (s[j] > m)
+                            m = s[j];
+                    }
+                    double l = 0.0;
+                    for (int j = 0; j <= last; ++j)
+                        l += exp(s[j] - m);
+                    const double lse = m + log(l);
+                    /* weights, dP and D_i */
+                    double Di = 0.0;
+                    for (int j = 0; j <= last; ++j) {
+                        p[j] = exp(s[j] - lse);
+                        double dot = 0.0;
+                        for (int d = 0; d < D; ++d)
+                            dot += bf16_to_double(do_row[d]) * bf16_to_double(v_head[(size_t)j * D + d]);
+                        dp[j] = dot;
+                        Di += p[j] * dp[j];
+                    }
+                    /* gradients */
+                    for (int d = 0; d < D; ++d)
+                        dq_row[d] = 0.0;
+                    for (int j = 0; j <= last; ++j) {
+                        const double ds = p[j] * (dp[j] - Di);
+                        for (int d = 0; d < D; ++d) {
+                            dq_row[d] += scale_d * ds * bf16_to_double(k_head[(size_t)j * D + d]);
+                            dk_head[(size_t)j * D + d] += scale_d * ds * bf16_to_double(q_row[d]);
+                            dv_head[(size_t)j * D + d] += p[j] * bf16_to_double(do_row[d]);
+                        }
+                    }
+                }
+            }
+        }
+        free(s);
+        free(p);
+        free(dp);
+    }
+    return failed ? ORACLE_ERR_NOMEM : ORACLE_OK;
+}
