@@ -16,9 +16,10 @@ SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), 
 
 # (name, original text, replacement, expected number of occurrences replaced)
 MUTANTS = [
-    ("mask_top_left_alignment", "causal ? i + offset : Skv - 1", "causal ? i : Skv - 1", 1),
-    ("mask_off_by_one", "causal ? i + offset : Skv - 1", "causal ? i + offset - 1 + (i == 0) : Skv - 1", 1),
-    ("mask_offset_sign", "const int offset = Skv - Sq;", "const int offset = Sq - Skv;", 1),
+    ("mask_top_left_alignment", "last_visible = causal ? i + offset : Skv - 1", "last_visible = causal ? i : Skv - 1", 1),
+    ("mask_off_by_one", "last_visible = causal ? i + offset : Skv - 1",
+     "last_visible = causal ? i + offset - 1 + (i == 0) : Skv - 1", 1),
+    ("mask_offset_sign", "const int offset = Skv - Sq; /* the mask", "const int offset = Sq - Skv; /* the mask", 1),
     ("scale_dropped", "scores[j] = scale * dot;", "scores[j] = dot;", 1),
     ("max_not_subtracted", "l += exp(scores[j] - m);", "l += exp(scores[j]);", 1),
     ("lse_without_max", "*lse_out = m + log(l);", "*lse_out = log(l);", 1),
