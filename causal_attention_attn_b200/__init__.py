@@ -9,7 +9,8 @@ __version__ = "0.2.0"
 
 
 def __getattr__(name):
-    if name in ("attn_fwd", "attn_fwd_host", "attn_decode_paged", "AttnError", "library_path", "load_library"):
+    if name in ("attn_fwd", "attn_fwd_host", "attn_decode_paged", "attn_bwd", "AttnError", "library_path",
+                "load_library"):
         from . import attn as _attn
 
         return getattr(_attn, name)

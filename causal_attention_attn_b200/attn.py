@@ -25,7 +25,7 @@ STATUS_NAMES = {
     -13: "ATTN_ERR_SCRATCH_LIMIT",
 }
 EXPORTED = ("attn_fwd", "attn_fwd_ex", "attn_decode_ctas", "attn_status_string", "attn_version",
-            "attn_device_status", "attn_decode_noalloc", "attn_decode_paged")
+            "attn_device_status", "attn_decode_noalloc", "attn_decode_paged", "attn_bwd")
 
 _lock = threading.Lock()
 _lib = None
@@ -64,6 +64,8 @@ def load_library(path: str | None = None):
         lib.attn_decode_noalloc.restype = i
         lib.attn_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, vp]
         lib.attn_decode_paged.restype = i
+        lib.attn_bwd.restype = i
+        lib.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp]
         lib.attn_decode_paged.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, vp]
         if path is None:
             _lib = lib
@@ -238,6 +240,32 @@ def attn_decode_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Ten
                                               int(decode_ctas), _stream_handle(stream))
     _check(rc)
     return out, lse
+
+
+def attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse: torch.Tensor,
+             dout: torch.Tensor, scale: float | None = None, causal: bool = True, dq: torch.Tensor | None = None,
+             dk: torch.Tensor | None = None, dv: torch.Tensor | None = None, stream=None):
+    """Backward pass through ``attn_bwd``: gradients for q, k, v given dout = dL/do, the forward's
+    inputs and its outputs o and lse. Head dim 128. Returns (dq, dk, dv), bf16."""
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout)):
+        _check_tensor(name, t, torch.bfloat16, 4)
+    _check_tensor("lse", lse, torch.float32, 3)
+    B, Hq, Sq, D = q.shape
+    Bk, Hkv, Skv, Dk = k.shape
+    if tuple(v.shape) != tuple(k.shape) or Bk != B or Dk != D or tuple(o.shape) != tuple(q.shape) \
+            or tuple(dout.shape) != tuple(q.shape) or tuple(lse.shape) != (B, Hq, Sq):
+        raise ValueError("shapes of q, k, v, o, lse, dout disagree")
+    if scale is None:
+        scale = D ** -0.5
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    with torch.cuda.device(q.device):
+        rc = load_library().attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(),
+                                     lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, Sq, Skv, D,
+                                     float(scale), int(bool(causal)), _stream_handle(stream))
+    _check(rc)
+    return dq, dk, dv
 
 
 def decode_ctas(B: int, Hq: int, Hkv: int, Skv: int, D: int) -> int:

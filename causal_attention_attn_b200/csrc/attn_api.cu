@@ -30,6 +30,8 @@ struct DeviceState {
     size_t counter_count = 0;
     float *partials = nullptr;
     size_t partial_floats = 0;
+    void *bwd_block = nullptr;  // backward pass: dq accumulator and per-row vectors
+    size_t bwd_bytes = 0;
 };
 
 std::mutex g_mutex;
@@ -382,3 +384,74 @@ extern "C" int attn_decode_paged(const void *q, const void *k_pages, const void 
     }
     return ATTN_OK;
 }
+
+extern "C" int attn_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout, const float *lse,
+                        void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int Sq, int Skv, int D, float scale,
+                        int causal, void *stream_ptr)
+{
+    using namespace attn_b200;
+    int rc = validate(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, D, scale, causal);
+    if (rc != ATTN_OK)
+        return rc;
+    if (!dout || !dq || !dk || !dv)
+        return ATTN_ERR_NULL;
+    if (!aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+        return ATTN_ERR_ALIGN;
+    if (D != 128)
+        return ATTN_ERR_HEADDIM;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+    std::lock_guard<std::mutex> lock(g_mutex);
+    int err = ATTN_OK;
+    DeviceState *s = device_state(&err);
+    if (!s)
+        return err;
+    rc = ensure_workspace(*s, 0, 0, stream);  // the status word
+    if (rc != ATTN_OK)
+        return rc;
+    const size_t need = bwd_workspace_bytes(B, Hq, Sq, D);
+    if (s->bwd_bytes < need) {
+        void *block = nullptr;
+        if (cudaMalloc(&block, need) != cudaSuccess) {
+            cudaGetLastError();
+            return ATTN_ERR_WORKSPACE;
+        }
+        if (s->bwd_block) {
+            // The old block may still be read by queued kernels.
+            if (cudaDeviceSynchronize() != cudaSuccess) {
+                cudaGetLastError();
+                cudaFree(block);
+                return ATTN_ERR_WORKSPACE;
+            }
+            cudaFree(s->bwd_block);
+        }
+        s->bwd_block = block;
+        s->bwd_bytes = need;
+    }
+    BwdArgs a;
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.o = o;
+    a.dout = dout;
+    a.lse = lse;
+    a.dq = dq;
+    a.dk = dk;
+    a.dv = dv;
+    a.B = B;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.Sq = Sq;
+    a.Skv = Skv;
+    a.D = D;
+    a.scale = scale;
+    a.causal = causal;
+    a.ws = s->bwd_block;
+    a.status = s->status;
+    int encode_error = 0;
+    if (launch_bwd(a, stream, &encode_error) != cudaSuccess) {
+        cudaGetLastError();
+        return encode_error ? ATTN_ERR_CUDA : ATTN_ERR_LAUNCH;
+    }
+    return ATTN_OK;
+}
+

@@ -1,0 +1,531 @@
+/*
+ * bwd_sm100.cu — backward pass of the fused attention (head dim 128) on sm_100a: given dO, the
+ * gradients dQ, dK, dV, with the softmax weights recomputed from the LSE saved by the forward.
+ *
+ * Per row i and visible key j (P_ij = exp(s_ij - lse_i), D_i = dO_i . O_i):
+ *   dV_j += P_ij dO_i,   dS_ij = P_ij (dO_i . v_j - D_i),
+ *   dQ_i += scale dS_ij k_j,   dK_j += scale dS_ij q_i.
+ *
+ * Kernels:
+ *   bwd_pre_kernel   D_i = dO_i . O_i and lse_i in log2 units, per row, into the workspace (rows
+ *                    padded to whole 128-row tiles per (batch, head));
+ *   bwd_kernel       one CTA per (128-key tile of K and V, batch, kv head); it walks every query
+ *                    head of the kv head's group and every 128-row query tile that sees any of its
+ *                    keys. Per step (one query tile), with keys in TMEM lanes:
+ *                      S^T  = K Q^T      and  dP^T = V dO^T     (tcgen05.mma, both operands TMA tiles)
+ *                      P^T, dS^T         the softmax warps (thread = key) recompute the weights from
+ *                                        the LSE, apply the causal mask, form dS, and write P^T and
+ *                                        dS^T back into TMEM as bf16 and dS into shared memory;
+ *                      dV  += P^T dO     (A = P^T from TMEM, B = dO read MN-major)
+ *                      dK  += dS^T Q     (A = dS^T from TMEM, B = Q read MN-major)
+ *                      dQ   = dS K       (A = dS from shared memory, B = K read MN-major)
+ *                    a second warpgroup (thread = query row) drains dQ with fp32 vector reductions
+ *                    into the workspace; dK and dV stay in TMEM until the last step;
+ *   bwd_dq_kernel    dQ (fp32 workspace) -> bf16.
+ *
+ * TMEM (512 columns): [0,128) S^T, then P^T (bf16) in [0,64), then dQ; [128,256) dP^T, then dS^T
+ * in [128,192); [256,384) dV; [384,512) dK. The MMAs of one thread run in issue order, so dV's read
+ * of P^T is done before dQ overwrites those columns, and dK's read of dS^T before the next dP^T.
+ *
+ * Sources (page title, section): the backward pass recomputes the weights from the LSE the forward
+ * saved instead of storing them — "AI Infra 入门：RMSNorm、Softmax、Causal Mask、Sampling 的数学与底层
+ * 优化", §3 (LSE paragraph); the causal mask and its alignment to the last Sq keys — same page §3 and
+ * "第11节：Attention 实现（Flash vs Fallback）", §3; bf16 operands with fp32 accumulation — "MLA 矩阵
+ * 乘法吸收的数值稳定性治理", §二.2. The gradient formulas are the derivative of the forward definition.
+ */
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+
+#include "kernels.h"
+#include "sm100_ptx.cuh"
+#include "tma_host.h"
+
+namespace attn_b200 {
+namespace {
+
+constexpr int kD = 128;
+constexpr int kBK = 128;  // keys per CTA tile (TMEM lanes of S^T, dP^T, dV, dK)
+constexpr int kBQ = 128;  // query rows per step
+constexpr int kThreads = 384;
+constexpr int kWarpTma = 8;
+constexpr int kWarpMma = 9;
+constexpr float kLog2e = 1.4426950408889634f;
+
+constexpr int kHalf = 128 * 128;      // 128 rows x 64 dims (or 64 keys) of bf16, 128-byte swizzle
+constexpr int kTile = 2 * kHalf;      // one 128 x 128 bf16 tile
+constexpr int kOffK = 0;
+constexpr int kOffV = kOffK + kTile;
+constexpr int kOffStage = kOffV + kTile;  // two stages of Q_i, dO_i
+constexpr int kStageBytes = 2 * kTile;
+constexpr int kOffDS = kOffStage + 2 * kStageBytes;  // dS (queries x keys), A operand of dQ
+constexpr int kOffVec = kOffDS + kTile;              // two stages of [lse2 | D] (128 floats each)
+constexpr int kVecBytes = 2 * kBQ * 4;
+constexpr int kOffBar = kOffVec + 2 * kVecBytes;
+enum BwdBar : int {
+    kBarKV = 0,
+    kBarStageFull0 = 1,   // [2]
+    kBarStageEmpty0 = 3,  // [2]
+    kBarSD = 5,           // S^T and dP^T ready
+    kBarP = 6,            // P^T, dS^T, dS written (128 arrivals)
+    kBarDQ = 7,           // dQ ready
+    kBarDQFree = 8,       // dQ drained (128 arrivals)
+    kBarFinal = 9,        // every MMA done
+    kNumBwdBars = 10,
+};
+constexpr int kOffMisc = kOffBar + kNumBwdBars * 8;
+constexpr int kSmem = kOffMisc + 64;  // the dynamic window starts 1024-aligned (no static smem)
+static_assert(kSmem <= 227 * 1024, "shared memory budget");
+constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 384;
+
+struct BwdParams {
+    __nv_bfloat16 *dk, *dv;
+    float *dq_acc;       // [B*Hq*Sq][D] fp32, zeroed before the launch
+    const float *vec;    // [2][B*Hq][Sq_pad]: lse2 then D
+    int *status;
+    int B, Hq, Hkv, Sq, Skv, Sq_pad, group, offset, causal, n_ktiles;
+    float scale, scale_log2;
+};
+
+__device__ __forceinline__ float ex2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
+{
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// acc[0..3] += (a, b, c, d): one vector reduction into global memory (16-byte aligned).
+__device__ __forceinline__ void red_add_v4(float *acc, float a, float b, float c, float d)
+{
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(acc), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity, uint64_t limit_ns)
+{
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > limit_ns)
+            return false;
+    }
+    return true;
+}
+
+// First query tile whose rows see key k0 (causal: row q sees k0 iff k0 <= q + offset).
+__device__ __forceinline__ int first_qtile(const BwdParams &p, int k0)
+{
+    if (!p.causal)
+        return 0;
+    const int q_min = k0 - p.offset;  // smallest row that sees key k0
+    return q_min <= 0 ? 0 : q_min / kBQ;
+}
+
+__global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16 *o, const __nv_bfloat16 *dout,
+                                                     const float *lse, float *vec, int rows, int Sq, int Sq_pad,
+                                                     int total_pad)
+{
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (warp >= rows)
+        return;
+    const uint2 a = reinterpret_cast<const uint2 *>(o + static_cast<size_t>(warp) * kD)[lane];
+    const uint2 b = reinterpret_cast<const uint2 *>(dout + static_cast<size_t>(warp) * kD)[lane];
+    auto lo = [](uint32_t w) { return __uint_as_float(w << 16); };
+    auto hi = [](uint32_t w) { return __uint_as_float(w & 0xffff0000u); };
+    float d = lo(a.x) * lo(b.x) + hi(a.x) * hi(b.x) + lo(a.y) * lo(b.y) + hi(a.y) * hi(b.y);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+        d += __shfl_xor_sync(0xffffffffu, d, off);
+    if (lane == 0) {
+        const int bh = warp / Sq, i = warp % Sq;
+        const size_t idx = static_cast<size_t>(bh) * Sq_pad + i;
+        vec[idx] = lse[warp] * kLog2e;
+        vec[static_cast<size_t>(total_pad) + idx] = d;
+    }
+}
+
+__global__ void __launch_bounds__(256) bwd_dq_kernel(const float4 *acc, uint2 *dq, long long n4)
+{
+    for (long long t = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; t < n4;
+         t += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const float4 a = acc[t];
+        dq[t] = make_uint2(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w));
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+               const BwdParams p)
+{
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const uint32_t s_base = smem_u32(smem);
+    const uint32_t sK = s_base + kOffK, sV = s_base + kOffV, sStage = s_base + kOffStage, sDS = s_base + kOffDS;
+    const uint32_t bar0 = s_base + kOffBar;
+#define BAR(i) (bar0 + 8u * static_cast<uint32_t>(i))
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffMisc);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffMisc + 4);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    // The swizzled tiles need the 1024-byte alignment the window starts with; refuse to run
+    // otherwise (the status word tells the caller).
+    if (s_base & 1023u) {
+        if (threadIdx.x == 0)
+            atomicExch(p.status, kSiteBwd);
+        return;
+    }
+
+    // Work decode: kv heads fastest, then batch, then key tiles from the first (the most rows see them).
+    int t = blockIdx.x;
+    const int g = t % p.Hkv;
+    t /= p.Hkv;
+    const int b = t % p.B;
+    const int kt = t / p.B;
+    const int k0 = kt * kBK;
+    const int bh_kv = b * p.Hkv + g;
+    const int n_qtiles = (p.Sq + kBQ - 1) / kBQ;
+    const int qt0 = first_qtile(p, k0);
+    const int steps_per_head = (qt0 < n_qtiles) ? n_qtiles - qt0 : 0;
+    const int n_steps = steps_per_head * p.group;
+    auto step_head = [&](int s) { return g * p.group + s / steps_per_head; };
+    auto step_q0 = [&](int s) { return (qt0 + s % steps_per_head) * kBQ; };
+
+    if (threadIdx.x == 0) {
+        mbar_init(BAR(kBarKV), 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(BAR(kBarStageFull0 + s), 1);
+            mbar_init(BAR(kBarStageEmpty0 + s), 1);
+        }
+        mbar_init(BAR(kBarSD), 1);
+        mbar_init(BAR(kBarP), 128);
+        mbar_init(BAR(kBarDQ), 1);
+        mbar_init(BAR(kBarDQFree), 128);
+        mbar_init(BAR(kBarFinal), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == kWarpMma) {
+        tmem_alloc(smem_u32(tmem_slot), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == kWarpTma) {
+        // ---------------------------------------------------------------- TMA producer
+        if (lane == 0 && n_steps > 0) {
+            mbar_arrive_expect_tx(BAR(kBarKV), 2 * kTile);
+            for (int hf = 0; hf < 2; ++hf) {
+                tma_load_3d(sK + hf * kHalf, &tm_k, BAR(kBarKV), hf * 64, k0, bh_kv);
+                tma_load_3d(sV + hf * kHalf, &tm_v, BAR(kBarKV), hf * 64, k0, bh_kv);
+            }
+            int s = 0;
+            for (; s < n_steps; ++s) {
+                const int st = s & 1;
+                if (!mbar_wait(BAR(kBarStageEmpty0 + st), (static_cast<uint32_t>(s >> 1) & 1u) ^ 1u, abort_flag, p.status,
+                               kSiteBwd))
+                    break;
+                const int h = step_head(s), q0 = step_q0(s);
+                const int bh_q = b * p.Hq + h;
+                const uint32_t dst = sStage + st * kStageBytes;
+                const size_t vec_off = static_cast<size_t>(bh_q) * p.Sq_pad + q0;
+                const size_t total_pad = static_cast<size_t>(p.B) * p.Hq * p.Sq_pad;
+                mbar_arrive_expect_tx(BAR(kBarStageFull0 + st), kStageBytes + kVecBytes);
+                for (int hf = 0; hf < 2; ++hf) {
+                    tma_load_3d(dst + hf * kHalf, &tm_q, BAR(kBarStageFull0 + st), hf * 64, q0, bh_q);
+                    tma_load_3d(dst + kTile + hf * kHalf, &tm_do, BAR(kBarStageFull0 + st), hf * 64, q0, bh_q);
+                }
+                const uint32_t vdst = s_base + kOffVec + st * kVecBytes;
+                bulk_load(vdst, p.vec + vec_off, kBQ * 4, BAR(kBarStageFull0 + st));
+                bulk_load(vdst + kBQ * 4, p.vec + total_pad + vec_off, kBQ * 4, BAR(kBarStageFull0 + st));
+            }
+            if (*abort_flag) {
+                wait_drain(BAR(kBarKV), 0, 100000000ull);
+                for (int c = (s > 2 ? s - 2 : 0); c < s; ++c)
+                    wait_drain(BAR(kBarStageFull0 + (c & 1)), static_cast<uint32_t>(c >> 1) & 1u, 100000000ull);
+            }
+        }
+    } else if (warp == kWarpMma) {
+        // ---------------------------------------------------------------- MMA issuer
+        const bool leader = elect_one();
+        constexpr uint32_t kIdSS = idesc_bf16_f32_ab(128, 128, false, false);  // S^T, dP^T
+        constexpr uint32_t kIdTS = idesc_bf16_f32_ab(128, 128, false, true);   // dV, dK: B read MN-major
+        constexpr uint32_t kIdQ = idesc_bf16_f32_ab(128, 128, false, true);    // dQ: A = dS, B = K read MN-major
+        auto kmaj = [](uint32_t base, int kk) {  // K-major tile, K step kk (16 elements)
+            return smem_desc(base + (kk >> 2) * kHalf + (kk & 3) * 32, 16, 1024, kSwizzle128B);
+        };
+        auto mnmaj = [](uint32_t base, int kk) {  // MN-major tile, K step kk (16 rows of 128 bytes)
+            return smem_desc(base + kk * 16 * 128, kHalf, 1024, kSwizzle128B);
+        };
+        auto commit = [&](int bar) {
+            if (leader)
+                tc_commit(BAR(bar));
+        };
+        bool ok = n_steps > 0 && mbar_wait(BAR(kBarKV), 0, abort_flag, p.status, kSiteBwd);
+        for (int s = 0; ok && s < n_steps; ++s) {
+            const int st = s & 1;
+            const uint32_t sQ = sStage + st * kStageBytes, sDO = sQ + kTile;
+            if (!(ok = mbar_wait(BAR(kBarStageFull0 + st), static_cast<uint32_t>(s >> 1) & 1u, abort_flag, p.status,
+                                 kSiteBwd)))
+                break;
+            // S^T goes where the previous step's dQ was: wait until it is drained.
+            if (s > 0 && !(ok = mbar_wait(BAR(kBarDQFree), static_cast<uint32_t>(s - 1) & 1u, abort_flag, p.status,
+                                          kSiteBwd)))
+                break;
+            tc_fence_after_sync();
+            if (leader) {
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk)
+                    tc_mma_ss(tmem + kColS, kmaj(sK, kk), kmaj(sQ, kk), kIdSS, kk > 0 ? 1u : 0u);
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk)
+                    tc_mma_ss(tmem + kColDP, kmaj(sV, kk), kmaj(sDO, kk), kIdSS, kk > 0 ? 1u : 0u);
+            }
+            commit(kBarSD);
+            if (!(ok = mbar_wait(BAR(kBarP), static_cast<uint32_t>(s) & 1u, abort_flag, p.status, kSiteBwd)))
+                break;
+            tc_fence_after_sync();
+            if (leader) {
+#pragma unroll
+                for (int kk = 0; kk < kBQ / 16; ++kk)  // dV += P^T dO
+                    tc_mma_ts(tmem + kColDV, tmem + kColS + kk * 8, mnmaj(sDO, kk), kIdTS, (s > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+                for (int kk = 0; kk < kBQ / 16; ++kk)  // dK += dS^T Q
+                    tc_mma_ts(tmem + kColDK, tmem + kColDP + kk * 8, mnmaj(sQ, kk), kIdTS, (s > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+                for (int kk = 0; kk < kBK / 16; ++kk)  // dQ = dS K (queries in TMEM lanes)
+                    tc_mma_ss(tmem + kColS, kmaj(sDS, kk), mnmaj(sK, kk), kIdQ, kk > 0 ? 1u : 0u);
+            }
+            commit(kBarDQ);
+            commit(kBarStageEmpty0 + st);
+        }
+        commit(kBarFinal);
+        if (!wait_drain(BAR(kBarFinal), 0, kWaitLimitNs) && leader) {
+            *abort_flag = 1;
+            atomicExch(p.status, kSiteBwd);
+        }
+        __syncwarp();
+    } else if (warp < 4) {
+        // ---------------------------------------------------------------- softmax warps: thread = key
+        const int kr = threadIdx.x;  // key within the tile == TMEM lane
+        const int key = k0 + kr;
+        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+        const uint32_t tS = tmem + lane_base + kColS, tDP = tmem + lane_base + kColDP;
+        bool ok = true;
+        for (int s = 0; s < n_steps; ++s) {
+            const int st = s & 1;
+            // tcgen05.ld/st are warp-collective: the warp goes on or stops as one.
+            if (!(ok = __all_sync(0xffffffffu, mbar_wait(BAR(kBarSD), static_cast<uint32_t>(s) & 1u, abort_flag,
+                                                         p.status, kSiteBwd))))
+                break;
+            tc_fence_after_sync();
+            const int q0 = step_q0(s);
+            const float *lse2 = reinterpret_cast<const float *>(smem + kOffVec + st * kVecBytes);
+            const float *dvec = lse2 + kBQ;
+            // Columns of this step's query tile that this key may feed: visible and inside Sq.
+            int last_q = min(kBQ, p.Sq - q0) - 1;  // last valid column
+            int first_q = 0;
+            if (p.causal)
+                first_q = max(0, key - p.offset - q0);  // row q sees key iff key <= q + offset
+            const bool key_ok = key < p.Skv;
+            uint8_t *dsrow_base = smem + kOffDS + (kr >> 6) * kHalf;
+            const int kk = kr & 63;
+#pragma unroll 1
+            for (int c = 0; c < kBQ / 32; ++c) {
+                uint32_t sr[32], dr[32];
+                tmem_ld32_wait(tS + c * 32, sr);
+                tmem_ld32_wait(tDP + c * 32, dr);
+                uint32_t pk[16], dk[16];
+#pragma unroll
+                for (int i = 0; i < 32; i += 2) {
+                    float pe[2], ds[2];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int q = c * 32 + i + u;
+                        const bool vis = key_ok && q >= first_q && q <= last_q;
+                        // Masked entries are exact zeros (lse2 and D of padding rows are never read).
+                        const float w = vis ? ex2(__uint_as_float(sr[i + u]) * p.scale_log2 - lse2[q]) : 0.f;
+                        pe[u] = w;
+                        ds[u] = vis ? w * (__uint_as_float(dr[i + u]) - dvec[q]) : 0.f;
+                    }
+                    pk[i >> 1] = pack_bf16x2(pe[0], pe[1]);
+                    dk[i >> 1] = pack_bf16x2(ds[0], ds[1]);
+                    // dS (row q, column key) for the dQ product: K-major, 128-byte swizzle.
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int q = c * 32 + i + u;
+                        const __nv_bfloat16 v = __float2bfloat16_rn(ds[u]);
+                        *reinterpret_cast<__nv_bfloat16 *>(dsrow_base + q * 128 +
+                                                           ((((kk >> 3) ^ (q & 7)) << 4) | ((kk & 7) << 1))) = v;
+                    }
+                }
+                // P^T and dS^T over the columns this warp has already read (in-place packing).
+                tmem_st16_wait(tS + c * 16, pk);
+                tmem_st16_wait(tDP + c * 16, dk);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before_sync();
+            mbar_arrive(BAR(kBarP));
+        }
+        // Epilogue: dK (scaled) and dV rows of this key. The whole warp loads (tcgen05.ld is
+        // warp-collective); only the stores of keys past Skv are skipped.
+        const bool okf = __all_sync(0xffffffffu, ok && mbar_wait(BAR(kBarFinal), 0, abort_flag, p.status, kSiteBwd));
+        const bool key_store = key < p.Skv;
+        if (okf) {
+            tc_fence_after_sync();
+            const size_t row = static_cast<size_t>(bh_kv) * p.Skv + (key_store ? key : 0);
+            __nv_bfloat16 *dk_row = p.dk + row * kD;
+            __nv_bfloat16 *dv_row = p.dv + row * kD;
+#pragma unroll 1
+            for (int c = 0; c < kD / 32; ++c) {
+                uint32_t kv[32], vv[32];
+                if (n_steps > 0) {
+                    tmem_ld32_wait(tmem + lane_base + kColDK + c * 32, kv);
+                    tmem_ld32_wait(tmem + lane_base + kColDV + c * 32, vv);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        kv[i] = vv[i] = 0u;
+                }
+                uint32_t pkk[16], pkv[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    pkk[i] = pack_bf16x2(__uint_as_float(kv[2 * i]) * p.scale, __uint_as_float(kv[2 * i + 1]) * p.scale);
+                    pkv[i] = pack_bf16x2(__uint_as_float(vv[2 * i]), __uint_as_float(vv[2 * i + 1]));
+                }
+                if (key_store) {
+                    uint4 *dkk = reinterpret_cast<uint4 *>(dk_row + c * 32);
+                    uint4 *dvv = reinterpret_cast<uint4 *>(dv_row + c * 32);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        dkk[i] = make_uint4(pkk[4 * i], pkk[4 * i + 1], pkk[4 * i + 2], pkk[4 * i + 3]);
+                        dvv[i] = make_uint4(pkv[4 * i], pkv[4 * i + 1], pkv[4 * i + 2], pkv[4 * i + 3]);
+                    }
+                }
+                __syncwarp();
+            }
+        }
+    } else if (warp < 8) {
+        // ---------------------------------------------------------------- dQ warps: thread = query row
+        // (warps 4-7 only: warps 10 and 11 have no role and go straight to the final barrier)
+        const int qr = threadIdx.x - 128;  // row within the query tile == TMEM lane
+        const uint32_t lane_base = static_cast<uint32_t>((warp - 4) * 32) << 16;
+        const uint32_t tQ = tmem + lane_base + kColS;
+        for (int s = 0; s < n_steps; ++s) {
+            if (!__all_sync(0xffffffffu, mbar_wait(BAR(kBarDQ), static_cast<uint32_t>(s) & 1u, abort_flag, p.status,
+                                                   kSiteBwd)))
+                break;
+            tc_fence_after_sync();
+            const int h = step_head(s), q0 = step_q0(s);
+            const bool valid = q0 + qr < p.Sq;
+            float *acc = p.dq_acc + ((static_cast<size_t>(b) * p.Hq + h) * p.Sq + (valid ? q0 + qr : 0)) * kD;
+#pragma unroll 1
+            for (int c = 0; c < kD / 32; ++c) {
+                uint32_t v[32];
+                tmem_ld32_wait(tQ + c * 32, v);
+                if (valid) {
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4)
+                        red_add_v4(acc + c * 32 + i, __uint_as_float(v[i]) * p.scale, __uint_as_float(v[i + 1]) * p.scale,
+                                   __uint_as_float(v[i + 2]) * p.scale, __uint_as_float(v[i + 3]) * p.scale);
+                }
+                __syncwarp();
+            }
+            tc_fence_before_sync();
+            mbar_arrive(BAR(kBarDQFree));
+        }
+    }
+
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == kWarpMma) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, 512);
+    }
+#undef BAR
+}
+
+}  // namespace
+
+size_t bwd_workspace_bytes(int B, int Hq, int Sq, int D)
+{
+    const size_t sq_pad = (static_cast<size_t>(Sq) + kBQ - 1) / kBQ * kBQ;
+    return static_cast<size_t>(B) * Hq * Sq * D * sizeof(float) + 2 * static_cast<size_t>(B) * Hq * sq_pad * sizeof(float);
+}
+
+cudaError_t launch_bwd(const BwdArgs &a, cudaStream_t stream, int *encode_error)
+{
+    if (a.D != kD)
+        return cudaErrorInvalidValue;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+        if (e != cudaSuccess)
+            return e;
+        attr_set = true;
+    }
+    auto encode = get_encode_fn();
+    if (!encode) {
+        *encode_error = -1;
+        return cudaErrorInitializationError;
+    }
+    CUtensorMap tq, tk, tv, tdo;
+    if (!make_map(encode, &tq, a.q, kD, a.Sq, a.B * a.Hq, 64, kBQ, CU_TENSOR_MAP_SWIZZLE_128B, encode_error) ||
+        !make_map(encode, &tdo, a.dout, kD, a.Sq, a.B * a.Hq, 64, kBQ, CU_TENSOR_MAP_SWIZZLE_128B, encode_error) ||
+        !make_map(encode, &tk, a.k, kD, a.Skv, a.B * a.Hkv, 64, kBK, CU_TENSOR_MAP_SWIZZLE_128B, encode_error) ||
+        !make_map(encode, &tv, a.v, kD, a.Skv, a.B * a.Hkv, 64, kBK, CU_TENSOR_MAP_SWIZZLE_128B, encode_error))
+        return cudaErrorInvalidValue;
+
+    const int Sq_pad = (a.Sq + kBQ - 1) / kBQ * kBQ;
+    const size_t rows = static_cast<size_t>(a.B) * a.Hq * a.Sq;
+    float *dq_acc = static_cast<float *>(a.ws);
+    float *vec = dq_acc + rows * kD;
+    cudaError_t e = cudaMemsetAsync(dq_acc, 0, rows * kD * sizeof(float), stream);
+    if (e != cudaSuccess)
+        return e;
+    const int total_pad = a.B * a.Hq * Sq_pad;
+    bwd_pre_kernel<<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16 *>(a.o), static_cast<const __nv_bfloat16 *>(a.dout), a.lse, vec,
+        static_cast<int>(rows), a.Sq, Sq_pad, total_pad);
+    if ((e = cudaGetLastError()) != cudaSuccess)
+        return e;
+
+    BwdParams p;
+    p.dk = static_cast<__nv_bfloat16 *>(a.dk);
+    p.dv = static_cast<__nv_bfloat16 *>(a.dv);
+    p.dq_acc = dq_acc;
+    p.vec = vec;
+    p.status = a.status;
+    p.B = a.B;
+    p.Hq = a.Hq;
+    p.Hkv = a.Hkv;
+    p.Sq = a.Sq;
+    p.Skv = a.Skv;
+    p.Sq_pad = Sq_pad;
+    p.group = a.Hq / a.Hkv;
+    p.offset = a.Skv - a.Sq;
+    p.causal = a.causal;
+    p.n_ktiles = (a.Skv + kBK - 1) / kBK;
+    p.scale = a.scale;
+    p.scale_log2 = a.scale * kLog2e;
+    const long long grid = static_cast<long long>(p.n_ktiles) * a.B * a.Hkv;
+    bwd_kernel<<<static_cast<unsigned>(grid), kThreads, kSmem, stream>>>(tq, tk, tv, tdo, p);
+    if ((e = cudaGetLastError()) != cudaSuccess)
+        return e;
+    const long long n4 = static_cast<long long>(rows) * kD / 4;
+    bwd_dq_kernel<<<296, 256, 0, stream>>>(reinterpret_cast<const float4 *>(dq_acc), static_cast<uint2 *>(a.dq), n4);
+    return cudaGetLastError();
+}
+
+}  // namespace attn_b200

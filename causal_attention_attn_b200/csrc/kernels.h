@@ -22,6 +22,7 @@ enum WaitSite : int {
     kSitePrefillDrain = 9,
     kSiteDecodeProducer = 16,
     kSiteDecodeConsumer = 17,
+    kSiteBwd = 24,
 };
 
 struct PrefillArgs {
@@ -69,6 +70,20 @@ struct DecodeArgs {
 
 // Returns a cudaError_t value (cudaSuccess on success); never synchronises.
 cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t stream, int *encode_error);
+
+// Backward pass (head dim 128): dq, dk, dv from q, k, v, o, dout and the forward's lse.
+struct BwdArgs {
+    const void *q, *k, *v, *o, *dout;
+    const float *lse;
+    void *dq, *dk, *dv;
+    int B, Hq, Hkv, Sq, Skv, D;
+    float scale;
+    int causal;
+    void *ws;     // bwd_workspace_bytes(B, Hq, Sq, D) bytes, 256-byte aligned
+    int *status;  // device status word
+};
+size_t bwd_workspace_bytes(int B, int Hq, int Sq, int D);
+cudaError_t launch_bwd(const BwdArgs &a, cudaStream_t stream, int *encode_error);
 
 // Decode planning and launch. requested_ctas <= 0 means one CTA per resident slot on the device.
 int decode_heads_per_cta(int group, int D);  // G: 1, 2, 4 or 8 (up to 16 for D = 128)

@@ -163,6 +163,22 @@ int attn_decode_noalloc(const void *q, const void *k, const void *v, void *o, fl
  * never synchronises, so block_table and seq_lens may be written by earlier work on `stream`.
  * Returns ATTN_OK or a negative attn_status (argument errors before any launch).
  */
+/*
+ * attn_bwd — backward pass of attn_fwd: given dout = dL/do for a loss L, the gradients
+ *   dq = dL/dq [B, Hq, Sq, D], dk = dL/dk and dv = dL/dv [B, Hkv, Skv, D] (bf16, written entirely;
+ *   for grouped heads dk and dv sum over the query heads that share a kv head).
+ * Inputs are those of the forward call plus its outputs o (bf16 [B, Hq, Sq, D]) and lse (fp32
+ * [B, Hq, Sq], natural log), and dout (bf16, layout of o). The softmax weights are recomputed from
+ * lse rather than stored — "AI Infra 入门…", §3 (LSE paragraph); the gradients are the derivative of
+ * the operation defined at the top of this file. Head dim 128 only; the other sizes, the causal flag
+ * and the scale as attn_fwd. The library keeps an fp32 accumulator for dq and two per-row vectors in
+ * its workspace (grown with cudaMalloc like attn_fwd's). Every pointer is a caller-owned device
+ * pointer, 16-byte aligned. Returns ATTN_OK or a negative attn_status; never synchronises.
+ */
+int attn_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout, const float *lse,
+             void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int Sq, int Skv, int D,
+             float scale, int causal, void *stream);
+
 int attn_decode_paged(const void *q, const void *k_pages, const void *v_pages, const int *block_table,
                       const int *seq_lens, void *o, float *lse, int B, int Hq, int Hkv, int num_pages,
                       int page_size, int pages_per_seq, int max_seq_len, float scale, int decode_ctas,
