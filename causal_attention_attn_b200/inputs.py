@@ -107,6 +107,28 @@ def generate(w: Workload):
     return q, k, v
 
 
+def generate_fp8(w: Workload):
+    """An e4m3 K/V cache for workload ``w``: ``(q, k8, v8, k_scale, v_scale)``.
+
+    q is drawn as by :func:`generate` (the same bytes); k and v too, then each (kv head, channel)
+    gets the coefficient max|x| / 448 over every batch entry and key (1 where that is 0), and the
+    codes are x / coefficient converted to e4m3 by torch (round to nearest even). k8, v8: uint8
+    [B, Hkv, Skv, D]; k_scale, v_scale: fp32 [Hkv, D]. This is input preparation for a quantised
+    cache, not part of the attention it feeds.
+    """
+    q, k, v = generate(w)
+
+    def quantise(x):
+        amax = x.float().abs().amax(dim=(0, 2))  # [Hkv, D]
+        coef = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax)).to(torch.float32)
+        codes = (x.float() / coef[None, :, None, :]).to(torch.float8_e4m3fn).view(torch.uint8)
+        return codes.contiguous(), coef.contiguous()
+
+    k8, k_scale = quantise(k)
+    v8, v_scale = quantise(v)
+    return q, k8, v8, k_scale, v_scale
+
+
 def sample_rows(w: Workload, every: int = 64, seed: int = 7) -> torch.Tensor:
     """Deterministic sample of flat row ids ``(b*Hq + h)*Sq + i`` covering every (b, h):
     every ``every``-th row plus the first row, the row at the cache offset and the last row."""

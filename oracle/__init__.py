@@ -13,7 +13,10 @@ compiles it with gcc and marshals arrays through ctypes. What it computes, with 
   ``j <= i + Skv - Sq``) -- "第11节：Attention 实现（Flash vs Fallback）", §3;
 * softmax in three passes (max, denominator, result) and ``LSE = m + ln l`` -- "AI Infra 入门：
   RMSNorm、Softmax、Causal Mask、Sampling 的数学与底层优化", §3;
-* masked keys get weight exactly zero -- "Bộ 06 · Bên trong model", Q2.
+* masked keys get weight exactly zero -- "Bộ 06 · Bên trong model", Q2;
+* an FP8 (e4m3) K/V cache with one fp32 coefficient per (kv head, channel), dequantised before the
+  plain definition -- "MLA 矩阵乘法吸收的数值稳定性治理", §五 (FP8 storage, higher-precision
+  accumulation) and §二.1 (per-channel scaling).
 """
 from __future__ import annotations
 
@@ -67,6 +70,19 @@ def _bind(path: str):
         ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
         ctypes.c_float, ctypes.c_int, ctypes.c_int,
     ]
+    fp8 = lib.oracle_attn_fp8kv
+    fp8.restype = ctypes.c_int
+    fp8.argtypes = [
+        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,  # q (bf16 bits), k8, v8 (e4m3 codes)
+        ctypes.c_void_p, ctypes.c_void_p,  # k_scale, v_scale (fp32 [Hkv, D])
+        ctypes.c_void_p, ctypes.c_void_p,  # o lse (fp64)
+        ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+        ctypes.c_float, ctypes.c_int,
+        ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
+    ]
+    dec = lib.oracle_decode_e4m3
+    dec.restype = None
+    dec.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64]
     return lib
 
 
@@ -155,3 +171,67 @@ def attention_bwd(q, k, v, dout, scale: float, causal: bool, threads: int | None
         raise ValueError(f"oracle_attn_bwd rejected its arguments (code {rc})")
     return dq, dk, dv
 
+
+
+def _as_u8(x) -> np.ndarray:
+    """Accept a torch uint8 / float8_e4m3fn tensor or a numpy uint8 array of e4m3 codes."""
+    if isinstance(x, np.ndarray):
+        if x.dtype != np.uint8:
+            raise TypeError("numpy fp8 inputs must be uint8 arrays of e4m3 codes")
+        return np.ascontiguousarray(x)
+    import torch
+
+    if not isinstance(x, torch.Tensor) or x.dtype not in (torch.uint8, torch.float8_e4m3fn):
+        raise TypeError("fp8 inputs must be torch uint8 / float8_e4m3fn tensors or uint8 numpy arrays")
+    return x.detach().to("cpu").contiguous().view(torch.uint8).numpy()
+
+
+def _as_f32(x) -> np.ndarray:
+    if isinstance(x, np.ndarray):
+        return np.ascontiguousarray(x, dtype=np.float32)
+    return x.detach().to("cpu").contiguous().float().numpy()
+
+
+def decode_e4m3(codes, lib=None) -> np.ndarray:
+    """The oracle's e4m3 decoder applied to an array of codes (float64 result, same shape)."""
+    c = _as_u8(codes)
+    out = np.empty(c.shape, dtype=np.float64)
+    lib = lib if lib is not None else load()
+    lib.oracle_decode_e4m3(c.ctypes.data, out.ctypes.data, int(c.size))
+    return out
+
+
+def attention_fp8kv(q, k8, v8, k_scale, v_scale, scale: float, causal: bool, rows=None,
+                    threads: int | None = None, lib=None):
+    """Oracle attention over an e4m3 K/V cache: k = e4m3(k8) * k_scale[kv head, channel], likewise v.
+
+    q: [B, Hq, Sq, D] bf16; k8/v8: [B, Hkv, Skv, D] e4m3 codes; k_scale/v_scale: [Hkv, D] fp32.
+    Returns ``(o, lse)`` as :func:`attention` does.
+    """
+    qb, kb, vb = _as_bf16_bits(q), _as_u8(k8), _as_u8(v8)
+    ks, vs = _as_f32(k_scale), _as_f32(v_scale)
+    if qb.ndim != 4 or kb.ndim != 4 or vb.shape != kb.shape:
+        raise ValueError("expected q [B,Hq,Sq,D] and k8, v8 [B,Hkv,Skv,D]")
+    B, Hq, Sq, D = qb.shape
+    Bk, Hkv, Skv, Dk = kb.shape
+    if Bk != B or Dk != D or ks.shape != (Hkv, D) or vs.shape != (Hkv, D):
+        raise ValueError("q, k8/v8 and the scales [Hkv, D] disagree")
+    if rows is None:
+        n_rows = B * Hq * Sq
+        rows_arr = None
+    else:
+        rows_arr = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1))
+        n_rows = int(rows_arr.shape[0])
+    o = np.empty((n_rows, D), dtype=np.float64)
+    lse = np.empty((n_rows,), dtype=np.float64)
+    lib = lib if lib is not None else load()
+    rc = lib.oracle_attn_fp8kv(
+        qb.ctypes.data, kb.ctypes.data, vb.ctypes.data, ks.ctypes.data, vs.ctypes.data,
+        o.ctypes.data, lse.ctypes.data, B, Hq, Hkv, Sq, Skv, D, ctypes.c_float(scale), int(bool(causal)),
+        rows_arr.ctypes.data if rows_arr is not None else None, n_rows, int(threads or 0),
+    )
+    if rc != 0:
+        raise ValueError(f"oracle_attn_fp8kv rejected its arguments (code {rc})")
+    if rows is None:
+        return o.reshape(B, Hq, Sq, D), lse.reshape(B, Hq, Sq)
+    return o, lse

@@ -268,3 +268,128 @@ int oracle_attn_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, con
     }
     return failed ? ORACLE_ERR_NOMEM : ORACLE_OK;
 }
+
+/*
+ * Attention over an FP8 (e4m3) K/V cache with per-channel scales, in fp64.
+ *
+ * TEST INFRASTRUCTURE, like the functions above.
+ *
+ * "MLA 矩阵乘法吸收的数值稳定性治理", §五: the KV cache may be stored in FP8 to save bandwidth,
+ * with the products accumulated in higher precision; §二.1 of the same page scales each feature
+ * channel by a coefficient. Reading taken here: one fp32 coefficient per (kv head, channel) for K
+ * and one for V, and the cached value is code * coefficient:
+ *
+ *   k~[b,g,j,d] = e4m3(k8[b,g,j,d]) * k_scale[g,d],   v~[b,g,j,d] = e4m3(v8[b,g,j,d]) * v_scale[g,d]
+ *
+ * after which the result is the plain definition above with k~, v~ in place of k, v.
+ *
+ * e4m3 (the OCP 8-bit format with 4 exponent and 3 mantissa bits, bias 7, no infinities): bit 7
+ * sign, bits 6-3 exponent e, bits 2-0 mantissa m. e = 0: (m / 8) * 2^-6; otherwise
+ * (1 + m / 8) * 2^(e - 7), except e = 15 with m = 7, which is NaN. Largest finite value 448.
+ */
+static double e4m3_to_double(uint8_t code)
+{
+    const int sign = code >> 7;
+    const int e = (code >> 3) & 15;
+    const int m = code & 7;
+    double mag;
+    if (e == 15 && m == 7)
+        return NAN;
+    if (e == 0)
+        mag = ldexp((double)m / 8.0, -6);
+    else
+        mag = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return sign ? -mag : mag;
+}
+
+/* Decodes n e4m3 codes (exposed for the tests that pin the decoder). */
+void oracle_decode_e4m3(const uint8_t *codes, double *out, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = e4m3_to_double(codes[i]);
+}
+
+/* One query row over the dequantised cache; n_vis keys (0..n_vis-1) are visible. */
+static void fp8kv_row(const uint16_t *qv, const uint8_t *kc, const uint8_t *vc, const float *ks,
+                      const float *vs, int D, int n_vis, double scale, double *sc, double *out,
+                      double *lse_out)
+{
+    /* scaled scores against the dequantised keys k~ = e4m3(code) * ks[channel] */
+    for (int j = 0; j < n_vis; ++j) {
+        double acc = 0.0;
+        for (int d = 0; d < D; ++d) {
+            const double kd = e4m3_to_double(kc[(size_t)j * D + d]) * (double)ks[d];
+            acc += bf16_to_double(qv[d]) * kd;
+        }
+        sc[j] = acc * scale;
+    }
+    double mx = -INFINITY;
+    for (int j = 0; j < n_vis; ++j)
+        mx = sc[j] > mx ? sc[j] : mx;
+    double den = 0.0;
+    for (int j = 0; j < n_vis; ++j)
+        den += exp(sc[j] - mx);
+    for (int d = 0; d < D; ++d)
+        out[d] = 0.0;
+    for (int j = 0; j < n_vis; ++j) {
+        const double wj = exp(sc[j] - mx) / den;
+        for (int d = 0; d < D; ++d) {
+            const double vd = e4m3_to_double(vc[(size_t)j * D + d]) * (double)vs[d];
+            out[d] += wj * vd;
+        }
+    }
+    *lse_out = mx + log(den);
+}
+
+/*
+ * q: [B, Hq, Sq, D] bf16 bits; k8/v8: [B, Hkv, Skv, D] e4m3 codes; k_scale/v_scale: [Hkv, D] fp32.
+ * rows, o, lse, n_threads: as oracle_attn.
+ */
+int oracle_attn_fp8kv(const uint16_t *q, const uint8_t *k8, const uint8_t *v8, const float *k_scale,
+                      const float *v_scale, double *o, double *lse,
+                      int B, int Hq, int Hkv, int Sq, int Skv, int D,
+                      float scale, int causal,
+                      const int64_t *rows, int64_t n_rows, int n_threads)
+{
+    if (!q || !k8 || !v8 || !k_scale || !v_scale || !o || !lse)
+        return ORACLE_ERR_ARGS;
+    if (B < 1 || Hq < 1 || Hkv < 1 || Sq < 1 || Skv < 1 || D < 1 || Hq % Hkv != 0)
+        return ORACLE_ERR_ARGS;
+    if (causal && Sq > Skv)
+        return ORACLE_ERR_ARGS;
+    const int64_t n_all = (int64_t)B * Hq * Sq;
+    if (rows == NULL)
+        n_rows = n_all;
+    if (n_rows < 0)
+        return ORACLE_ERR_ARGS;
+    for (int64_t r = 0; rows && r < n_rows; ++r)
+        if (rows[r] < 0 || rows[r] >= n_all)
+            return ORACLE_ERR_ARGS;
+    int failed = 0;
+
+#pragma omp parallel num_threads(n_threads > 0 ? n_threads : omp_get_max_threads())
+    {
+        double *sc = (double *)malloc(sizeof(double) * (size_t)Skv);
+        if (!sc) {
+#pragma omp atomic write
+            failed = 1;
+        }
+#pragma omp for schedule(dynamic, 8)
+        for (int64_t r = 0; r < n_rows; ++r) {
+            if (!sc)
+                continue;
+            const int64_t row = rows ? rows[r] : r;
+            const int64_t bh = row / Sq;
+            const int i = (int)(row - bh * Sq);
+            const int b = (int)(bh / Hq);
+            const int h = (int)(bh - (int64_t)b * Hq);
+            const int g = h / (Hq / Hkv); /* kv head of query head h */
+            const int n_vis = causal ? i + (Skv - Sq) + 1 : Skv;
+            const size_t cache = ((size_t)b * Hkv + g) * (size_t)Skv * D;
+            fp8kv_row(q + (size_t)row * D, k8 + cache, v8 + cache, k_scale + (size_t)g * D,
+                      v_scale + (size_t)g * D, D, n_vis, (double)scale, sc, o + (size_t)r * D, lse + r);
+        }
+        free(sc);
+    }
+    return failed ? ORACLE_ERR_NOMEM : ORACLE_OK;
+}
