@@ -264,6 +264,33 @@ def run_ours(args):
         e2e_ms = t.item()
         torch.distributed.barrier()
     e2e_tflops = world * e2e_steps * PREFILL.flops() / (e2e_ms * 1e-3) / 1e12
+
+    # The same decode over an e4m3 cache (per-channel coefficients), timed on its own: inputs
+    # resident, L2 flushed before every launch, CUDA events around each launch.
+    fq, fk8, fv8, fks, fvs = (t.to(dev) for t in inputs.generate_fp8(DECODE))
+    fo = torch.empty_like(fq)
+    fl = torch.empty(fq.shape[:3], dtype=torch.float32, device=dev)
+    fp8_bytes = fp8_decode_bytes(DECODE)
+    for _ in range(args.warmup):
+        clear_l2()
+        attn.attn_decode_fp8(fq, fk8, fv8, fks, fvs, scale=DECODE.scale, out=fo, lse=fl, stream=stream)
+    fp8_steps = max(3, min(args.steps, 500))
+    fev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(fp8_steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    for s in range(fp8_steps):
+        clear_l2()
+        fev[s][0].record(stream)
+        attn.attn_decode_fp8(fq, fk8, fv8, fks, fvs, scale=DECODE.scale, out=fo, lse=fl, stream=stream)
+        fev[s][1].record(stream)
+    torch.cuda.synchronize(dev)
+    fp8_ms = sum(a.elapsed_time(b) for a, b in fev)
+    if world > 1:
+        t = torch.tensor([fp8_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        fp8_ms = t.item()
+    fp8_launch_s = fp8_ms * 1e-3 / fp8_steps
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
     d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
 
@@ -289,6 +316,17 @@ def run_ours(args):
                 "us_per_launch": dec_launch_s * 1e6,
                 "ctas": attn.decode_ctas(DECODE.B, DECODE.Hq, DECODE.Hkv, DECODE.Skv, DECODE.D),
             },
+            "decode_fp8": {
+                "metric": "decode KV-read GB/s, e4m3 K/V cache", "value": world * fp8_bytes / fp8_launch_s / 1e9,
+                "unit": "GB/s", "config": dict(DECODE.config(), kv_dtype="e4m3", scales="fp32 per (kv head, channel)"),
+                "steps": fp8_steps,
+                "roofline": {"bound": "hbm", "achieved": fp8_bytes / fp8_launch_s / 1e9, "peak": hbm_peak,
+                             "unit": "GB/s", "frac": fp8_bytes / fp8_launch_s / 1e9 / hbm_peak,
+                             "traffic": read_traffic("decode_tc_kernel_fp8", DECODE.name),
+                             "peak_kind": f"{peak_kind} HBM copy", "kernel": "decode_tc_kernel<4, e4m3>"},
+                "us_per_launch": fp8_launch_s * 1e6,
+                "bytes_per_launch": fp8_bytes,
+            },
             "prefill_us_per_launch": pre_launch_s * 1e6,
             "timed_region_ms": region_ms,
             "e2e": {"value": e2e_tflops, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -310,6 +348,7 @@ def run_ours(args):
 KERNEL_SOURCES = {
     "prefill_kernel": ["prefill_sm100.cu", "sm100_ptx.cuh"],
     "decode_tc_kernel": ["decode_tc_sm100.cu", "sm100_ptx.cuh"],
+    "decode_tc_kernel_fp8": ["decode_tc_sm100.cu", "sm100_ptx.cuh"],
 }
 
 
@@ -345,11 +384,33 @@ def read_traffic(kernel: str, workload: str):
         return None
 
 
+def fp8_decode_bytes(w) -> int:
+    """Bytes the e4m3 decode must move once: K and V codes, q, o, lse and both coefficient tables."""
+    kv = 2 * w.B * w.Hkv * w.Skv * w.D
+    return kv + 2 * w.B * w.Hq * w.D * 2 + w.B * w.Hq * 4 + 2 * w.Hkv * w.D * 4
+
+
 def run_case(args):
     """Run one named workload `--repeat` times through attn_fwd (no L2 flush, no JSON line): the
     command the committed ncu summaries were captured with."""
     from causal_attention_attn_b200 import attn
 
+    if args.case == "decode_fp8":
+        w = inputs.DECODE_GQA
+        q, k8, v8, ks, vs = (t.cuda() for t in inputs.generate_fp8(w))
+        o = torch.empty_like(q)
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        ev[0].record()
+        for _ in range(args.repeat):
+            attn.attn_decode_fp8(q, k8, v8, ks, vs, scale=w.scale, out=o, lse=lse)
+        ev[1].record()
+        torch.cuda.synchronize()
+        ms = ev[0].elapsed_time(ev[1]) / args.repeat
+        print(json.dumps({"case": w.name + "_e4m3", "repeat": args.repeat, "us_per_launch": ms * 1e3,
+                          "io_gbs": fp8_decode_bytes(w) / (ms * 1e-3) / 1e9,
+                          "device_status": attn.device_status()}), flush=True)
+        return 0
     w = inputs.SHORT_NAMES[args.case]
     q, k, v = (t.cuda() for t in inputs.generate(w))
     o = torch.empty_like(q)
@@ -373,7 +434,7 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--case", choices=sorted(inputs.SHORT_NAMES), default=None,
+    ap.add_argument("--case", choices=sorted(inputs.SHORT_NAMES) + ["decode_fp8"], default=None,
                     help="only run this workload --repeat times (for profiling); prints no bench line")
     ap.add_argument("--repeat", type=int, default=3)
     args = ap.parse_args()

@@ -25,7 +25,8 @@ STATUS_NAMES = {
     -13: "ATTN_ERR_SCRATCH_LIMIT",
 }
 EXPORTED = ("attn_fwd", "attn_fwd_ex", "attn_decode_ctas", "attn_status_string", "attn_version",
-            "attn_device_status", "attn_decode_noalloc", "attn_decode_paged", "attn_bwd")
+            "attn_device_status", "attn_decode_noalloc", "attn_decode_paged", "attn_bwd", "attn_decode_fp8",
+            "attn_decode_paged_fp8")
 
 _lock = threading.Lock()
 _lib = None
@@ -67,6 +68,8 @@ def load_library(path: str | None = None):
         lib.attn_bwd.restype = i
         lib.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp]
         lib.attn_decode_paged.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, vp]
+        lib.attn_decode_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
+        lib.attn_decode_paged_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, vp]
         if path is None:
             _lib = lib
         return lib
@@ -238,6 +241,78 @@ def attn_decode_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Ten
                                               lse.data_ptr(), B, Hq, Hkv, num_pages, page_size,
                                               int(block_table.shape[1]), int(max_seq_len), float(scale),
                                               int(decode_ctas), _stream_handle(stream))
+    _check(rc)
+    return out, lse
+
+
+def _as_codes(name, t):
+    """e4m3 codes: a uint8 tensor, or a float8_e4m3fn tensor viewed as its bytes."""
+    if isinstance(t, torch.Tensor) and t.dtype == torch.float8_e4m3fn:
+        t = t.view(torch.uint8)
+    _check_tensor(name, t, torch.uint8, 4)
+    return t
+
+
+def attn_decode_fp8(q: torch.Tensor, k8: torch.Tensor, v8: torch.Tensor, k_scale: torch.Tensor,
+                    v_scale: torch.Tensor, scale: float | None = None, out: torch.Tensor | None = None,
+                    lse: torch.Tensor | None = None, stream=None, decode_ctas: int = 0):
+    """Single-token decode over an e4m3 K/V cache through ``attn_decode_fp8``.
+    q: [B, Hq, 1, 128] bf16; k8, v8: [B, Hkv, Skv, 128] e4m3 codes (uint8 or float8_e4m3fn);
+    k_scale, v_scale: fp32 [Hkv, 128] (value = code * coefficient). Returns (o, lse)."""
+    _check_tensor("q", q, torch.bfloat16, 4)
+    k8, v8 = _as_codes("k8", k8), _as_codes("v8", v8)
+    _check_tensor("k_scale", k_scale, torch.float32, 2)
+    _check_tensor("v_scale", v_scale, torch.float32, 2)
+    B, Hq, Sq, D = q.shape
+    Bk, Hkv, Skv, Dk = k8.shape
+    if Sq != 1 or tuple(v8.shape) != tuple(k8.shape) or Bk != B or Dk != D \
+            or tuple(k_scale.shape) != (Hkv, D) or tuple(v_scale.shape) != (Hkv, D):
+        raise ValueError("expected q [B,Hq,1,D], k8, v8 [B,Hkv,Skv,D] and scales [Hkv,D]")
+    if scale is None:
+        scale = D ** -0.5
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, Hq, 1), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check_tensor("out", out, torch.bfloat16, 4)
+    _check_tensor("lse", lse, torch.float32, 3)
+    with torch.cuda.device(q.device):
+        rc = load_library().attn_decode_fp8(q.data_ptr(), k8.data_ptr(), v8.data_ptr(), k_scale.data_ptr(),
+                                            v_scale.data_ptr(), out.data_ptr(), lse.data_ptr(), B, Hq, Hkv, Skv, D,
+                                            float(scale), int(decode_ctas), _stream_handle(stream))
+    _check(rc)
+    return out, lse
+
+
+def attn_decode_paged_fp8(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor, k_scale: torch.Tensor,
+                          v_scale: torch.Tensor, block_table: torch.Tensor, seq_lens: torch.Tensor, max_seq_len: int,
+                          scale: float | None = None, out: torch.Tensor | None = None,
+                          lse: torch.Tensor | None = None, stream=None, decode_ctas: int = 0):
+    """attn_decode_paged over e4m3 pages: k_pages, v_pages [num_pages, Hkv, page_size, 128] e4m3
+    codes; k_scale, v_scale fp32 [Hkv, 128]; the rest as :func:`attn_decode_paged`."""
+    _check_tensor("q", q, torch.bfloat16, 4)
+    k_pages, v_pages = _as_codes("k_pages", k_pages), _as_codes("v_pages", v_pages)
+    _check_tensor("k_scale", k_scale, torch.float32, 2)
+    _check_tensor("v_scale", v_scale, torch.float32, 2)
+    _check_tensor("block_table", block_table, torch.int32, 2)
+    _check_tensor("seq_lens", seq_lens, torch.int32, 1)
+    B, Hq, Sq, D = q.shape
+    num_pages, Hkv, page_size, Dk = k_pages.shape
+    if Sq != 1 or tuple(v_pages.shape) != tuple(k_pages.shape) or Dk != D \
+            or tuple(k_scale.shape) != (Hkv, D) or tuple(v_scale.shape) != (Hkv, D):
+        raise ValueError("expected q [B,Hq,1,D], pages [P,Hkv,page,D] and scales [Hkv,D]")
+    if block_table.shape[0] != B or seq_lens.shape[0] != B:
+        raise ValueError("block_table and seq_lens need one row / entry per batch element")
+    if scale is None:
+        scale = D ** -0.5
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, Hq, 1), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check_tensor("out", out, torch.bfloat16, 4)
+    _check_tensor("lse", lse, torch.float32, 3)
+    with torch.cuda.device(q.device):
+        rc = load_library().attn_decode_paged_fp8(q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(),
+                                                  k_scale.data_ptr(), v_scale.data_ptr(), block_table.data_ptr(),
+                                                  seq_lens.data_ptr(), out.data_ptr(), lse.data_ptr(), B, Hq, Hkv,
+                                                  num_pages, page_size, int(block_table.shape[1]), int(max_seq_len),
+                                                  float(scale), int(decode_ctas), _stream_handle(stream))
     _check(rc)
     return out, lse
 

@@ -16,7 +16,7 @@
 namespace attn_b200 {
 namespace {
 
-constexpr int kVersion = 200;  // 0.2.0: adds attn_decode_paged
+constexpr int kVersion = 300;  // 0.3.0: adds attn_bwd, attn_decode_fp8, attn_decode_paged_fp8
 constexpr int kMaxDevices = 64;
 
 struct DeviceState {
@@ -316,13 +316,16 @@ extern "C" int attn_device_status(void *stream_ptr)
     return ATTN_OK;
 }
 
-extern "C" int attn_decode_paged(const void *q, const void *k_pages, const void *v_pages, const int *block_table,
-                                 const int *seq_lens, void *o, float *lse, int B, int Hq, int Hkv, int num_pages,
-                                 int page_size, int pages_per_seq, int max_seq_len, float scale, int decode_ctas,
-                                 void *stream_ptr)
+namespace {
+
+// Shared by attn_decode_paged and attn_decode_paged_fp8 (k_scale, v_scale non-null for the latter).
+int decode_paged_impl(const void *q, const void *k_pages, const void *v_pages, const float *k_scale,
+                      const float *v_scale, const int *block_table, const int *seq_lens, void *o, float *lse, int B,
+                      int Hq, int Hkv, int num_pages, int page_size, int pages_per_seq, int max_seq_len, float scale,
+                      int decode_ctas, void *stream_ptr, bool fp8)
 {
     using namespace attn_b200;
-    if (!q || !k_pages || !v_pages || !block_table || !seq_lens || !o || !lse)
+    if (!q || !k_pages || !v_pages || !block_table || !seq_lens || !o || !lse || (fp8 && (!k_scale || !v_scale)))
         return ATTN_ERR_NULL;
     if (B < 1 || B > kPagedMaxBatch || Hq < 1 || Hkv < 1 || num_pages < 1 || pages_per_seq < 1 || max_seq_len < 0 ||
         decode_ctas < 0)
@@ -338,7 +341,8 @@ extern "C" int attn_decode_paged(const void *q, const void *k_pages, const void 
         static_cast<long long>(pages_per_seq) * page_size > INT_MAX || static_cast<long long>(B) * Hq > INT_MAX)
         return ATTN_ERR_SHAPE;
     if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(o) || !aligned16(lse) ||
-        (reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
+        (reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u) ||
+        (fp8 && (!aligned16(k_scale) || !aligned16(v_scale))))
         return ATTN_ERR_ALIGN;
     if (!(scale > 0.f) || !std::isfinite(scale))
         return ATTN_ERR_SCALE;
@@ -378,6 +382,91 @@ extern "C" int attn_decode_paged(const void *q, const void *k_pages, const void 
     a.page_size = page_size;
     a.pages_per_seq = pages_per_seq;
     a.max_seq_len = max_seq_len;
+    a.fp8 = fp8;
+    a.k_scale = k_scale;
+    a.v_scale = v_scale;
+    if (launch_decode_tc(a, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_LAUNCH;
+    }
+    return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" int attn_decode_paged(const void *q, const void *k_pages, const void *v_pages, const int *block_table,
+                                 const int *seq_lens, void *o, float *lse, int B, int Hq, int Hkv, int num_pages,
+                                 int page_size, int pages_per_seq, int max_seq_len, float scale, int decode_ctas,
+                                 void *stream_ptr)
+{
+    return decode_paged_impl(q, k_pages, v_pages, nullptr, nullptr, block_table, seq_lens, o, lse, B, Hq, Hkv,
+                             num_pages, page_size, pages_per_seq, max_seq_len, scale, decode_ctas, stream_ptr, false);
+}
+
+extern "C" int attn_decode_paged_fp8(const void *q, const void *k_pages, const void *v_pages, const float *k_scale,
+                                     const float *v_scale, const int *block_table, const int *seq_lens, void *o,
+                                     float *lse, int B, int Hq, int Hkv, int num_pages, int page_size,
+                                     int pages_per_seq, int max_seq_len, float scale, int decode_ctas,
+                                     void *stream_ptr)
+{
+    return decode_paged_impl(q, k_pages, v_pages, k_scale, v_scale, block_table, seq_lens, o, lse, B, Hq, Hkv,
+                             num_pages, page_size, pages_per_seq, max_seq_len, scale, decode_ctas, stream_ptr, true);
+}
+
+extern "C" int attn_decode_fp8(const void *q, const void *k8, const void *v8, const float *k_scale,
+                               const float *v_scale, void *o, float *lse, int B, int Hq, int Hkv, int Skv, int D,
+                               float scale, int decode_ctas, void *stream_ptr)
+{
+    using namespace attn_b200;
+    if (!q || !k8 || !v8 || !k_scale || !v_scale || !o || !lse)
+        return ATTN_ERR_NULL;
+    if (B < 1 || Hq < 1 || Hkv < 1 || Skv < 1 || decode_ctas < 0)
+        return ATTN_ERR_SHAPE;
+    if (Hq % Hkv != 0)
+        return ATTN_ERR_GQA;
+    if (D != 128)
+        return ATTN_ERR_HEADDIM;
+    // Tensor-map coordinates (rows of a kv head, b * Hkv + h) and output rows must fit in 32 bits.
+    if (static_cast<long long>(B) * Hkv > INT_MAX || static_cast<long long>(B) * Hq > INT_MAX)
+        return ATTN_ERR_SHAPE;
+    if (!aligned16(q) || !aligned16(k8) || !aligned16(v8) || !aligned16(k_scale) || !aligned16(v_scale) ||
+        !aligned16(o) || !aligned16(lse))
+        return ATTN_ERR_ALIGN;
+    if (!(scale > 0.f) || !std::isfinite(scale))
+        return ATTN_ERR_SCALE;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+    std::lock_guard<std::mutex> lock(g_mutex);
+    int err = ATTN_OK;
+    DeviceState *s = device_state(&err);
+    if (!s)
+        return err;
+    DecodePlan plan;
+    if (decode_plan(B, Hq, Hkv, Skv, D, decode_ctas, s->sm_count, &plan) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_SHAPE;
+    }
+    int rc = ensure_workspace(*s, static_cast<size_t>(plan.pairs), plan.partial_floats, stream);
+    if (rc != ATTN_OK)
+        return rc;
+    DecodeArgs a;
+    a.q = q;
+    a.k = k8;
+    a.v = v8;
+    a.o = o;
+    a.lse = lse;
+    a.B = B;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.Skv = Skv;
+    a.D = D;
+    a.scale = scale;
+    a.plan = plan;
+    a.ws = s->partials;
+    a.counters = s->counters;
+    a.status = s->status;
+    a.fp8 = true;
+    a.k_scale = k_scale;
+    a.v_scale = v_scale;
     if (launch_decode_tc(a, stream) != cudaSuccess) {
         cudaGetLastError();
         return ATTN_ERR_LAUNCH;

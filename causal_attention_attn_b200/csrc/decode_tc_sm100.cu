@@ -39,6 +39,8 @@
  */
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -53,7 +55,6 @@ namespace {
 constexpr int kD = 128;         // head dim (the only one this kernel serves)
 constexpr int kCK = 128;        // keys per chunk = M of S^T = K of O^T
 constexpr int kN = 16;          // MMA N: query heads of one pair, padded
-constexpr int kStages = 3;      // K/V chunks in flight
 constexpr int kWarpTma = 4;
 constexpr int kWarpMma = 5;
 constexpr int kSoftmaxThreads = 128;
@@ -61,39 +62,58 @@ constexpr int kThreads = 192;
 constexpr int kBarSoftmax = 1;  // named barrier of the softmax warps
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
-constexpr float kRescaleThreshold = 8.0f;
 
-constexpr int kHalfBytes = kCK * 128;          // 128 rows x 64 dims: one swizzled half of a K or V chunk
-constexpr int kTileBytes = 2 * kHalfBytes;     // one K or V chunk
-constexpr int kStageBytes = 2 * kTileBytes;    // K chunk, then V chunk
-constexpr int kSmallHalf = kN * 128;           // 16 rows x 128 bytes: half of Q^T or of P^T
-constexpr int kSmallBytes = 2 * kSmallHalf;
-constexpr int kOffRing = 0;
-constexpr int kOffQ = kOffRing + kStages * kStageBytes;  // two Q^T slots (one per segment parity)
-constexpr int kOffP = kOffQ + 2 * kSmallBytes;           // two P^T buffers (one per chunk parity)
-constexpr int kOffRedMax = kOffP + 2 * kSmallBytes;      // [chunk parity][warp][head] chunk maxima
-constexpr int kOffRedSum = kOffRedMax + 2 * 4 * kN * 4;  // [warp][head][2] running sums
-constexpr int kOffBar = kOffRedSum + 4 * kN * 2 * 4;
+constexpr int kHalfBytes = kCK * 128;  // 128 rows x 128 bytes: one swizzled box column of a K or V chunk
+constexpr int kSmallHalf = kN * 128;   // 16 rows x 128 bytes: half of a bf16 Q^T or P^T, or one e4m3 part
+constexpr int kMaxStages = 5;
 enum TcBar : int {
-    kBarFull0 = 0,                      // [stage] K/V chunk landed
-    kBarEmpty0 = kBarFull0 + kStages,   // [stage] chunk consumed by both MMAs
-    kBarQFull0 = kBarEmpty0 + kStages,  // [segment parity] Q^T landed
-    kBarQEmpty0 = kBarQFull0 + 2,       // [segment parity] last S^T of the segment done
-    kBarSFull0 = kBarQEmpty0 + 2,       // [chunk parity] S^T ready
-    kBarPFull0 = kBarSFull0 + 2,        // [chunk parity] P^T written (128 arrivals)
-    kBarODone0 = kBarPFull0 + 2,        // [chunk parity] O^T += V^T P^T done
-    kBarOFree = kBarODone0 + 2,         // segment's O^T read out (128 arrivals)
+    kBarFull0 = 0,                         // [stage] K/V chunk landed
+    kBarEmpty0 = kBarFull0 + kMaxStages,   // [stage] chunk consumed by both MMAs
+    kBarQFull0 = kBarEmpty0 + kMaxStages,  // [segment parity] Q^T in place
+    kBarQEmpty0 = kBarQFull0 + 2,          // [segment parity] last S^T of the segment done
+    kBarSFull0 = kBarQEmpty0 + 2,          // [chunk parity] S^T ready
+    kBarPFull0 = kBarSFull0 + 2,           // [chunk parity] P^T written (128 arrivals)
+    kBarODone0 = kBarPFull0 + 2,           // [chunk parity] O^T += V^T P^T done
+    kBarOFree = kBarODone0 + 2,            // segment's O^T read out (128 arrivals)
     kBarDrain = kBarOFree + 1,
-    kNumTcBars = kBarDrain + 1,
+    kBarQScFree0 = kBarDrain + 1,          // [segment parity] e4m3 cache: the score scales read (128 arrivals)
+    kNumTcBars = kBarQScFree0 + 2,
 };
-constexpr int kOffMisc = kOffBar + kNumTcBars * 8;  // tmem slot, abort flag, merge bookkeeping
-// Paged decode only: first unit of each batch entry (and the total), then the clamped lengths.
-constexpr int kOffBatchStart = kOffMisc + 64;
-constexpr int kOffBatchLen = kOffBatchStart + 8 * (kPagedMaxBatch + 1);
-constexpr int kUsed = kOffBatchLen + 4 * kPagedMaxBatch;
-constexpr int kSmem = kUsed + 1024;  // + alignment of the base to the 1024-byte swizzle repeat
-static_assert(kSmem <= 227 * 1024, "shared memory budget");
-static_assert(kOffQ % 1024 == 0 && kOffP % 1024 == 0, "swizzled tiles sit on 1024-byte boundaries");
+
+// Shared-memory layout of one variant. bf16 cache: K and V chunks of 32 KB (two 64-dim box
+// columns each), three in flight, Q^T and P^T in bf16. e4m3 cache: chunks of 16 KB (one 128-byte
+// box column), five in flight, Q^T and P^T each as three e4m3 parts (hi, mid, lo) of 16 x 128 bytes.
+template <bool kFp8>
+struct Lay {
+    static constexpr int kStages = kFp8 ? 5 : 3;
+    static constexpr int kBoxCols = kFp8 ? 1 : 2;          // 128-byte box columns per K or V row
+    static constexpr int kTileBytes = kBoxCols * kHalfBytes;  // one K or V chunk
+    static constexpr int kStageBytes = 2 * kTileBytes;        // K chunk, then V chunk
+    static constexpr int kSmallBytes = kFp8 ? 3 * kSmallHalf : 2 * kSmallHalf;  // one Q^T slot or P^T buffer
+    static constexpr int kOffRing = 0;
+    static constexpr int kOffQ = kOffRing + kStages * kStageBytes;  // two Q^T slots (one per segment parity)
+    static constexpr int kOffP = kOffQ + 2 * kSmallBytes;           // two P^T buffers (one per chunk parity)
+    static constexpr int kOffQScale = kOffP + 2 * kSmallBytes;      // [segment parity][head] score scales
+    static constexpr int kOffRedMax = kOffQScale + 2 * kN * 4;      // [chunk parity][warp][head] chunk maxima
+    static constexpr int kOffRedSum = kOffRedMax + 2 * 4 * kN * 4;  // [warp][head][2] running sums
+    static constexpr int kOffBar = kOffRedSum + 4 * kN * 2 * 4;
+    static constexpr int kOffMisc = kOffBar + kNumTcBars * 8;  // tmem slot, abort flag, merge bookkeeping
+    // Paged decode only: first unit of each batch entry (and the total), then the clamped lengths.
+    static constexpr int kOffBatchStart = kOffMisc + 64;
+    static constexpr int kOffBatchLen = kOffBatchStart + 8 * (kPagedMaxBatch + 1);
+    static constexpr int kUsed = kOffBatchLen + 4 * kPagedMaxBatch;
+    static constexpr int kSmem = kUsed + 1024;  // + alignment of the base to the 1024-byte swizzle repeat
+    static_assert(kSmem <= 227 * 1024, "shared memory budget");
+    static_assert(kOffQ % 1024 == 0 && kOffP % 1024 == 0 && kSmallBytes % 1024 == 0,
+                  "swizzled tiles sit on 1024-byte boundaries");
+    static_assert(kStages <= kMaxStages, "barrier arrays");
+    // The reference max moves when a chunk's max exceeds it by more than this (log2 units). With the
+    // e4m3 cache the weights are scaled by 16 before they are split, and 16 * 2^4 = 256 stays below
+    // the e4m3 maximum of 448.
+    static constexpr float kRescaleThreshold = kFp8 ? 4.0f : 8.0f;
+    static constexpr float kPScale = kFp8 ? 16.0f : 1.0f;
+};
+static_assert(Lay<false>::kStageBytes == 65536 && Lay<false>::kSmallBytes == 4096, "bf16 layout");
 constexpr uint32_t kTmemCols = 64;  // S^T [0,16) and [16,32), O^T [32,48)
 constexpr uint32_t kColO = 32;
 
@@ -108,6 +128,9 @@ struct TcParams {
     // paged, variable-length cache
     const int *seq_lens, *block_table;
     int B, num_pages, page_size, pages_per_seq, max_seq_len;
+    // e4m3 cache: the bf16 queries, read by the producer, and the per-(kv head, channel) coefficients
+    const __nv_bfloat16 *q;
+    const float *k_scale, *v_scale;
 };
 
 __device__ __forceinline__ float ex2(float x)
@@ -115,6 +138,52 @@ __device__ __forceinline__ float ex2(float x)
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// ---- e4m3 cache: splitting a fp32 value into three e4m3 parts ---------------------------------
+// x ~ c1 + c2 + c3 with c_t = e4m3(x - c1 - ... - c_{t-1}) rounded to nearest even. Each
+// subtraction is exact (a value and its 3-bit rounding lie within a factor of two of each other),
+// so the parts carry x to about 12 significant bits wherever x, scaled as below, is above the
+// e4m3 subnormal range (2^-6).
+
+// Codes of (a, b), a in the low byte.
+__device__ __forceinline__ uint32_t e4m3x2(float a, float b)
+{
+    return __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+}
+
+__device__ __forceinline__ float2 e4m3x2_value(uint32_t codes)
+{
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(codes), __NV_E4M3);
+    return __half22float2(__half2(h));
+}
+
+// One split step over four values: their codes (value u in byte u), and x -= the codes' values.
+__device__ __forceinline__ uint32_t split_step4(float (&x)[4])
+{
+    const uint32_t lo = e4m3x2(x[0], x[1]), hi = e4m3x2(x[2], x[3]);
+    const float2 vl = e4m3x2_value(lo), vh = e4m3x2_value(hi);
+    x[0] -= vl.x;
+    x[1] -= vl.y;
+    x[2] -= vh.x;
+    x[3] -= vh.y;
+    return lo | (hi << 16);
+}
+
+// 2^e for |e| <= 126.
+__device__ __forceinline__ float exp2_int(int e) { return __uint_as_float(static_cast<uint32_t>(e + 127) << 23); }
+
+// The power of two e that brings mx (the largest magnitude of one query head's q * k_scale) into
+// (224, 448], the top of the e4m3 range: 0 for a zero head, clamped to [-100, 100].
+__device__ __forceinline__ int q_exponent(float mx)
+{
+    if (!(mx > 0.f))
+        return 0;
+    const uint32_t bits = __float_as_uint(mx);
+    const int E = static_cast<int>((bits >> 23) & 255u) - 127;
+    const float mant = __uint_as_float((bits & 0x007fffffu) | 0x3f800000u);  // in [1, 2)
+    const int e = (mant <= 1.75f ? 8 : 7) - E;
+    return min(max(e, -100), 100);
 }
 
 __device__ __forceinline__ long long range_start(long long c, long long total, int ctas) { return c * total / ctas; }
@@ -145,12 +214,17 @@ struct UnitPos {
     int local, cpp;
 };
 
-template <int G, bool kPaged>
+template <int G, bool kPaged, bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const TcParams p)
 {
     static_assert(G >= 1 && G <= kN, "one pair's heads fit the MMA's N");
+    using L = Lay<kFp8>;
+    constexpr int kStages = L::kStages, kStageBytes = L::kStageBytes, kTileBytes = L::kTileBytes;
+    constexpr int kSmallBytes = L::kSmallBytes, kOffRing = L::kOffRing, kOffQ = L::kOffQ, kOffP = L::kOffP;
+    constexpr int kOffRedMax = L::kOffRedMax, kOffRedSum = L::kOffRedSum, kOffBar = L::kOffBar;
+    constexpr int kOffMisc = L::kOffMisc, kOffBatchStart = L::kOffBatchStart, kOffBatchLen = L::kOffBatchLen;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t s_base = smem_u32(smem);
@@ -160,6 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t bar0 = s_base + kOffBar;
 #define BAR(i) (bar0 + 8u * static_cast<uint32_t>(i))
     float *red_max = reinterpret_cast<float *>(smem + kOffRedMax);
+    float *q_scale = reinterpret_cast<float *>(smem + L::kOffQScale);  // [segment parity][kN], e4m3 cache
     float *red_sum = reinterpret_cast<float *>(smem + kOffRedSum);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffMisc + 4);
@@ -181,7 +256,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(BAR(kBarEmpty0 + s), 1);
         }
         for (int x = 0; x < 2; ++x) {
-            mbar_init(BAR(kBarQFull0 + x), 1);
+            mbar_init(BAR(kBarQFull0 + x), kFp8 ? 32 : 1);  // e4m3: every producer lane writes Q^T
+            mbar_init(BAR(kBarQScFree0 + x), kSoftmaxThreads);
             mbar_init(BAR(kBarQEmpty0 + x), 1);
             mbar_init(BAR(kBarSFull0 + x), 1);
             mbar_init(BAR(kBarPFull0 + x), kSoftmaxThreads);
@@ -192,9 +268,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         *abort_flag = 0;
         fence_mbar_init();
     }
-    // P^T rows G..15 are never written by the softmax: keep them zero.
-    for (int i = threadIdx.x; i < 2 * kSmallBytes / 16; i += kThreads)
-        reinterpret_cast<uint4 *>(smem + kOffP)[i] = make_uint4(0u, 0u, 0u, 0u);
+    // P^T rows G..15 are never written by the softmax, nor (e4m3 cache) Q^T rows G..15 by the
+    // producer: keep them zero. Q^T and P^T are adjacent.
+    {
+        constexpr int kZeroFrom = kFp8 ? kOffQ : kOffP;
+        for (int i = threadIdx.x; i < (kOffP + 2 * kSmallBytes - kZeroFrom) / 16; i += kThreads)
+            reinterpret_cast<uint4 *>(smem + kZeroFrom)[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
     fence_proxy_async_smem();
     if (warp == kWarpTma && lane == 0) {
         tma_prefetch_desc(&tm_q);
@@ -291,17 +371,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         int bk = 0;
         int tab_row = -1, tab_base = 0, tab_val = 0;  // this lane holds entry tab_base + lane of row tab_row
         for (long long g = g_begin; g < g_end; ++g) {
-            if (g == g_begin || local == 0) {
+            const bool new_seg = (g == g_begin || local == 0);
+            const int qs = seg & 1;
+            uint2 qraw[kFp8 ? G : 1];  // e4m3 cache: this lane's dims 4*lane .. 4*lane+3 of each head
+            float4 ksv = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (new_seg) {
                 // A new segment: Q^T of its pair (G heads, padded to 16 rows) into the segment's slot.
-                const int qs = seg & 1;
-                if (!__all_sync(0xffffffffu, mbar_wait(BAR(kBarQEmpty0 + qs), (static_cast<uint32_t>(seg >> 1) & 1u) ^ 1u,
-                                                       abort_flag, p.status, kSiteDecodeProducer)))
+                const uint32_t free_parity = (static_cast<uint32_t>(seg >> 1) & 1u) ^ 1u;
+                if (!__all_sync(0xffffffffu, mbar_wait(BAR(kBarQEmpty0 + qs), free_parity, abort_flag, p.status,
+                                                       kSiteDecodeProducer)))
+                    break;
+                // e4m3 cache: the softmax warps also have read the slot's score scales.
+                if (kFp8 && !__all_sync(0xffffffffu, mbar_wait(BAR(kBarQScFree0 + qs), free_parity, abort_flag,
+                                                               p.status, kSiteDecodeProducer)))
                     break;
                 const int hg = static_cast<int>(pair % p.head_groups);
                 bk = static_cast<int>(pair / p.head_groups);  // b * Hkv + kv head
                 const int b = bk / p.Hkv;
                 const int h0 = (bk % p.Hkv) * p.group + hg * G;
-                if (issuer) {
+                if constexpr (kFp8) {
+                    // Loads only; Q^T is built once this chunk's copies are on their way.
+                    const __nv_bfloat16 *qrow = p.q + (static_cast<size_t>(b) * p.Hq + h0) * kD;
+#pragma unroll
+                    for (int h = 0; h < (kFp8 ? G : 1); ++h)
+                        qraw[h] = reinterpret_cast<const uint2 *>(qrow + static_cast<size_t>(h) * kD)[lane];
+                    ksv = reinterpret_cast<const float4 *>(p.k_scale + static_cast<size_t>(bk % p.Hkv) * kD)[lane];
+                } else if (issuer) {
                     mbar_arrive_expect_tx(BAR(kBarQFull0 + qs), kSmallBytes);
                     for (int hf = 0; hf < 2; ++hf)
                         tma_load_3d(sQ + qs * kSmallBytes + hf * kSmallHalf, &tm_q, BAR(kBarQFull0 + qs), hf * 64,
@@ -342,7 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         page = p.num_pages;
                     const int coord = static_cast<int>(static_cast<long long>(page) * p.Hkv + kvh);
                     const int in_page = key % p.page_size;
-                    for (int hf = 0; hf < 2; ++hf) {
+                    for (int hf = 0; hf < L::kBoxCols; ++hf) {
                         tma_load_3d(dst + hf * kHalfBytes + lane * rows * 128, &tm_k, BAR(kBarFull0 + slot), hf * 64,
                                     in_page, coord);
                         tma_load_3d(dst + kTileBytes + hf * kHalfBytes + lane * rows * 128, &tm_v, BAR(kBarFull0 + slot),
@@ -350,9 +445,45 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             } else if (issuer) {
-                for (int hf = 0; hf < 2; ++hf) {
+                for (int hf = 0; hf < L::kBoxCols; ++hf) {
                     tma_load_3d(dst + hf * kHalfBytes, &tm_k, BAR(kBarFull0 + slot), hf * 64, key0, bk);
                     tma_load_3d(dst + kTileBytes + hf * kHalfBytes, &tm_v, BAR(kBarFull0 + slot), hf * 64, key0, bk);
+                }
+            }
+            if constexpr (kFp8) {
+                if (new_seg) {
+                    // Q^T parts: per head, q * k_scale scaled by 2^e into the top of the e4m3 range,
+                    // then split into three e4m3 parts (rows h of three 16 x 128-byte K-major tiles
+                    // with the 128-byte swizzle: dims 4*lane..4*lane+3 sit in 16-byte unit
+                    // (lane / 4) XOR (h % 8), bytes 4*(lane % 4)..+3). The scores come out scaled by
+                    // 2^e; the softmax undoes that with the factor left in q_scale.
+                    uint8_t *qbase = smem + kOffQ + qs * kSmallBytes;
+                    const uint32_t unit = static_cast<uint32_t>(lane >> 2), sub = static_cast<uint32_t>(lane & 3) * 4u;
+                    auto lo = [](uint32_t w) { return __uint_as_float(w << 16); };
+                    auto hi = [](uint32_t w) { return __uint_as_float(w & 0xffff0000u); };
+#pragma unroll
+                    for (int h = 0; h < (kFp8 ? G : 1); ++h) {
+                        float x[4] = {lo(qraw[h].x) * ksv.x, hi(qraw[h].x) * ksv.y, lo(qraw[h].y) * ksv.z,
+                                      hi(qraw[h].y) * ksv.w};
+                        float mx = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1)
+                            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                        const int e = q_exponent(mx);
+                        const float f = exp2_int(e);
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            x[u] *= f;
+                        const uint32_t off = static_cast<uint32_t>((h >> 3) * 1024 + (h & 7) * 128) +
+                                             (((unit ^ static_cast<uint32_t>(h & 7)) << 4) | sub);
+#pragma unroll
+                        for (int t = 0; t < 3; ++t)
+                            *reinterpret_cast<uint32_t *>(qbase + t * kSmallHalf + off) = split_step4(x);
+                        if (lane == 0)
+                            q_scale[qs * kN + h] = p.scale_log2 * exp2_int(-e);
+                    }
+                    fence_proxy_async_smem();
+                    mbar_arrive(BAR(kBarQFull0 + qs));
                 }
             }
             ++issued;
@@ -367,13 +498,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             // Let every copy already issued land before the CTA exits.
             for (int c = (issued > kStages ? issued - kStages : 0); c < issued; ++c)
                 wait_drain(BAR(kBarFull0 + c % kStages), static_cast<uint32_t>(c / kStages) & 1u, 100000000ull);
-            for (int s = (seg > 2 ? seg - 2 : 0); s < seg; ++s)
+            for (int s = (seg > 2 ? seg - 2 : 0); !kFp8 && s < seg; ++s)  // e4m3 Q^T is not copied by TMA
                 wait_drain(BAR(kBarQFull0 + (s & 1)), static_cast<uint32_t>(s >> 1) & 1u, 100000000ull);
         }
     } else if (warp == kWarpMma) {
         // ---------------------------------------------------------------- MMA issuer
-        constexpr uint32_t kIdS = idesc_bf16_f32_ab(kCK, kN, false, false);  // A = K chunk, B = Q^T
-        constexpr uint32_t kIdO = idesc_bf16_f32_ab(kD, kN, true, false);    // A = V chunk read MN-major, B = P^T
+        // A = K chunk, B = Q^T; then A = V chunk read MN-major, B = P^T. e4m3 cache: both operands e4m3.
+        constexpr uint32_t kIdS = kFp8 ? idesc_e4m3_f32_ab(kCK, kN, false, false) : idesc_bf16_f32_ab(kCK, kN, false, false);
+        constexpr uint32_t kIdO = kFp8 ? idesc_e4m3_f32_ab(kD, kN, true, false) : idesc_bf16_f32_ab(kD, kN, true, false);
         const bool leader = elect_one();
         // A K step moves the start address, the low field of a descriptor (address >> 4): every
         // address here is below 2^18, so the field never overflows.
@@ -388,6 +520,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         auto issue_s = [&](int c, int qs) {
             const uint64_t dk = desc_k0 + static_cast<uint64_t>((c % kStages) * (kStageBytes >> 4));
             const uint64_t dq = desc_q0 + static_cast<uint64_t>(qs * (kSmallBytes >> 4));
+            if constexpr (kFp8) {
+                // S^T = K (Q^T_hi + Q^T_mid + Q^T_lo): per part four K steps of 32 dims (32 bytes).
+                if (leader) {
+#pragma unroll
+                    for (int t = 0; t < 3; ++t)
+#pragma unroll
+                        for (int kk = 0; kk < kD / 32; ++kk)
+                            tc_mma_f8_ss(tmem + 16u * static_cast<uint32_t>(c & 1), dk + static_cast<uint64_t>((kk * 32) >> 4),
+                                         dq + static_cast<uint64_t>((t * kSmallHalf + kk * 32) >> 4), kIdS,
+                                         (t > 0 || kk > 0) ? 1u : 0u);
+                }
+                return;
+            }
             if (leader) {
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk) {
@@ -400,6 +545,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         auto issue_o = [&](int c, bool accumulate) {
             const uint64_t dv = desc_v0 + static_cast<uint64_t>((c % kStages) * (kStageBytes >> 4));
             const uint64_t dp = desc_p0 + static_cast<uint64_t>((c & 1) * (kSmallBytes >> 4));
+            if constexpr (kFp8) {
+                // O^T += V^T (P^T_hi + P^T_mid + P^T_lo): per part four K steps of 32 keys (32 rows of
+                // 128 bytes of the MN-major V chunk; 32 bytes of a P^T row).
+                if (leader) {
+#pragma unroll
+                    for (int t = 0; t < 3; ++t)
+#pragma unroll
+                        for (int kk = 0; kk < kCK / 32; ++kk)
+                            tc_mma_f8_ss(tmem + kColO, dv + static_cast<uint64_t>((kk * 32 * 128) >> 4),
+                                         dp + static_cast<uint64_t>((t * kSmallHalf + kk * 32) >> 4), kIdO,
+                                         (accumulate || t > 0 || kk > 0) ? 1u : 0u);
+                }
+                return;
+            }
             if (leader) {
 #pragma unroll
                 for (int kk = 0; kk < kCK / 16; ++kk) {
@@ -490,7 +649,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         bool ok = true;
-        int c = 0, n_deferred = 0;
+        int c = 0, n_deferred = 0, sg = 0;
         for (long long g = g_begin; g < g_end;) {
             const UnitPos pos = locate(g);
             const long long pair = pos.pair;
@@ -503,6 +662,28 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int h0 = (bk % p.Hkv) * p.group + static_cast<int>(pair % p.head_groups) * G;
             const int seq_len = kPaged ? batch_len[b] : p.Skv;
 
+            // Factor from a score to log2 units, per head: the softmax scale times log2(e), and with
+            // the e4m3 cache also 2^-e for the power of two the producer folded into that head's
+            // Q^T parts (k_scale is folded into Q^T as well). v_coef: V's coefficient for dim i.
+            float sl2[G];
+            float v_coef = 1.f;
+#pragma unroll
+            for (int h = 0; h < G; ++h)
+                sl2[h] = p.scale_log2;
+            if constexpr (kFp8) {
+                const int qs = sg & 1;
+                const bool okq = mbar_wait(BAR(kBarQFull0 + qs), static_cast<uint32_t>(sg >> 1) & 1u, abort_flag,
+                                           p.status, kSiteDecodeConsumer);
+                if (okq) {
+#pragma unroll
+                    for (int h = 0; h < G; ++h)
+                        sl2[h] = q_scale[qs * kN + h];
+                }
+                mbar_arrive(BAR(kBarQScFree0 + qs));
+                ok = ok && okq;
+                v_coef = p.v_scale[static_cast<size_t>(bk % p.Hkv) * kD + i];
+                ++sg;
+            }
             float m[G], l[G], lpv[G];
 #pragma unroll
             for (int h = 0; h < G; ++h) {
@@ -521,7 +702,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const bool valid = (local0 + j) * kCK + i < seq_len;
 #pragma unroll
                     for (int h = 0; h < G; ++h) {
-                        x[h] = valid ? __uint_as_float(r[h]) * p.scale_log2 : -INFINITY;
+                        x[h] = valid ? __uint_as_float(r[h]) * sl2[h] : -INFINITY;
                         float v = x[h];
 #pragma unroll
                         for (int o = 16; o > 0; o >>= 1)
@@ -539,7 +720,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int h = 0; h < G; ++h) {
                     cmax[h] = fmaxf(fmaxf(rm[h], rm[kN + h]), fmaxf(rm[2 * kN + h], rm[3 * kN + h]));
-                    rescale = rescale || (cmax[h] > m[h] + kRescaleThreshold);
+                    rescale = rescale || (cmax[h] > m[h] + L::kRescaleThreshold);
                 }
                 if (j == 0) {
 #pragma unroll
@@ -573,16 +754,49 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // Weights, both running sums, and P^T (row h, column i) for the PV product. P^T is
                 // K-major with the 128-byte swizzle: key i sits in half i / 64 of row h, in 16-byte
                 // unit ((i % 64) / 8) XOR (h % 8).
-                uint8_t *pbuf = smem + kOffP + (c & 1) * kSmallBytes + (i >> 6) * kSmallHalf;
-                const int kk = i & 63;
+                if constexpr (kFp8) {
+                    // e4m3 cache: the weight times 16 as three e4m3 parts, each in its own 16 x 128-byte
+                    // tile: key i is byte (i % 16) of 16-byte unit (i / 16) XOR (h % 8) in row h. lpv sums
+                    // what the PV product uses (in units of 1/16, like O^T).
+                    uint8_t *pbuf = smem + kOffP + (c & 1) * kSmallBytes;
+                    auto off_of = [&](int h) { return (h >> 3) * 1024 + (h & 7) * 128 + ((((i >> 4) ^ (h & 7)) << 4) | (i & 15)); };
 #pragma unroll
-                for (int h = 0; h < G; ++h) {
-                    const float pe = ex2(x[h] - m[h]);
-                    l[h] += pe;
-                    const __nv_bfloat16 pb = __float2bfloat16_rn(pe);
-                    lpv[h] += __bfloat162float(pb);
-                    const int off = (h >> 3) * 1024 + (h & 7) * 128 + ((((kk >> 3) ^ (h & 7)) << 4) | ((kk & 7) << 1));
-                    *reinterpret_cast<__nv_bfloat16 *>(pbuf + off) = pb;
+                    for (int h = 0; h < G; h += 2) {  // two heads per conversion
+                        constexpr bool kPair = G > 1;
+                        const float pa = ex2(x[h] - m[h]);
+                        const float pb = kPair ? ex2(x[h + (kPair ? 1 : 0)] - m[h + (kPair ? 1 : 0)]) : 0.f;
+                        float wa = pa * L::kPScale, wb = pb * L::kPScale;
+                        const float ua = wa, ub = wb;
+#pragma unroll
+                        for (int t = 0; t < 3; ++t) {
+                            const uint32_t cd = e4m3x2(wa, wb);
+                            const float2 v = e4m3x2_value(cd);
+                            wa -= v.x;
+                            wb -= v.y;
+                            pbuf[t * kSmallHalf + off_of(h)] = static_cast<uint8_t>(cd & 0xffu);
+                            if (kPair)
+                                pbuf[t * kSmallHalf + off_of(h + 1)] = static_cast<uint8_t>((cd >> 8) & 0xffu);
+                        }
+                        // The parts' sum is the weight minus what is left over (exact: it needs ~12 bits).
+                        l[h] += pa;
+                        lpv[h] += ua - wa;
+                        if (kPair) {
+                            l[h + (kPair ? 1 : 0)] += pb;
+                            lpv[h + (kPair ? 1 : 0)] += ub - wb;
+                        }
+                    }
+                } else {
+                    uint8_t *pbuf = smem + kOffP + (c & 1) * kSmallBytes + (i >> 6) * kSmallHalf;
+                    const int kk = i & 63;
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        const float pe = ex2(x[h] - m[h]);
+                        l[h] += pe;
+                        const __nv_bfloat16 pb = __float2bfloat16_rn(pe);
+                        lpv[h] += __bfloat162float(pb);
+                        const int off = (h >> 3) * 1024 + (h & 7) * 128 + ((((kk >> 3) ^ (h & 7)) << 4) | ((kk & 7) << 1));
+                        *reinterpret_cast<__nv_bfloat16 *>(pbuf + off) = pb;
+                    }
                 }
                 if constexpr (kPaged) {
                     // Rows past the sequence's length in its last page hold whatever the cache holds
@@ -591,7 +805,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         uint4 *vrow = reinterpret_cast<uint4 *>(smem + kOffRing + (c % kStages) * kStageBytes + kTileBytes +
                                                                 i * 128);
 #pragma unroll
-                        for (int hf = 0; hf < 2; ++hf)
+                        for (int hf = 0; hf < L::kBoxCols; ++hf)
 #pragma unroll
                             for (int u = 0; u < 8; ++u)
                                 vrow[hf * (kHalfBytes / 16) + u] = make_uint4(0u, 0u, 0u, 0u);
@@ -640,7 +854,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     L += red_sum[(w * kN + h) * 2];
                     LPV += red_sum[(w * kN + h) * 2 + 1];
                 }
-                const float o = __uint_as_float(ov[h]) / LPV;
+                const float o = __uint_as_float(ov[h]) / LPV * v_coef;
                 const size_t bh = static_cast<size_t>(b) * p.Hq + h0 + h;
                 if (whole_pair) {
                     p.o[bh * kD + i] = __float2bfloat16_rn(o);
@@ -746,16 +960,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 #undef BAR
 }
 
-template <int G, bool kPaged>
+template <int G, bool kPaged, bool kFp8>
 cudaError_t prepare_g(int *ctas_per_sm)
 {
     static int cached = 0;
+    constexpr int kSmem = Lay<kFp8>::kSmem;
     if (cached == 0) {
-        cudaError_t e =
-            cudaFuncSetAttribute(decode_tc_kernel<G, kPaged>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+        cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<G, kPaged, kFp8>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
         int n = 0;
         if (e == cudaSuccess)
-            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_tc_kernel<G, kPaged>, kThreads, kSmem);
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_tc_kernel<G, kPaged, kFp8>, kThreads, kSmem);
         if (e != cudaSuccess)
             return e;
         cached = n > 0 ? n : 1;
@@ -765,10 +980,10 @@ cudaError_t prepare_g(int *ctas_per_sm)
     return cudaSuccess;
 }
 
-template <int G, bool kPaged>
+template <int G, bool kPaged, bool kFp8>
 cudaError_t launch_g(const DecodeArgs &a, cudaStream_t stream)
 {
-    cudaError_t e = prepare_g<G, kPaged>(nullptr);
+    cudaError_t e = prepare_g<G, kPaged, kFp8>(nullptr);
     if (e != cudaSuccess)
         return e;
     auto encode = get_encode_fn();
@@ -777,14 +992,22 @@ cudaError_t launch_g(const DecodeArgs &a, cudaStream_t stream)
     int err = 0;
     CUtensorMap tq, tk, tv;
     // q as [1][B*Hq][D] (one row per query head); k and v as [B*Hkv][Skv][D], or, paged, as
-    // [num_pages*Hkv][page_size][D] read in boxes of min(page_size, 128) rows.
+    // [num_pages*Hkv][page_size][D] read in boxes of min(page_size, 128) rows and 128 bytes of D
+    // (64 bf16 or 128 e4m3 elements).
     const int kv_rows = kPaged ? a.page_size : a.Skv;
     const int kv_bh = kPaged ? a.num_pages * a.Hkv : a.B * a.Hkv;
     const int box_rows = kPaged ? (a.page_size < kCK ? a.page_size : kCK) : kCK;
-    if (!make_map(encode, &tq, a.q, kD, a.B * a.Hq, 1, 64, kN, CU_TENSOR_MAP_SWIZZLE_128B, &err) ||
-        !make_map(encode, &tk, a.k, kD, kv_rows, kv_bh, 64, box_rows, CU_TENSOR_MAP_SWIZZLE_128B, &err) ||
-        !make_map(encode, &tv, a.v, kD, kv_rows, kv_bh, 64, box_rows, CU_TENSOR_MAP_SWIZZLE_128B, &err))
+    if (!make_map(encode, &tq, a.q, kD, a.B * a.Hq, 1, 64, kN, CU_TENSOR_MAP_SWIZZLE_128B, &err))
         return cudaErrorInvalidValue;
+    if constexpr (kFp8) {
+        if (!make_map_u8(encode, &tk, a.k, kD, kv_rows, kv_bh, 128, box_rows, CU_TENSOR_MAP_SWIZZLE_128B, &err) ||
+            !make_map_u8(encode, &tv, a.v, kD, kv_rows, kv_bh, 128, box_rows, CU_TENSOR_MAP_SWIZZLE_128B, &err))
+            return cudaErrorInvalidValue;
+    } else {
+        if (!make_map(encode, &tk, a.k, kD, kv_rows, kv_bh, 64, box_rows, CU_TENSOR_MAP_SWIZZLE_128B, &err) ||
+            !make_map(encode, &tv, a.v, kD, kv_rows, kv_bh, 64, box_rows, CU_TENSOR_MAP_SWIZZLE_128B, &err))
+            return cudaErrorInvalidValue;
+    }
     const DecodePlan &pl = a.plan;
     TcParams p;
     p.o = static_cast<__nv_bfloat16 *>(a.o);
@@ -808,7 +1031,11 @@ cudaError_t launch_g(const DecodeArgs &a, cudaStream_t stream)
     p.page_size = a.page_size;
     p.pages_per_seq = a.pages_per_seq;
     p.max_seq_len = a.max_seq_len;
-    decode_tc_kernel<G, kPaged><<<static_cast<unsigned>(pl.ctas), kThreads, kSmem, stream>>>(tq, tk, tv, p);
+    p.q = static_cast<const __nv_bfloat16 *>(a.q);
+    p.k_scale = a.k_scale;
+    p.v_scale = a.v_scale;
+    decode_tc_kernel<G, kPaged, kFp8>
+        <<<static_cast<unsigned>(pl.ctas), kThreads, Lay<kFp8>::kSmem, stream>>>(tq, tk, tv, p);
     return cudaGetLastError();
 }
 
@@ -816,8 +1043,10 @@ template <int G>
 cudaError_t dispatch_g(const DecodeArgs *a, cudaStream_t stream, int *ctas_per_sm)
 {
     if (!a)
-        return prepare_g<G, false>(ctas_per_sm);
-    return a->seq_lens ? launch_g<G, true>(*a, stream) : launch_g<G, false>(*a, stream);
+        return prepare_g<G, false, false>(ctas_per_sm);
+    if (a->fp8)
+        return a->seq_lens ? launch_g<G, true, true>(*a, stream) : launch_g<G, false, true>(*a, stream);
+    return a->seq_lens ? launch_g<G, true, false>(*a, stream) : launch_g<G, false, false>(*a, stream);
 }
 
 cudaError_t dispatch_tc(int G, const DecodeArgs *a, cudaStream_t stream, int *ctas_per_sm)
@@ -871,7 +1100,7 @@ cudaError_t decode_plan_paged(int B, int Hq, int Hkv, int max_seq_len, int reque
     long long ctas = requested_ctas;
     if (ctas <= 0) {
         int per_sm = 1;
-        const cudaError_t e = prepare_g<1, true>(&per_sm);
+        const cudaError_t e = prepare_g<1, true, false>(&per_sm);
         if (e != cudaSuccess)
             return e;
         // As for the dense cache: one CTA per pair when the pairs alone fill most of the GPU

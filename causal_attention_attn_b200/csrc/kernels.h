@@ -66,6 +66,10 @@ struct DecodeArgs {
     const int *seq_lens = nullptr;
     const int *block_table = nullptr;
     int num_pages = 0, page_size = 0, pages_per_seq = 0, max_seq_len = 0;
+    // e4m3 cache (tensor-core decode only): k, v hold e4m3 codes; k_scale, v_scale are device fp32
+    // [Hkv][D] coefficients (value = code * coefficient of its kv head and channel).
+    bool fp8 = false;
+    const float *k_scale = nullptr, *v_scale = nullptr;
 };
 
 // Returns a cudaError_t value (cudaSuccess on success); never synchronises.

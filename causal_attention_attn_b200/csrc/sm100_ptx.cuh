@@ -214,6 +214,17 @@ __device__ __forceinline__ void tc_mma_ss(uint32_t d_tmem, uint64_t a_desc, uint
                  : "memory");
 }
 
+// As tc_mma_ss for 8-bit floating-point operands (kind::f8f6f4; both e4m3 here): the K extent of
+// one instruction is 32 elements, i.e. 32 bytes of a K-major row.
+__device__ __forceinline__ void tc_mma_f8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate)
+{
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+                 "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+                 : "memory");
+}
+
 // D[tmem] (+)= A[tmem] * B[smem]: the A operand (M x K, K-major) is read from tensor memory, row i
 // in lane i, two 16-bit elements per 32-bit column (element 2c in the low half of column c).
 __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
@@ -257,6 +268,14 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_ma
 __host__ __device__ constexpr uint32_t idesc_bf16_f32_ab(int M, int N, bool a_mn_major, bool b_mn_major)
 {
     return idesc_bf16_f32(M, N, b_mn_major) | ((a_mn_major ? 1u : 0u) << 15);
+}
+
+// Instruction descriptor for kind::f8f6f4 with e4m3 A and B (format code 0 in bits 7-9 and 10-12)
+// and an fp32 accumulator; majors, N and M as for idesc_bf16_f32_ab. MN-major is valid for e4m3.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32_ab(int M, int N, bool a_mn_major, bool b_mn_major)
+{
+    return (1u << 4) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
+           (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
 // TMEM address: lane in bits 31-16, column in bits 15-0.

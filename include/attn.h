@@ -163,6 +163,11 @@ int attn_decode_noalloc(const void *q, const void *k, const void *v, void *o, fl
  * never synchronises, so block_table and seq_lens may be written by earlier work on `stream`.
  * Returns ATTN_OK or a negative attn_status (argument errors before any launch).
  */
+int attn_decode_paged(const void *q, const void *k_pages, const void *v_pages, const int *block_table,
+                      const int *seq_lens, void *o, float *lse, int B, int Hq, int Hkv, int num_pages,
+                      int page_size, int pages_per_seq, int max_seq_len, float scale, int decode_ctas,
+                      void *stream);
+
 /*
  * attn_bwd — backward pass of attn_fwd: given dout = dL/do for a loss L, the gradients
  *   dq = dL/dq [B, Hq, Sq, D], dk = dL/dk and dv = dL/dv [B, Hkv, Skv, D] (bf16, written entirely;
@@ -179,10 +184,42 @@ int attn_bwd(const void *q, const void *k, const void *v, const void *o, const v
              void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int Sq, int Skv, int D,
              float scale, int causal, void *stream);
 
-int attn_decode_paged(const void *q, const void *k_pages, const void *v_pages, const int *block_table,
-                      const int *seq_lens, void *o, float *lse, int B, int Hq, int Hkv, int num_pages,
-                      int page_size, int pages_per_seq, int max_seq_len, float scale, int decode_ctas,
-                      void *stream);
+/*
+ * attn_decode_fp8 — single-token decode (Sq == 1) over a K/V cache stored as FP8 (e4m3) codes with
+ * one fp32 coefficient per (kv head, channel): the cached key is k~[b,g,j,d] = e4m3(k8[b,g,j,d]) *
+ * k_scale[g,d], likewise v~ with v_scale, and the result is attn_fwd's decode over k~, v~.
+ *
+ * Source (page title, section): "MLA 矩阵乘法吸收的数值稳定性治理", §五 — the KV cache may be kept in
+ * FP8 to save bandwidth provided the products accumulate in higher precision (fp32 here, in tensor
+ * memory); §二.1 — a coefficient per feature channel. The coefficient's granularity (per kv head and
+ * channel, shared by all batch entries) is this library's reading.
+ *
+ * Layout (device pointers owned by the caller, 16-byte aligned):
+ *   q            bf16 [B, Hq, 1, 128]; o bf16 [B, Hq, 1, 128]; lse fp32 [B, Hq, 1] (natural log).
+ *   k8, v8       e4m3 codes (1 byte each; the OCP format with bias 7, NaN = S.1111.111)
+ *                [B, Hkv, Skv, 128].
+ *   k_scale,     fp32 [Hkv, 128].
+ *   v_scale
+ * The tensor core reads the codes as they are. q * k_scale and the softmax weights enter the
+ * products as sums of three e4m3 parts (about 12 significant bits; q is first scaled per head by a
+ * power of two into the top of the e4m3 range, which the softmax undoes), so the result matches
+ * the dequantised cache to about the accuracy of the bf16 path. Non-finite codes, coefficients or
+ * q values give undefined results. Head dim 128 only; Hq % Hkv == 0; decode_ctas as attn_decode_paged.
+ * Returns ATTN_OK or a negative attn_status (argument errors before any launch); never synchronises.
+ */
+int attn_decode_fp8(const void *q, const void *k8, const void *v8, const float *k_scale, const float *v_scale,
+                    void *o, float *lse, int B, int Hq, int Hkv, int Skv, int D, float scale, int decode_ctas,
+                    void *stream);
+
+/*
+ * attn_decode_paged_fp8 — attn_decode_paged over an e4m3 cache: k_pages, v_pages hold e4m3 codes
+ * [num_pages, Hkv, page_size, 128] and k_scale, v_scale are as for attn_decode_fp8. Every other
+ * argument, rule and return value is attn_decode_paged's.
+ */
+int attn_decode_paged_fp8(const void *q, const void *k_pages, const void *v_pages, const float *k_scale,
+                          const float *v_scale, const int *block_table, const int *seq_lens, void *o, float *lse,
+                          int B, int Hq, int Hkv, int num_pages, int page_size, int pages_per_seq, int max_seq_len,
+                          float scale, int decode_ctas, void *stream);
 
 #ifdef __cplusplus
 }

@@ -21,7 +21,7 @@ def lib():
 def declared_functions():
     text = open(HEADER, encoding="utf-8").read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(attn_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(attn_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_header_declares_the_entry_points():
@@ -37,7 +37,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.attn_version() == 200
+    assert lib.attn_version() == 300
     for code, name in attn.STATUS_NAMES.items():
         s = attn.status_string(code)
         assert s and s != "unknown status", (code, name)
@@ -126,3 +126,40 @@ def test_paged_argument_errors(lib, name, override, expected):
                                a["max_seq_len"], a["scale"], a["ctas"], None)
     assert rc == expected, (name, rc)
 
+
+
+# attn_decode_fp8(q, k8, v8, k_scale, v_scale, o, lse, B, Hq, Hkv, Skv, D, scale, ctas, stream)
+FP8_GOOD = dict(B=2, Hq=8, Hkv=2, Skv=300, D=128, scale=0.1, ctas=0)
+FP8_PTRS = [A[0], A[1], A[2], A[3], A[4], A[0] + 0x100000, A[1] + 0x100000]
+FP8_CASES = [
+    ("null k_scale", dict(ptrs=FP8_PTRS[:3] + [0] + FP8_PTRS[4:]), -1),
+    ("null v_scale", dict(ptrs=FP8_PTRS[:4] + [0] + FP8_PTRS[5:]), -1),
+    ("zero keys", dict(Skv=0), -2),
+    ("negative cta count", dict(ctas=-1), -2),
+    ("gqa not divisible", dict(Hq=6, Hkv=4), -3),
+    ("head dim 64", dict(D=64), -4),
+    ("misaligned k_scale", dict(ptrs=FP8_PTRS[:3] + [A[3] + 4] + FP8_PTRS[4:]), -5),
+    ("misaligned k8", dict(ptrs=[A[0], A[1] + 8] + FP8_PTRS[2:]), -5),
+    ("zero scale", dict(scale=0.0), -11),
+]
+
+
+@pytest.mark.parametrize("name,override,expected", FP8_CASES, ids=[c[0] for c in FP8_CASES])
+def test_fp8_argument_errors(lib, name, override, expected):
+    a = dict(FP8_GOOD)
+    a.update({k: v for k, v in override.items() if k != "ptrs"})
+    ptrs = override.get("ptrs", FP8_PTRS)
+    rc = lib.attn_decode_fp8(*ptrs, a["B"], a["Hq"], a["Hkv"], a["Skv"], a["D"], a["scale"], a["ctas"], None)
+    assert rc == expected, (name, rc)
+
+
+def test_paged_fp8_argument_errors(lib):
+    # q, k_pages, v_pages, k_scale, v_scale, block_table, seq_lens, o, lse
+    ptrs = [A[0], A[1], A[2], A[3], A[4], A[3], A[4], A[0] + 0x100000, A[1] + 0x100000]
+    args = (2, 8, 2, 4, 64, 2, 128, 0.1, 0, None)
+    bad_scale = list(ptrs)
+    bad_scale[3] = 0
+    assert lib.attn_decode_paged_fp8(*bad_scale, *args) == -1
+    bad_scale[3] = A[3] + 4
+    assert lib.attn_decode_paged_fp8(*bad_scale, *args) == -5
+    assert lib.attn_decode_paged_fp8(*ptrs, 2, 8, 2, 4, 48, 2, 128, 0.1, 0, None) == -2
