@@ -52,6 +52,41 @@ def dist_env():
     return world, rank, local
 
 
+class Ranks:
+    """Host-side plumbing of the replicas: a barrier and a max over ranks of device-timed values.
+
+    The ranks exchange only timings (no data-path collective: every rank runs the whole workload on
+    its own GPU). NCCL on GPU tensors when the process group uses it, gloo on CPU tensors otherwise;
+    with one process both are no-ops.
+    """
+
+    def __init__(self, world: int, device):
+        self.world = world
+        self.device = device
+
+    def barrier(self):
+        if self.world > 1:
+            import torch.distributed as dist
+
+            dist.barrier()
+
+    def max(self, values):
+        """Element-wise maximum of `values` (a list of floats) over all ranks."""
+        if self.world == 1:
+            return list(values)
+        import torch.distributed as dist
+
+        t = torch.tensor(list(values), dtype=torch.float64, device=self.device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return t.tolist()
+
+
+def whole_job_rate(world: int, units_per_rank: float, seconds: float) -> float:
+    """Units all ranks processed per second: every rank did `units_per_rank`; `seconds` is the
+    slowest rank's device time."""
+    return world * units_per_rank / seconds
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle-reason samples taken every 100 ms while the timed region runs."""
 
@@ -148,7 +183,7 @@ def run_reference(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,1) bf16 inputs)", "config": PREFILL.config(),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                         "sample": f"every {every}th query row of the workload per step (rows offset by the step "
+                         "sample": f"one query row in {every} of the workload per step (rows offset by the step "
                                    f"index), {n} rows; fp64 three-pass oracle"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -166,6 +201,7 @@ def run_ours(args):
         import torch.distributed as dist
 
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    ranks = Ranks(world, dev)
     from causal_attention_attn_b200 import attn
 
     attn.load_library()
@@ -211,8 +247,7 @@ def run_ours(args):
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     t_all0 = torch.cuda.Event(enable_timing=True)
     t_all1 = torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        torch.distributed.barrier()
+    ranks.barrier()
     torch.cuda.synchronize(dev)
     with ClockSampler(local) as clocks:
         t_all0.record(stream)
@@ -220,19 +255,15 @@ def run_ours(args):
             step(events[s])
         t_all1.record(stream)
         torch.cuda.synchronize(dev)
-    if world > 1:
-        torch.distributed.barrier()
+    ranks.barrier()
     pre_ms = sum(e[0].elapsed_time(e[1]) for e in events)
     dec_ms = sum(e[2].elapsed_time(e[3]) for e in events)
     region_ms = t_all0.elapsed_time(t_all1)
-    if world > 1:
-        t = torch.tensor([pre_ms, dec_ms, region_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        pre_ms, dec_ms, region_ms = t.tolist()
+    pre_ms, dec_ms, region_ms = ranks.max([pre_ms, dec_ms, region_ms])
 
-    prefill_tflops = world * args.steps * PREFILL.flops() / (pre_ms * 1e-3) / 1e12
+    prefill_tflops = whole_job_rate(world, args.steps * PREFILL.flops(), pre_ms * 1e-3) / 1e12
     decode_bytes = DECODE.io_bytes()  # K and V read once, plus q, o and lse
-    decode_gbs = world * args.steps * decode_bytes / (dec_ms * 1e-3) / 1e9
+    decode_gbs = whole_job_rate(world, args.steps * decode_bytes, dec_ms * 1e-3) / 1e9
     pre_launch_s = pre_ms * 1e-3 / args.steps
     dec_launch_s = dec_ms * 1e-3 / args.steps
     tensor_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
@@ -248,8 +279,7 @@ def run_ours(args):
                            dev_bufs=bufs)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e2e_steps = max(3, min(args.steps, 10))
-    if world > 1:
-        torch.distributed.barrier()
+    ranks.barrier()
     torch.cuda.synchronize(dev)
     e0.record(stream)
     for _ in range(e2e_steps):
@@ -258,12 +288,9 @@ def run_ours(args):
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = t.item()
-        torch.distributed.barrier()
-    e2e_tflops = world * e2e_steps * PREFILL.flops() / (e2e_ms * 1e-3) / 1e12
+    e2e_ms = ranks.max([e2e_ms])[0]
+    ranks.barrier()
+    e2e_tflops = whole_job_rate(world, e2e_steps * PREFILL.flops(), e2e_ms * 1e-3) / 1e12
 
     # The same decode over an e4m3 cache (per-channel coefficients), timed on its own: inputs
     # resident, L2 flushed before every launch, CUDA events around each launch.
@@ -276,8 +303,7 @@ def run_ours(args):
         attn.attn_decode_fp8(fq, fk8, fv8, fks, fvs, scale=DECODE.scale, out=fo, lse=fl, stream=stream)
     fp8_steps = max(3, min(args.steps, 500))
     fev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(fp8_steps)]
-    if world > 1:
-        torch.distributed.barrier()
+    ranks.barrier()
     torch.cuda.synchronize(dev)
     for s in range(fp8_steps):
         clear_l2()
@@ -285,11 +311,7 @@ def run_ours(args):
         attn.attn_decode_fp8(fq, fk8, fv8, fks, fvs, scale=DECODE.scale, out=fo, lse=fl, stream=stream)
         fev[s][1].record(stream)
     torch.cuda.synchronize(dev)
-    fp8_ms = sum(a.elapsed_time(b) for a, b in fev)
-    if world > 1:
-        t = torch.tensor([fp8_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        fp8_ms = t.item()
+    fp8_ms = ranks.max([sum(a.elapsed_time(b) for a, b in fev)])[0]
     fp8_launch_s = fp8_ms * 1e-3 / fp8_steps
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
     d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
@@ -317,7 +339,7 @@ def run_ours(args):
                 "ctas": attn.decode_ctas(DECODE.B, DECODE.Hq, DECODE.Hkv, DECODE.Skv, DECODE.D),
             },
             "decode_fp8": {
-                "metric": "decode KV-read GB/s, e4m3 K/V cache", "value": world * fp8_bytes / fp8_launch_s / 1e9,
+                "metric": "decode KV-read GB/s, e4m3 K/V cache", "value": whole_job_rate(world, fp8_bytes, fp8_launch_s) / 1e9,
                 "unit": "GB/s", "config": dict(DECODE.config(), kv_dtype="e4m3", scales="fp32 per (kv head, channel)"),
                 "steps": fp8_steps,
                 "roofline": {"bound": "hbm", "achieved": fp8_bytes / fp8_launch_s / 1e9, "peak": hbm_peak,

@@ -25,14 +25,17 @@
  *
  * Ownership: every pointer is a DEVICE pointer owned by the caller. The library keeps no pointer
  * after the work completes on `stream`. The library owns one small per-device workspace (the
- * split-KV partials of the decode kernel and a status word); it grows on the first call that needs
- * more, with cudaMalloc (so that first call is not stream-ordered and cannot be graph-captured).
- * Concurrent decode calls on different streams of one device share that workspace and must be
- * serialised by the caller.
+ * split-KV partials of the decode kernel and a status word; attn_bwd keeps a second one); it grows
+ * on the first call that needs more, with cudaMalloc, and when it replaces a smaller block it waits
+ * for the device (cudaDeviceSynchronize) before freeing the old one, which queued kernels may still
+ * read. A growing call is therefore neither stream-ordered nor graph-capturable; make one call of
+ * the largest size before capturing. Concurrent decode calls on different streams of one device
+ * share that workspace and must be serialised by the caller.
  *
  * Errors: argument errors are detected on the host before any launch and returned as a negative
- * attn_status; nothing is launched then. Launch failures return ATTN_ERR_LAUNCH. The call never
- * synchronises the stream, never aborts the process and never traps on the device. Kernel-side
+ * attn_status; nothing is launched then. Launch failures return ATTN_ERR_LAUNCH. Apart from a call
+ * that grows the workspace (above), no call synchronises; none aborts the process or traps on the
+ * device. Kernel-side
  * waits are bounded: a wait that runs out sets the device status word, which attn_device_status()
  * reads.
  */
@@ -159,8 +162,8 @@ int attn_decode_noalloc(const void *q, const void *k, const void *v, void *o, fl
  *   max_seq_len  host-side upper bound of the lengths (sizes nothing larger than it needs).
  *   page_size    16, 32, 64 or a multiple of 128.
  *   decode_ctas  CTAs to launch (0: one per resident slot). A performance parameter only.
- * Head dim 128 only; 1 <= B <= 1024; Hq % Hkv == 0. Lengths are read on the device: the call
- * never synchronises, so block_table and seq_lens may be written by earlier work on `stream`.
+ * Head dim 128 only; 1 <= B <= 1024; Hq % Hkv == 0. Lengths are read on the device and never on
+ * the host, so block_table and seq_lens may be written by earlier work on `stream`.
  * Returns ATTN_OK or a negative attn_status (argument errors before any launch).
  */
 int attn_decode_paged(const void *q, const void *k_pages, const void *v_pages, const int *block_table,
@@ -178,7 +181,8 @@ int attn_decode_paged(const void *q, const void *k_pages, const void *v_pages, c
  * the operation defined at the top of this file. Head dim 128 only; the other sizes, the causal flag
  * and the scale as attn_fwd. The library keeps an fp32 accumulator for dq and two per-row vectors in
  * its workspace (grown with cudaMalloc like attn_fwd's). Every pointer is a caller-owned device
- * pointer, 16-byte aligned. Returns ATTN_OK or a negative attn_status; never synchronises.
+ * pointer, 16-byte aligned. Returns ATTN_OK or a negative attn_status; synchronises only when it
+ * grows its workspace.
  */
 int attn_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout, const float *lse,
              void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int Sq, int Skv, int D,
@@ -205,7 +209,7 @@ int attn_bwd(const void *q, const void *k, const void *v, const void *o, const v
  * power of two into the top of the e4m3 range, which the softmax undoes), so the result matches
  * the dequantised cache to about the accuracy of the bf16 path. Non-finite codes, coefficients or
  * q values give undefined results. Head dim 128 only; Hq % Hkv == 0; decode_ctas as attn_decode_paged.
- * Returns ATTN_OK or a negative attn_status (argument errors before any launch); never synchronises.
+ * Returns ATTN_OK or a negative attn_status (argument errors before any launch).
  */
 int attn_decode_fp8(const void *q, const void *k8, const void *v8, const float *k_scale, const float *v_scale,
                     void *o, float *lse, int B, int Hq, int Hkv, int Skv, int D, float scale, int decode_ctas,
