@@ -26,7 +26,7 @@ STATUS_NAMES = {
 }
 EXPORTED = ("attn_fwd", "attn_fwd_ex", "attn_decode_ctas", "attn_status_string", "attn_version",
             "attn_device_status", "attn_decode_noalloc", "attn_decode_paged", "attn_bwd", "attn_decode_fp8",
-            "attn_decode_paged_fp8")
+            "attn_decode_paged_fp8", "attn_lse_merge")
 
 _lock = threading.Lock()
 _lib = None
@@ -70,6 +70,8 @@ def load_library(path: str | None = None):
         lib.attn_decode_paged.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, vp]
         lib.attn_decode_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
         lib.attn_decode_paged_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, vp]
+        lib.attn_lse_merge.restype = i
+        lib.attn_lse_merge.argtypes = [vp, vp, vp, vp, vp, ctypes.c_longlong, i, vp]
         if path is None:
             _lib = lib
         return lib
@@ -315,6 +317,31 @@ def attn_decode_paged_fp8(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch
                                                   float(scale), int(decode_ctas), _stream_handle(stream))
     _check(rc)
     return out, lse
+
+
+def attn_lse_merge(o_acc: torch.Tensor, lse_acc: torch.Tensor, o_part: torch.Tensor, lse_part: torch.Tensor,
+                   out: torch.Tensor | None = None, stream=None):
+    """Merge one attention result over a block of keys (o_part bf16 [..., D], lse_part fp32 [...])
+    into a running result (o_acc fp32, lse_acc fp32, same shapes; updated in place) through
+    ``attn_lse_merge``. ``out`` (bf16, shape of o_part) optionally receives the merged O."""
+    _check_tensor("o_part", o_part, torch.bfloat16, o_part.dim())
+    _check_tensor("o_acc", o_acc, torch.float32, o_part.dim())
+    _check_tensor("lse_part", lse_part, torch.float32, o_part.dim() - 1)
+    _check_tensor("lse_acc", lse_acc, torch.float32, o_part.dim() - 1)
+    if o_acc.shape != o_part.shape or lse_acc.shape != lse_part.shape or tuple(lse_part.shape) != tuple(o_part.shape[:-1]):
+        raise ValueError("o_acc, o_part [..., D] and lse_acc, lse_part [...] must agree")
+    if out is not None:
+        _check_tensor("out", out, torch.bfloat16, o_part.dim())
+        if out.shape != o_part.shape:
+            raise ValueError("out must have the shape of o_part")
+    D = int(o_part.shape[-1])
+    rows = o_part.numel() // D if D else 0
+    with torch.cuda.device(o_part.device):
+        rc = load_library().attn_lse_merge(o_acc.data_ptr(), lse_acc.data_ptr(), o_part.data_ptr(), lse_part.data_ptr(),
+                                           out.data_ptr() if out is not None else None, rows, D,
+                                           _stream_handle(stream))
+    _check(rc)
+    return o_acc, lse_acc
 
 
 def attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse: torch.Tensor,

@@ -16,7 +16,7 @@
 namespace attn_b200 {
 namespace {
 
-constexpr int kVersion = 300;  // 0.3.0: adds attn_bwd, attn_decode_fp8, attn_decode_paged_fp8
+constexpr int kVersion = 400;  // 0.4.0: adds attn_lse_merge (after 0.3.0: attn_bwd, the e4m3 decodes)
 constexpr int kMaxDevices = 64;
 
 struct DeviceState {
@@ -468,6 +468,37 @@ extern "C" int attn_decode_fp8(const void *q, const void *k8, const void *v8, co
     a.k_scale = k_scale;
     a.v_scale = v_scale;
     if (launch_decode_tc(a, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_LAUNCH;
+    }
+    return ATTN_OK;
+}
+
+extern "C" int attn_lse_merge(float *o_acc, float *lse_acc, const void *o_part, const float *lse_part, void *o_out,
+                              long long rows, int D, void *stream_ptr)
+{
+    using namespace attn_b200;
+    if (!o_acc || !lse_acc || !o_part || !lse_part)
+        return ATTN_ERR_NULL;
+    if (rows < 0 || rows > (1LL << 40))
+        return ATTN_ERR_SHAPE;
+    if (D != 32 && D != 64 && D != 128)
+        return ATTN_ERR_HEADDIM;
+    if (!aligned16(o_acc) || !aligned16(o_part) || !aligned16(lse_acc) || !aligned16(lse_part) ||
+        (o_out && !aligned16(o_out)))
+        return ATTN_ERR_ALIGN;
+    if (rows == 0)
+        return ATTN_OK;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+    int err = ATTN_OK;
+    DeviceState *s = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        s = device_state(&err);
+    }
+    if (!s)
+        return err;
+    if (launch_lse_merge(o_acc, lse_acc, o_part, lse_part, o_out, rows, D, s->sm_count, stream) != cudaSuccess) {
         cudaGetLastError();
         return ATTN_ERR_LAUNCH;
     }

@@ -89,6 +89,11 @@ struct BwdArgs {
 size_t bwd_workspace_bytes(int B, int Hq, int Sq, int D);
 cudaError_t launch_bwd(const BwdArgs &a, cudaStream_t stream, int *encode_error);
 
+// LSE merge of a partial result (bf16 o_part, fp32 lse_part) into an fp32 accumulator, rows x D
+// (D in {32, 64, 128}); o_out (bf16, may be null) receives the merged O.
+cudaError_t launch_lse_merge(float *o_acc, float *lse_acc, const void *o_part, const float *lse_part, void *o_out,
+                             long long rows, int D, int sm_count, cudaStream_t stream);
+
 // Decode planning and launch. requested_ctas <= 0 means one CTA per resident slot on the device.
 int decode_heads_per_cta(int group, int D);  // G: 1, 2, 4 or 8 (up to 16 for D = 128)
 cudaError_t decode_plan(int B, int Hq, int Hkv, int Skv, int D, int requested_ctas, int sm_count, DecodePlan *plan);

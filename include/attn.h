@@ -225,6 +225,25 @@ int attn_decode_paged_fp8(const void *q, const void *k_pages, const void *v_page
                           int B, int Hq, int Hkv, int num_pages, int page_size, int pages_per_seq, int max_seq_len,
                           float scale, int decode_ctas, void *stream);
 
+/*
+ * attn_lse_merge — merges attention over one block of keys into a running result over other keys
+ * (the LSE merge of split keys; ring attention calls it once per key block it receives).
+ *
+ * Source (page title, section): "AI Infra 入门…", §3 (LSE paragraph). Per row, natural logs:
+ *   M = max(lse_acc, lse_part), w_a = e^(lse_acc - M), w_p = e^(lse_part - M),
+ *   o_acc <- (w_a o_acc + w_p o_part) / (w_a + w_p), lse_acc <- M + ln(w_a + w_p).
+ * A side with lse = -inf (no key) has weight 0; a row empty on both sides stays as it is. Start an
+ * accumulator at o_acc = 0, lse_acc = -inf.
+ *
+ * Layout (device pointers owned by the caller, 16-byte aligned): o_acc fp32 [rows, D] and lse_acc
+ * fp32 [rows], updated in place; o_part bf16 [rows, D] and lse_part fp32 [rows] (an attn_fwd
+ * result); o_out bf16 [rows, D] or NULL: when given, also receives the merged O rounded to bf16.
+ * rows = B * Hq * Sq of the attention call; D in {32, 64, 128}. rows = 0 launches nothing.
+ * Returns ATTN_OK or a negative attn_status (argument errors before any launch); never allocates.
+ */
+int attn_lse_merge(float *o_acc, float *lse_acc, const void *o_part, const float *lse_part, void *o_out,
+                   long long rows, int D, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

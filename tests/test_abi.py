@@ -37,7 +37,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.attn_version() == 300
+    assert lib.attn_version() == 400
     for code, name in attn.STATUS_NAMES.items():
         s = attn.status_string(code)
         assert s and s != "unknown status", (code, name)
@@ -163,3 +163,20 @@ def test_paged_fp8_argument_errors(lib):
     bad_scale[3] = A[3] + 4
     assert lib.attn_decode_paged_fp8(*bad_scale, *args) == -5
     assert lib.attn_decode_paged_fp8(*ptrs, 2, 8, 2, 4, 48, 2, 128, 0.1, 0, None) == -2
+
+
+# attn_lse_merge(o_acc, lse_acc, o_part, lse_part, o_out, rows, D, stream)
+MERGE_CASES = [
+    ("null accumulator", [0, A[1], A[2], A[3], None], 10, 128, -1),
+    ("null part lse", [A[0], A[1], A[2], 0, None], 10, 128, -1),
+    ("negative rows", [A[0], A[1], A[2], A[3], None], -1, 128, -2),
+    ("head dim 48", [A[0], A[1], A[2], A[3], None], 10, 48, -4),
+    ("misaligned part", [A[0], A[1], A[2] + 2, A[3], None], 10, 64, -5),
+    ("misaligned output", [A[0], A[1], A[2], A[3], A[4] + 8], 10, 32, -5),
+    ("no rows: nothing to do", [A[0], A[1], A[2], A[3], None], 0, 128, 0),
+]
+
+
+@pytest.mark.parametrize("name,ptrs,rows,D,expected", MERGE_CASES, ids=[c[0] for c in MERGE_CASES])
+def test_lse_merge_argument_errors(lib, name, ptrs, rows, D, expected):
+    assert lib.attn_lse_merge(*ptrs, rows, D, None) == expected, name

@@ -1,0 +1,130 @@
+"""GPU parity of the LSE merge kernel (``attn_lse_merge``) and of ring attention's per-block work.
+
+Every run here has one GPU, so no test waits on another rank: the ring's schedule is emulated on
+one GPU (the chunks are indexed instead of received), which runs exactly the kernels and the
+merge order a rank runs; the distributed driver itself is run with one rank, and with two and
+three gloo ranks on the CPU in ``test_ring_cpu.py``.
+"""
+import datetime
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from causal_attention_attn_b200 import attn, build, inputs
+from causal_attention_attn_b200.ring import DIAG, SKIP, ring_schedule
+from tests.compare import compare
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    if torch.cuda.get_device_capability(0) != (10, 0):
+        pytest.skip("needs an sm_100 device")
+    build.build()
+    attn.load_library()
+    yield
+    torch.cuda.synchronize()
+    assert attn.device_status() == 0, "a kernel-side wait ran out during the ring tests"
+
+
+@pytest.mark.parametrize("D", [32, 64, 128])
+def test_merge_of_two_key_blocks_equals_attention_over_both(D):
+    """Attention over keys [0, h) and over [h, Skv), merged, equals attention over all keys."""
+    w = inputs.custom(2, 4, 2, 96, 200, D, False, seed=D)
+    q, k, v = inputs.generate(w)
+    h = 77
+    parts = [oracle.attention(q, k[:, :, :h].contiguous(), v[:, :, :h].contiguous(), w.scale, False),
+             oracle.attention(q, k[:, :, h:].contiguous(), v[:, :, h:].contiguous(), w.scale, False)]
+    o_acc = torch.zeros(q.shape, dtype=torch.float32, device="cuda")
+    lse_acc = torch.full(q.shape[:-1], float("-inf"), dtype=torch.float32, device="cuda")
+    out = torch.empty(q.shape, dtype=torch.bfloat16, device="cuda")
+    for n, (o_p, l_p) in enumerate(parts):
+        attn.attn_lse_merge(o_acc, lse_acc, torch.from_numpy(o_p).to(torch.bfloat16).cuda(),
+                            torch.from_numpy(l_p).float().cuda(), out=out if n == 1 else None)
+    torch.cuda.synchronize()
+    ro, rl = oracle.attention(q, k, v, w.scale, False)
+    rep = compare(out, lse_acc, ro, rl)
+    assert rep.ok(), str(rep)
+
+
+def test_merge_with_empty_sides():
+    """lse = -inf means no key: such a side has weight 0; a row empty on both sides stays empty."""
+    rows, D = 40, 128
+    g = torch.Generator().manual_seed(1)
+    o_a = torch.randn((rows, D), generator=g)
+    l_a = torch.randn((rows,), generator=g)
+    o_p = torch.randn((rows, D), generator=g).to(torch.bfloat16)
+    l_p = torch.randn((rows,), generator=g)
+    l_a[:10] = float("-inf")
+    o_a[:10] = 0.0
+    l_p[10:20] = float("-inf")
+    l_a[20:30] = float("-inf")
+    l_p[20:30] = float("-inf")
+    o_a[20:30] = 0.0
+    acc, lacc = o_a.clone().cuda(), l_a.clone().cuda()
+    attn.attn_lse_merge(acc, lacc, o_p.cuda(), l_p.cuda())
+    torch.cuda.synchronize()
+    acc, lacc = acc.cpu(), lacc.cpu()
+    assert torch.equal(acc[:10], o_p[:10].float()) and torch.equal(lacc[:10], l_p[:10])   # empty accumulator
+    assert torch.equal(acc[10:20], o_a[10:20]) and torch.equal(lacc[10:20], l_a[10:20])   # empty part
+    assert torch.equal(acc[20:30], o_a[20:30]) and bool(torch.isneginf(lacc[20:30]).all())  # both empty
+    m = torch.maximum(l_a[30:], l_p[30:]).double()
+    wa, wp = torch.exp(l_a[30:].double() - m), torch.exp(l_p[30:].double() - m)
+    want = (wa[:, None] * o_a[30:].double() + wp[:, None] * o_p[30:].double()) / (wa + wp)[:, None]
+    assert torch.allclose(acc[30:].double(), want, rtol=1e-5, atol=1e-5)
+    assert torch.allclose(lacc[30:].double(), m + torch.log(wa + wp), rtol=0, atol=1e-5)
+
+
+@pytest.mark.parametrize("world,S,causal", [(4, 128, True), (3, 100, True), (2, 64, False)])
+def test_ring_schedule_on_one_gpu_matches_oracle(world, S, causal):
+    """Every virtual rank runs its schedule's blocks through attn_fwd and attn_lse_merge."""
+    w = inputs.custom(1, 8, 2, world * S, world * S, 128, causal, seed=world * S)
+    q, k, v = (t.cuda() for t in inputs.generate(w))
+    ro, rl = oracle.attention(*(t.cpu() for t in (q, k, v)), w.scale, causal)
+    for rank in range(world):
+        sl = slice(rank * S, (rank + 1) * S)
+        qr = q[:, :, sl].contiguous()
+        o_acc = torch.zeros(qr.shape, dtype=torch.float32, device="cuda")
+        lse_acc = torch.full(qr.shape[:-1], float("-inf"), dtype=torch.float32, device="cuda")
+        out = torch.empty(qr.shape, dtype=torch.bfloat16, device="cuda")
+        sched = ring_schedule(rank, world, causal)
+        last = max(t for t, _, mode in sched if mode != SKIP)
+        for t, j, mode in sched:
+            if mode == SKIP:
+                continue
+            kj = k[:, :, j * S:(j + 1) * S].contiguous()
+            vj = v[:, :, j * S:(j + 1) * S].contiguous()
+            o_p, l_p = attn.attn_fwd(qr, kj, vj, scale=w.scale, causal=(mode == DIAG))
+            attn.attn_lse_merge(o_acc, lse_acc, o_p, l_p, out=out if t == last else None)
+        torch.cuda.synchronize()
+        rep = compare(out, lse_acc, ro[:, :, sl], rl[:, :, sl])
+        assert rep.ok(), f"rank {rank}: {rep}"
+
+
+def test_ring_driver_with_one_rank_equals_attn_fwd():
+    import torch.distributed as dist
+
+    from causal_attention_attn_b200.ring import ring_attention
+
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=0, world_size=1, timeout=datetime.timedelta(seconds=60))
+    try:
+        w = inputs.custom(1, 4, 2, 200, 200, 128, True, seed=4)
+        q, k, v = (t.cuda() for t in inputs.generate(w))
+        o, lse = ring_attention(q, k, v, scale=w.scale, causal=True)
+        ro, rl = oracle.attention(*(t.cpu() for t in (q, k, v)), w.scale, True)
+        rep = compare(o, lse, ro, rl)
+        assert rep.ok(), str(rep)
+    finally:
+        dist.destroy_process_group()
