@@ -128,3 +128,40 @@ def test_ring_driver_with_one_rank_equals_attn_fwd():
         assert rep.ok(), str(rep)
     finally:
         dist.destroy_process_group()
+
+
+def test_merge_reproduces_the_pages_online_softmax_example():
+    """The blocks [2, 1] and [3, 0] of the worked online-softmax example ("05 · Tích vô hướng,
+    Softmax và toán của Attention", §6), with one-hot value rows so that O is the weight vector:
+    the partial LSEs ln(e^2 + e) and ln(e^3 + 1) merge to ln(e^2 + e + e^3 + 1) = 3.440190 and O to
+    softmax(2, 1, 3, 0)."""
+    import json
+    import math
+
+    with open(os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "pages_worked_examples.json")) as f:
+        blocks = json.load(f)["online_softmax_blocks"]["blocks"]
+    D = 32
+
+    def partial(scores, first_key):
+        lse = math.log(sum(math.exp(s) for s in scores))
+        o = torch.zeros(D)
+        for n, s in enumerate(scores):
+            o[first_key + n] = math.exp(s - lse)  # value row of key j is the unit vector e_j
+        return o.to(torch.bfloat16), lse
+
+    (o1, l1), (o2, l2) = partial(blocks[0], 0), partial(blocks[1], len(blocks[0]))
+    o_acc = o1.float().reshape(1, D).cuda()
+    lse_acc = torch.tensor([l1], dtype=torch.float32, device="cuda")
+    out = torch.empty((1, D), dtype=torch.bfloat16, device="cuda")
+    attn.attn_lse_merge(o_acc, lse_acc, o2.reshape(1, D).cuda(), torch.tensor([l2], dtype=torch.float32, device="cuda"),
+                        out=out)
+    torch.cuda.synchronize()
+    scores = blocks[0] + blocks[1]
+    want_lse = math.log(sum(math.exp(s) for s in scores))
+    assert abs(want_lse - 3.440190) < 1e-6
+    assert abs(lse_acc.item() - want_lse) < 1e-5
+    want = [math.exp(s - want_lse) for s in scores]
+    got = out.float().cpu()[0]
+    for j, wj in enumerate(want):
+        assert abs(got[j].item() - wj) <= 5e-3 * wj, (j, got[j].item(), wj)  # two bf16 roundings: <= 2^-8
+    assert torch.all(got[len(scores):] == 0)
