@@ -180,3 +180,26 @@ MERGE_CASES = [
 @pytest.mark.parametrize("name,ptrs,rows,D,expected", MERGE_CASES, ids=[c[0] for c in MERGE_CASES])
 def test_lse_merge_argument_errors(lib, name, ptrs, rows, D, expected):
     assert lib.attn_lse_merge(*ptrs, rows, D, None) == expected, name
+
+
+# attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Sq, Skv, D, scale, causal, stream)
+BWD_PTRS = [A[0], A[1], A[2], A[3], A[4], A[0] + 0x100000, A[1] + 0x100000, A[2] + 0x100000, A[3] + 0x100000]
+BWD_GOOD = (1, 4, 2, 128, 128, 128, 0.1, 1)
+BWD_CASES = [
+    ("null dout", 4, 0, BWD_GOOD, -1),
+    ("null dv", 8, 0, BWD_GOOD, -1),
+    ("null q", 0, 0, BWD_GOOD, -1),
+    ("head dim 64", None, None, (1, 4, 2, 128, 128, 64, 0.1, 1), -4),
+    ("gqa not divisible", None, None, (1, 6, 4, 128, 128, 128, 0.1, 1), -3),
+    ("causal with Sq > Skv", None, None, (1, 4, 2, 129, 128, 128, 0.1, 1), -6),
+    ("misaligned dq", 6, A[1] + 0x100000 + 4, BWD_GOOD, -5),
+    ("zero scale", None, None, (1, 4, 2, 128, 128, 128, 0.0, 1), -11),
+]
+
+
+@pytest.mark.parametrize("name,slot,value,args,expected", BWD_CASES, ids=[c[0] for c in BWD_CASES])
+def test_bwd_argument_errors(lib, name, slot, value, args, expected):
+    ptrs = list(BWD_PTRS)
+    if slot is not None:
+        ptrs[slot] = value
+    assert lib.attn_bwd(*ptrs, *args, None) == expected, name
