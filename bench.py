@@ -313,6 +313,13 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     fp8_ms = ranks.max([sum(a.elapsed_time(b) for a, b in fev)])[0]
     fp8_launch_s = fp8_ms * 1e-3 / fp8_steps
+
+    # The backward pass of the prefill workload (dq, dk, dv from dout and the forward's o, lse),
+    # timed the same way. Reported beside the step, not part of it.
+    try:
+        backward = backward_leg(attn, args, ranks, dev, stream, clear_l2, pq, pk, pv, po, pl, world)
+    except Exception as e:  # an extra leg that fails is reported in its object, not allowed to drop the line
+        backward = {"metric": "backward TFLOP/s (dq, dk, dv)", "error": f"{type(e).__name__}: {e}"}
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
     d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
 
@@ -349,6 +356,7 @@ def run_ours(args):
                 "us_per_launch": fp8_launch_s * 1e6,
                 "bytes_per_launch": fp8_bytes,
             },
+            "backward": backward,
             "prefill_us_per_launch": pre_launch_s * 1e6,
             "timed_region_ms": region_ms,
             "e2e": {"value": e2e_tflops, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -404,6 +412,42 @@ def read_traffic(kernel: str, workload: str):
         return entry.get("dram_bytes_per_launch")
     except (OSError, ValueError):
         return None
+
+
+def backward_leg(attn, args, ranks, dev, stream, clear_l2, q, k, v, o, lse, world):
+    """Time attn_bwd on the prefill workload: inputs resident, L2 flushed before every launch, CUDA
+    events around each launch, max over ranks. FLOPs: five products of 2*D per visible pair (S, dP,
+    dV, dK, dQ), 2.5x the forward's. Returns the JSON object of the leg."""
+    peaks, peak_kind = load_peaks()
+    tensor_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    flops = 5 * PREFILL.flops() // 2
+    g = torch.Generator().manual_seed(7)
+    dout = torch.randn(q.shape, generator=g).to(torch.bfloat16).to(dev)
+    attn.attn_fwd(q, k, v, scale=PREFILL.scale, causal=True, out=o, lse=lse, stream=stream)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    for _ in range(args.warmup):
+        clear_l2()
+        attn.attn_bwd(q, k, v, o, lse, dout, scale=PREFILL.scale, causal=True, dq=dq, dk=dk, dv=dv, stream=stream)
+    steps = max(3, min(args.steps, 20))
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+    ranks.barrier()
+    torch.cuda.synchronize(dev)
+    for s in range(steps):
+        clear_l2()
+        ev[s][0].record(stream)
+        attn.attn_bwd(q, k, v, o, lse, dout, scale=PREFILL.scale, causal=True, dq=dq, dk=dk, dv=dv, stream=stream)
+        ev[s][1].record(stream)
+    torch.cuda.synchronize(dev)
+    ms = ranks.max([sum(a.elapsed_time(b) for a, b in ev)])[0]
+    launch_s = ms * 1e-3 / steps
+    achieved = flops / launch_s / 1e12
+    return {"metric": "backward TFLOP/s (dq, dk, dv)", "value": whole_job_rate(world, flops, launch_s) / 1e12,
+            "unit": "TFLOP/s", "config": PREFILL.config(), "steps": steps,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": tensor_peak, "unit": "TFLOP/s",
+                         "frac": achieved / tensor_peak, "traffic": None,
+                         "peak_kind": f"{peak_kind} bf16 dense (burst)", "kernel": "bwd_kernel"},
+            "us_per_launch": launch_s * 1e6, "flops_per_launch": flops,
+            "device_status": attn.device_status(stream)}
 
 
 def fp8_decode_bytes(w) -> int:
