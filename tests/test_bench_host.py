@@ -1,0 +1,72 @@
+"""Host logic of ``bench.py``'s extra legs on the CPU: the backward leg run with a stand-in library
+and stand-in CUDA events (every launch "takes" 1 ms), checking the call sequence and the arithmetic
+of its JSON object. No kernel runs here; the GPU runs of the bench exercise the real library."""
+import os
+import sys
+import types
+
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+
+class _Event:
+    clock = 0.0
+
+    def __init__(self, enable_timing=True):
+        self.t = None
+
+    def record(self, stream=None):
+        _Event.clock += 1.0  # ms: a launch's start and end events are 1 ms apart
+        self.t = _Event.clock
+
+    def elapsed_time(self, other):
+        return other.t - self.t
+
+
+def test_backward_leg_reports_rate_and_roofline(monkeypatch):
+    import bench
+
+    calls = []
+    fake = types.SimpleNamespace(
+        attn_fwd=lambda *a, **kw: calls.append("fwd"),
+        attn_bwd=lambda *a, **kw: calls.append("bwd"),
+        device_status=lambda stream=None: 0,
+    )
+    monkeypatch.setattr(torch.cuda, "Event", _Event)
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda *a, **kw: None)
+    args = types.SimpleNamespace(steps=2000, warmup=3)
+    ranks = bench.Ranks(1, torch.device("cpu"))
+    w = bench.PREFILL
+    q = torch.zeros((1, 1, 1, 1), dtype=torch.bfloat16)  # shapes only matter to the real library
+    flushes = []
+    out = bench.backward_leg(fake, args, ranks, torch.device("cpu"), None, lambda: flushes.append(1), q, q, q, q,
+                             torch.zeros((1, 1, 1)), world=1)
+    assert calls == ["fwd"] + ["bwd"] * (3 + 20)  # forward once, warm-up, then 20 timed launches
+    assert len(flushes) == 3 + 20  # L2 flushed before every launch
+    assert out["steps"] == 20 and out["device_status"] == 0
+    flops = 5 * w.flops() // 2
+    assert out["flops_per_launch"] == flops
+    # each timed launch spans 1 ms between its events in the stand-in clock
+    assert abs(out["us_per_launch"] - 1000.0) < 1e-9
+    assert abs(out["value"] - flops / 1e-3 / 1e12) < 1e-6
+    assert abs(out["roofline"]["frac"] - out["roofline"]["achieved"] / out["roofline"]["peak"]) < 1e-12
+    assert out["roofline"]["bound"] == "tensor" and out["roofline"]["traffic"] is None
+
+
+def test_whole_job_rate_scales_with_ranks_for_the_backward_leg(monkeypatch):
+    import bench
+
+    fake = types.SimpleNamespace(attn_fwd=lambda *a, **kw: None, attn_bwd=lambda *a, **kw: None,
+                                 device_status=lambda stream=None: 0)
+    monkeypatch.setattr(torch.cuda, "Event", _Event)
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda *a, **kw: None)
+    ranks = bench.Ranks(1, torch.device("cpu"))
+    q = torch.zeros((1, 1, 1, 1), dtype=torch.bfloat16)
+    args = types.SimpleNamespace(steps=5, warmup=3)
+    one = bench.backward_leg(fake, args, ranks, torch.device("cpu"), None, lambda: None, q, q, q, q,
+                             torch.zeros((1, 1, 1)), world=1)
+    two = bench.backward_leg(fake, args, ranks, torch.device("cpu"), None, lambda: None, q, q, q, q,
+                             torch.zeros((1, 1, 1)), world=2)
+    assert one["steps"] == 5 and abs(two["value"] - 2 * one["value"]) < 1e-9
