@@ -59,3 +59,40 @@ def test_backward_matches_oracle(shape):
         assert np.isfinite(g).all(), name
         assert err.max() <= 1e-2 * top and err.mean() <= 1e-3 * top, (
             f"{name}: max|err| {err.max():.3e} mean|err| {err.mean():.3e} vs max|ref| {top:.3e}")
+
+
+def test_backward_reads_and_writes_only_in_bounds():
+    """q, k, v, o, dout and lse inside NaN-filled buffers, dq, dk, dv inside sentinel-filled ones:
+    no NaN may leak into the gradients (nothing outside the tensors is read, ragged tails included)
+    and the sentinels must survive (nothing is written out of bounds)."""
+    B, Hq, Hkv, Sq, Skv = 1, 4, 2, 300, 300
+    w = inputs.custom(B, Hq, Hkv, Sq, Skv, 128, True, seed=sum((B, Hq, Hkv, Sq, Skv)))
+    q, k, v = inputs.generate(w)
+    dout = torch.randn(q.shape, generator=torch.Generator().manual_seed(7)).to(torch.bfloat16)
+    pad = 4096
+
+    def inside(t, fill):
+        buf = torch.full((2 * pad + t.numel(),), fill, dtype=t.dtype, device="cuda")
+        buf[pad:pad + t.numel()] = t.reshape(-1).to("cuda")
+        return buf, buf[pad:pad + t.numel()].view(t.shape)
+
+    nan = float("nan")
+    _, qd = inside(q, nan)
+    _, kd = inside(k, nan)
+    _, vd = inside(v, nan)
+    _, dd = inside(dout, nan)
+    o, lse = attn.attn_fwd(qd, kd, vd, scale=w.scale, causal=True)
+    _, od = inside(o, nan)
+    _, lsed = inside(lse, nan)
+    bufs = [inside(torch.full(t.shape, 7.0, dtype=torch.bfloat16), 7.0) for t in (q, k, v)]
+    attn.attn_bwd(qd, kd, vd, od, lsed, dd, scale=w.scale, causal=True, dq=bufs[0][1], dk=bufs[1][1], dv=bufs[2][1])
+    torch.cuda.synchronize()
+    ref = oracle.attention_bwd(q, k, v, dout, w.scale, True)
+    for (buf, view), want, name in zip(bufs, ref, ("dq", "dk", "dv")):
+        n = view.numel()
+        assert (buf[:pad] == 7.0).all() and (buf[pad + n:] == 7.0).all(), name
+        g = view.cpu().double().numpy()
+        assert np.isfinite(g).all(), name
+        err = np.abs(g - want)
+        top = np.abs(want).max()
+        assert err.max() <= 1e-2 * top and err.mean() <= 1e-3 * top, name

@@ -159,3 +159,32 @@ def test_paged_fp8_decode_matches_oracle(case):
             assert rep.o_max_ulps <= 0.5 + 1e-6 and rep.lse_max_abs <= 1e-3, f"batch {b} (length 1): {rep}"
             continue
         assert rep.ok(), f"batch {b} (length {n}): {rep}"
+
+
+def test_fp8_decode_reads_and_writes_only_in_bounds():
+    """The e4m3 cache sits inside buffers of NaN codes and the coefficient tables inside NaN floats;
+    O and LSE inside sentinel-filled buffers: no NaN may leak in (nothing past Skv or past the
+    tables is read) and the sentinels must survive (nothing is written out of bounds)."""
+    B, Hq, Hkv, Skv = 1, 4, 2, 333
+    w = inputs.custom(B, Hq, Hkv, 1, Skv, 128, True, seed=333)
+    q, k8, v8, ks, vs = inputs.generate_fp8(w)
+    pad = 4096
+
+    def inside(t, fill):
+        buf = torch.full((2 * pad + t.numel(),), fill, dtype=t.dtype, device="cuda")
+        buf[pad:pad + t.numel()] = t.reshape(-1).cuda()
+        return buf, buf[pad:pad + t.numel()].view(t.shape)
+
+    _, kd = inside(k8, E4M3_NAN)
+    _, vd = inside(v8, E4M3_NAN)
+    _, ksd = inside(ks, float("nan"))
+    _, vsd = inside(vs, float("nan"))
+    obuf, od = inside(torch.full(q.shape, 7.0, dtype=torch.bfloat16), 7.0)
+    lbuf, ld = inside(torch.full((B, Hq, 1), 7.0), 7.0)
+    attn.attn_decode_fp8(q.cuda(), kd, vd, ksd, vsd, scale=w.scale, out=od, lse=ld)
+    torch.cuda.synchronize()
+    assert torch.isfinite(od.float()).all() and torch.isfinite(ld).all()
+    assert (obuf[:pad] == 7.0).all() and (obuf[pad + q.numel():] == 7.0).all()
+    assert (lbuf[:pad] == 7.0).all() and (lbuf[pad + B * Hq:] == 7.0).all()
+    rep = compare(od, ld, *oracle.attention_fp8kv(q, k8, v8, ks, vs, w.scale, True))
+    assert rep.ok(), str(rep)

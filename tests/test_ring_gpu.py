@@ -165,3 +165,33 @@ def test_merge_reproduces_the_pages_online_softmax_example():
     for j, wj in enumerate(want):
         assert abs(got[j].item() - wj) <= 5e-3 * wj, (j, got[j].item(), wj)  # two bf16 roundings: <= 2^-8
     assert torch.all(got[len(scores):] == 0)
+
+
+def test_merge_reads_and_writes_only_in_bounds():
+    """The part inside NaN-filled buffers, the accumulator and the output inside sentinel-filled
+    ones: the sentinels must survive and no NaN may leak into the merged rows."""
+    rows, D, pad = 37, 128, 4096
+    g = torch.Generator().manual_seed(2)
+    o_a, l_a = torch.randn((rows, D), generator=g), torch.randn((rows,), generator=g)
+    o_p, l_p = torch.randn((rows, D), generator=g).to(torch.bfloat16), torch.randn((rows,), generator=g)
+
+    def inside(t, fill):
+        buf = torch.full((2 * pad + t.numel(),), fill, dtype=t.dtype, device="cuda")
+        buf[pad:pad + t.numel()] = t.reshape(-1).cuda()
+        return buf, buf[pad:pad + t.numel()].view(t.shape)
+
+    abuf, acc = inside(o_a, 7.0)
+    lbuf, lacc = inside(l_a, 7.0)
+    _, part = inside(o_p, float("nan"))
+    _, lpart = inside(l_p, float("nan"))
+    obuf, out = inside(torch.full((rows, D), 7.0, dtype=torch.bfloat16), 7.0)
+    attn.attn_lse_merge(acc, lacc, part, lpart, out=out)
+    torch.cuda.synchronize()
+    for buf, n in ((abuf, rows * D), (lbuf, rows), (obuf, rows * D)):
+        assert (buf[:pad] == 7.0).all() and (buf[pad + n:] == 7.0).all()
+    assert torch.isfinite(acc).all() and torch.isfinite(lacc).all() and torch.isfinite(out.float()).all()
+    m = torch.maximum(l_a, l_p).double()
+    wa, wp = torch.exp(l_a.double() - m), torch.exp(l_p.double() - m)
+    want = (wa[:, None] * o_a.double() + wp[:, None] * o_p.double()) / (wa + wp)[:, None]
+    assert torch.allclose(acc.cpu().double(), want, rtol=1e-5, atol=1e-5)
+    assert torch.allclose(out.cpu().double(), want, rtol=2.0 ** -8, atol=1e-6)
