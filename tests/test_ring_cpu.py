@@ -1,7 +1,7 @@
-"""Ring (context-parallel) attention on the CPU: the schedule, and the distributed driver run by two
+"""Ring (context-parallel) attention on the CPU: the schedule, and the distributed ring loop run by two
 and three gloo ranks against the oracle over the whole sequence.
 
-The driver (``causal_attention_attn_b200.ring.ring_attention``) is the one the GPUs run; only the
+The ring loop (``causal_attention_attn_b200.ring.ring_attention``) is the one the GPUs run; only the
 per-block compute and the merge are replaced here by CPU stand-ins: the oracle for a block's
 attention (its O rounded to bf16 and its LSE to fp32, as the GPU kernel returns them) and the LSE
 merge written out in fp64. The schedule, the exchange and the bookkeeping are the product's.

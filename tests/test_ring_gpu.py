@@ -2,7 +2,7 @@
 
 Every run here has one GPU, so no test waits on another rank: the ring's schedule is emulated on
 one GPU (the chunks are indexed instead of received), which runs exactly the kernels and the
-merge order a rank runs; the distributed driver itself is run with one rank, and with two and
+merge order a rank runs; the distributed ring loop itself is run with one rank, and with two and
 three gloo ranks on the CPU in ``test_ring_cpu.py``.
 """
 import datetime
@@ -108,7 +108,7 @@ def test_ring_schedule_on_one_gpu_matches_oracle(world, S, causal):
         assert rep.ok(), f"rank {rank}: {rep}"
 
 
-def test_ring_driver_with_one_rank_equals_attn_fwd():
+def test_ring_loop_with_one_rank_equals_attn_fwd():
     import torch.distributed as dist
 
     from causal_attention_attn_b200.ring import ring_attention
