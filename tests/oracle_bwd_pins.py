@@ -6,6 +6,8 @@ Kinds of pin:
   * numerical derivative: central differences of an independent numpy forward (a materialised
     score matrix with an explicit cache-aligned mask, softmax, weighted sum of V) on tiny shapes,
     for every element of q, k and v;
+  * the exact derivative: torch autograd in fp64 through a materialised forward (score matrix,
+    explicit cache-aligned mask, softmax, weighted sum of V), written independently of the oracle;
   * invariants that follow from the softmax: every row of dS sums to zero, so the key gradients sum
     to zero and a shift of every key by the same vector changes no gradient; every row of P sums to
     one, so the value gradients sum to the sum of dO over the rows that read them.
@@ -127,7 +129,39 @@ def pin_bwd_key_shift_changes_nothing(lib):
         assert np.abs(a - b).max() < 1e-12
 
 
+def _autograd_check(lib, B, Hq, Hkv, Sq, Skv, D, causal, seed):
+    q = _rand_bf16((B, Hq, Sq, D), seed)
+    k = _rand_bf16((B, Hkv, Skv, D), seed + 1)
+    v = _rand_bf16((B, Hkv, Skv, D), seed + 2)
+    do = _rand_bf16((B, Hq, Sq, D), seed + 3)
+    scale = float(np.float32(D ** -0.5))
+    got = oracle.attention_bwd(q, k, v, do, scale, causal, lib=lib)
+    qt, kt, vt = (t.double().requires_grad_(True) for t in (q, k, v))
+    g = Hq // Hkv
+    kr, vr = kt.repeat_interleave(g, dim=1), vt.repeat_interleave(g, dim=1)  # query head h reads kv head h // g
+    s = scale * qt @ kr.transpose(-1, -2)
+    i = torch.arange(Sq)[:, None]
+    j = torch.arange(Skv)[None, :]
+    visible = (j <= i + (Skv - Sq)) if causal else torch.ones((Sq, Skv), dtype=torch.bool)
+    p = torch.softmax(s.masked_fill(~visible, float("-inf")), dim=-1)
+    ((p @ vr) * do.double()).sum().backward()
+    for name, mine, ref in zip(("dq", "dk", "dv"), got, (qt.grad, kt.grad, vt.grad)):
+        err = np.abs(mine - ref.numpy()).max()
+        assert err <= 1e-12 * max(1.0, np.abs(ref.numpy()).max()), (name, err)
+
+
+def pin_bwd_autograd_causal_gqa_cached(lib):
+    # GQA group 3, a cache offset of 5 (Sq = 7 over Skv = 12), causal
+    _autograd_check(lib, 2, 6, 2, 7, 12, 16, True, seed=71)
+
+
+def pin_bwd_autograd_noncausal_more_queries(lib):
+    _autograd_check(lib, 1, 4, 1, 9, 5, 8, False, seed=81)
+
+
 BWD_PINS = [
+    pin_bwd_autograd_causal_gqa_cached,
+    pin_bwd_autograd_noncausal_more_queries,
     pin_bwd_finite_differences_causal_gqa,
     pin_bwd_finite_differences_noncausal,
     pin_bwd_finite_differences_square_causal,
