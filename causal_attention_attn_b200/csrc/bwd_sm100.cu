@@ -128,27 +128,29 @@ __device__ __forceinline__ int first_qtile(const BwdParams &p, int k0)
     return q_min <= 0 ? 0 : q_min / kBQ;
 }
 
+// One warp per query row (grid-stride, 64-bit row indices): D_i = dO_i . O_i and lse_i in log2 units.
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16 *o, const __nv_bfloat16 *dout,
-                                                     const float *lse, float *vec, int rows, int Sq, int Sq_pad,
-                                                     int total_pad)
+                                                     const float *lse, float *vec, long long rows, int Sq, int Sq_pad,
+                                                     size_t total_pad)
 {
-    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
-    if (warp >= rows)
-        return;
-    const uint2 a = reinterpret_cast<const uint2 *>(o + static_cast<size_t>(warp) * kD)[lane];
-    const uint2 b = reinterpret_cast<const uint2 *>(dout + static_cast<size_t>(warp) * kD)[lane];
-    auto lo = [](uint32_t w) { return __uint_as_float(w << 16); };
-    auto hi = [](uint32_t w) { return __uint_as_float(w & 0xffff0000u); };
-    float d = lo(a.x) * lo(b.x) + hi(a.x) * hi(b.x) + lo(a.y) * lo(b.y) + hi(a.y) * hi(b.y);
+    const long long n_warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
+    for (long long row = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; row < rows;
+         row += n_warps) {
+        const uint2 a = reinterpret_cast<const uint2 *>(o + static_cast<size_t>(row) * kD)[lane];
+        const uint2 b = reinterpret_cast<const uint2 *>(dout + static_cast<size_t>(row) * kD)[lane];
+        auto lo = [](uint32_t w) { return __uint_as_float(w << 16); };
+        auto hi = [](uint32_t w) { return __uint_as_float(w & 0xffff0000u); };
+        float d = lo(a.x) * lo(b.x) + hi(a.x) * hi(b.x) + lo(a.y) * lo(b.y) + hi(a.y) * hi(b.y);
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1)
-        d += __shfl_xor_sync(0xffffffffu, d, off);
-    if (lane == 0) {
-        const int bh = warp / Sq, i = warp % Sq;
-        const size_t idx = static_cast<size_t>(bh) * Sq_pad + i;
-        vec[idx] = lse[warp] * kLog2e;
-        vec[static_cast<size_t>(total_pad) + idx] = d;
+        for (int off = 16; off > 0; off >>= 1)
+            d += __shfl_xor_sync(0xffffffffu, d, off);
+        if (lane == 0) {
+            const long long bh = row / Sq, i = row % Sq;
+            const size_t idx = static_cast<size_t>(bh) * Sq_pad + static_cast<size_t>(i);
+            vec[idx] = lse[row] * kLog2e;
+            vec[total_pad + idx] = d;
+        }
     }
 }
 
@@ -468,12 +470,15 @@ cudaError_t launch_bwd(const BwdArgs &a, cudaStream_t stream, int *encode_error)
 {
     if (a.D != kD)
         return cudaErrorInvalidValue;
-    static bool attr_set = false;
-    if (!attr_set) {
+    static bool attr_set[kMaxDevices] = {};  // per device: the attribute applies to the current one
+    const int dev = current_device_index();
+    if (dev < 0)
+        return cudaErrorInvalidDevice;
+    if (!attr_set[dev]) {
         cudaError_t e = cudaFuncSetAttribute(bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
         if (e != cudaSuccess)
             return e;
-        attr_set = true;
+        attr_set[dev] = true;
     }
     auto encode = get_encode_fn();
     if (!encode) {
@@ -494,10 +499,11 @@ cudaError_t launch_bwd(const BwdArgs &a, cudaStream_t stream, int *encode_error)
     cudaError_t e = cudaMemsetAsync(dq_acc, 0, rows * kD * sizeof(float), stream);
     if (e != cudaSuccess)
         return e;
-    const int total_pad = a.B * a.Hq * Sq_pad;
-    bwd_pre_kernel<<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0, stream>>>(
+    const size_t total_pad = static_cast<size_t>(a.B) * a.Hq * Sq_pad;
+    const size_t pre_blocks = (rows + 7) / 8;  // eight warps (rows) per block, at most 64K blocks (grid-stride)
+    bwd_pre_kernel<<<static_cast<unsigned>(pre_blocks < 65536 ? pre_blocks : 65536), 256, 0, stream>>>(
         static_cast<const __nv_bfloat16 *>(a.o), static_cast<const __nv_bfloat16 *>(a.dout), a.lse, vec,
-        static_cast<int>(rows), a.Sq, Sq_pad, total_pad);
+        static_cast<long long>(rows), a.Sq, Sq_pad, total_pad);
     if ((e = cudaGetLastError()) != cudaSuccess)
         return e;
 

@@ -621,7 +621,11 @@ template <int D, int G>
 cudaError_t prepare_dg(int *ctas_per_sm)
 {
     using C = DecCfg<D, G>;
-    static int cached = 0;
+    static int cached_per_dev[kMaxDevices] = {};  // per device: attributes apply to the current one
+    const int dev = current_device_index();
+    if (dev < 0)
+        return cudaErrorInvalidDevice;
+    int &cached = cached_per_dev[dev];
     if (cached == 0) {
         cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
         if (e == cudaSuccess)

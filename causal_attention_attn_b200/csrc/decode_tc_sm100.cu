@@ -433,7 +433,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int e = (lane < n_box) ? key / p.page_size : e0;
                 int page = __shfl_sync(0xffffffffu, tab_val, e - tab_base);
                 if (lane < n_box) {
-                    if (key >= batch_len[b])
+                    // Keys past the length, and a table entry outside [0, num_pages) (which could
+                    // otherwise wrap page * Hkv onto another sequence's page), read the zero-filled
+                    // page beyond the last one.
+                    if (key >= batch_len[b] || page < 0 || page >= p.num_pages)
                         page = p.num_pages;
                     const int coord = static_cast<int>(static_cast<long long>(page) * p.Hkv + kvh);
                     const int in_page = key % p.page_size;
@@ -692,8 +695,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 lpv[h] = 0.f;
             }
             for (int j = 0; j < n_chunks; ++j, ++c) {
-                const bool okw = mbar_wait(BAR(kBarSFull0 + (c & 1)), static_cast<uint32_t>(c >> 1) & 1u, abort_flag,
-                                           p.status, kSiteDecodeConsumer);
+                // Agreed by the warp: it gates the warp-collective TMEM load.
+                const bool okw = __all_sync(0xffffffffu, mbar_wait(BAR(kBarSFull0 + (c & 1)), static_cast<uint32_t>(c >> 1) & 1u,
+                                                                   abort_flag, p.status, kSiteDecodeConsumer));
                 float x[G];
                 if (okw) {
                     tc_fence_after_sync();
@@ -738,8 +742,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         l[h] *= alpha[h];
                         lpv[h] *= alpha[h];
                     }
-                    if (mbar_wait(BAR(kBarODone0 + ((c - 1) & 1)), static_cast<uint32_t>((c - 1) >> 1) & 1u,
-                                  abort_flag, p.status, kSiteDecodeConsumer)) {
+                    if (__all_sync(0xffffffffu, mbar_wait(BAR(kBarODone0 + ((c - 1) & 1)),
+                                                          static_cast<uint32_t>((c - 1) >> 1) & 1u, abort_flag,
+                                                          p.status, kSiteDecodeConsumer))) {
                         tc_fence_after_sync();
                         uint32_t ov[16];
                         tmem_ld16_wait(tO, ov);
@@ -963,8 +968,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int G, bool kPaged, bool kFp8>
 cudaError_t prepare_g(int *ctas_per_sm)
 {
-    static int cached = 0;
+    static int cached_per_dev[kMaxDevices] = {};  // per device: attributes apply to the current one
     constexpr int kSmem = Lay<kFp8>::kSmem;
+    const int dev = current_device_index();
+    if (dev < 0)
+        return cudaErrorInvalidDevice;
+    int &cached = cached_per_dev[dev];
     if (cached == 0) {
         cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<G, kPaged, kFp8>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);

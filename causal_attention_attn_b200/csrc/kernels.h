@@ -8,6 +8,22 @@
 
 namespace attn_b200 {
 
+// Devices the library keeps state for (function attributes, occupancy, workspaces), by index.
+constexpr int kMaxDevices = 64;
+
+// Index of the current device, or -1 if it cannot be read or is kMaxDevices or beyond. Function
+// attributes such as the dynamic shared-memory limit take effect on the device that is current
+// when they are set, so the launchers keep them per device.
+inline int current_device_index()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return -1;
+    }
+    return (dev >= 0 && dev < kMaxDevices) ? dev : -1;
+}
+
 // Device status word values: 0 = fine, otherwise the site of the first wait that ran out.
 enum WaitSite : int {
     kSiteNone = 0,
@@ -110,5 +126,9 @@ constexpr int kPagedMaxBatch = 1024;  // batch entries a paged decode may have (
 cudaError_t decode_plan_paged(int B, int Hq, int Hkv, int max_seq_len, int requested_ctas, int sm_count,
                               DecodePlan *plan);
 cudaError_t launch_decode_tc(const DecodeArgs &a, cudaStream_t stream);
+
+// The status word of attn_decode_noalloc's fixed scratch array on the current device, or nullptr
+// if that entry point has not run on it (its address is only looked up by its first call there).
+int *noalloc_status_word();
 
 }  // namespace attn_b200

@@ -409,8 +409,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
 
         for (int j = 0; j < n; ++j) {
-            if (!(ok = mbar_wait(BAR(kBarSFull0 + x), static_cast<uint32_t>(j) & 1u, abort_flag, p.status,
-                                 kSitePrefillSoftmaxSFull)))
+            // The wait's result gates the warp-collective TMEM load below: the warp agrees on it.
+            if (!(ok = __all_sync(0xffffffffu, mbar_wait(BAR(kBarSFull0 + x), static_cast<uint32_t>(j) & 1u,
+                                                         abort_flag, p.status, kSitePrefillSoftmaxSFull))))
                 break;
             tc_fence_after_sync();
             uint32_t s_raw[kBN];
@@ -505,7 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
 
         if (ok && n > 0)
-            ok = mbar_wait(BAR(kBarOFinal0 + x), 0, abort_flag, p.status, kSitePrefillEpilogue);
+            ok = __all_sync(0xffffffffu, mbar_wait(BAR(kBarOFinal0 + x), 0, abort_flag, p.status, kSitePrefillEpilogue));
         if (ok && n > 0) {
             tc_fence_after_sync();
             const float inv_l = 1.f / l_pv;
@@ -558,8 +559,13 @@ cudaError_t launch(const PrefillArgs &a, cudaStream_t stream, int *encode_error)
         !make_map(encode, &tv, a.v, D, a.Skv, a.B * a.Hkv, C::kChunkElems, 128, swz, encode_error))
         return cudaErrorInvalidValue;
 
-    static bool attr_set = false;  // benign race: every caller sets the same value
-    if (!attr_set) {
+    // Per device: the attribute applies to the device current when it is set (benign race between
+    // host threads: every caller sets the same value).
+    static bool attr_set[kMaxDevices] = {};
+    const int dev = current_device_index();
+    if (dev < 0)
+        return cudaErrorInvalidDevice;
+    if (!attr_set[dev]) {
         // The setmaxnreg split inside the kernel is only valid for the register count it was
         // written for; refuse to launch a build that was compiled to anything else.
         cudaFuncAttributes fa;
@@ -571,7 +577,7 @@ cudaError_t launch(const PrefillArgs &a, cudaStream_t stream, int *encode_error)
         e = cudaFuncSetAttribute(prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
         if (e != cudaSuccess)
             return e;
-        attr_set = true;
+        attr_set[dev] = true;
     }
     Params p;
     p.o = static_cast<__nv_bfloat16 *>(a.o);

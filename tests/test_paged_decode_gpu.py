@@ -101,3 +101,25 @@ def test_paged_lengths_beyond_the_table_are_clamped():
     o_ref, l_ref = oracle.attention(q[:1], k[:1], v[:1], w.scale, True)
     rep = compare(o.cpu()[:1], lse.cpu()[:1], o_ref, l_ref)
     assert rep.ok(), str(rep)
+
+
+def test_table_entries_outside_the_pages_read_as_zeros():
+    """A block-table entry outside [0, num_pages) reads as zeros, even one whose page * Hkv would
+    wrap in 32 bits onto a valid page of another sequence (2^29 + 3 with Hkv = 8 -> page 3)."""
+    B, Hq, Hkv, cap, page_size = 2, 32, 8, 512, 64
+    lens = [512, 300]
+    w = inputs.custom(B, Hq, Hkv, 1, cap, 128, True, seed=78)
+    q, k, v, kp, vp, table, seq_lens = make_paged(w, lens, page_size, seed=4)
+    table[0, 2] = (1 << 29) + 3   # wraps onto page 3 if not range-checked
+    table[1, 1] = -5
+    o, lse = attn.attn_decode_paged(q.cuda(), kp.cuda(), vp.cuda(), table.cuda(), seq_lens.cuda(), max(lens),
+                                    scale=w.scale)
+    torch.cuda.synchronize()
+    o, lse = o.cpu(), lse.cpu()
+    for b, n in ((0, 2), (1, 1)):
+        kz, vz = k[b:b + 1, :, :lens[b]].clone(), v[b:b + 1, :, :lens[b]].clone()
+        kz[:, :, n * page_size:(n + 1) * page_size] = 0
+        vz[:, :, n * page_size:(n + 1) * page_size] = 0
+        o_ref, l_ref = oracle.attention(q[b:b + 1], kz, vz, w.scale, True)
+        rep = compare(o[b:b + 1], lse[b:b + 1], o_ref, l_ref)
+        assert rep.ok(), f"sequence {b}: {rep}"
