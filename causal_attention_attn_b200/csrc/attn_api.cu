@@ -16,8 +16,7 @@
 namespace attn_b200 {
 namespace {
 
-constexpr int kVersion = 400;  // 0.4.0: adds attn_lse_merge (after 0.3.0: attn_bwd, the e4m3 decodes)
-constexpr int kMaxDevices = 64;
+constexpr int kVersion = 500;  // 0.5.0: stream-ordered workspace growth (after 0.4.0: attn_lse_merge)
 
 struct DeviceState {
     bool probed = false;
@@ -95,6 +94,10 @@ DeviceState *device_state(int *err)
 }
 
 // Make sure the workspace holds `counters` ints and `partials` floats (plus the status word).
+// Growth is stream-ordered: the new block comes from the device's stream-ordered pool on `stream`
+// (cudaMallocAsync), is cleared there, and the old block is released on `stream` after the work
+// already queued on it (cudaFreeAsync). Nothing waits on the host. A status word that a kernel set in
+// the old block (a wait that ran out) is carried into the new one on the stream.
 int ensure_workspace(DeviceState &s, size_t counters, size_t partials, cudaStream_t stream)
 {
     if (s.block && counters <= s.counter_count && partials <= s.partial_floats)
@@ -107,26 +110,19 @@ int ensure_workspace(DeviceState &s, size_t counters, size_t partials, cudaStrea
     const size_t cbytes = ((nc * sizeof(int) + 255) / 256) * 256;
     const size_t bytes = head + cbytes + np * sizeof(float);
     void *block = nullptr;
-    if (cudaMalloc(&block, bytes) != cudaSuccess) {
+    if (cudaMallocAsync(&block, bytes, stream) != cudaSuccess) {
         cudaGetLastError();
         return ATTN_ERR_WORKSPACE;
     }
-    // The old block may still be read by queued kernels: wait for the device before freeing it.
-    if (s.block) {
-        if (cudaDeviceSynchronize() != cudaSuccess) {
-            cudaGetLastError();
-            cudaFree(block);
-            return ATTN_ERR_WORKSPACE;
-        }
-        cudaFree(s.block);
-    }
-    if (cudaMemsetAsync(block, 0, head + cbytes, stream) != cudaSuccess) {
+    if (cudaMemsetAsync(block, 0, head + cbytes, stream) != cudaSuccess ||
+        (s.block && cudaMemcpyAsync(block, s.block, sizeof(int), cudaMemcpyDeviceToDevice, stream) != cudaSuccess)) {
         cudaGetLastError();
-        cudaFree(block);
-        s.block = nullptr;
-        s.bytes = s.counter_count = s.partial_floats = 0;
+        cudaFreeAsync(block, stream);
+        cudaGetLastError();
         return ATTN_ERR_WORKSPACE;
     }
+    if (s.block && cudaFreeAsync(s.block, stream) != cudaSuccess)
+        cudaGetLastError();  // the old block stays allocated; nothing reads it any more
     s.block = block;
     s.bytes = bytes;
     s.status = static_cast<int *>(block);
@@ -296,24 +292,30 @@ extern "C" int attn_device_status(void *stream_ptr)
     DeviceState *s = device_state(&err);
     if (!s)
         return err;
-    if (!s->block)
-        return ATTN_OK;
-    int value = 0;
-    if (cudaMemcpyAsync(&value, s->status, sizeof(int), cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
-        cudaStreamSynchronize(stream) != cudaSuccess) {
-        cudaGetLastError();
-        return ATTN_ERR_CUDA;
-    }
-    if (value != 0) {
-        const int zero = 0;
-        if (cudaMemcpyAsync(s->status, &zero, sizeof(int), cudaMemcpyHostToDevice, stream) != cudaSuccess ||
+    // Two status words: the workspace's (every entry point but attn_decode_noalloc) and the one at
+    // the start of attn_decode_noalloc's fixed array (once that entry point has run on this device).
+    int *words[2] = {s->block ? s->status : nullptr, noalloc_status_word()};
+    bool timed_out = false;
+    for (int *word : words) {
+        if (!word)
+            continue;
+        int value = 0;
+        if (cudaMemcpyAsync(&value, word, sizeof(int), cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
             cudaStreamSynchronize(stream) != cudaSuccess) {
             cudaGetLastError();
             return ATTN_ERR_CUDA;
         }
-        return ATTN_ERR_DEVICE_TIMEOUT;
+        if (value != 0) {
+            const int zero = 0;
+            if (cudaMemcpyAsync(word, &zero, sizeof(int), cudaMemcpyHostToDevice, stream) != cudaSuccess ||
+                cudaStreamSynchronize(stream) != cudaSuccess) {
+                cudaGetLastError();
+                return ATTN_ERR_CUDA;
+            }
+            timed_out = true;
+        }
     }
-    return ATTN_OK;
+    return timed_out ? ATTN_ERR_DEVICE_TIMEOUT : ATTN_OK;
 }
 
 namespace {
@@ -530,20 +532,15 @@ extern "C" int attn_bwd(const void *q, const void *k, const void *v, const void 
         return rc;
     const size_t need = bwd_workspace_bytes(B, Hq, Sq, D);
     if (s->bwd_bytes < need) {
+        // Stream-ordered, as for the forward workspace: the old block is released on `stream` after
+        // the work queued on it; nothing waits on the host.
         void *block = nullptr;
-        if (cudaMalloc(&block, need) != cudaSuccess) {
+        if (cudaMallocAsync(&block, need, stream) != cudaSuccess) {
             cudaGetLastError();
             return ATTN_ERR_WORKSPACE;
         }
-        if (s->bwd_block) {
-            // The old block may still be read by queued kernels.
-            if (cudaDeviceSynchronize() != cudaSuccess) {
-                cudaGetLastError();
-                cudaFree(block);
-                return ATTN_ERR_WORKSPACE;
-            }
-            cudaFree(s->bwd_block);
-        }
+        if (s->bwd_block && cudaFreeAsync(s->bwd_block, stream) != cudaSuccess)
+            cudaGetLastError();
         s->bwd_block = block;
         s->bwd_bytes = need;
     }

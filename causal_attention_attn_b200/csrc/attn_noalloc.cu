@@ -7,8 +7,12 @@
  * absorb mid-request, and some processes hand all device memory to one allocator at start-up (a
  * framework's caching allocator or a fixed memory budget), so an allocation made behind that
  * allocator's back either fails or breaks its accounting. attn_decode_noalloc serves those callers:
- * the scratch lives in a fixed-size array in the library's own device memory, reserved when the
- * library is loaded, and the call makes no allocation and frees nothing.
+ * the scratch lives in a fixed-size array in the library's own device memory, and the call makes no
+ * allocation and frees nothing. The runtime places the array on a device when it loads this file's
+ * module there; with lazy module loading (the CUDA 12.2+ default) that happens at the first
+ * cudaGetSymbolAddress below, i.e. in the first call on each device, so a caller that budgets
+ * device memory makes that first call at start-up. A kernel-side wait that runs out is recorded in
+ * the array's status word, which attn_device_status reads and clears.
  *
  * The array is shared by every call on a device and keeps the last call's contents. The arrival
  * counters, which must start at zero, are cleared on the stream before each launch; calls that
@@ -36,7 +40,6 @@ constexpr size_t kStatusBytes = 256;  // status word, padded to keep what follow
 // address: it is a host-side stand-in; the device address comes from cudaGetSymbolAddress below.
 static __device__ __align__(256) unsigned char g_decode_scratch[kScratchBytes];
 
-constexpr int kMaxDevices = 64;
 std::mutex g_setup_mutex;
 unsigned char *g_scratch_addr[kMaxDevices];  // device address of g_decode_scratch, per device
 
@@ -64,6 +67,16 @@ int scratch_for_current_device(unsigned char **out)
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 }  // namespace
+
+int *noalloc_status_word()
+{
+    const int dev = current_device_index();
+    if (dev < 0)
+        return nullptr;
+    std::lock_guard<std::mutex> lock(g_setup_mutex);
+    return reinterpret_cast<int *>(g_scratch_addr[dev]);
+}
+
 }  // namespace attn_b200
 
 using namespace attn_b200;

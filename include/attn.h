@@ -25,19 +25,18 @@
  *
  * Ownership: every pointer is a DEVICE pointer owned by the caller. The library keeps no pointer
  * after the work completes on `stream`. The library owns one small per-device workspace (the
- * split-KV partials of the decode kernel and a status word; attn_bwd keeps a second one); it grows
- * on the first call that needs more, with cudaMalloc, and when it replaces a smaller block it waits
- * for the device (cudaDeviceSynchronize) before freeing the old one, which queued kernels may still
- * read. A growing call is therefore neither stream-ordered nor graph-capturable; make one call of
- * the largest size before capturing. Concurrent decode calls on different streams of one device
- * share that workspace and must be serialised by the caller.
+ * split-KV partials of the decode kernel and a status word; attn_bwd keeps a second one). It grows
+ * on the first call that needs more, stream-ordered: the new block is taken from the device's
+ * stream-ordered pool on `stream` (cudaMallocAsync) and the old one released on `stream` after the
+ * work queued before it (cudaFreeAsync); the host never waits. Make one call of the largest size
+ * before capturing a stream into a CUDA graph. Calls on different streams of one device share the
+ * workspace and must be serialised by the caller (an event between the streams suffices).
  *
  * Errors: argument errors are detected on the host before any launch and returned as a negative
- * attn_status; nothing is launched then. Launch failures return ATTN_ERR_LAUNCH. Apart from a call
- * that grows the workspace (above), no call synchronises; none aborts the process or traps on the
- * device. Kernel-side
- * waits are bounded: a wait that runs out sets the device status word, which attn_device_status()
- * reads.
+ * attn_status; nothing is launched then. Launch failures return ATTN_ERR_LAUNCH. No call other
+ * than attn_device_status synchronises; none aborts the process or traps on the device.
+ * Kernel-side waits are bounded: a wait that runs out sets a device status word, which
+ * attn_device_status() reads.
  */
 #ifndef ATTN_B200_ATTN_H
 #define ATTN_B200_ATTN_H
@@ -102,7 +101,9 @@ int attn_version(void);
 
 /*
  * attn_device_status — synchronises `stream`, then reads and clears the current device's status
- * word. Returns ATTN_OK if no kernel-side wait has run out since the last call,
+ * words: the workspace's (every entry point except attn_decode_noalloc) and, once
+ * attn_decode_noalloc has run on the device, the one in its fixed array. Returns ATTN_OK if no
+ * kernel-side wait has run out since the last call,
  * ATTN_ERR_DEVICE_TIMEOUT if one has, or ATTN_ERR_CUDA if the stream could not be synchronised.
  * This is a diagnostic call: it blocks the host, so it does not belong on a hot path.
  */
@@ -112,13 +113,13 @@ int attn_device_status(void *stream);
  * attn_decode_noalloc — single-token decode (Sq == 1) that allocates no memory.
  *
  * The pages have no counterpart to this entry point: it is an interface addition for callers that
- * must not have a library allocate device memory — a serving loop that cannot absorb the device
- * synchronisation and latency of cudaMalloc in the middle of a request, or a process whose device
- * memory is owned by one allocator or a budget fixed at start-up, where an allocation behind that
- * allocator's back fails or breaks its accounting. attn_fwd grows a workspace with cudaMalloc on
- * first use; this call instead uses a fixed array of ATTN_DECODE_NOALLOC_SCRATCH_BYTES in the
- * library's own device memory, reserved on every GPU that loads the library until the process
- * exits. It calls no cudaMalloc, cudaFree or other allocating routine.
+ * must not have a library allocate device memory — a serving loop that cannot absorb the latency
+ * of an allocation in the middle of a request, or a process whose device memory is owned by one
+ * allocator or a budget fixed at start-up, where an allocation behind that allocator's back fails
+ * or breaks its accounting. attn_fwd grows a workspace (cudaMallocAsync) on first use; this call
+ * instead uses a fixed array of ATTN_DECODE_NOALLOC_SCRATCH_BYTES in the library's own device
+ * memory, held on every GPU where it has been placed until the process exits. It calls no
+ * cudaMalloc, cudaFree or other allocating routine.
  *
  * Arguments are those of attn_fwd with Sq = 1 and no causal flag (a single new query sees every
  * cached key): q [B, Hq, 1, D], k and v [B, Hkv, Skv, D], o [B, Hq, 1, D] bf16; lse [B, Hq, 1] fp32;
@@ -127,10 +128,14 @@ int attn_device_status(void *stream);
  * (batch, kv head) key ranges instead, which needs none).
  *
  * The first call on a device looks up that device's address of the array (cudaGetSymbolAddress,
- * with the device current); make that first call before any stream capture. Every call on a device
- * shares the array and it keeps the last call's contents; the counters that must start at zero are
- * cleared on `stream` before each launch. Calls that overlap on the GPU (different streams with no
- * ordering between them) race on the array: serialise them.
+ * with the device current); make that first call before any stream capture. With CUDA's lazy
+ * module loading (the default since CUDA 12.2) that first call is also when the runtime loads the
+ * array onto the device, so the array's memory is taken then: a caller that budgets device memory
+ * makes the first call at start-up. Every later call leaves the device's free memory unchanged.
+ * Every call on a device shares the array and it keeps the last call's contents; the counters that
+ * must start at zero are cleared on `stream` before each launch. Calls that overlap on the GPU
+ * (different streams with no ordering between them) race on the array: serialise them. A kernel-side
+ * wait that runs out is recorded in the array's status word, which attn_device_status reports.
  *
  * Returns ATTN_OK, an argument error as attn_fwd does, or ATTN_ERR_SCRATCH_LIMIT when the
  * arrival counters alone (one int per (batch, kv head, group of up to 8 query heads)) do not fit in
@@ -180,9 +185,8 @@ int attn_decode_paged(const void *q, const void *k_pages, const void *v_pages, c
  * lse rather than stored — "AI Infra 入门…", §3 (LSE paragraph); the gradients are the derivative of
  * the operation defined at the top of this file. Head dim 128 only; the other sizes, the causal flag
  * and the scale as attn_fwd. The library keeps an fp32 accumulator for dq and two per-row vectors in
- * its workspace (grown with cudaMalloc like attn_fwd's). Every pointer is a caller-owned device
- * pointer, 16-byte aligned. Returns ATTN_OK or a negative attn_status; synchronises only when it
- * grows its workspace.
+ * its workspace (grown stream-ordered like attn_fwd's). Every pointer is a caller-owned device
+ * pointer, 16-byte aligned. Returns ATTN_OK or a negative attn_status; never synchronises.
  */
 int attn_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout, const float *lse,
              void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int Sq, int Skv, int D,

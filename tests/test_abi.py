@@ -37,7 +37,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.attn_version() == 400
+    assert lib.attn_version() == 500
     for code, name in attn.STATUS_NAMES.items():
         s = attn.status_string(code)
         assert s and s != "unknown status", (code, name)
