@@ -15,7 +15,7 @@ import torch
 
 import oracle
 from causal_attention_attn_b200 import attn, build, inputs
-from causal_attention_attn_b200.ring import DIAG, SKIP, ring_schedule
+from causal_attention_attn_b200.ring import DIAG, ring_schedule, zigzag_shard
 from tests.compare import compare
 
 pytestmark = pytest.mark.gpu
@@ -84,27 +84,32 @@ def test_merge_with_empty_sides():
 
 @pytest.mark.parametrize("world,S,causal", [(4, 128, True), (3, 100, True), (2, 64, False)])
 def test_ring_schedule_on_one_gpu_matches_oracle(world, S, causal):
-    """Every virtual rank runs its schedule's blocks through attn_fwd and attn_lse_merge."""
+    """Every virtual rank runs its zigzag schedule's blocks through attn_fwd and attn_lse_merge.
+    S: tokens per rank (two chunks of S / 2)."""
     w = inputs.custom(1, 8, 2, world * S, world * S, 128, causal, seed=world * S)
     q, k, v = (t.cuda() for t in inputs.generate(w))
     ro, rl = oracle.attention(*(t.cpu() for t in (q, k, v)), w.scale, causal)
+    c = S // 2
+
+    def halves(x):
+        return x[:, :, :c].contiguous(), x[:, :, c:].contiguous()
+
     for rank in range(world):
-        sl = slice(rank * S, (rank + 1) * S)
-        qr = q[:, :, sl].contiguous()
-        o_acc = torch.zeros(qr.shape, dtype=torch.float32, device="cuda")
-        lse_acc = torch.full(qr.shape[:-1], float("-inf"), dtype=torch.float32, device="cuda")
-        out = torch.empty(qr.shape, dtype=torch.bfloat16, device="cuda")
+        qs = halves(zigzag_shard(q, rank, world))
+        o_acc = [torch.zeros(x.shape, dtype=torch.float32, device="cuda") for x in qs]
+        lse_acc = [torch.full(x.shape[:-1], float("-inf"), dtype=torch.float32, device="cuda") for x in qs]
+        out = [torch.empty(x.shape, dtype=torch.bfloat16, device="cuda") for x in qs]
         sched = ring_schedule(rank, world, causal)
-        last = max(t for t, _, mode in sched if mode != SKIP)
-        for t, j, mode in sched:
-            if mode == SKIP:
-                continue
-            kj = k[:, :, j * S:(j + 1) * S].contiguous()
-            vj = v[:, :, j * S:(j + 1) * S].contiguous()
-            o_p, l_p = attn.attn_fwd(qr, kj, vj, scale=w.scale, causal=(mode == DIAG))
-            attn.attn_lse_merge(o_acc, lse_acc, o_p, l_p, out=out if t == last else None)
+        last = {qh: (t, b) for t, _, blocks in sched for b, (qh, _, _) in enumerate(blocks)}
+        for t, j, blocks in sched:
+            ks, vs = halves(zigzag_shard(k, j, world)), halves(zigzag_shard(v, j, world))
+            for b, (qh, kh, mode) in enumerate(blocks):
+                o_p, l_p = attn.attn_fwd(qs[qh], ks[kh], vs[kh], scale=w.scale, causal=(mode == DIAG))
+                attn.attn_lse_merge(o_acc[qh], lse_acc[qh], o_p, l_p, out=out[qh] if last[qh] == (t, b) else None)
         torch.cuda.synchronize()
-        rep = compare(out, lse_acc, ro[:, :, sl], rl[:, :, sl])
+        want_o = zigzag_shard(torch.from_numpy(ro), rank, world).numpy()
+        want_l = zigzag_shard(torch.from_numpy(rl), rank, world).numpy()
+        rep = compare(torch.cat(out, dim=2), torch.cat(lse_acc, dim=2), want_o, want_l)
         assert rep.ok(), f"rank {rank}: {rep}"
 
 
