@@ -1,13 +1,19 @@
 """Benchmark: fused causal attention on B200, prefill TFLOP/s and decode KV-read GB/s.
 
-One step = one pass of the whole hot path over one batch of synthetic input: the causal prefill of
-an 8B-shaped layer (B=1, Hq=32, Hkv=8, S=4096, D=128) through the prefill kernel, then the GQA
-decode over a 16 x 4096-token KV cache through the tensor-core split-KV decode kernel. Inputs are resident in
-HBM before timing; L2 is flushed before each of the two kernels (a 256 MiB write, then a 256 MiB read
-so that the written lines are cleaned before the kernel starts), outside the kernel events.
+One step = one pass of the whole hot path over the five synthetic workloads, each once: the tiny
+causal prefill (B1 H2 S64 D32), the causal prefill of an 8B-shaped layer (B1 Hq32 Hkv8 S4096 D128),
+the GQA decode over a 16 x 4096-token KV cache, the chunked prefill (B8, 256 new tokens over a
+768-token cache) and the long-context prefill (B1 Hq32 Hkv8 S32768 D128, 1% of the keys x8). Inputs
+are resident in HBM before timing; L2 is flushed before every launch (a 256 MiB write, then a
+256 MiB read so that the written lines are cleaned before the kernel starts), outside the kernel
+events. Each launch is timed with CUDA events on the launching stream.
+
+The line's ``value`` is the prefill TFLOP/s of the largest single-GPU workload (the 32K prefill);
+``configs`` holds every workload's own throughput, roofline fraction, DRAM traffic and oracle
+baseline, and ``decode`` repeats the GQA decode's.
 
 ``python bench.py --gpus N --steps K --warmup W`` prints one JSON line (rank 0). For N > 1 it is
-launched with torchrun, one rank per GPU; every rank processes its own copy of the workload (the
+launched with torchrun, one rank per GPU; every rank processes its own copy of the workloads (the
 (batch, head) problems are independent, so there is no data-path collective) and the time is the
 max over ranks. ``--impl reference`` times the CPU oracle instead (rank 0 only).
 """
@@ -32,6 +38,10 @@ from causal_attention_attn_b200 import inputs  # noqa: E402
 METRIC = "prefill attn TFLOP/s & decode KV-read GB/s, as fraction of B200 roofline"
 PREFILL = inputs.PREFILL_8B
 DECODE = inputs.DECODE_GQA
+HEADLINE = inputs.LONG_PREFILL  # the largest workload that fits one GPU: the line's value
+STEP_WORKLOADS = (inputs.TINY_PREFILL, inputs.PREFILL_8B, inputs.DECODE_GQA, inputs.CHUNKED_PREFILL,
+                  inputs.LONG_PREFILL)
+SHORT = {w.name: n for n, w in inputs.SHORT_NAMES.items()}
 L2_FLUSH_BYTES = 256 * 1024 * 1024
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -88,11 +98,13 @@ def whole_job_rate(world: int, units_per_rank: float, seconds: float) -> float:
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples taken every 100 ms while the timed region runs."""
+    """nvidia-smi clock / power / throttle-reason samples taken every 20 ms while the timed region
+    runs."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    LOAD_WATTS = 300.0  # a sample drawing at least this much is taken while a kernel runs
 
     def __init__(self, device_index: int):
         self.device_index = device_index
@@ -104,7 +116,7 @@ class ClockSampler:
             self.out = open(os.devnull, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.device_index}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=subprocess.PIPE, stderr=self.out, text=True)
         except (OSError, FileNotFoundError):
             self.proc = None
@@ -125,22 +137,36 @@ class ClockSampler:
             self.out.close()
 
     def summary(self):
-        sm, smax, reasons = [], 0.0, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in getattr(self, "lines", []):
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                smax = max(smax, float(parts[2]))
-            except ValueError:
-                continue
-            for name, val in zip(names, parts[5:9]):
-                if val.lower() == "active":
-                    reasons.add(name)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax or None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        return summarise_clock_lines(getattr(self, "lines", []), self.LOAD_WATTS)
+
+
+def summarise_clock_lines(lines, load_watts):
+    """Median SM clock over every sample and over the samples drawing >= load_watts (under load),
+    the highest max clock seen, and the throttle reasons active in any sample."""
+    sm, sm_load, smax, reasons = [], [], 0.0, set()
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    for ln in lines:
+        parts = [p.strip() for p in ln.split(",")]
+        if len(parts) < 9:
+            continue
+        try:
+            mhz = float(parts[1])
+            smax = max(smax, float(parts[2]))
+        except ValueError:
+            continue
+        sm.append(mhz)
+        try:
+            if float(parts[3]) >= load_watts:
+                sm_load.append(mhz)
+        except ValueError:
+            pass
+        for name, val in zip(names, parts[5:9]):
+            if val.lower() == "active":
+                reasons.add(name)
+    return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax or None,
+            "reasons": sorted(reasons), "samples": len(sm),
+            "sm_mhz_under_load": statistics.median(sm_load) if sm_load else None,
+            "samples_under_load": len(sm_load)}
 
 
 def prefill_sample_flops(w, rows):
@@ -149,30 +175,50 @@ def prefill_sample_flops(w, rows):
     return int(4 * w.D * int(visible.sum()))
 
 
-def cpu_baseline(w, every: int, offset: int = 0, threads=None):
-    """Time the oracle on every `every`-th row of workload `w` (rows offset, offset+every, ...)."""
+def cpu_baseline(w, every: int, offset: int = 0, threads=None, data=None):
+    """Time the oracle on every `every`-th row of workload `w` (rows offset, offset+every, ...).
+    Returns (TFLOP/s, seconds, cores, rows)."""
     import oracle  # the CPU baseline is the oracle as it stands
 
-    q, k, v = inputs.generate(w)
+    q, k, v = data if data is not None else inputs.generate(w)
     total = w.B * w.Hq * w.Sq
     rows = torch.arange(offset % every, total, every, dtype=torch.int64)
     cores = len(os.sched_getaffinity(0))
     t0 = time.perf_counter()
-    oracle.attention(q, k, v, w.scale, w.causal, rows=rows.numpy(), threads=threads or cores)
+    oracle.attention(q, k, v, w.scale, w.causal, rows=rows.numpy() if every > 1 else None,
+                     threads=threads or cores)
     dt = time.perf_counter() - t0
     flops = prefill_sample_flops(w, rows)
     return flops / dt / 1e12, dt, cores, rows.numel()
+
+
+# Rows of each workload the oracle baseline times in the bench: every row, except the long
+# prefill's every 64th (its full 8.8 TFLOP would take minutes of fp64).
+BASELINE_EVERY = {inputs.LONG_PREFILL.name: 64}
+
+
+def workload_baseline(w, data=None):
+    every = BASELINE_EVERY.get(w.name, 1)
+    tf, dt, cores, n = cpu_baseline(w, every, data=data)
+    d = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "seconds": dt,
+         "sample": (f"every query row ({n} rows, {dt:.2f} s); fp64 three-pass oracle" if every == 1 else
+                    f"every {every}th query row ({n} rows, {dt:.2f} s), rate extrapolated to the whole "
+                    f"workload; fp64 three-pass oracle")}
+    if w.Sq == 1:  # the decode's own unit: K/V bytes per second
+        d["value_gbs"] = w.io_bytes() / (dt * (w.B * w.Hq * w.Sq) / n) / 1e9
+    return d
 
 
 def run_reference(args):
     world, rank, _ = dist_env()
     if rank != 0:
         return 0
-    w = PREFILL
-    every = 32
+    w = HEADLINE
+    every = 1024
+    data = inputs.generate(w)
     times, flops = [], []
     for s in range(args.warmup + args.steps):
-        tf, dt, cores, n = cpu_baseline(w, every, offset=s)
+        tf, dt, cores, n = cpu_baseline(w, every, offset=97 * s, data=data)
         if s >= args.warmup:
             times.append(dt)
             flops.append(tf * dt * 1e12)
@@ -181,14 +227,43 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sum(times) / len(times),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic (seeded N(0,1) bf16 inputs)", "config": PREFILL.config(),
+        "data": "synthetic (seeded N(0,1) bf16 inputs)", "config": HEADLINE.config(),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                         "sample": f"one query row in {every} of the workload per step (rows offset by the step "
-                                   f"index), {n} rows; fp64 three-pass oracle"},
+                         "sample": f"one query row in {every} of the workload per step (rows offset by 97 x the "
+                                   f"step index), {n} rows; fp64 three-pass oracle"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def config_entry(w, launch_s, world, peaks, peak_kind, baseline=None):
+    """The JSON object of one workload: throughput, roofline of its kernel, oracle baseline."""
+    tensor_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    kernel = "decode_tc_kernel" if w.Sq == 1 else "prefill_kernel"
+    if w.Sq == 1:
+        achieved = w.io_bytes() / launch_s / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
+                "peak_kind": f"{peak_kind} HBM copy", "bytes_per_launch": w.io_bytes()}
+        value, unit = whole_job_rate(world, w.io_bytes(), launch_s) / 1e9, "GB/s"
+    else:
+        achieved = w.flops() / launch_s / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": tensor_peak, "unit": "TFLOP/s",
+                "frac": achieved / tensor_peak, "peak_kind": f"{peak_kind} bf16 dense (burst)",
+                "flops_per_launch": w.flops()}
+        value, unit = whole_job_rate(world, w.flops(), launch_s) / 1e12, "TFLOP/s"
+    roof["traffic"] = read_traffic(kernel, w.name)
+    roof["kernel"] = f"{kernel}<{w.D}>" if w.Sq > 1 else "decode_tc_kernel<4>"
+    e = {"workload": w.name, "value": value, "unit": unit, "us_per_launch": launch_s * 1e6, "roofline": roof,
+         "config": w.config()}
+    if w.name == inputs.TINY_PREFILL.name:
+        e["note"] = "launch-latency bound (0.5 MFLOP); the roofline fraction is reported but is not the measure"
+    if baseline is not None:
+        e["cpu_baseline"] = baseline
+        if unit == "TFLOP/s":
+            e["vs_oracle"] = value / baseline["value"]
+    return e
 
 
 def run_ours(args):
@@ -207,14 +282,11 @@ def run_ours(args):
     attn.load_library()
     peaks, peak_kind = load_peaks()
 
-    qp, kp, vp = inputs.generate(PREFILL)
-    qd, kd, vd = inputs.generate(DECODE)
-    pq, pk, pv = (t.to(dev) for t in (qp, kp, vp))
-    dq, dk, dv = (t.to(dev) for t in (qd, kd, vd))
-    po = torch.empty_like(pq)
-    pl = torch.empty(pq.shape[:3], dtype=torch.float32, device=dev)
-    do = torch.empty_like(dq)
-    dl = torch.empty(dq.shape[:3], dtype=torch.float32, device=dev)
+    host = {w.name: inputs.generate(w) for w in STEP_WORKLOADS}
+    bufs = {}
+    for w in STEP_WORKLOADS:
+        q, k, v = (t.to(dev) for t in host[w.name])
+        bufs[w.name] = (q, k, v, torch.empty_like(q), torch.empty(q.shape[:3], dtype=torch.float32, device=dev))
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     flush_clean = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     flush_sum = torch.empty((), dtype=torch.float32, device=dev)
@@ -226,25 +298,26 @@ def run_ours(args):
         flush.zero_()
         torch.sum(flush_clean, dim=0, out=flush_sum)
 
+    def launch(w):
+        q, k, v, o, lse = bufs[w.name]
+        attn.attn_fwd(q, k, v, scale=w.scale, causal=w.causal, out=o, lse=lse, stream=stream)
+
     def step(evs=None):
-        clear_l2()
-        if evs:
-            evs[0].record(stream)
-        attn.attn_fwd(pq, pk, pv, scale=PREFILL.scale, causal=True, out=po, lse=pl, stream=stream)
-        if evs:
-            evs[1].record(stream)
-        clear_l2()
-        if evs:
-            evs[2].record(stream)
-        attn.attn_fwd(dq, dk, dv, scale=DECODE.scale, causal=True, out=do, lse=dl, stream=stream)
-        if evs:
-            evs[3].record(stream)
+        for i, w in enumerate(STEP_WORKLOADS):
+            clear_l2()
+            if evs:
+                evs[i][0].record(stream)
+            launch(w)
+            if evs:
+                evs[i][1].record(stream)
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
 
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    n_w = len(STEP_WORKLOADS)
+    events = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n_w)]
+              for _ in range(args.steps)]
     t_all0 = torch.cuda.Event(enable_timing=True)
     t_all1 = torch.cuda.Event(enable_timing=True)
     ranks.barrier()
@@ -256,41 +329,44 @@ def run_ours(args):
         t_all1.record(stream)
         torch.cuda.synchronize(dev)
     ranks.barrier()
-    pre_ms = sum(e[0].elapsed_time(e[1]) for e in events)
-    dec_ms = sum(e[2].elapsed_time(e[3]) for e in events)
+    per_w_ms = [sum(events[s][i][0].elapsed_time(events[s][i][1]) for s in range(args.steps)) for i in range(n_w)]
     region_ms = t_all0.elapsed_time(t_all1)
-    pre_ms, dec_ms, region_ms = ranks.max([pre_ms, dec_ms, region_ms])
+    timed = ranks.max(per_w_ms + [region_ms])
+    per_w_ms, region_ms = timed[:n_w], timed[n_w]
+    launch_s = {w.name: per_w_ms[i] * 1e-3 / args.steps for i, w in enumerate(STEP_WORKLOADS)}
+    status = attn.device_status(stream)
 
-    prefill_tflops = whole_job_rate(world, args.steps * PREFILL.flops(), pre_ms * 1e-3) / 1e12
-    decode_bytes = DECODE.io_bytes()  # K and V read once, plus q, o and lse
-    decode_gbs = whole_job_rate(world, args.steps * decode_bytes, dec_ms * 1e-3) / 1e9
-    pre_launch_s = pre_ms * 1e-3 / args.steps
-    dec_launch_s = dec_ms * 1e-3 / args.steps
+    head_s = launch_s[HEADLINE.name]
+    head_tflops = whole_job_rate(world, args.steps * HEADLINE.flops(), head_s * args.steps) / 1e12
     tensor_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
 
-    # End to end through the public call on HOST buffers: pinned H2D of q, k, v, the kernel, D2H of o, lse.
-    hq, hk, hv = (t.pin_memory() for t in (qp, kp, vp))
-    ho = torch.empty(qp.shape, dtype=torch.bfloat16, pin_memory=True)
-    hl = torch.empty(qp.shape[:3], dtype=torch.float32, pin_memory=True)
-    bufs = (pq, pk, pv, po, pl)
+    # End to end through the public call on HOST buffers: pinned H2D of q, k, v, the kernel, D2H of
+    # o and lse, for the headline workload.
+    hq, hk, hv = (t.pin_memory() for t in host[HEADLINE.name])
+    ho = torch.empty(hq.shape, dtype=torch.bfloat16, pin_memory=True)
+    hl = torch.empty(hq.shape[:3], dtype=torch.float32, pin_memory=True)
+    head_bufs = bufs[HEADLINE.name]
     for _ in range(2):
-        attn.attn_fwd_host(hq, hk, hv, scale=PREFILL.scale, causal=True, stream=stream, out_host=ho, lse_host=hl,
-                           dev_bufs=bufs)
+        attn.attn_fwd_host(hq, hk, hv, scale=HEADLINE.scale, causal=True, stream=stream, out_host=ho, lse_host=hl,
+                           dev_bufs=head_bufs)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e2e_steps = max(3, min(args.steps, 10))
     ranks.barrier()
     torch.cuda.synchronize(dev)
     e0.record(stream)
     for _ in range(e2e_steps):
-        attn.attn_fwd_host(hq, hk, hv, scale=PREFILL.scale, causal=True, stream=stream, out_host=ho, lse_host=hl,
-                           dev_bufs=bufs)
+        attn.attn_fwd_host(hq, hk, hv, scale=HEADLINE.scale, causal=True, stream=stream, out_host=ho, lse_host=hl,
+                           dev_bufs=head_bufs)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1)
     e2e_ms = ranks.max([e2e_ms])[0]
     ranks.barrier()
-    e2e_tflops = whole_job_rate(world, e2e_steps * PREFILL.flops(), e2e_ms * 1e-3) / 1e12
+    e2e_tflops = whole_job_rate(world, e2e_steps * HEADLINE.flops(), e2e_ms * 1e-3) / 1e12
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+    d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+    del hq, hk, hv, ho, hl
 
     # The same decode over an e4m3 cache (per-channel coefficients), timed on its own: inputs
     # resident, L2 flushed before every launch, CUDA events around each launch.
@@ -314,37 +390,36 @@ def run_ours(args):
     fp8_ms = ranks.max([sum(a.elapsed_time(b) for a, b in fev)])[0]
     fp8_launch_s = fp8_ms * 1e-3 / fp8_steps
 
-    # The backward pass of the prefill workload (dq, dk, dv from dout and the forward's o, lse),
+    # The backward pass of the 8B prefill workload (dq, dk, dv from dout and the forward's o, lse),
     # timed the same way. Reported beside the step, not part of it.
     try:
+        pq, pk, pv, po, pl = bufs[PREFILL.name]
         backward = backward_leg(attn, args, ranks, dev, stream, clear_l2, pq, pk, pv, po, pl, world)
     except Exception as e:  # an extra leg that fails is reported in its object, not allowed to drop the line
         backward = {"metric": "backward TFLOP/s (dq, dk, dv)", "error": f"{type(e).__name__}: {e}"}
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
-    d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
 
     if rank == 0:
-        base_tf, base_dt, cores, n_rows = cpu_baseline(PREFILL, every=1) if world == 1 else (None, None, None, None)
-        traffic = read_traffic("prefill_kernel", PREFILL.name)
+        baselines = {w.name: workload_baseline(w, host[w.name]) for w in STEP_WORKLOADS} if world == 1 else {}
+        configs = {SHORT[w.name]: config_entry(w, launch_s[w.name], world, peaks, peak_kind, baselines.get(w.name))
+                   for w in STEP_WORKLOADS}
+        head = configs[SHORT[HEADLINE.name]]
+        dec = configs[SHORT[DECODE.name]]
+        clk = clocks.summary()
+        if clk.get("sm_mhz_under_load"):
+            clk["headline_kcycles_at_load_clock"] = head_s * 1e6 * clk["sm_mhz_under_load"] / 1e3
         line = {
-            "metric": METRIC, "value": prefill_tflops, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": (pre_ms + dec_ms) / args.steps, "higher_is_better": True,
+            "metric": METRIC, "value": head_tflops, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": sum(per_w_ms) / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16 inputs)",
-            "config": dict(PREFILL.config(), l2="flushed before every kernel (256 MiB write, then 256 MiB read)",
+            "config": dict(HEADLINE.config(),
+                           step="the five workloads, each launched once (tiny, 8B prefill, GQA decode, chunked, 32K)",
+                           l2="flushed before every kernel (256 MiB write, then 256 MiB read)",
                            parallelism=f"replicas x{world}"),
-            "roofline": {"bound": "tensor", "achieved": PREFILL.flops() / pre_launch_s / 1e12, "peak": tensor_peak,
-                         "unit": "TFLOP/s", "frac": PREFILL.flops() / pre_launch_s / 1e12 / tensor_peak,
-                         "traffic": traffic, "peak_kind": f"{peak_kind} bf16 dense (burst)",
-                         "kernel": "prefill_kernel<128>"},
-            "decode": {
-                "metric": "decode KV-read GB/s", "value": decode_gbs, "unit": "GB/s", "config": DECODE.config(),
-                "roofline": {"bound": "hbm", "achieved": decode_bytes / dec_launch_s / 1e9, "peak": hbm_peak,
-                             "unit": "GB/s", "frac": decode_bytes / dec_launch_s / 1e9 / hbm_peak,
-                             "traffic": read_traffic("decode_tc_kernel", DECODE.name),
-                             "peak_kind": f"{peak_kind} HBM copy", "kernel": "decode_tc_kernel<4>"},
-                "us_per_launch": dec_launch_s * 1e6,
-                "ctas": attn.decode_ctas(DECODE.B, DECODE.Hq, DECODE.Hkv, DECODE.Skv, DECODE.D),
-            },
+            "roofline": dict(head["roofline"]),
+            "configs": configs,
+            "decode": {"metric": "decode KV-read GB/s", "value": dec["value"], "unit": "GB/s",
+                       "config": DECODE.config(), "roofline": dec["roofline"], "us_per_launch": dec["us_per_launch"],
+                       "ctas": attn.decode_ctas(DECODE.B, DECODE.Hq, DECODE.Hkv, DECODE.Skv, DECODE.D)},
             "decode_fp8": {
                 "metric": "decode KV-read GB/s, e4m3 K/V cache", "value": whole_job_rate(world, fp8_bytes, fp8_launch_s) / 1e9,
                 "unit": "GB/s", "config": dict(DECODE.config(), kv_dtype="e4m3", scales="fp32 per (kv head, channel)"),
@@ -357,17 +432,17 @@ def run_ours(args):
                 "bytes_per_launch": fp8_bytes,
             },
             "backward": backward,
-            "prefill_us_per_launch": pre_launch_s * 1e6,
             "timed_region_ms": region_ms,
             "e2e": {"value": e2e_tflops, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "steps": e2e_steps, "what": "prefill through attn_fwd on pinned host buffers, copies included"},
-            "gpu_launches": 2 * args.steps,
-            "clocks": clocks.summary(),
+                    "steps": e2e_steps,
+                    "what": "32K prefill through attn_fwd on pinned host buffers, copies included"},
+            "gpu_launches": n_w * args.steps,
+            "device_status": status,
+            "clocks": clk,
         }
-        if base_tf is not None:
-            line["cpu_baseline"] = {"value": base_tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                                    "sample": f"every query row of the prefill workload ({n_rows} rows, "
-                                              f"{base_dt:.1f} s); fp64 three-pass oracle"}
+        if baselines:
+            b = baselines[HEADLINE.name]
+            line["cpu_baseline"] = {k: b[k] for k in ("value", "unit", "cores", "kind", "sample")}
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.barrier()
@@ -399,18 +474,19 @@ def kernel_source_hash(kernel: str) -> str:
 
 
 def read_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch for `kernel` from the committed ncu summary (profiles/traffic.json),
-    or None when there is none for this workload or the kernel's source changed since the capture."""
+    """DRAM bytes per launch for `kernel` on `workload` from the committed ncu summaries
+    (profiles/traffic.json: kernel -> workload -> entry), or None when there is no capture for it
+    or the kernel's source changed since the capture."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     try:
         with open(path) as f:
-            entry = json.load(f).get(kernel, {})
-        if entry.get("workload") != workload or entry.get("source_hash") != kernel_source_hash(kernel):
+            entry = json.load(f).get(kernel, {}).get(workload, {})
+        if entry.get("source_hash") != kernel_source_hash(kernel):
             return None
         return entry.get("dram_bytes_per_launch")
-    except (OSError, ValueError):
+    except (OSError, ValueError, AttributeError):
         return None
 
 

@@ -70,3 +70,34 @@ def test_whole_job_rate_scales_with_ranks_for_the_backward_leg(monkeypatch):
     two = bench.backward_leg(fake, args, ranks, torch.device("cpu"), None, lambda: None, q, q, q, q,
                              torch.zeros((1, 1, 1)), world=2)
     assert one["steps"] == 5 and abs(two["value"] - 2 * one["value"]) < 1e-9
+
+
+def test_config_entry_reports_rate_roofline_and_baseline():
+    import bench
+    from causal_attention_attn_b200 import inputs
+
+    peaks = {"bf16_tflops": 1000.0, "hbm_gbs": 5000.0}
+    w = inputs.CHUNKED_PREFILL
+    base = {"value": 0.05, "unit": "TFLOP/s", "cores": 4, "kind": "oracle", "sample": "all"}
+    e = bench.config_entry(w, 1e-3, 2, peaks, "measured", base)
+    assert abs(e["value"] - 2 * w.flops() / 1e-3 / 1e12) < 1e-9  # two ranks, 1 ms each
+    assert abs(e["roofline"]["achieved"] - w.flops() / 1e-3 / 1e12) < 1e-9
+    assert abs(e["roofline"]["frac"] - e["roofline"]["achieved"] / 1000.0) < 1e-12
+    assert e["roofline"]["bound"] == "tensor" and e["us_per_launch"] == 1000.0
+    assert abs(e["vs_oracle"] - e["value"] / 0.05) < 1e-9
+    d = bench.config_entry(inputs.DECODE_GQA, 1e-3, 1, peaks, "measured")
+    assert d["roofline"]["bound"] == "hbm" and d["unit"] == "GB/s"
+    assert abs(d["roofline"]["frac"] - inputs.DECODE_GQA.io_bytes() / 1e-3 / 1e9 / 5000.0) < 1e-12
+
+
+def test_clock_summary_separates_samples_under_load():
+    import bench
+
+    lines = ["0, 1965, 1965, 120.5, 0x0, Not Active, Not Active, Not Active, Not Active",
+             "0, 1700, 1965, 900.0, 0x4, Not Active, Not Active, Not Active, Active",
+             "0, 1650, 1965, 950.0, 0x4, Not Active, Not Active, Not Active, Active",
+             "0, 1600, 1965, 980.0, 0x4, Not Active, Not Active, Not Active, Active"]
+    s = bench.summarise_clock_lines(lines, 300.0)
+    assert s["samples"] == 4 and s["samples_under_load"] == 3
+    assert s["sm_mhz_under_load"] == 1650.0 and s["sm_mhz"] == 1675.0
+    assert s["reasons"] == ["sw_power_cap"] and s["sm_max_mhz"] == 1965.0

@@ -271,3 +271,90 @@ def test_binding_rejects_bad_tensors():
     with pytest.raises(attn.AttnError) as e:
         attn.attn_fwd(q, q[:, :, :4].contiguous(), q[:, :, :4].contiguous(), causal=True)
     assert e.value.status == -6
+
+
+# ------------------------------------------------------------------------------ scale other than 1/sqrt(D)
+# The boundary takes any finite scale > 0 and applies it as given ("05 · Tích vô hướng…", "Vì sao
+# chia cho √128" explains 1/sqrt(d) as the usual choice, not the only one). V is multiplied by 1/4
+# (exact in bf16) so that |O| < 2: a peaked softmax puts O close to single V rows, and for |O| >= 4
+# half a bf16 ulp of the output alone would exceed the 1e-2 bound.
+
+SCALE_SHAPES = [
+    # B, Hq, Hkv, Sq, Skv, D, causal
+    (1, 4, 2, 300, 300, 128, True),
+    (1, 4, 2, 100, 500, 128, True),    # cache offset 400
+    (1, 2, 2, 200, 456, 64, False),
+    (1, 2, 1, 257, 257, 32, True),
+    (2, 8, 2, 1, 777, 128, True),      # decode, tensor core
+    (2, 8, 8, 1, 300, 64, True),       # decode, CUDA cores
+    (1, 6, 1, 1, 300, 32, True),
+]
+
+
+@pytest.mark.parametrize("scale", [0.05, 0.3, 2.0])
+@pytest.mark.parametrize("shape", SCALE_SHAPES, ids=lambda s: "b{}_hq{}_hkv{}_sq{}_skv{}_d{}_{}".format(
+    *s[:6], "c" if s[6] else "nc"))
+def test_scale_other_than_inverse_sqrt_d(shape, scale):
+    B, Hq, Hkv, Sq, Skv, D, causal = shape
+    w = inputs.custom(B, Hq, Hkv, Sq, Skv, D, causal, seed=sum(shape[:6]) + int(100 * scale))
+    q, k, v = inputs.generate(w)
+    v = (v.float() * 0.25).to(torch.bfloat16)
+    scale32 = float(np.float32(scale))
+    check(q, k, v, scale32, causal)
+
+
+@pytest.mark.parametrize("shape", [(1, 4, 2, 1024, 1024, 128, True), (4, 32, 8, 1, 4096, 128, True),
+                                   (1, 4, 4, 600, 600, 64, True)],
+                         ids=["prefill_d128", "decode_d128", "prefill_d64"])
+def test_high_variance_scores_drive_the_lazy_rescale(shape):
+    """Q and K drawn N(0, 4^2) (the N(0,1) draws times 4, exact in bf16): with scale 1/sqrt(D) the
+    scores have a standard deviation of 16, so the running max of ordinary rows jumps past the
+    rescale threshold again and again, not only on the 32K workload's outlier keys."""
+    B, Hq, Hkv, Sq, Skv, D, causal = shape
+    w = inputs.custom(B, Hq, Hkv, Sq, Skv, D, causal, seed=4242 + Sq)
+    q, k, v = inputs.generate(w)
+    q = (q.float() * 4).to(torch.bfloat16)
+    k = (k.float() * 4).to(torch.bfloat16)
+    v = (v.float() * 0.25).to(torch.bfloat16)
+    check(q, k, v, w.scale, causal)
+
+
+def test_workspace_growth_does_not_synchronise():
+    """A decode that needs a larger workspace than any call before it returns while earlier work on
+    its stream is still running: the workspace grows stream-ordered (no device synchronisation)."""
+    # Both shapes run the same kernel instantiation (D = 32, one head per kv head), so the first
+    # call has loaded it; the second needs 65536 arrival counters, more than any test before it.
+    small = inputs.custom(1, 4, 4, 1, 8, 32, True, seed=1)
+    big = inputs.custom(16384, 4, 4, 1, 8, 32, True, seed=2)
+    qs, ks, vs = (t.cuda() for t in inputs.generate(small))
+    qb, kb, vb = (t.cuda() for t in inputs.generate(big))
+    ob = torch.empty_like(qb)
+    lb = torch.empty(qb.shape[:3], dtype=torch.float32, device="cuda")
+    attn.attn_fwd(qs, ks, vs, scale=small.scale)  # loads the kernels and creates the workspace
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    done = torch.cuda.Event()
+    torch.cuda._sleep(2_000_000_000)  # about one second of device time
+    done.record(stream)
+    attn.attn_fwd(qb, kb, vb, scale=big.scale, out=ob, lse=lb)  # grows the workspace
+    still_running = not done.query()
+    torch.cuda.synchronize()
+    assert still_running, "attn_fwd waited for earlier work while growing its workspace"
+    o_ref, lse_ref = oracle.attention(qb.cpu(), kb.cpu(), vb.cpu(), big.scale, True)
+    rep = compare(ob, lb, o_ref, lse_ref)
+    assert rep.ok(), str(rep)
+
+
+@pytest.mark.skipif(not torch.cuda.is_available() or torch.cuda.device_count() < 2, reason="needs two devices")
+def test_second_device_gets_its_own_kernel_attributes():
+    """Function attributes (the dynamic shared-memory limit) are set per device: a prefill and a
+    decode on a second device run after the first device has used both."""
+    w = inputs.custom(1, 4, 2, 300, 300, 128, True, seed=12)
+    q, k, v = inputs.generate(w)
+    for dev in (0, 1):
+        with torch.cuda.device(dev):
+            o, lse = attn.attn_fwd(q.to(dev), k.to(dev), v.to(dev), scale=w.scale, causal=True)
+            od, ld = attn.attn_fwd(q[:, :, -1:].contiguous().to(dev), k.to(dev), v.to(dev), scale=w.scale)
+            torch.cuda.synchronize(dev)
+        o_ref, lse_ref = oracle.attention(q, k, v, w.scale, True)
+        assert compare(o, lse, o_ref, lse_ref).ok()
