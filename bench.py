@@ -537,6 +537,23 @@ def run_case(args):
     command the committed ncu summaries were captured with."""
     from causal_attention_attn_b200 import attn
 
+    if args.case == "backward":
+        w = inputs.PREFILL_8B
+        q, k, v = (t.cuda() for t in inputs.generate(w))
+        o, lse = attn.attn_fwd(q, k, v, scale=w.scale, causal=True)
+        dout = torch.randn(q.shape, generator=torch.Generator().manual_seed(7)).to(torch.bfloat16).cuda()
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        ev[0].record()
+        for _ in range(args.repeat):
+            attn.attn_bwd(q, k, v, o, lse, dout, scale=w.scale, causal=True, dq=dq, dk=dk, dv=dv)
+        ev[1].record()
+        torch.cuda.synchronize()
+        ms = ev[0].elapsed_time(ev[1]) / args.repeat
+        print(json.dumps({"case": w.name + "_backward", "repeat": args.repeat, "us_per_launch": ms * 1e3,
+                          "tflops": 5 * w.flops() / 2 / (ms * 1e-3) / 1e12,
+                          "device_status": attn.device_status()}), flush=True)
+        return 0
     if args.case == "decode_fp8":
         w = inputs.DECODE_GQA
         q, k8, v8, ks, vs = (t.cuda() for t in inputs.generate_fp8(w))
@@ -576,7 +593,7 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--case", choices=sorted(inputs.SHORT_NAMES) + ["decode_fp8"], default=None,
+    ap.add_argument("--case", choices=sorted(inputs.SHORT_NAMES) + ["decode_fp8", "backward"], default=None,
                     help="only run this workload --repeat times (for profiling); prints no bench line")
     ap.add_argument("--repeat", type=int, default=3)
     args = ap.parse_args()

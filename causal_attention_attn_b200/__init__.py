@@ -9,7 +9,7 @@ __version__ = "0.5.0"
 
 
 def __getattr__(name):
-    if name in ("attn_fwd", "attn_fwd_host", "attn_decode_paged", "attn_bwd", "attn_decode_fp8",
+    if name in ("attn_fwd", "attn_fwd_host", "attn_decode_paged", "attn_prefill_paged", "attn_bwd", "attn_decode_fp8",
                 "attn_decode_paged_fp8", "attn_lse_merge", "AttnError", "library_path", "load_library"):
         from . import attn as _attn
 

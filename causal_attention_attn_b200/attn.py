@@ -24,8 +24,8 @@ STATUS_NAMES = {
     -9: "ATTN_ERR_LAUNCH", -10: "ATTN_ERR_DEVICE_TIMEOUT", -11: "ATTN_ERR_SCALE", -12: "ATTN_ERR_CUDA",
     -13: "ATTN_ERR_SCRATCH_LIMIT",
 }
-EXPORTED = ("attn_fwd", "attn_fwd_ex", "attn_decode_ctas", "attn_status_string", "attn_version",
-            "attn_device_status", "attn_decode_noalloc", "attn_decode_paged", "attn_bwd", "attn_decode_fp8",
+EXPORTED = ("attn_fwd", "attn_fwd_ex", "attn_fwd_strided", "attn_decode_ctas", "attn_status_string", "attn_version",
+            "attn_device_status", "attn_decode_noalloc", "attn_decode_paged", "attn_prefill_paged", "attn_bwd", "attn_decode_fp8",
             "attn_decode_paged_fp8", "attn_lse_merge")
 
 _lock = threading.Lock()
@@ -54,6 +54,9 @@ def load_library(path: str | None = None):
         lib.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp]
         lib.attn_fwd_ex.restype = i
         lib.attn_fwd_ex.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, vp]
+        ll3 = ctypes.POINTER(ctypes.c_longlong)
+        lib.attn_fwd_strided.restype = i
+        lib.attn_fwd_strided.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, ll3, ll3, ll3, ll3, f, i, vp]
         lib.attn_decode_ctas.restype = i
         lib.attn_decode_ctas.argtypes = [i, i, i, i, i]
         lib.attn_status_string.restype = ctypes.c_char_p
@@ -68,6 +71,8 @@ def load_library(path: str | None = None):
         lib.attn_bwd.restype = i
         lib.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp]
         lib.attn_decode_paged.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, vp]
+        lib.attn_prefill_paged.restype = i
+        lib.attn_prefill_paged.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, f, i, vp]
         lib.attn_decode_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
         lib.attn_decode_paged_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, vp]
         lib.attn_lse_merge.restype = i
@@ -105,6 +110,27 @@ def _check_tensor(name, t, dtype, ndim):
         raise ValueError(f"{name} must be contiguous")
 
 
+def _check_rows(name, t, dtype):
+    """A [batch, head, row, dim] tensor in any layout whose last (dim) axis is contiguous."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must live on a CUDA device")
+    if t.dim() != 4:
+        raise ValueError(f"{name} must have 4 dims, got {tuple(t.shape)}")
+    if t.shape[-1] > 1 and t.stride(-1) != 1:
+        raise ValueError(f"{name} must have a contiguous last (head-dim) axis")
+
+
+def _strides3(t):
+    """(batch, head, row) element strides of a [B, H, S, D] view; an axis of extent 1 gets D
+    (its stride is never used, and the library wants a multiple of 8)."""
+    D = int(t.shape[-1])
+    return tuple(int(t.stride(i)) if t.shape[i] > 1 else D for i in range(3))
+
+
 def attn_fwd_raw(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, lse_ptr: int, B: int, Hq: int, Hkv: int,
                  Sq: int, Skv: int, D: int, scale: float, causal: bool, stream: int = 0,
                  decode_ctas: int = 0) -> int:
@@ -122,12 +148,15 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: float | N
              decode_ctas: int = 0):
     """Fused causal attention forward on the GPU.
 
-    q: [B, Hq, Sq, D], k/v: [B, Hkv, Skv, D], bf16, contiguous, on one CUDA device.
-    Returns (o [B, Hq, Sq, D] bf16, lse [B, Hq, Sq] fp32). ``scale`` defaults to 1/sqrt(D).
+    q: [B, Hq, Sq, D], k/v: [B, Hkv, Skv, D], bf16, on one CUDA device, each either contiguous or any
+    view with a contiguous last axis (e.g. a token-major [B, S, H, D] tensor passed as
+    ``x.transpose(1, 2)``); views go through ``attn_fwd_strided``. ``out`` (shape of q) may be such a
+    view too. Returns (o [B, Hq, Sq, D] bf16, lse [B, Hq, Sq] fp32, contiguous). ``scale``
+    defaults to 1/sqrt(D).
     """
-    _check_tensor("q", q, torch.bfloat16, 4)
-    _check_tensor("k", k, torch.bfloat16, 4)
-    _check_tensor("v", v, torch.bfloat16, 4)
+    _check_rows("q", q, torch.bfloat16)
+    _check_rows("k", k, torch.bfloat16)
+    _check_rows("v", v, torch.bfloat16)
     B, Hq, Sq, D = q.shape
     Bk, Hkv, Skv, Dk = k.shape
     if tuple(v.shape) != tuple(k.shape) or Bk != B or Dk != D:
@@ -135,9 +164,9 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: float | N
     if scale is None:
         scale = D ** -0.5
     if out is None:
-        out = torch.empty_like(q)
+        out = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
     else:
-        _check_tensor("out", out, torch.bfloat16, 4)
+        _check_rows("out", out, torch.bfloat16)
         if out.shape != q.shape:
             raise ValueError("out must have the shape of q")
     if lse is None:
@@ -146,9 +175,16 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: float | N
         _check_tensor("lse", lse, torch.float32, 3)
         if tuple(lse.shape) != (B, Hq, Sq):
             raise ValueError("lse must be [B, Hq, Sq]")
+    strided = not all(t.is_contiguous() for t in (q, k, v, out))
     with torch.cuda.device(q.device):
-        rc = attn_fwd_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, Hq, Hkv,
-                          Sq, Skv, D, scale, causal, _stream_handle(stream), decode_ctas)
+        if strided:
+            arr = [(ctypes.c_longlong * 3)(*_strides3(t)) for t in (q, k, v, out)]
+            rc = load_library().attn_fwd_strided(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                                 lse.data_ptr(), B, Hq, Hkv, Sq, Skv, D, *arr, float(scale),
+                                                 int(causal), _stream_handle(stream))
+        else:
+            rc = attn_fwd_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, Hq, Hkv,
+                              Sq, Skv, D, scale, causal, _stream_handle(stream), decode_ctas)
     _check(rc)
     return out, lse
 
@@ -243,6 +279,42 @@ def attn_decode_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Ten
                                               lse.data_ptr(), B, Hq, Hkv, num_pages, page_size,
                                               int(block_table.shape[1]), int(max_seq_len), float(scale),
                                               int(decode_ctas), _stream_handle(stream))
+    _check(rc)
+    return out, lse
+
+
+def attn_prefill_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor, block_table: torch.Tensor,
+                       seq_lens: torch.Tensor, max_seq_len: int, scale: float | None = None, causal: bool = True,
+                       out: torch.Tensor | None = None, lse: torch.Tensor | None = None, stream=None):
+    """Chunked prefill over a paged, variable-length KV cache through ``attn_prefill_paged``:
+    sequence b's Sq new queries attend to its first seq_lens[b] cached keys, the causal mask aligned
+    to the last Sq of them. q: [B, Hq, Sq, 128] bf16; k_pages, v_pages: [num_pages, Hkv, page_size,
+    128] bf16; block_table int32 [B, pages_per_seq]; seq_lens int32 [B] (all on the GPU).
+    Returns (o [B, Hq, Sq, 128], lse [B, Hq, Sq])."""
+    _check_tensor("q", q, torch.bfloat16, 4)
+    _check_tensor("k_pages", k_pages, torch.bfloat16, 4)
+    _check_tensor("v_pages", v_pages, torch.bfloat16, 4)
+    _check_tensor("block_table", block_table, torch.int32, 2)
+    _check_tensor("seq_lens", seq_lens, torch.int32, 1)
+    B, Hq, Sq, D = q.shape
+    num_pages, Hkv, page_size, Dk = k_pages.shape
+    if tuple(v_pages.shape) != tuple(k_pages.shape) or Dk != D:
+        raise ValueError(f"expected q [B,Hq,Sq,D] and k, v pages [P,Hkv,page,D]; got {tuple(q.shape)}, "
+                         f"{tuple(k_pages.shape)}")
+    if block_table.shape[0] != B or seq_lens.shape[0] != B:
+        raise ValueError("block_table and seq_lens need one row / entry per batch element")
+    if scale is None:
+        scale = D ** -0.5
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check_tensor("out", out, torch.bfloat16, 4)
+    _check_tensor("lse", lse, torch.float32, 3)
+    with torch.cuda.device(q.device):
+        rc = load_library().attn_prefill_paged(q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(),
+                                               block_table.data_ptr(), seq_lens.data_ptr(), out.data_ptr(),
+                                               lse.data_ptr(), B, Hq, Hkv, Sq, num_pages, page_size,
+                                               int(block_table.shape[1]), int(max_seq_len), float(scale),
+                                               int(bool(causal)), _stream_handle(stream))
     _check(rc)
     return out, lse
 

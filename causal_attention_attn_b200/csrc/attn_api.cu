@@ -16,7 +16,7 @@
 namespace attn_b200 {
 namespace {
 
-constexpr int kVersion = 500;  // 0.5.0: stream-ordered workspace growth (after 0.4.0: attn_lse_merge)
+constexpr int kVersion = 500;  // 0.5.0: attn_fwd_strided, attn_prefill_paged, stream-ordered workspace growth
 
 struct DeviceState {
     bool probed = false;
@@ -133,8 +133,23 @@ int ensure_workspace(DeviceState &s, size_t counters, size_t partials, cudaStrea
     return ATTN_OK;
 }
 
+// Element strides (batch, head, row) of q, k, v and o; `strided` false: the contiguous layouts.
+struct Layouts {
+    TensorStrides q, k, v, o;
+    bool strided;
+};
+
+Layouts contiguous_layouts(int Hq, int Hkv, int Sq, int Skv, int D)
+{
+    Layouts L;
+    L.q = L.o = TensorStrides{static_cast<long long>(Hq) * Sq * D, static_cast<long long>(Sq) * D, D};
+    L.k = L.v = TensorStrides{static_cast<long long>(Hkv) * Skv * D, static_cast<long long>(Skv) * D, D};
+    L.strided = false;
+    return L;
+}
+
 int run(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq, int Hkv, int Sq, int Skv,
-        int D, float scale, int causal, int decode_ctas, void *stream_ptr)
+        int D, float scale, int causal, int decode_ctas, const Layouts &st, void *stream_ptr)
 {
     int rc = validate(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, D, scale, causal);
     if (rc != ATTN_OK)
@@ -148,7 +163,9 @@ int run(const void *q, const void *k, const void *v, void *o, float *lse, int B,
     if (!s)
         return err;
 
-    if (Sq == 1) {
+    // Sq == 1 runs a decode kernel: the tensor-core one (D = 128) takes any layout, the CUDA-core one
+    // (D = 32, 64) only the contiguous one; a strided decode with D < 128 runs the prefill kernel.
+    if (Sq == 1 && (D == 128 || !st.strided)) {
         DecodePlan plan;
         if (decode_plan(B, Hq, Hkv, Skv, D, decode_ctas, s->sm_count, &plan) != cudaSuccess) {
             cudaGetLastError();
@@ -173,6 +190,11 @@ int run(const void *q, const void *k, const void *v, void *o, float *lse, int B,
         a.ws = s->partials;
         a.counters = s->counters;
         a.status = s->status;
+        a.strided = st.strided;
+        a.qs = st.q;
+        a.ks = st.k;
+        a.vs = st.v;
+        a.os = st.o;
         if (launch_decode(a, stream) != cudaSuccess) {
             cudaGetLastError();
             return ATTN_ERR_LAUNCH;
@@ -198,6 +220,11 @@ int run(const void *q, const void *k, const void *v, void *o, float *lse, int B,
     a.scale = scale;
     a.causal = causal;
     a.status = s->status;
+    a.sm_count = s->sm_count;
+    a.qs = st.q;
+    a.ks = st.k;
+    a.vs = st.v;
+    a.os = st.o;
     int encode_error = 0;
     const cudaError_t e = launch_prefill(a, stream, &encode_error);
     if (e != cudaSuccess) {
@@ -215,13 +242,47 @@ using namespace attn_b200;
 extern "C" int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq, int Hkv,
                         int Sq, int Skv, int D, float scale, int causal, void *stream)
 {
-    return run(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, D, scale, causal, 0, stream);
+    return run(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, D, scale, causal, 0, contiguous_layouts(Hq, Hkv, Sq, Skv, D),
+               stream);
 }
 
 extern "C" int attn_fwd_ex(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
                            int Hkv, int Sq, int Skv, int D, float scale, int causal, int decode_ctas, void *stream)
 {
-    return run(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, D, scale, causal, decode_ctas, stream);
+    return run(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, D, scale, causal, decode_ctas,
+               contiguous_layouts(Hq, Hkv, Sq, Skv, D), stream);
+}
+
+namespace {
+
+// A stride triple the kernels can use: every stride >= 1, a whole number of 16-byte units (8 bf16
+// elements: the TMA and the 16-byte output stores need it) and below 2^38 elements.
+bool strides_ok(const long long *st)
+{
+    for (int i = 0; i < 3; ++i)
+        if (st[i] < 1 || st[i] % 8 != 0 || st[i] >= (1LL << 38))
+            return false;
+    return true;
+}
+
+}  // namespace
+
+extern "C" int attn_fwd_strided(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
+                                int Hkv, int Sq, int Skv, int D, const long long *q_strides, const long long *k_strides,
+                                const long long *v_strides, const long long *o_strides, float scale, int causal,
+                                void *stream)
+{
+    if (!q_strides || !k_strides || !v_strides || !o_strides)
+        return ATTN_ERR_NULL;
+    if (!strides_ok(q_strides) || !strides_ok(k_strides) || !strides_ok(v_strides) || !strides_ok(o_strides))
+        return ATTN_ERR_ALIGN;
+    Layouts L;
+    L.q = TensorStrides{q_strides[0], q_strides[1], q_strides[2]};
+    L.k = TensorStrides{k_strides[0], k_strides[1], k_strides[2]};
+    L.v = TensorStrides{v_strides[0], v_strides[1], v_strides[2]};
+    L.o = TensorStrides{o_strides[0], o_strides[1], o_strides[2]};
+    L.strided = true;
+    return run(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, D, scale, causal, 0, L, stream);
 }
 
 extern "C" int attn_decode_ctas(int B, int Hq, int Hkv, int Skv, int D)
@@ -355,7 +416,7 @@ int decode_paged_impl(const void *q, const void *k_pages, const void *v_pages, c
     if (!s)
         return err;
     DecodePlan plan;
-    if (decode_plan_paged(B, Hq, Hkv, max_seq_len, decode_ctas, s->sm_count, &plan) != cudaSuccess) {
+    if (decode_plan_paged(B, Hq, Hkv, max_seq_len, decode_ctas, s->sm_count, &plan, fp8) != cudaSuccess) {
         cudaGetLastError();
         return ATTN_ERR_SHAPE;
     }
@@ -395,6 +456,75 @@ int decode_paged_impl(const void *q, const void *k_pages, const void *v_pages, c
 }
 
 }  // namespace
+
+extern "C" int attn_prefill_paged(const void *q, const void *k_pages, const void *v_pages, const int *block_table,
+                                  const int *seq_lens, void *o, float *lse, int B, int Hq, int Hkv, int Sq, int num_pages,
+                                  int page_size, int pages_per_seq, int max_seq_len, float scale, int causal,
+                                  void *stream_ptr)
+{
+    using namespace attn_b200;
+    if (!q || !k_pages || !v_pages || !block_table || !seq_lens || !o || !lse)
+        return ATTN_ERR_NULL;
+    if (B < 1 || Hq < 1 || Hkv < 1 || Sq < 1 || num_pages < 1 || pages_per_seq < 1 || max_seq_len < 0)
+        return ATTN_ERR_SHAPE;
+    if (causal != 0 && causal != 1)
+        return ATTN_ERR_SHAPE;
+    const bool page_ok = page_size == 16 || page_size == 32 || page_size == 64 ||
+                         (page_size >= 128 && page_size % 128 == 0);
+    if (!page_ok)
+        return ATTN_ERR_SHAPE;
+    if (Hq % Hkv != 0)
+        return ATTN_ERR_GQA;
+    // Rows (b*Hq + h)*Sq + i, block-table offsets and key positions must fit in 32 bits.
+    if (static_cast<long long>(B) * Hq * Sq > INT_MAX || static_cast<long long>(B) * pages_per_seq > INT_MAX ||
+        static_cast<long long>(pages_per_seq) * page_size > INT_MAX)
+        return ATTN_ERR_SHAPE;
+    if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(o) || !aligned16(lse) ||
+        (reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
+        return ATTN_ERR_ALIGN;
+    if (!(scale > 0.f) || !std::isfinite(scale))
+        return ATTN_ERR_SCALE;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+    std::lock_guard<std::mutex> lock(g_mutex);
+    int err = ATTN_OK;
+    DeviceState *s = device_state(&err);
+    if (!s)
+        return err;
+    int rc = ensure_workspace(*s, 0, 0, stream);  // the status word
+    if (rc != ATTN_OK)
+        return rc;
+    const int D = 128;
+    PrefillArgs a;
+    a.q = q;
+    a.k = k_pages;
+    a.v = v_pages;
+    a.o = o;
+    a.lse = lse;
+    a.B = B;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.Sq = Sq;
+    a.Skv = 0;
+    a.D = D;
+    a.scale = scale;
+    a.causal = causal;
+    a.status = s->status;
+    a.sm_count = s->sm_count;
+    a.qs = a.os = TensorStrides{static_cast<long long>(Hq) * Sq * D, static_cast<long long>(Sq) * D, D};
+    a.ks = a.vs = TensorStrides{0, 0, 0};  // unused: the pages have their own layout
+    a.seq_lens = seq_lens;
+    a.block_table = block_table;
+    a.num_pages = num_pages;
+    a.page_size = page_size;
+    a.pages_per_seq = pages_per_seq;
+    a.max_seq_len = max_seq_len;
+    int encode_error = 0;
+    if (launch_prefill(a, stream, &encode_error) != cudaSuccess) {
+        cudaGetLastError();
+        return encode_error ? ATTN_ERR_CUDA : ATTN_ERR_LAUNCH;
+    }
+    return ATTN_OK;
+}
 
 extern "C" int attn_decode_paged(const void *q, const void *k_pages, const void *v_pages, const int *block_table,
                                  const int *seq_lens, void *o, float *lse, int B, int Hq, int Hkv, int num_pages,
@@ -443,7 +573,7 @@ extern "C" int attn_decode_fp8(const void *q, const void *k8, const void *v8, co
     if (!s)
         return err;
     DecodePlan plan;
-    if (decode_plan(B, Hq, Hkv, Skv, D, decode_ctas, s->sm_count, &plan) != cudaSuccess) {
+    if (decode_plan(B, Hq, Hkv, Skv, D, decode_ctas, s->sm_count, &plan, true) != cudaSuccess) {
         cudaGetLastError();
         return ATTN_ERR_SHAPE;
     }

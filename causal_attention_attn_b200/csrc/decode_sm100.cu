@@ -699,7 +699,7 @@ cudaError_t dispatch(int D, int G, const DecodeArgs *a, cudaStream_t stream, int
     case 128:
         if (a)
             return launch_decode_tc(*a, stream);
-        return decode_tc_ctas_per_sm(G, ctas_per_sm);
+        return decode_tc_ctas_per_sm(G, false, ctas_per_sm);
     default:
         return cudaErrorInvalidValue;
     }
@@ -719,7 +719,8 @@ int decode_heads_per_cta(int group, int D)
     return g;
 }
 
-cudaError_t decode_plan(int B, int Hq, int Hkv, int Skv, int D, int requested_ctas, int sm_count, DecodePlan *plan)
+cudaError_t decode_plan(int B, int Hq, int Hkv, int Skv, int D, int requested_ctas, int sm_count, DecodePlan *plan,
+                        bool fp8)
 {
     DecodePlan pl;
     const int group = Hq / Hkv;
@@ -732,7 +733,8 @@ cudaError_t decode_plan(int B, int Hq, int Hkv, int Skv, int D, int requested_ct
     long long ctas = requested_ctas;
     if (ctas <= 0) {
         int per_sm = 1;
-        const cudaError_t e = dispatch(D, pl.G, nullptr, nullptr, &per_sm);
+        const cudaError_t e = (D == 128) ? decode_tc_ctas_per_sm(pl.G, fp8, &per_sm)
+                                         : dispatch(D, pl.G, nullptr, nullptr, &per_sm);
         if (e != cudaSuccess)
             return e;
         const long long slots = static_cast<long long>(sm_count) * per_sm;

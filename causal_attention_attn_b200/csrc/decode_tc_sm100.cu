@@ -81,11 +81,14 @@ enum TcBar : int {
 };
 
 // Shared-memory layout of one variant. bf16 cache: K and V chunks of 32 KB (two 64-dim box
-// columns each), three in flight, Q^T and P^T in bf16. e4m3 cache: chunks of 16 KB (one 128-byte
-// box column), five in flight, Q^T and P^T each as three e4m3 parts (hi, mid, lo) of 16 x 128 bytes.
+// columns each), three in flight, Q^T and P^T in bf16; one CTA per SM. e4m3 cache: chunks of 16 KB
+// (one 128-byte box column), two in flight, Q^T and P^T each as three e4m3 parts (hi, mid, lo) of
+// 16 x 128 bytes; about 100 KB, so two CTAs share an SM. The e4m3 decode streams half the bytes of
+// the bf16 one per key but pays the same per-chunk softmax chain, which then takes longer than the
+// chunk's memory time: a second resident CTA runs its chain in the gaps of the first.
 template <bool kFp8>
 struct Lay {
-    static constexpr int kStages = kFp8 ? 5 : 3;
+    static constexpr int kStages = kFp8 ? 2 : 3;
     static constexpr int kBoxCols = kFp8 ? 1 : 2;          // 128-byte box columns per K or V row
     static constexpr int kTileBytes = kBoxCols * kHalfBytes;  // one K or V chunk
     static constexpr int kStageBytes = 2 * kTileBytes;        // K chunk, then V chunk
@@ -119,6 +122,8 @@ constexpr uint32_t kColO = 32;
 
 struct TcParams {
     __nv_bfloat16 *o;
+    long long o_sb, o_sh;  // element strides of o (batch, head); each head's D values are contiguous
+    long long q_sb, q_sh;  // element strides of q (batch, head), read directly by the e4m3 producer
     float *lse;
     float *ws;  // partials: [CTA][first or last segment][G*D + G]
     int *counters, *status;
@@ -391,16 +396,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int h0 = (bk % p.Hkv) * p.group + hg * G;
                 if constexpr (kFp8) {
                     // Loads only; Q^T is built once this chunk's copies are on their way.
-                    const __nv_bfloat16 *qrow = p.q + (static_cast<size_t>(b) * p.Hq + h0) * kD;
+                    const __nv_bfloat16 *qrow = p.q + b * p.q_sb + h0 * p.q_sh;
 #pragma unroll
                     for (int h = 0; h < (kFp8 ? G : 1); ++h)
-                        qraw[h] = reinterpret_cast<const uint2 *>(qrow + static_cast<size_t>(h) * kD)[lane];
+                        qraw[h] = reinterpret_cast<const uint2 *>(qrow + h * p.q_sh)[lane];
                     ksv = reinterpret_cast<const float4 *>(p.k_scale + static_cast<size_t>(bk % p.Hkv) * kD)[lane];
                 } else if (issuer) {
                     mbar_arrive_expect_tx(BAR(kBarQFull0 + qs), kSmallBytes);
                     for (int hf = 0; hf < 2; ++hf)
-                        tma_load_3d(sQ + qs * kSmallBytes + hf * kSmallHalf, &tm_q, BAR(kBarQFull0 + qs), hf * 64,
-                                    b * p.Hq + h0, 0);
+                        tma_load_4d(sQ + qs * kSmallBytes + hf * kSmallHalf, &tm_q, BAR(kBarQFull0 + qs), hf * 64,
+                                    h0, 0, b);
                 }
                 ++seg;
             }
@@ -438,19 +443,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // page beyond the last one.
                     if (key >= batch_len[b] || page < 0 || page >= p.num_pages)
                         page = p.num_pages;
-                    const int coord = static_cast<int>(static_cast<long long>(page) * p.Hkv + kvh);
                     const int in_page = key % p.page_size;
                     for (int hf = 0; hf < L::kBoxCols; ++hf) {
-                        tma_load_3d(dst + hf * kHalfBytes + lane * rows * 128, &tm_k, BAR(kBarFull0 + slot), hf * 64,
-                                    in_page, coord);
-                        tma_load_3d(dst + kTileBytes + hf * kHalfBytes + lane * rows * 128, &tm_v, BAR(kBarFull0 + slot),
-                                    hf * 64, in_page, coord);
+                        tma_load_4d(dst + hf * kHalfBytes + lane * rows * 128, &tm_k, BAR(kBarFull0 + slot), hf * 64,
+                                    in_page, kvh, page);
+                        tma_load_4d(dst + kTileBytes + hf * kHalfBytes + lane * rows * 128, &tm_v, BAR(kBarFull0 + slot),
+                                    hf * 64, in_page, kvh, page);
                     }
                 }
             } else if (issuer) {
                 for (int hf = 0; hf < L::kBoxCols; ++hf) {
-                    tma_load_3d(dst + hf * kHalfBytes, &tm_k, BAR(kBarFull0 + slot), hf * 64, key0, bk);
-                    tma_load_3d(dst + kTileBytes + hf * kHalfBytes, &tm_v, BAR(kBarFull0 + slot), hf * 64, key0, bk);
+                    tma_load_4d(dst + hf * kHalfBytes, &tm_k, BAR(kBarFull0 + slot), hf * 64, key0, bk % p.Hkv,
+                                bk / p.Hkv);
+                    tma_load_4d(dst + kTileBytes + hf * kHalfBytes, &tm_v, BAR(kBarFull0 + slot), hf * 64, key0,
+                                bk % p.Hkv, bk / p.Hkv);
                 }
             }
             if constexpr (kFp8) {
@@ -645,7 +651,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (batch_len[b] != 0)
                     continue;
                 for (int h = 0; h < p.Hq; ++h) {
-                    p.o[(static_cast<size_t>(b) * p.Hq + h) * kD + i] = __float2bfloat16_rn(0.f);
+                    p.o[b * p.o_sb + h * p.o_sh + i] = __float2bfloat16_rn(0.f);
                     if (i == 0)
                         p.lse[static_cast<size_t>(b) * p.Hq + h] = -INFINITY;
                 }
@@ -862,7 +868,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float o = __uint_as_float(ov[h]) / LPV * v_coef;
                 const size_t bh = static_cast<size_t>(b) * p.Hq + h0 + h;
                 if (whole_pair) {
-                    p.o[bh * kD + i] = __float2bfloat16_rn(o);
+                    p.o[b * p.o_sb + (h0 + h) * p.o_sh + i] = __float2bfloat16_rn(o);
                     if (i == h)
                         p.lse[bh] = (m[h] + log2f(L)) * kLn2;
                 } else {
@@ -946,7 +952,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         O = fmaf(w, __ldcg(sb + idx), O);
                     }
                     const size_t bh = static_cast<size_t>(b) * p.Hq + h0 + h;
-                    p.o[bh * kD + d] = __float2bfloat16_rn(O / W);
+                    p.o[b * p.o_sb + (h0 + h) * p.o_sh + d] = __float2bfloat16_rn(O / W);
                     if (d == 0)
                         p.lse[bh] = (M + log2f(W)) * kLn2;
                 }
@@ -1000,26 +1006,40 @@ cudaError_t launch_g(const DecodeArgs &a, cudaStream_t stream)
         return cudaErrorInitializationError;
     int err = 0;
     CUtensorMap tq, tk, tv;
-    // q as [1][B*Hq][D] (one row per query head); k and v as [B*Hkv][Skv][D], or, paged, as
-    // [num_pages*Hkv][page_size][D] read in boxes of min(page_size, 128) rows and 128 bytes of D
+    // q: heads as the rows of a (dim, head, 1, batch) map, boxes of 16 heads; k and v: (dim, key,
+    // kv head, batch) with the caller's strides, or, paged, (dim, slot, kv head, page) over
+    // [num_pages][Hkv][page_size][D], read in boxes of min(page_size, 128) rows and 128 bytes of D
     // (64 bf16 or 128 e4m3 elements).
-    const int kv_rows = kPaged ? a.page_size : a.Skv;
-    const int kv_bh = kPaged ? a.num_pages * a.Hkv : a.B * a.Hkv;
+    const TensorStrides qs = a.strided ? a.qs : TensorStrides{static_cast<long long>(a.Hq) * kD, kD, kD};
     const int box_rows = kPaged ? (a.page_size < kCK ? a.page_size : kCK) : kCK;
-    if (!make_map(encode, &tq, a.q, kD, a.B * a.Hq, 1, 64, kN, CU_TENSOR_MAP_SWIZZLE_128B, &err))
+    if (!make_map4(encode, &tq, a.q, 2, kD, a.Hq, 1, a.B, Strides{qs.b, qs.b, qs.h}, 64, kN,
+                   CU_TENSOR_MAP_SWIZZLE_128B, &err))
         return cudaErrorInvalidValue;
-    if constexpr (kFp8) {
-        if (!make_map_u8(encode, &tk, a.k, kD, kv_rows, kv_bh, 128, box_rows, CU_TENSOR_MAP_SWIZZLE_128B, &err) ||
-            !make_map_u8(encode, &tv, a.v, kD, kv_rows, kv_bh, 128, box_rows, CU_TENSOR_MAP_SWIZZLE_128B, &err))
-            return cudaErrorInvalidValue;
+    constexpr int kElem = kFp8 ? 1 : 2;
+    constexpr int kBoxInner = kFp8 ? 128 : 64;
+    Strides kst, vst;
+    if (kPaged) {
+        kst = vst = Strides{static_cast<long long>(a.Hkv) * a.page_size * kD, static_cast<long long>(a.page_size) * kD, kD};
+    } else if (a.strided) {
+        kst = Strides{a.ks.b, a.ks.h, a.ks.s};
+        vst = Strides{a.vs.b, a.vs.h, a.vs.s};
     } else {
-        if (!make_map(encode, &tk, a.k, kD, kv_rows, kv_bh, 64, box_rows, CU_TENSOR_MAP_SWIZZLE_128B, &err) ||
-            !make_map(encode, &tv, a.v, kD, kv_rows, kv_bh, 64, box_rows, CU_TENSOR_MAP_SWIZZLE_128B, &err))
-            return cudaErrorInvalidValue;
+        kst = vst = contiguous_strides(a.Hkv, a.Skv, kD);
     }
+    const int kv_rows = kPaged ? a.page_size : a.Skv;
+    const int kv_outer = kPaged ? a.num_pages : a.B;
+    if (!make_map4(encode, &tk, a.k, kElem, kD, kv_rows, a.Hkv, kv_outer, kst, kBoxInner, box_rows,
+                   CU_TENSOR_MAP_SWIZZLE_128B, &err) ||
+        !make_map4(encode, &tv, a.v, kElem, kD, kv_rows, a.Hkv, kv_outer, vst, kBoxInner, box_rows,
+                   CU_TENSOR_MAP_SWIZZLE_128B, &err))
+        return cudaErrorInvalidValue;
     const DecodePlan &pl = a.plan;
     TcParams p;
     p.o = static_cast<__nv_bfloat16 *>(a.o);
+    p.o_sb = a.strided ? a.os.b : static_cast<long long>(a.Hq) * kD;
+    p.o_sh = a.strided ? a.os.h : kD;
+    p.q_sb = qs.b;
+    p.q_sh = qs.h;
     p.lse = a.lse;
     p.ws = a.ws;
     p.counters = a.counters;
@@ -1049,28 +1069,28 @@ cudaError_t launch_g(const DecodeArgs &a, cudaStream_t stream)
 }
 
 template <int G>
-cudaError_t dispatch_g(const DecodeArgs *a, cudaStream_t stream, int *ctas_per_sm)
+cudaError_t dispatch_g(const DecodeArgs *a, cudaStream_t stream, int *ctas_per_sm, bool fp8 = false)
 {
     if (!a)
-        return prepare_g<G, false, false>(ctas_per_sm);
+        return fp8 ? prepare_g<G, false, true>(ctas_per_sm) : prepare_g<G, false, false>(ctas_per_sm);
     if (a->fp8)
         return a->seq_lens ? launch_g<G, true, true>(*a, stream) : launch_g<G, false, true>(*a, stream);
     return a->seq_lens ? launch_g<G, true, false>(*a, stream) : launch_g<G, false, false>(*a, stream);
 }
 
-cudaError_t dispatch_tc(int G, const DecodeArgs *a, cudaStream_t stream, int *ctas_per_sm)
+cudaError_t dispatch_tc(int G, const DecodeArgs *a, cudaStream_t stream, int *ctas_per_sm, bool fp8 = false)
 {
     switch (G) {
     case 1:
-        return dispatch_g<1>(a, stream, ctas_per_sm);
+        return dispatch_g<1>(a, stream, ctas_per_sm, fp8);
     case 2:
-        return dispatch_g<2>(a, stream, ctas_per_sm);
+        return dispatch_g<2>(a, stream, ctas_per_sm, fp8);
     case 4:
-        return dispatch_g<4>(a, stream, ctas_per_sm);
+        return dispatch_g<4>(a, stream, ctas_per_sm, fp8);
     case 8:
-        return dispatch_g<8>(a, stream, ctas_per_sm);
+        return dispatch_g<8>(a, stream, ctas_per_sm, fp8);
     case 16:
-        return dispatch_g<16>(a, stream, ctas_per_sm);
+        return dispatch_g<16>(a, stream, ctas_per_sm, fp8);
     default:
         return cudaErrorInvalidValue;
     }
@@ -1089,14 +1109,17 @@ int decode_tc_heads_per_pair(int group)
 
 int decode_tc_chunk_keys() { return kCK; }
 
-cudaError_t decode_tc_ctas_per_sm(int G, int *ctas_per_sm) { return dispatch_tc(G, nullptr, nullptr, ctas_per_sm); }
+cudaError_t decode_tc_ctas_per_sm(int G, bool fp8, int *ctas_per_sm)
+{
+    return dispatch_tc(G, nullptr, nullptr, ctas_per_sm, fp8);
+}
 
 cudaError_t launch_decode_tc(const DecodeArgs &a, cudaStream_t stream) { return dispatch_tc(a.plan.G, &a, stream, nullptr); }
 
 size_t decode_tc_partial_floats(int G, int ctas) { return static_cast<size_t>(2) * ctas * (static_cast<size_t>(G) * kD + G); }
 
 cudaError_t decode_plan_paged(int B, int Hq, int Hkv, int max_seq_len, int requested_ctas, int sm_count,
-                              DecodePlan *plan)
+                              DecodePlan *plan, bool fp8)
 {
     DecodePlan pl;
     const int group = Hq / Hkv;
@@ -1109,7 +1132,7 @@ cudaError_t decode_plan_paged(int B, int Hq, int Hkv, int max_seq_len, int reque
     long long ctas = requested_ctas;
     if (ctas <= 0) {
         int per_sm = 1;
-        const cudaError_t e = prepare_g<1, true, false>(&per_sm);
+        const cudaError_t e = fp8 ? prepare_g<1, true, true>(&per_sm) : prepare_g<1, true, false>(&per_sm);
         if (e != cudaSuccess)
             return e;
         // As for the dense cache: one CTA per pair when the pairs alone fill most of the GPU

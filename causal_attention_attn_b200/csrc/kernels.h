@@ -41,14 +41,27 @@ enum WaitSite : int {
     kSiteBwd = 24,
 };
 
+// Element strides of a [batch][head][row][dim] tensor with a contiguous dim (see tma_host.h).
+struct TensorStrides {
+    long long b, h, s;
+};
+
 struct PrefillArgs {
     const void *q, *k, *v;
     void *o;
-    float *lse;
+    float *lse;  // [B][Hq][Sq], contiguous
     int B, Hq, Hkv, Sq, Skv, D;
     float scale;
     int causal;
-    int *status;  // device status word
+    int *status;       // device status word
+    int sm_count = 0;  // SMs of the device: the persistent grid's size
+    TensorStrides qs, ks, vs, os;  // element strides of q, k, v, o
+    // Paged, variable-length cache (seq_lens != nullptr; head dim 128): k, v are
+    // [num_pages][Hkv][page_size][D]; sequence b holds min(max(seq_lens[b], 0), cap) keys, cap =
+    // min(max_seq_len, pages_per_seq * page_size), in pages block_table[b][...]; Skv is unused.
+    const int *seq_lens = nullptr;
+    const int *block_table = nullptr;
+    int num_pages = 0, page_size = 0, pages_per_seq = 0, max_seq_len = 0;
 };
 
 // How a decode (Sq == 1) is spread over persistent CTAs. A "pair" is one (batch, kv head, group of
@@ -70,6 +83,10 @@ struct DecodeArgs {
     const void *q, *k, *v;
     void *o;
     float *lse;
+    // Element strides of q, k, v and o (dense cache, tensor-core kernel); `strided` false: the
+    // contiguous [B][H][S][D] layouts, which the CUDA-core kernel requires.
+    bool strided = false;
+    TensorStrides qs{}, ks{}, vs{}, os{};
     int B, Hq, Hkv, Skv, D;
     float scale;
     DecodePlan plan;
@@ -112,19 +129,21 @@ cudaError_t launch_lse_merge(float *o_acc, float *lse_acc, const void *o_part, c
 
 // Decode planning and launch. requested_ctas <= 0 means one CTA per resident slot on the device.
 int decode_heads_per_cta(int group, int D);  // G: 1, 2, 4 or 8 (up to 16 for D = 128)
-cudaError_t decode_plan(int B, int Hq, int Hkv, int Skv, int D, int requested_ctas, int sm_count, DecodePlan *plan);
+// fp8: plan for the e4m3-cache variant of the tensor-core kernel (its own occupancy).
+cudaError_t decode_plan(int B, int Hq, int Hkv, int Skv, int D, int requested_ctas, int sm_count, DecodePlan *plan,
+                        bool fp8 = false);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream);
 
 // Head dim 128 decodes on the tensor core (decode_tc_sm100.cu); launch_decode routes there.
 int decode_tc_heads_per_pair(int group);  // G: largest power of two dividing the group, at most 16
 int decode_tc_chunk_keys();               // keys per chunk (128)
-cudaError_t decode_tc_ctas_per_sm(int G, int *ctas_per_sm);
+cudaError_t decode_tc_ctas_per_sm(int G, bool fp8, int *ctas_per_sm);
 size_t decode_tc_partial_floats(int G, int ctas);  // workspace floats for shared pairs' partials
 constexpr int kPagedMaxBatch = 1024;  // batch entries a paged decode may have (per-CTA scan in shared memory)
 // Plan of a paged, variable-length decode: lengths are only known on the device, so the plan holds
 // upper bounds (cpp from max_seq_len; total is computed by each CTA); every pair may be shared.
 cudaError_t decode_plan_paged(int B, int Hq, int Hkv, int max_seq_len, int requested_ctas, int sm_count,
-                              DecodePlan *plan);
+                              DecodePlan *plan, bool fp8 = false);
 cudaError_t launch_decode_tc(const DecodeArgs &a, cudaStream_t stream);
 
 // The status word of attn_decode_noalloc's fixed scratch array on the current device, or nullptr

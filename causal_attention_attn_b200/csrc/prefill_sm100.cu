@@ -51,6 +51,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <climits>
 #include <cmath>
 #include <mutex>
 
@@ -100,8 +101,9 @@ struct Cfg {
 };
 
 enum Bar : int {
-    kBarQ = 0,
-    kBarFull0 = 1,
+    kBarQFull = 0,
+    kBarQFree = 1,  // the Q tiles may be replaced (every S product of the item has completed)
+    kBarFull0 = 2,
     kBarEmpty0 = kBarFull0 + kRing,
     kBarSFull0 = kBarEmpty0 + kRing,  // [A, B]
     kBarPHalf0 = kBarSFull0 + 2,      // [A, B] first half of P_X stored
@@ -114,13 +116,25 @@ static_assert(kNumBars * 8 <= 192, "barrier area");
 
 struct Params {
     __nv_bfloat16 *o;
+    long long o_sb, o_sh, o_ss;  // element strides of o (batch, head, row)
     float *lse;
     int *status;
     int B, Hq, Hkv, Sq, Skv, group, offset, causal;
     int n_items;      // work items along the query dimension (see the work decode)
+    int n_work;       // work items in all: n_items * B * (Hq / heads per item)
     int pair_heads;   // 1: tiles A and B are the same query tile of two heads sharing a kv head
     float scale_log2;
+    // Paged, variable-length cache (the kernel's kPaged variant): K and V are
+    // [num_pages][Hkv][page_size][D], sequence b's keys are its first seq_lens[b] keys (clamped to
+    // [0, cap]) in the pages block_table[b][0..pages_per_seq).
+    const int *seq_lens = nullptr;
+    const int *block_table = nullptr;
+    int num_pages = 0, page_size = 0, pages_per_seq = 0, cap = 0;
 };
+
+// Reference max of a row that has seen no key yet (paged variant): finite, so that the weights of
+// masked scores are 2^(-inf) = 0 rather than NaN, and far below any real score.
+constexpr float kNoKeyMax = -1e30f;
 
 __device__ __forceinline__ float ex2(float x)
 {
@@ -165,18 +179,88 @@ __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, u
     return true;
 }
 
-// Number of KV tiles a 128-row query tile starting at q0 needs (0 if the tile lies past Sq).
-__device__ __forceinline__ int kv_tiles_for(const Params &p, int q0)
+// Number of KV tiles a 128-row query tile starting at q0 needs over skv keys with the causal
+// offset off (0 if the tile lies past Sq, or, paged, if none of its rows sees a key).
+__device__ __forceinline__ int kv_tiles_for(const Params &p, int q0, int skv, int off)
 {
     if (q0 >= p.Sq)
         return 0;
-    int kv_end = p.Skv;
+    int kv_end = skv;
     if (p.causal)
-        kv_end = min(p.Skv, q0 + kBM + p.offset);  // last visible key of the tile's last row, + 1
-    return (kv_end + kBN - 1) / kBN;
+        kv_end = min(skv, q0 + kBM + off);  // last visible key of the tile's last row, + 1
+    return kv_end > 0 ? (kv_end + kBN - 1) / kBN : 0;
 }
 
-template <int D>
+// The r-th work item of this CTA, or -1. Persistent CTAs take the heaviest-first list in snake
+// order (round r left to right when r is even, right to left when odd), which balances the
+// decreasing item sizes over the CTAs as well as a dynamic queue would, with no shared counter.
+__device__ __forceinline__ int work_index(const Params &p, int r)
+{
+    const int g = static_cast<int>(gridDim.x);
+    const int c = static_cast<int>(blockIdx.x);
+    const long long w = static_cast<long long>(r) * g + ((r & 1) ? (g - 1 - c) : c);
+    return w < p.n_work ? static_cast<int>(w) : -1;
+}
+
+// One work item: two 128-row query tiles X = 0 (A), 1 (B) that stream the same K/V tiles.
+struct Item {
+    int q0[2];     // first query row of each tile
+    int hq[2];     // query head of each tile
+    int b, kvh;    // batch entry and kv head
+    int skv, off;  // keys of the sequence, and the causal offset skv - Sq
+    int n[2];      // KV tiles each tile needs (0: the tile lies past Sq or sees no key)
+    __device__ __forceinline__ int n_max() const { return max(n[0], n[1]); }
+};
+
+// Work item w, heaviest first (query tiles from the last). With pair_heads (the GQA group is even),
+// tiles A and B are the same 128 query rows of heads 2k and 2k+1, which share a kv head: both need
+// the same number of KV tiles, so they ping-pong to the last one. Otherwise they are two
+// consecutive query tiles of one head, and B needs one KV tile more than A.
+template <bool kPaged>
+__device__ __forceinline__ Item decode_item(const Params &p, int w)
+{
+    const int heads_per_item = p.pair_heads ? 2 : 1;
+    const int hpu = p.Hq / heads_per_item;
+    int t = w;
+    const int hu = t % hpu;
+    t /= hpu;
+    const int b = t % p.B;
+    t /= p.B;
+    const int item = p.n_items - 1 - t;
+    const int h_a = hu * heads_per_item;
+    Item it;
+    it.q0[0] = p.pair_heads ? item * kBM : item * 2 * kBM;
+    it.q0[1] = p.pair_heads ? it.q0[0] : it.q0[0] + kBM;
+    it.hq[0] = h_a;
+    it.hq[1] = h_a + (p.pair_heads ? 1 : 0);
+    it.b = b;
+    it.kvh = h_a / p.group;
+    if constexpr (kPaged) {
+        it.skv = min(max(__ldg(p.seq_lens + b), 0), p.cap);
+        it.off = it.skv - p.Sq;
+    } else {
+        it.skv = p.Skv;
+        it.off = p.offset;
+    }
+    it.n[0] = kv_tiles_for(p, it.q0[0], it.skv, it.off);
+    it.n[1] = kv_tiles_for(p, it.q0[1], it.skv, it.off);
+    return it;
+}
+
+// The first of this CTA's items from the r-th on that has a KV tile to stream, or -1. Without a
+// paged cache every item has one; with it, an item whose rows see no key at all is written by the
+// softmax warps alone (O = 0, LSE = -inf) and the producer and the MMA issuer skip it.
+template <bool kPaged>
+__device__ __forceinline__ int next_active(const Params &p, int r)
+{
+    for (;; ++r) {
+        const int w = work_index(p, r);
+        if (w < 0 || !kPaged || decode_item<kPaged>(p, w).n_max() > 0)
+            return w < 0 ? -1 : r;
+    }
+}
+
+template <int D, bool kPaged>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const Params p)
@@ -195,29 +279,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // Work decode, heaviest items first (query tiles from the last). With pair_heads (the GQA group
-    // is even), tiles A and B are the same 128 query rows of heads 2k and 2k+1, which share a kv head:
-    // both need the same number of KV tiles, so they ping-pong to the last one. Otherwise they are
-    // two consecutive query tiles of one head, and B needs one KV tile more than A.
-    int t = blockIdx.x;
-    const int heads_per_item = p.pair_heads ? 2 : 1;
-    const int hu = t % (p.Hq / heads_per_item);
-    t /= p.Hq / heads_per_item;
-    const int b = t % p.B;
-    t /= p.B;
-    const int item = p.n_items - 1 - t;
-    const int h_a = hu * heads_per_item;                       // head of tile A
-    const int q0_a = p.pair_heads ? item * kBM : item * 2 * kBM;  // first query row of tile A
-    auto q0_of = [&](int x) { return p.pair_heads ? q0_a : q0_a + x * kBM; };
-    auto bh_q_of = [&](int x) { return b * p.Hq + h_a + (p.pair_heads ? x : 0); };
-    const int n_a = kv_tiles_for(p, q0_of(0));
-    const int n_b = kv_tiles_for(p, q0_of(1));
-    const int n_max = max(n_a, n_b);
-    auto n_of = [&](int x) { return x ? n_b : n_a; };
-    const int bh_kv = b * p.Hkv + h_a / p.group;
-
     if (threadIdx.x == 0) {
-        mbar_init(BAR(kBarQ), 1);
+        mbar_init(BAR(kBarQFull), 1);
+        mbar_init(BAR(kBarQFree), 1);
         for (int r = 0; r < kRing; ++r) {
             mbar_init(BAR(kBarFull0 + r), 1);
             mbar_init(BAR(kBarEmpty0 + r), 1);
@@ -251,38 +315,82 @@ __global__ void __launch_bounds__(kThreads, 1)
       asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
       if (warp == kWarpTma) {
         // ---------------------------------------------------------------- TMA producer
+        // Per item: Q_A (and Q_B) once the previous item's last S products have read the Q tiles,
+        // then K0, V0, K1, V1, ... through the ring, whose position runs on across items.
         if (lane == 0) {
             const uint64_t pol = l2_policy_evict_last();  // K/V tiles are re-read by sibling CTAs
-            const int n_q = (n_b > 0) ? 2 : 1;
-            mbar_arrive_expect_tx(BAR(kBarQ), n_q * C::kTileBytes);
-            for (int x = 0; x < n_q; ++x)
-#pragma unroll
-                for (int c = 0; c < C::kChunks; ++c)
-                    tma_load_3d(sQ + x * C::kTileBytes + c * C::kChunkBytes, &tm_q, BAR(kBarQ), c * C::kChunkElems,
-                                q0_of(x), bh_q_of(x));
-            // Items in consumption order: K0, V0, K1, V1, ...
-            const int n_items = 2 * n_max;
-            int issued = 0;
-            for (int it = 0; it < n_items; ++it) {
-                const int slot = it % kRing;
-                const uint32_t round = static_cast<uint32_t>(it / kRing);
-                if (!mbar_wait(BAR(kBarEmpty0 + slot), (round & 1u) ^ 1u, abort_flag, p.status, kSitePrefillTmaEmpty))
+            uint32_t kv = 0;   // K/V loads issued so far
+            int q_issued = 0;  // Q loads issued so far (one per item with a KV tile)
+            bool ok = true;
+            int pg[8], ip[8];  // paged: page and first slot of each box of the current KV tile
+            for (int k = next_active<kPaged>(p, 0); ok && k >= 0; k = next_active<kPaged>(p, k + 1)) {
+                const Item it = decode_item<kPaged>(p, work_index(p, k));
+                if (q_issued > 0 && !(ok = mbar_wait(BAR(kBarQFree), static_cast<uint32_t>(q_issued - 1) & 1u,
+                                                     abort_flag, p.status, kSitePrefillTmaEmpty)))
                     break;
-                mbar_arrive_expect_tx(BAR(kBarFull0 + slot), C::kTileBytes);
-                const CUtensorMap *map = (it & 1) ? &tm_v : &tm_k;
-                const uint32_t dst = sRing + slot * C::kTileBytes;
+                const int n_q = (it.n[1] > 0) ? 2 : 1;
+                mbar_arrive_expect_tx(BAR(kBarQFull), n_q * C::kTileBytes);
 #pragma unroll
-                for (int c = 0; c < C::kChunks; ++c)
-                    tma_load_3d_hint(dst + c * C::kChunkBytes, map, BAR(kBarFull0 + slot), c * C::kChunkElems,
-                                     (it >> 1) * kBN, bh_kv, pol);
-                ++issued;
+                for (int x = 0; x < 2; ++x)
+                    if (x < n_q)
+#pragma unroll
+                        for (int c = 0; c < C::kChunks; ++c)
+                            tma_load_4d(sQ + x * C::kTileBytes + c * C::kChunkBytes, &tm_q, BAR(kBarQFull),
+                                        c * C::kChunkElems, it.q0[x], it.hq[x], it.b);
+                ++q_issued;
+                const int n_loads = 2 * it.n_max();  // K0, V0, K1, V1, ...
+                for (int i = 0; i < n_loads; ++i, ++kv) {
+                    const uint32_t slot = kv % kRing;
+                    if (!(ok = mbar_wait(BAR(kBarEmpty0 + slot), ((kv / kRing) & 1u) ^ 1u, abort_flag, p.status,
+                                         kSitePrefillTmaEmpty)))
+                        break;
+                    mbar_arrive_expect_tx(BAR(kBarFull0 + slot), C::kTileBytes);
+                    const CUtensorMap *map = (i & 1) ? &tm_v : &tm_k;
+                    const uint32_t dst = sRing + slot * C::kTileBytes;
+                    if constexpr (kPaged) {
+                        // The tile's keys come page by page, in boxes of min(page_size, 128) rows. A
+                        // box past the sequence's length, or whose block-table entry lies outside
+                        // [0, num_pages), reads the page beyond the last one: zeros.
+                        const int rows = min(p.page_size, kBN);
+                        const int n_box = kBN / rows;
+                        if ((i & 1) == 0) {  // K: look the pages up; V reuses them
+                            const int k0 = (i >> 1) * kBN;
+#pragma unroll
+                            for (int l = 0; l < 8; ++l) {
+                                const int key = k0 + l * rows;
+                                int page = p.num_pages;
+                                if (l < n_box && key < it.skv) {
+                                    page = __ldg(p.block_table + static_cast<size_t>(it.b) * p.pages_per_seq +
+                                                 key / p.page_size);
+                                    if (page < 0 || page >= p.num_pages)
+                                        page = p.num_pages;
+                                }
+                                pg[l] = page;
+                                ip[l] = key % p.page_size;
+                            }
+                        }
+#pragma unroll
+                        for (int l = 0; l < 8; ++l)
+                            if (l < n_box)
+#pragma unroll
+                                for (int c = 0; c < C::kChunks; ++c)
+                                    tma_load_4d_hint(dst + c * C::kChunkBytes + l * rows * C::kSwizzleBytes, map,
+                                                     BAR(kBarFull0 + slot), c * C::kChunkElems, ip[l], it.kvh, pg[l],
+                                                     pol);
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < C::kChunks; ++c)
+                            tma_load_4d_hint(dst + c * C::kChunkBytes, map, BAR(kBarFull0 + slot), c * C::kChunkElems,
+                                             (i >> 1) * kBN, it.kvh, it.b, pol);
+                    }
+                }
             }
             if (*abort_flag) {
                 // Let every copy already issued land before the CTA exits.
-                mbar_wait_drain(BAR(kBarQ), 0, 100000000ull);
-                for (int it = (issued > kRing ? issued - kRing : 0); it < issued; ++it)
-                    mbar_wait_drain(BAR(kBarFull0 + it % kRing), static_cast<uint32_t>(it / kRing) & 1u,
-                                    100000000ull);
+                if (q_issued > 0)
+                    mbar_wait_drain(BAR(kBarQFull), static_cast<uint32_t>(q_issued - 1) & 1u, 100000000ull);
+                for (uint32_t i = (kv > kRing ? kv - kRing : 0); i < kv; ++i)
+                    mbar_wait_drain(BAR(kBarFull0 + i % kRing), (i / kRing) & 1u, 100000000ull);
             }
         }
     } else if (warp == kWarpMma) {
@@ -296,34 +404,39 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool leader = elect_one();
             // Descriptors of the tile bases; a K step moves the start address, which is the low
             // field (address >> 4, 14 bits) of the descriptor: every address here is below 2^18.
+            // The three descriptors share their high word (stride offset, version, swizzle); only the
+            // low word (start address >> 4, leading-dimension offset) differs, and a K step or a
+            // ring slot only adds to the start address.
             const uint64_t desc_q0 = smem_desc(sQ, 16, kSbo, C::kSwizzleMode);
-            const uint64_t desc_k0 = smem_desc(sRing, 16, kSbo, C::kSwizzleMode);
-            const uint64_t desc_v0 = smem_desc(sRing, C::kChunkBytes, kSbo, C::kSwizzleMode);
-            constexpr uint64_t kSlotStep = static_cast<uint64_t>(C::kTileBytes >> 4);  // one tile, in descriptor units
+            const uint32_t desc_hi = static_cast<uint32_t>(desc_q0 >> 32);
+            const uint32_t q_lo = static_cast<uint32_t>(desc_q0);
+            const uint32_t k_lo = static_cast<uint32_t>(smem_desc(sRing, 16, kSbo, C::kSwizzleMode));
+            const uint32_t v_lo = static_cast<uint32_t>(smem_desc(sRing, C::kChunkBytes, kSbo, C::kSwizzleMode));
+            constexpr uint32_t kSlotStep = static_cast<uint32_t>(C::kTileBytes >> 4);  // one tile, in descriptor units
 
-            auto issue_s = [&](int x, int item) {
-                const uint64_t dq = desc_q0 + static_cast<uint64_t>(x) * kSlotStep;  // Q_B follows Q_A
-                const uint64_t dk = desc_k0 + static_cast<uint64_t>(item % kRing) * kSlotStep;
+            auto issue_s = [&](int x, uint32_t slot) {
+                const uint32_t dq = q_lo + static_cast<uint32_t>(x) * kSlotStep;  // Q_B follows Q_A
+                const uint32_t dk = k_lo + slot * kSlotStep;
                 if (leader) {
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const int c = kk / (C::kChunkElems / 16);
                         const int w = kk % (C::kChunkElems / 16);
-                        const uint64_t off = static_cast<uint64_t>((c * C::kChunkBytes + w * 32) >> 4);
-                        tc_mma_ss(tmem + col_s(x), dq + off, dk + off, kIdS, kk > 0 ? 1u : 0u);
+                        const uint32_t off = static_cast<uint32_t>((c * C::kChunkBytes + w * 32) >> 4);
+                        tc_mma_ss_lo(tmem + col_s(x), dq + off, dk + off, desc_hi, kIdS, kk > 0 ? 1u : 0u);
                     }
                 }
             };
             // PV for the keys of one half of the tile: kk in [half * kBN / 32, (half + 1) * kBN / 32).
-            auto issue_pv = [&](int x, int item, bool accumulate, int half) {
-                const uint64_t dv = desc_v0 + static_cast<uint64_t>(item % kRing) * kSlotStep;
+            auto issue_pv = [&](int x, uint32_t slot, bool accumulate, int half) {
+                const uint32_t dv = v_lo + slot * kSlotStep;
                 if (leader) {
 #pragma unroll
                     for (int kk = half * (kBN / 32); kk < (half + 1) * (kBN / 32); ++kk) {
                         // P_X: 16 keys = 8 packed columns per step, in the first half of S_X's columns.
-                        const uint64_t off = static_cast<uint64_t>((kk * 16 * C::kSwizzleBytes) >> 4);
-                        tc_mma_ts(tmem + col_o(x), tmem + col_s(x) + kk * 8, dv + off, kIdO,
-                                  (accumulate || kk > 0) ? 1u : 0u);
+                        const uint32_t off = static_cast<uint32_t>((kk * 16 * C::kSwizzleBytes) >> 4);
+                        tc_mma_ts_lo(tmem + col_o(x), tmem + col_s(x) + kk * 8, dv + off, desc_hi, kIdO,
+                                     (accumulate || kk > 0) ? 1u : 0u);
                     }
                 }
             };
@@ -331,57 +444,151 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (leader)
                     tc_commit(BAR(bar));
             };
-            auto wait_item = [&](int item) -> bool {
-                return mbar_wait(BAR(kBarFull0 + item % kRing), static_cast<uint32_t>(item / kRing) & 1u, abort_flag,
-                                 p.status, kSitePrefillMmaFull);
+            auto wait_kv = [&](uint32_t i) -> bool {
+                return mbar_wait(BAR(kBarFull0 + i % kRing), (i / kRing) & 1u, abort_flag, p.status,
+                                 kSitePrefillMmaFull);
             };
 
-            bool ok = mbar_wait(BAR(kBarQ), 0, abort_flag, p.status, kSitePrefillMmaQ);
-            if (ok && n_max > 0) {
-                ok = wait_item(0);
+            bool ok = true;
+            int r_cur = next_active<kPaged>(p, 0);  // this CTA's item index (items with KV tiles only)
+            Item it{};
+            if (r_cur >= 0) {
+                // The first item's S_X(0); every later item's are issued during the item before it.
+                it = decode_item<kPaged>(p, work_index(p, r_cur));
+                ok = mbar_wait(BAR(kBarQFull), 0, abort_flag, p.status, kSitePrefillMmaQ) && wait_kv(0);
                 if (ok) {
                     tc_fence_after_sync();
                     for (int x = 0; x < 2; ++x)
-                        if (n_of(x) > 0) {
+                        if (it.n[x] > 0) {
                             issue_s(x, 0);
                             commit(kBarSFull0 + x);
                         }
                     commit(kBarEmpty0 + 0);
                 }
             }
-            for (int j = 0; ok && j < n_max; ++j) {
-                const int item_v = 2 * j + 1, item_k = 2 * j + 2;
-                for (int x = 0; ok && x < 2; ++x) {
-                    if (j >= n_of(x))
-                        continue;
-                    // The first half of PV_X(j) runs while the softmax finishes the second half of P_X(j).
-                    if (!(ok = mbar_wait(BAR(kBarPHalf0 + x), static_cast<uint32_t>(j) & 1u, abort_flag, p.status,
-                                         kSitePrefillMmaPFull)))
-                        break;
-                    if (!(ok = wait_item(item_v)))
-                        break;
-                    tc_fence_after_sync();
-                    issue_pv(x, item_v, j > 0, 0);
-                    if (!(ok = mbar_wait(BAR(kBarPFull0 + x), static_cast<uint32_t>(j) & 1u, abort_flag, p.status,
-                                         kSitePrefillMmaPFull)))
-                        break;
-                    tc_fence_after_sync();
-                    issue_pv(x, item_v, true, 1);
-                    if (j + 1 < n_of(x)) {
-                        if (!(ok = wait_item(item_k)))
-                            break;
-                        tc_fence_after_sync();
-                        issue_s(x, item_k);
-                        commit(kBarSFull0 + x);
-                    } else {
-                        commit(kBarOFinal0 + x);
+            uint32_t kv_base = 0;           // ring position of the current item's K0
+            uint32_t p_cnt[2] = {0u, 0u};   // P_X tiles consumed so far (phase of PHalf_X / PFull_X)
+            for (int k = 0; ok && r_cur >= 0; ++k) {  // k: Q loads consumed so far (phase of QFull)
+                const int r_next = next_active<kPaged>(p, r_cur + 1);
+                const int w_next = (r_next >= 0) ? work_index(p, r_next) : -1;
+                const Item nx = (w_next >= 0) ? decode_item<kPaged>(p, w_next) : Item{};
+                const uint32_t kv_next = kv_base + 2u * static_cast<uint32_t>(it.n_max());  // next item's K0
+                // The Q tiles may be replaced once every S product of this item has been issued (and,
+                // by the commit, completed): the last S_X is S_X(n_X - 1), issued at j = n_X - 2.
+                int last_s_left = (it.n[0] >= 2 ? 1 : 0) + (it.n[1] >= 2 ? 1 : 0);
+                bool q_free = false;
+                // Tile X is done with this item once its last PV is issued: then the next item's
+                // S_X(0) may overwrite S_X (in-order execution keeps it behind that PV).
+                bool pending[2] = {it.n[0] == 0, it.n[1] == 0};
+                int next_s_left = (w_next >= 0) ? (nx.n[0] > 0 ? 1 : 0) + (nx.n[1] > 0 ? 1 : 0) : 0;
+                bool next_ready = false;  // next item's Q and K0 have landed
+                auto try_commit_q_free = [&]() {
+                    if (!q_free && last_s_left == 0) {
+                        commit(kBarQFree);
+                        q_free = true;
                     }
+                };
+                // Issue the next item's pending S_X(0) products. Non-blocking unless `block`: a Q or
+                // K0 still in flight leaves them pending, so the current item's PVs are not held up.
+                auto flush_next = [&](bool block) -> bool {
+                    if (!q_free)
+                        return true;
+#pragma unroll
+                    for (int y = 0; y < 2; ++y) {
+                        if (!pending[y])
+                            continue;
+                        if (w_next < 0 || nx.n[y] == 0) {
+                            pending[y] = false;
+                            continue;
+                        }
+                        if (!next_ready) {
+                            const uint32_t qpar = static_cast<uint32_t>(k + 1) & 1u;
+                            const uint32_t kpar = (kv_next / kRing) & 1u;
+                            const uint32_t kbar = BAR(kBarFull0 + kv_next % kRing);
+                            if (block) {
+                                if (!mbar_wait(BAR(kBarQFull), qpar, abort_flag, p.status, kSitePrefillMmaQ) ||
+                                    !mbar_wait(kbar, kpar, abort_flag, p.status, kSitePrefillMmaFull))
+                                    return false;
+                            } else if (!__all_sync(0xffffffffu, mbar_try_wait(BAR(kBarQFull), qpar) &&
+                                                                    mbar_try_wait(kbar, kpar))) {
+                                return true;
+                            }
+                            next_ready = true;
+                            tc_fence_after_sync();
+                        }
+                        issue_s(y, kv_next % kRing);
+                        commit(kBarSFull0 + y);
+                        pending[y] = false;
+                        if (--next_s_left == 0)
+                            commit(kBarEmpty0 + kv_next % kRing);  // both S products have read K0
+                    }
+                    return true;
+                };
+                try_commit_q_free();
+                ok = flush_next(false);
+                for (int j = 0; ok && j < it.n_max(); ++j) {
+                    const uint32_t item_v = kv_base + 2u * j + 1u, item_k = kv_base + 2u * j + 2u;
+                    if constexpr (kPaged) {
+                        // Rows of V_j past the sequence's length hold whatever the cache holds in the
+                        // last page's unused slots; their weights are 0, but 0 * NaN is not: zero them
+                        // before the first PV product reads the tile.
+                        const int r0 = it.skv - j * kBN;
+                        if (r0 < kBN) {
+                            if (!(ok = wait_kv(item_v)))
+                                break;
+                            uint4 *vt = reinterpret_cast<uint4 *>(smem + C::kOffRing + (item_v % kRing) * C::kTileBytes);
+                            constexpr int kUnitsPerRow = C::kSwizzleBytes / 16;
+                            for (int c = 0; c < C::kChunks; ++c)
+                                for (int u = r0 * kUnitsPerRow + lane; u < kBN * kUnitsPerRow; u += 32)
+                                    vt[c * (C::kChunkBytes / 16) + u] = make_uint4(0u, 0u, 0u, 0u);
+                            fence_proxy_async_smem();
+                            __syncwarp();
+                        }
+                    }
+#pragma unroll
+                    for (int x = 0; x < 2; ++x) {
+                        if (!ok || j >= it.n[x])
+                            continue;
+                        // The first half of PV_X(j) runs while the softmax finishes the second half of P_X(j).
+                        if (!(ok = mbar_wait(BAR(kBarPHalf0 + x), p_cnt[x] & 1u, abort_flag, p.status,
+                                             kSitePrefillMmaPFull)))
+                            continue;
+                        if (!(ok = wait_kv(item_v)))
+                            continue;
+                        tc_fence_after_sync();
+                        issue_pv(x, item_v % kRing, j > 0, 0);
+                        if (!(ok = mbar_wait(BAR(kBarPFull0 + x), p_cnt[x] & 1u, abort_flag, p.status,
+                                             kSitePrefillMmaPFull)))
+                            continue;
+                        ++p_cnt[x];
+                        tc_fence_after_sync();
+                        issue_pv(x, item_v % kRing, true, 1);
+                        if (j + 1 < it.n[x]) {
+                            if (!(ok = wait_kv(item_k)))
+                                continue;
+                            tc_fence_after_sync();
+                            issue_s(x, item_k % kRing);
+                            commit(kBarSFull0 + x);
+                            if (j + 2 == it.n[x])
+                                --last_s_left;
+                        } else {
+                            commit(kBarOFinal0 + x);
+                            pending[x] = true;
+                        }
+                        try_commit_q_free();
+                        ok = flush_next(false);
+                    }
+                    if (!ok)
+                        break;
+                    commit(kBarEmpty0 + item_v % kRing);
+                    if (j + 1 < it.n_max())
+                        commit(kBarEmpty0 + item_k % kRing);
                 }
-                if (!ok)
-                    break;
-                commit(kBarEmpty0 + item_v % kRing);
-                if (j + 1 < n_max)
-                    commit(kBarEmpty0 + item_k % kRing);
+                if (ok)
+                    ok = flush_next(true);
+                kv_base = kv_next;
+                it = nx;
+                r_cur = r_next;
             }
             // Every MMA issued above has completed once this barrier flips.
             commit(kBarDrain);
@@ -395,124 +602,165 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
         // ---------------------------------------------------------------- softmax / correction / epilogue
-        const int x = warp >> 2;        // query tile: 0 = A, 1 = B
+        const int x = warp >> 2;          // query tile: 0 = A, 1 = B
         const int r = threadIdx.x & 127;  // row within the tile == TMEM lane
-        const int row = q0_of(x) + r;
-        const int n = n_of(x);
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const uint32_t tS = tmem + lane_base + col_s(x);
         const uint32_t tO = tmem + lane_base + col_o(x);
         const float sl2 = p.scale_log2;
-        float m = -INFINITY;  // reference max, log2-scaled units
-        float l = 0.f;        // running sum of the exact fp32 weights (gives the LSE)
-        float l_pv = 0.f;     // running sum of the bf16-rounded weights the PV product uses (normalises O)
+        uint32_t phases = 0;  // bit 0: phase of SFull_X (one per S_X tile); bit 1: of OFinal_X (one per item)
         bool ok = true;
 
-        for (int j = 0; j < n; ++j) {
-            // The wait's result gates the warp-collective TMEM load below: the warp agrees on it.
-            if (!(ok = __all_sync(0xffffffffu, mbar_wait(BAR(kBarSFull0 + x), static_cast<uint32_t>(j) & 1u,
-                                                         abort_flag, p.status, kSitePrefillSoftmaxSFull))))
+        for (int k = 0; ok; ++k) {
+            const int w = work_index(p, k);
+            if (w < 0)
                 break;
-            tc_fence_after_sync();
-            uint32_t s_raw[kBN];
-            tmem_ld128_wait(tS, s_raw);
-            float s[kBN];
+            int n, q0, skv, off;
+            {
+                const Item it = decode_item<kPaged>(p, w);
+                n = x ? it.n[1] : it.n[0];
+                q0 = x ? it.q0[1] : it.q0[0];
+                skv = it.skv;
+                off = it.off;
+            }
+            const int row = q0 + r;
+            if (kPaged && n == 0 && q0 < p.Sq) {
+                // Paged: a tile none of whose rows sees a key (the sequence holds fewer keys than
+                // the rows before it): O = 0 and LSE = -inf, with no product to wait for.
+                if (row < p.Sq) {
+                    const Item it = decode_item<kPaged>(p, w);
+                    const int hq = x ? it.hq[1] : it.hq[0];
+                    uint4 *dst = reinterpret_cast<uint4 *>(p.o + it.b * p.o_sb + hq * p.o_sh + row * p.o_ss);
 #pragma unroll
-            for (int c = 0; c < kBN; ++c)
-                s[c] = __uint_as_float(s_raw[c]);
+                    for (int i = 0; i < D / 8; ++i)
+                        dst[i] = make_uint4(0u, 0u, 0u, 0u);
+                    p.lse[(static_cast<size_t>(it.b) * p.Hq + hq) * p.Sq + row] = -INFINITY;
+                }
+                continue;
+            }
+            float m = -INFINITY;  // reference max, log2-scaled units
+            float l = 0.f;        // running sum of the exact fp32 weights (gives the LSE)
+            float l_pv = 0.f;     // running sum of the bf16-rounded weights the PV product uses (normalises O)
 
-            const int k0 = j * kBN;
-            const bool need_mask = (k0 + kBN > p.Skv) || (p.causal && k0 + kBN - 1 > q0_of(x) + p.offset);
-            if (need_mask) {
-                int limit = p.Skv - 1 - k0;  // last visible column of this tile for this row
-                if (p.causal)
-                    limit = min(limit, row + p.offset - k0);
+            for (int j = 0; j < n; ++j) {
+                // The wait's result gates the warp-collective TMEM load below: the warp agrees on it.
+                if (!(ok = __all_sync(0xffffffffu, mbar_wait(BAR(kBarSFull0 + x), phases & 1u, abort_flag, p.status,
+                                                             kSitePrefillSoftmaxSFull))))
+                    break;
+                phases ^= 1u;
+                tc_fence_after_sync();
+                uint32_t s_raw[kBN];
+                tmem_ld128_wait(tS, s_raw);
+                float s[kBN];
 #pragma unroll
                 for (int c = 0; c < kBN; ++c)
-                    if (c > limit)
-                        s[c] = -INFINITY;
-            }
-            // Row max: eight independent chains of three-input maxima.
-            static_assert(kBN % 16 == 0, "row max walks the tile 16 columns at a time");
-            float mx8[8];
+                    s[c] = __uint_as_float(s_raw[c]);
+
+                const int k0 = j * kBN;
+                const bool need_mask = (k0 + kBN > skv) || (p.causal && k0 + kBN - 1 > q0 + off);
+                if (need_mask) {
+                    int limit = skv - 1 - k0;  // last visible column of this tile for this row
+                    if (p.causal)
+                        limit = min(limit, row + off - k0);
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                mx8[i] = fmaxf(s[2 * i], s[2 * i + 1]);
-#pragma unroll
-            for (int c = 16; c < kBN; c += 16)
+                    for (int c = 0; c < kBN; ++c)
+                        if (c > limit)
+                            s[c] = -INFINITY;
+                }
+                // Row max: eight independent chains of three-input maxima.
+                static_assert(kBN % 16 == 0, "row max walks the tile 16 columns at a time");
+                float mx8[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
-                    mx8[i] = fmax3(mx8[i], s[c + 2 * i], s[c + 2 * i + 1]);
-            const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
-            const float mx2 = mx * sl2;  // scale > 0, so the max commutes with scaling
-
-            float alpha = 1.f;
-            bool rescale = false;
-            if (j == 0) {
-                m = mx2;  // key 0 is visible to every row, so this is finite
-            } else {
-                const float m_new = fmaxf(m, mx2);
-                rescale = __any_sync(0xffffffffu, m_new > m + kRescaleThreshold);
-                if (rescale) {
-                    alpha = ex2(m - m_new);
-                    m = m_new;
-                }
-            }
-            // O_X is stable here (the commit announcing S_X(j) came after PV_X(j-1)), and PV_X(j) is
-            // not issued before the first arrival below, so the (rare) rescale fits in between.
-            if (rescale) {
-#pragma unroll 1
-                for (int cc = 0; cc < D / 32; ++cc) {
-                    uint32_t ov[32];
-                    tmem_ld32_wait(tO + cc * 32, ov);
+                    mx8[i] = fmaxf(s[2 * i], s[2 * i + 1]);
 #pragma unroll
-                    for (int i = 0; i < 32; i += 2) {
-                        const float2 v2 = __fmul2_rn(make_float2(__uint_as_float(ov[i]), __uint_as_float(ov[i + 1])),
-                                                     make_float2(alpha, alpha));
-                        ov[i] = __float_as_uint(v2.x);
-                        ov[i + 1] = __float_as_uint(v2.y);
+                for (int c = 16; c < kBN; c += 16)
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        mx8[i] = fmax3(mx8[i], s[c + 2 * i], s[c + 2 * i + 1]);
+                const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                                       fmaxf(mx8[6], mx8[7]));
+                const float mx2 = mx * sl2;  // scale > 0, so the max commutes with scaling
+
+                float alpha = 1.f;
+                bool rescale = false;
+                if (j == 0) {
+                    // Key 0 is visible to every row, so this is finite; with a paged cache a row may
+                    // see no key yet, and the floor keeps its weights 2^(-inf) = 0.
+                    m = kPaged ? fmaxf(mx2, kNoKeyMax) : mx2;
+                } else {
+                    const float m_new = fmaxf(m, mx2);
+                    rescale = __any_sync(0xffffffffu, m_new > m + kRescaleThreshold);
+                    if (rescale) {
+                        alpha = ex2(m - m_new);
+                        m = m_new;
                     }
-                    tmem_st32_wait(tO + cc * 32, ov);
                 }
-            }
-            // Exponentials, packed bf16 weights, and both running sums; P_X -> TMEM in two halves,
-            // each announced as soon as it is stored so that the tensor core can start on it.
-            const float2 sl2x2 = make_float2(sl2, sl2);
-            const float2 negm2 = make_float2(-m, -m);
-            float2 sum[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                             make_float2(0.f, 0.f)};
-            float sum_pv[4] = {0.f, 0.f, 0.f, 0.f};
+                // O_X is stable here (the commit announcing S_X(j) came after PV_X(j-1)), and PV_X(j) is
+                // not issued before the first arrival below, so the (rare) rescale fits in between.
+                if (rescale) {
+#pragma unroll 1
+                    for (int cc = 0; cc < D / 32; ++cc) {
+                        uint32_t ov[32];
+                        tmem_ld32_wait(tO + cc * 32, ov);
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t pk[32];
-#pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    const int col = half * 64 + 2 * c;
-                    const float2 e = __ffma2_rn(make_float2(s[col], s[col + 1]), sl2x2, negm2);
-                    const float2 pe = make_float2(ex2(e.x), ex2(e.y));
-                    pk[c] = pack_bf16x2(pe.x, pe.y);
-                    sum[c & 3] = __fadd2_rn(sum[c & 3], pe);
-                    sum_pv[c & 3] = add_bf16x2(sum_pv[c & 3], pk[c]);
+                        for (int i = 0; i < 32; i += 2) {
+                            const float2 v2 = __fmul2_rn(make_float2(__uint_as_float(ov[i]), __uint_as_float(ov[i + 1])),
+                                                         make_float2(alpha, alpha));
+                            ov[i] = __float_as_uint(v2.x);
+                            ov[i + 1] = __float_as_uint(v2.y);
+                        }
+                        tmem_st32_wait(tO + cc * 32, ov);
+                    }
                 }
-                tmem_st32(tS + half * 32, pk);
-                tmem_wait_st();
-                tc_fence_before_sync();
-                mbar_arrive(BAR((half == 0 ? kBarPHalf0 : kBarPFull0) + x));
+                // Exponentials, packed bf16 weights, and both running sums; P_X -> TMEM in two halves,
+                // each announced as soon as it is stored so that the tensor core can start on it.
+                const float2 sl2x2 = make_float2(sl2, sl2);
+                const float2 negm2 = make_float2(-m, -m);
+                float2 sum[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                                 make_float2(0.f, 0.f)};
+                float sum_pv[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) {
+                        const int col = half * 64 + 2 * c;
+                        const float2 e = __ffma2_rn(make_float2(s[col], s[col + 1]), sl2x2, negm2);
+                        const float2 pe = make_float2(ex2(e.x), ex2(e.y));
+                        pk[c] = pack_bf16x2(pe.x, pe.y);
+                        sum[c & 3] = __fadd2_rn(sum[c & 3], pe);
+                        sum_pv[c & 3] = add_bf16x2(sum_pv[c & 3], pk[c]);
+                    }
+                    tmem_st32(tS + half * 32, pk);
+                    tmem_wait_st();
+                    tc_fence_before_sync();
+                    mbar_arrive(BAR((half == 0 ? kBarPHalf0 : kBarPFull0) + x));
+                }
+                const float2 s01 = __fadd2_rn(__fadd2_rn(sum[0], sum[1]), __fadd2_rn(sum[2], sum[3]));
+                const float q01 = (sum_pv[0] + sum_pv[1]) + (sum_pv[2] + sum_pv[3]);
+                l = l * alpha + (s01.x + s01.y);
+                l_pv = l_pv * alpha + q01;
             }
-            const float2 s01 = __fadd2_rn(__fadd2_rn(sum[0], sum[1]), __fadd2_rn(sum[2], sum[3]));
-            const float q01 = (sum_pv[0] + sum_pv[1]) + (sum_pv[2] + sum_pv[3]);
-            l = l * alpha + (s01.x + s01.y);
-            l_pv = l_pv * alpha + q01;
-        }
+            if (!ok || n == 0)
+                continue;
 
-        if (ok && n > 0)
-            ok = __all_sync(0xffffffffu, mbar_wait(BAR(kBarOFinal0 + x), 0, abort_flag, p.status, kSitePrefillEpilogue));
-        if (ok && n > 0) {
+            // Epilogue. It overlaps the next item's first S product, which the issuer may start as
+            // soon as PV_X(n-1) is issued; the next PV_X, which overwrites O_X, waits for this
+            // warpgroup's first P arrival of the next item, which comes after these TMEM loads.
+            ok = __all_sync(0xffffffffu, mbar_wait(BAR(kBarOFinal0 + x), (phases >> 1) & 1u, abort_flag, p.status,
+                                                   kSitePrefillEpilogue));
+            phases ^= 2u;
+            if (!ok)
+                break;
             tc_fence_after_sync();
-            const float inv_l = 1.f / l_pv;
+            // Paged: a row that saw no key has l = 0: O = 0 and LSE = m + log2(0) = -inf.
+            const float inv_l = (kPaged && !(l_pv > 0.f)) ? 0.f : 1.f / l_pv;
             const bool store = row < p.Sq;
-            const size_t bh_q = static_cast<size_t>(bh_q_of(x));
-            __nv_bfloat16 *orow = p.o + (bh_q * p.Sq + (store ? row : 0)) * D;
+            const Item it = decode_item<kPaged>(p, w);
+            const int hq = x ? it.hq[1] : it.hq[0];
+            const size_t bh_q = static_cast<size_t>(it.b) * p.Hq + hq;
+            __nv_bfloat16 *orow = p.o + it.b * p.o_sb + hq * p.o_sh + (store ? row : 0) * p.o_ss;
 #pragma unroll 1
             for (int cc = 0; cc < D / 32; ++cc) {
                 uint32_t ov[32];
@@ -530,6 +778,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (store)
                 p.lse[bh_q * p.Sq + row] = (m + log2f(l)) * kLn2;
+            tc_fence_before_sync();
         }
     }
 
@@ -542,7 +791,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #undef BAR
 }
 
-template <int D>
+template <int D, bool kPaged>
 cudaError_t launch(const PrefillArgs &a, cudaStream_t stream, int *encode_error)
 {
     using C = Cfg<D>;
@@ -554,10 +803,24 @@ cudaError_t launch(const PrefillArgs &a, cudaStream_t stream, int *encode_error)
     const CUtensorMapSwizzle swz =
         (C::kSwizzleBytes == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
     CUtensorMap tq, tk, tv;
-    if (!make_map(encode, &tq, a.q, D, a.Sq, a.B * a.Hq, C::kChunkElems, 128, swz, encode_error) ||
-        !make_map(encode, &tk, a.k, D, a.Skv, a.B * a.Hkv, C::kChunkElems, 128, swz, encode_error) ||
-        !make_map(encode, &tv, a.v, D, a.Skv, a.B * a.Hkv, C::kChunkElems, 128, swz, encode_error))
+    auto st = [](const TensorStrides &t) { return Strides{t.b, t.h, t.s}; };
+    if (!make_map4(encode, &tq, a.q, 2, D, a.Sq, a.Hq, a.B, st(a.qs), C::kChunkElems, 128, swz, encode_error))
         return cudaErrorInvalidValue;
+    if constexpr (kPaged) {
+        // Pages [num_pages][Hkv][page_size][D] as (dim, slot, kv head, page), boxes of
+        // min(page_size, 128) slots; the page index num_pages lies past the end: zeros.
+        const Strides pst{static_cast<long long>(a.Hkv) * a.page_size * D, static_cast<long long>(a.page_size) * D, D};
+        const int rows = a.page_size < kBN ? a.page_size : kBN;
+        if (!make_map4(encode, &tk, a.k, 2, D, a.page_size, a.Hkv, a.num_pages, pst, C::kChunkElems, rows, swz,
+                       encode_error) ||
+            !make_map4(encode, &tv, a.v, 2, D, a.page_size, a.Hkv, a.num_pages, pst, C::kChunkElems, rows, swz,
+                       encode_error))
+            return cudaErrorInvalidValue;
+    } else {
+        if (!make_map4(encode, &tk, a.k, 2, D, a.Skv, a.Hkv, a.B, st(a.ks), C::kChunkElems, 128, swz, encode_error) ||
+            !make_map4(encode, &tv, a.v, 2, D, a.Skv, a.Hkv, a.B, st(a.vs), C::kChunkElems, 128, swz, encode_error))
+            return cudaErrorInvalidValue;
+    }
 
     // Per device: the attribute applies to the device current when it is set (benign race between
     // host threads: every caller sets the same value).
@@ -569,18 +832,21 @@ cudaError_t launch(const PrefillArgs &a, cudaStream_t stream, int *encode_error)
         // The setmaxnreg split inside the kernel is only valid for the register count it was
         // written for; refuse to launch a build that was compiled to anything else.
         cudaFuncAttributes fa;
-        cudaError_t e = cudaFuncGetAttributes(&fa, prefill_kernel<D>);
+        cudaError_t e = cudaFuncGetAttributes(&fa, prefill_kernel<D, kPaged>);
         if (e != cudaSuccess)
             return e;
         if (fa.numRegs != kLaunchRegs)
             return cudaErrorInvalidConfiguration;
-        e = cudaFuncSetAttribute(prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+        e = cudaFuncSetAttribute(prefill_kernel<D, kPaged>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
         if (e != cudaSuccess)
             return e;
         attr_set[dev] = true;
     }
     Params p;
     p.o = static_cast<__nv_bfloat16 *>(a.o);
+    p.o_sb = a.os.b;
+    p.o_sh = a.os.h;
+    p.o_ss = a.os.s;
     p.lse = a.lse;
     p.status = a.status;
     p.B = a.B;
@@ -591,12 +857,26 @@ cudaError_t launch(const PrefillArgs &a, cudaStream_t stream, int *encode_error)
     p.group = a.Hq / a.Hkv;
     p.offset = a.Skv - a.Sq;
     p.causal = a.causal;
+    if constexpr (kPaged) {
+        p.seq_lens = a.seq_lens;
+        p.block_table = a.block_table;
+        p.num_pages = a.num_pages;
+        p.page_size = a.page_size;
+        p.pages_per_seq = a.pages_per_seq;
+        const long long cap = static_cast<long long>(a.pages_per_seq) * a.page_size;
+        p.cap = static_cast<int>(cap < a.max_seq_len ? cap : a.max_seq_len);
+    }
     const int n_qtiles = (a.Sq + kBM - 1) / kBM;
     p.pair_heads = (p.group % 2 == 0) ? 1 : 0;
     p.n_items = p.pair_heads ? n_qtiles : (n_qtiles + 1) / 2;
     p.scale_log2 = a.scale * kLog2e;
-    const long long grid = static_cast<long long>(p.n_items) * a.B * (a.Hq / (p.pair_heads ? 2 : 1));
-    prefill_kernel<D><<<static_cast<unsigned>(grid), kThreads, C::kSmem, stream>>>(tq, tk, tv, p);
+    const long long n_work = static_cast<long long>(p.n_items) * a.B * (a.Hq / (p.pair_heads ? 2 : 1));
+    if (n_work > INT_MAX)
+        return cudaErrorInvalidValue;
+    p.n_work = static_cast<int>(n_work);
+    // Persistent: one CTA per SM (each holds all 512 TMEM columns), never more than the items.
+    const int grid = static_cast<int>(n_work < a.sm_count ? n_work : a.sm_count);
+    prefill_kernel<D, kPaged><<<static_cast<unsigned>(grid), kThreads, C::kSmem, stream>>>(tq, tk, tv, p);
     return cudaGetLastError();
 }
 
@@ -605,13 +885,15 @@ cudaError_t launch(const PrefillArgs &a, cudaStream_t stream, int *encode_error)
 cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t stream, int *encode_error)
 {
     *encode_error = 0;
+    if (a.seq_lens)  // paged, variable-length cache: head dim 128
+        return a.D == 128 ? launch<128, true>(a, stream, encode_error) : cudaErrorInvalidValue;
     switch (a.D) {
     case 32:
-        return launch<32>(a, stream, encode_error);
+        return launch<32, false>(a, stream, encode_error);
     case 64:
-        return launch<64>(a, stream, encode_error);
+        return launch<64, false>(a, stream, encode_error);
     case 128:
-        return launch<128>(a, stream, encode_error);
+        return launch<128, false>(a, stream, encode_error);
     default:
         return cudaErrorInvalidValue;
     }

@@ -89,6 +89,29 @@ int attn_fwd_ex(const void *q, const void *k, const void *v, void *o, float *lse
                 int B, int Hq, int Hkv, int Sq, int Skv, int D,
                 float scale, int causal, int decode_ctas, void *stream);
 
+/*
+ * attn_fwd_strided — attn_fwd over tensors in any layout whose head dim is contiguous, e.g. the
+ * token-major [B, S, H, D] that a projection writes, as well as the heads-major [B, H, S, D].
+ *
+ * Source (page title, section): the operation is attn_fwd's; the layout [B, H, Q_len, K_len] of the
+ * scores in "第11节：Attention 实现（Flash vs Fallback）", §4 fixes no memory layout for q, k, v and o,
+ * which is the caller's.
+ *
+ *   q_strides, k_strides, v_strides, o_strides   host arrays of three element strides each:
+ *       {batch, head, row} — element (b, h, i, d) of q is q[b*s[0] + h*s[1] + i*s[2] + d]. Every
+ *       stride must be >= 1, a multiple of 8 elements (16 bytes) and below 2^38; o's strides must
+ *       not make two output elements share an address (not checked).
+ *   lse       fp32 [B, Hq, Sq], contiguous, as for attn_fwd.
+ * Every other argument, rule and return value is attn_fwd's; a stride triple that breaks the rule
+ * above returns ATTN_ERR_ALIGN and NULL stride arrays ATTN_ERR_NULL, before any launch. A decode
+ * (Sq == 1) with D = 32 or 64 in a layout other than the contiguous one runs the prefill kernel (the
+ * CUDA-core decode kernel streams contiguous K/V rows only): correct, slower than attn_fwd's decode.
+ */
+int attn_fwd_strided(const void *q, const void *k, const void *v, void *o, float *lse,
+                     int B, int Hq, int Hkv, int Sq, int Skv, int D,
+                     const long long *q_strides, const long long *k_strides, const long long *v_strides,
+                     const long long *o_strides, float scale, int causal, void *stream);
+
 /* attn_decode_ctas — the number of CTAs attn_fwd would launch for a decode of this shape on the
  * current device (>= 1), or a negative attn_status. */
 int attn_decode_ctas(int B, int Hq, int Hkv, int Skv, int D);
@@ -175,6 +198,29 @@ int attn_decode_paged(const void *q, const void *k_pages, const void *v_pages, c
                       const int *seq_lens, void *o, float *lse, int B, int Hq, int Hkv, int num_pages,
                       int page_size, int pages_per_seq, int max_seq_len, float scale, int decode_ctas,
                       void *stream);
+
+/*
+ * attn_prefill_paged — chunked prefill over a paged, variable-length KV cache: for each sequence b,
+ * its Sq new query rows attend to the first len_b keys of its cache, the causal mask aligned to the
+ * cache's last Sq keys (query i sees key j iff j <= i + len_b - Sq).
+ *
+ * Source (page title, section): K = [past K, current K] with the -inf upper triangle on the last
+ * seq_len key columns — "第11节：Attention 实现（Flash vs Fallback）", §3; attending only to the filled
+ * part of a cache allocated for more tokens — same page, §3, and "Bộ 06 · Bên trong model", Q2–Q3.
+ * The cache layout is attn_decode_paged's (this library's choice; the pages describe none).
+ *
+ *   q            bf16 [B, Hq, Sq, 128] (the new tokens' queries; every sequence has Sq of them).
+ *   o, lse       bf16 [B, Hq, Sq, 128] and fp32 [B, Hq, Sq], written entirely.
+ *   k_pages, v_pages, block_table, seq_lens, max_seq_len, page_size   as attn_decode_paged: the
+ *                new tokens' keys and values must already be in the cache (len_b counts them).
+ *   causal       0 or 1. A row that sees no key (len_b < Sq under the mask, or len_b = 0) gets
+ *                o = 0 and lse = -inf.
+ * Head dim 128 only; Hq % Hkv == 0. Lengths are read on the device, never on the host. Returns
+ * ATTN_OK or a negative attn_status (argument errors before any launch).
+ */
+int attn_prefill_paged(const void *q, const void *k_pages, const void *v_pages, const int *block_table,
+                       const int *seq_lens, void *o, float *lse, int B, int Hq, int Hkv, int Sq, int num_pages,
+                       int page_size, int pages_per_seq, int max_seq_len, float scale, int causal, void *stream);
 
 /*
  * attn_bwd — backward pass of attn_fwd: given dout = dL/do for a loss L, the gradients

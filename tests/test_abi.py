@@ -203,3 +203,48 @@ def test_bwd_argument_errors(lib, name, slot, value, args, expected):
     if slot is not None:
         ptrs[slot] = value
     assert lib.attn_bwd(*ptrs, *args, None) == expected, name
+
+
+def _strided_call(lib, strides, D=64, B=1, Hq=4, Hkv=2, Sq=8, Skv=8):
+    import ctypes
+
+    arrs = [None if s is None else (ctypes.c_longlong * 3)(*s) for s in strides]
+    return lib.attn_fwd_strided(A[0], A[1], A[2], A[3], A[4], B, Hq, Hkv, Sq, Skv, D, *arrs, 0.125, 1, None)
+
+
+@pytest.mark.parametrize("name,strides,D,expected", [
+    ("null q strides", [None, (512, 64, 256), (512, 64, 256), (512, 64, 256)], 64, -1),
+    ("null o strides", [(512, 64, 256)] * 3 + [None], 64, -1),
+    ("stride not a multiple of 8", [(512, 64, 260)] + [(512, 64, 256)] * 3, 64, -5),
+    ("zero stride", [(512, 0, 256)] + [(512, 64, 256)] * 3, 64, -5),
+    ("negative stride", [(512, 64, 256)] * 3 + [(-512, 64, 256)], 64, -5),
+    ("huge stride", [(1 << 40, 64, 256)] + [(512, 64, 256)] * 3, 64, -5),
+    ("valid strides, bad head dim", [(512, 64, 256)] * 4, 48, -4),
+])
+def test_strided_argument_errors(lib, name, strides, D, expected):
+    assert _strided_call(lib, strides, D=D) == expected, name
+
+
+def _prefill_paged_call(lib, **kw):
+    a = dict(ptrs=[A[0], A[1], A[2], 0x60000, 0x70000, A[3], A[4]], B=2, Hq=8, Hkv=2, Sq=64, num_pages=10,
+             page_size=64, pages_per_seq=4, max_seq_len=256, scale=0.1, causal=1)
+    a.update(kw)
+    return lib.attn_prefill_paged(*a["ptrs"], a["B"], a["Hq"], a["Hkv"], a["Sq"], a["num_pages"], a["page_size"],
+                                  a["pages_per_seq"], a["max_seq_len"], a["scale"], a["causal"], None)
+
+
+@pytest.mark.parametrize("name,override,expected", [
+    ("null seq_lens", dict(ptrs=[A[0], A[1], A[2], 0x60000, 0, A[3], A[4]]), -1),
+    ("null o", dict(ptrs=[A[0], A[1], A[2], 0x60000, 0x70000, 0, A[4]]), -1),
+    ("zero queries", dict(Sq=0), -2),
+    ("page size 48", dict(page_size=48), -2),
+    ("page size 192", dict(page_size=192), -2),
+    ("negative max_seq_len", dict(max_seq_len=-1), -2),
+    ("causal 2", dict(causal=2), -2),
+    ("gqa", dict(Hkv=3), -3),
+    ("unaligned q", dict(ptrs=[A[0] + 8, A[1], A[2], 0x60000, 0x70000, A[3], A[4]]), -5),
+    ("unaligned table", dict(ptrs=[A[0], A[1], A[2], 0x60002, 0x70000, A[3], A[4]]), -5),
+    ("zero scale", dict(scale=0.0), -11),
+])
+def test_prefill_paged_argument_errors(lib, name, override, expected):
+    assert _prefill_paged_call(lib, **override) == expected, name
