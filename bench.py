@@ -390,6 +390,13 @@ def run_ours(args):
     fp8_ms = ranks.max([sum(a.elapsed_time(b) for a, b in fev)])[0]
     fp8_launch_s = fp8_ms * 1e-3 / fp8_steps
 
+    # Chunked prefill over a paged cache with per-sequence lengths (attn_prefill_paged), timed the
+    # same way: inputs resident, L2 flushed before every launch.
+    try:
+        paged = paged_prefill_leg(attn, args, ranks, dev, stream, clear_l2, world, peaks, peak_kind)
+    except Exception as e:  # an extra leg that fails is reported in its object, not allowed to drop the line
+        paged = {"metric": "paged chunked prefill TFLOP/s", "error": f"{type(e).__name__}: {e}"}
+
     # The backward pass of the 8B prefill workload (dq, dk, dv from dout and the forward's o, lse),
     # timed the same way. Reported beside the step, not part of it.
     try:
@@ -432,6 +439,7 @@ def run_ours(args):
                 "bytes_per_launch": fp8_bytes,
             },
             "backward": backward,
+            "paged_prefill": paged,
             "timed_region_ms": region_ms,
             "e2e": {"value": e2e_tflops, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": e2e_steps,
@@ -452,6 +460,8 @@ def run_ours(args):
 
 KERNEL_SOURCES = {
     "prefill_kernel": ["prefill_sm100.cu", "sm100_ptx.cuh"],
+    "prefill_kernel_paged": ["prefill_sm100.cu", "sm100_ptx.cuh"],
+    "bwd_kernel": ["bwd_sm100.cu", "sm100_ptx.cuh"],
     "decode_tc_kernel": ["decode_tc_sm100.cu", "sm100_ptx.cuh"],
     "decode_tc_kernel_fp8": ["decode_tc_sm100.cu", "sm100_ptx.cuh"],
 }
@@ -520,10 +530,54 @@ def backward_leg(attn, args, ranks, dev, stream, clear_l2, q, k, v, o, lse, worl
     return {"metric": "backward TFLOP/s (dq, dk, dv)", "value": whole_job_rate(world, flops, launch_s) / 1e12,
             "unit": "TFLOP/s", "config": PREFILL.config(), "steps": steps,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": tensor_peak, "unit": "TFLOP/s",
-                         "frac": achieved / tensor_peak, "traffic": None,
+                         "frac": achieved / tensor_peak, "traffic": read_traffic("bwd_kernel", PREFILL.name),
                          "peak_kind": f"{peak_kind} bf16 dense (burst)", "kernel": "bwd_kernel"},
             "us_per_launch": launch_s * 1e6, "flops_per_launch": flops,
             "device_status": attn.device_status(stream)}
+
+
+def paged_prefill_inputs(dev):
+    w = inputs.PAGED_CHUNKED
+    lens = inputs.paged_chunked_lengths()
+    q, k, v = inputs.generate(w)
+    kp, vp, table = inputs.paged_cache(k, v, lens, inputs.PAGED_CHUNKED_PAGE, seed=w.seed)
+    seq = torch.tensor(lens, dtype=torch.int32)
+    return w, lens, [t.to(dev) for t in (q, kp, vp, table, seq)]
+
+
+def paged_prefill_leg(attn, args, ranks, dev, stream, clear_l2, world, peaks, peak_kind):
+    """Time attn_prefill_paged on the paged chunked-prefill workload (per-sequence cache lengths):
+    L2 flushed before every launch, CUDA events around each, max over ranks."""
+    w, lens, (q, kp, vp, table, seq) = paged_prefill_inputs(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+    flops = 4 * w.D * w.Hq * inputs.paged_visible_pairs(w.Sq, lens)
+    call = lambda: attn.attn_prefill_paged(q, kp, vp, table, seq, max(lens), scale=w.scale, causal=True, out=o,
+                                           lse=lse, stream=stream)
+    for _ in range(args.warmup):
+        clear_l2()
+        call()
+    steps = max(3, min(args.steps, 100))
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+    ranks.barrier()
+    torch.cuda.synchronize(dev)
+    for s in range(steps):
+        clear_l2()
+        ev[s][0].record(stream)
+        call()
+        ev[s][1].record(stream)
+    torch.cuda.synchronize(dev)
+    ms = ranks.max([sum(a.elapsed_time(b) for a, b in ev)])[0]
+    launch_s = ms * 1e-3 / steps
+    tensor_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    achieved = flops / launch_s / 1e12
+    return {"metric": "paged chunked prefill TFLOP/s", "value": whole_job_rate(world, flops, launch_s) / 1e12,
+            "unit": "TFLOP/s", "config": dict(w.config(), seq_lens=lens, page_size=inputs.PAGED_CHUNKED_PAGE),
+            "steps": steps,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": tensor_peak, "unit": "TFLOP/s",
+                         "frac": achieved / tensor_peak, "traffic": read_traffic("prefill_kernel_paged", w.name),
+                         "peak_kind": f"{peak_kind} bf16 dense (burst)", "kernel": "prefill_kernel<128, paged>"},
+            "us_per_launch": launch_s * 1e6, "flops_per_launch": flops}
 
 
 def fp8_decode_bytes(w) -> int:
@@ -553,6 +607,19 @@ def run_case(args):
         print(json.dumps({"case": w.name + "_backward", "repeat": args.repeat, "us_per_launch": ms * 1e3,
                           "tflops": 5 * w.flops() / 2 / (ms * 1e-3) / 1e12,
                           "device_status": attn.device_status()}), flush=True)
+        return 0
+    if args.case == "chunked_paged":
+        w, lens, (q, kp, vp, table, seq) = paged_prefill_inputs(torch.device("cuda"))
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        ev[0].record()
+        for _ in range(args.repeat):
+            attn.attn_prefill_paged(q, kp, vp, table, seq, max(lens), scale=w.scale, causal=True)
+        ev[1].record()
+        torch.cuda.synchronize()
+        ms = ev[0].elapsed_time(ev[1]) / args.repeat
+        flops = 4 * w.D * w.Hq * inputs.paged_visible_pairs(w.Sq, lens)
+        print(json.dumps({"case": w.name, "repeat": args.repeat, "us_per_launch": ms * 1e3,
+                          "tflops": flops / (ms * 1e-3) / 1e12, "device_status": attn.device_status()}), flush=True)
         return 0
     if args.case == "decode_fp8":
         w = inputs.DECODE_GQA
@@ -593,7 +660,8 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--case", choices=sorted(inputs.SHORT_NAMES) + ["decode_fp8", "backward"], default=None,
+    ap.add_argument("--case", choices=sorted(inputs.SHORT_NAMES) + ["decode_fp8", "backward", "chunked_paged"],
+                    default=None,
                     help="only run this workload --repeat times (for profiling); prints no bench line")
     ap.add_argument("--repeat", type=int, default=3)
     args = ap.parse_args()

@@ -13,19 +13,24 @@
  *                    head of the kv head's group and every 128-row query tile that sees any of its
  *                    keys. Per step (one query tile), with keys in TMEM lanes:
  *                      S^T  = K Q^T      and  dP^T = V dO^T     (tcgen05.mma, both operands TMA tiles)
- *                      P^T, dS^T         the softmax warps (thread = key) recompute the weights from
- *                                        the LSE, apply the causal mask, form dS, and write P^T and
- *                                        dS^T back into TMEM as bf16 and dS into shared memory;
+ *                      P^T, dS^T         warps 0-7 (thread = key; warpgroup g takes query columns
+ *                                        [64 g, 64 g + 64)) recompute the weights from the LSE,
+ *                                        apply the causal mask, form dS, and write P^T and dS^T back
+ *                                        into TMEM as bf16 and dS into shared memory;
  *                      dV  += P^T dO     (A = P^T from TMEM, B = dO read MN-major)
  *                      dK  += dS^T Q     (A = dS^T from TMEM, B = Q read MN-major)
  *                      dQ   = dS K       (A = dS from shared memory, B = K read MN-major)
- *                    a second warpgroup (thread = query row) drains dQ with fp32 vector reductions
- *                    into the workspace; dK and dV stay in TMEM until the last step;
+ *                    the same warps (thread = query row, warpgroup g: dQ columns [64 g, 64 g + 64))
+ *                    then drain dQ with fp32 vector reductions into the workspace; dK and dV stay in
+ *                    TMEM until the last step. Splitting each step's columns over two warpgroups
+ *                    halves the serial softmax and drain time of a step (a single warp per SM
+ *                    sub-partition left them latency-bound);
  *   bwd_dq_kernel    dQ (fp32 workspace) -> bf16.
  *
- * TMEM (512 columns): [0,128) S^T, then P^T (bf16) in [0,64), then dQ; [128,256) dP^T, then dS^T
- * in [128,192); [256,384) dV; [384,512) dK. The MMAs of one thread run in issue order, so dV's read
- * of P^T is done before dQ overwrites those columns, and dK's read of dS^T before the next dP^T.
+ * TMEM (512 columns): [0,128) S^T, then P^T (bf16: queries 0-63 in [0,32), 64-127 in [64,96)), then
+ * dQ; [128,256) dP^T, then dS^T (likewise in [128,160) and [192,224)); [256,384) dV; [384,512) dK.
+ * The MMAs of one thread run in issue order, so dV's read of P^T is done before dQ overwrites those
+ * columns, and dK's read of dS^T before the next dP^T.
  *
  * Sources (page title, section): the backward pass recomputes the weights from the LSE the forward
  * saved instead of storing them — "AI Infra 入门：RMSNorm、Softmax、Causal Mask、Sampling 的数学与底层
@@ -208,9 +213,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(BAR(kBarStageEmpty0 + s), 1);
         }
         mbar_init(BAR(kBarSD), 1);
-        mbar_init(BAR(kBarP), 128);
+        mbar_init(BAR(kBarP), 256);
         mbar_init(BAR(kBarDQ), 1);
-        mbar_init(BAR(kBarDQFree), 128);
+        mbar_init(BAR(kBarDQFree), 256);
         mbar_init(BAR(kBarFinal), 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -267,6 +272,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         auto kmaj = [](uint32_t base, int kk) {  // K-major tile, K step kk (16 elements)
             return smem_desc(base + (kk >> 2) * kHalf + (kk & 3) * 32, 16, 1024, kSwizzle128B);
         };
+        // Packed P^T / dS^T of queries [16 kk, 16 kk + 16): each query half's bf16 pairs sit at the start
+        // of that half's own 64 fp32 columns (see the softmax warps).
+        auto pcol = [](int kk) { return static_cast<uint32_t>((kk >> 2) * 64 + (kk & 3) * 8); };
         auto mnmaj = [](uint32_t base, int kk) {  // MN-major tile, K step kk (16 rows of 128 bytes)
             return smem_desc(base + kk * 16 * 128, kHalf, 1024, kSwizzle128B);
         };
@@ -301,10 +309,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (leader) {
 #pragma unroll
                 for (int kk = 0; kk < kBQ / 16; ++kk)  // dV += P^T dO
-                    tc_mma_ts(tmem + kColDV, tmem + kColS + kk * 8, mnmaj(sDO, kk), kIdTS, (s > 0 || kk > 0) ? 1u : 0u);
+                    tc_mma_ts(tmem + kColDV, tmem + kColS + pcol(kk), mnmaj(sDO, kk), kIdTS, (s > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
                 for (int kk = 0; kk < kBQ / 16; ++kk)  // dK += dS^T Q
-                    tc_mma_ts(tmem + kColDK, tmem + kColDP + kk * 8, mnmaj(sQ, kk), kIdTS, (s > 0 || kk > 0) ? 1u : 0u);
+                    tc_mma_ts(tmem + kColDK, tmem + kColDP + pcol(kk), mnmaj(sQ, kk), kIdTS, (s > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
                 for (int kk = 0; kk < kBK / 16; ++kk)  // dQ = dS K (queries in TMEM lanes)
                     tc_mma_ss(tmem + kColS, kmaj(sDS, kk), mnmaj(sK, kk), kIdQ, kk > 0 ? 1u : 0u);
@@ -318,12 +326,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             atomicExch(p.status, kSiteBwd);
         }
         __syncwarp();
-    } else if (warp < 4) {
-        // ---------------------------------------------------------------- softmax warps: thread = key
-        const int kr = threadIdx.x;  // key within the tile == TMEM lane
+    } else if (warp < 8) {
+        // ---------------------------------------------------------------- softmax and dQ warps
+        // Warps w and w + 4 share TMEM lanes 32 (w % 4) .. + 31 and split the 128 columns of a step:
+        // warpgroup g takes query columns [64 g, 64 g + 64) of S^T and dP^T (thread = key), then dQ
+        // columns [64 g, 64 g + 64) (thread = query row). Each half packs its P^T and dS^T (bf16) in
+        // place at the start of its own columns, so the halves never write what the other reads.
+        const int grp = warp >> 2;
+        const int kr = threadIdx.x & 127;  // key (softmax) or query row (dQ) within the tile == TMEM lane
         const int key = k0 + kr;
-        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-        const uint32_t tS = tmem + lane_base + kColS, tDP = tmem + lane_base + kColDP;
+        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t tS = tmem + lane_base + kColS + 64u * grp, tDP = tmem + lane_base + kColDP + 64u * grp;
+        const uint32_t tQ = tmem + lane_base + kColS + 64u * grp;
         bool ok = true;
         for (int s = 0; s < n_steps; ++s) {
             const int st = s & 1;
@@ -332,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                          p.status, kSiteBwd))))
                 break;
             tc_fence_after_sync();
-            const int q0 = step_q0(s);
+            const int h = step_head(s), q0 = step_q0(s);
             const float *lse2 = reinterpret_cast<const float *>(smem + kOffVec + st * kVecBytes);
             const float *dvec = lse2 + kBQ;
             // Columns of this step's query tile that this key may feed: visible and inside Sq.
@@ -344,7 +358,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint8_t *dsrow_base = smem + kOffDS + (kr >> 6) * kHalf;
             const int kk = kr & 63;
 #pragma unroll 1
-            for (int c = 0; c < kBQ / 32; ++c) {
+            for (int c = 0; c < 2; ++c) {
+                const int cq = (2 * grp + c) * 32;  // first query column of this chunk
                 uint32_t sr[32], dr[32];
                 tmem_ld32_wait(tS + c * 32, sr);
                 tmem_ld32_wait(tDP + c * 32, dr);
@@ -354,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     float pe[2], ds[2];
 #pragma unroll
                     for (int u = 0; u < 2; ++u) {
-                        const int q = c * 32 + i + u;
+                        const int q = cq + i + u;
                         const bool vis = key_ok && q >= first_q && q <= last_q;
                         // Masked entries are exact zeros (lse2 and D of padding rows are never read).
                         const float w = vis ? ex2(__uint_as_float(sr[i + u]) * p.scale_log2 - lse2[q]) : 0.f;
@@ -366,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // dS (row q, column key) for the dQ product: K-major, 128-byte swizzle.
 #pragma unroll
                     for (int u = 0; u < 2; ++u) {
-                        const int q = c * 32 + i + u;
+                        const int q = cq + i + u;
                         const __nv_bfloat16 v = __float2bfloat16_rn(ds[u]);
                         *reinterpret_cast<__nv_bfloat16 *>(dsrow_base + q * 128 +
                                                            ((((kk >> 3) ^ (q & 7)) << 4) | ((kk & 7) << 1))) = v;
@@ -379,22 +394,44 @@ __global__ void __launch_bounds__(kThreads, 1)
             fence_proxy_async_smem();
             tc_fence_before_sync();
             mbar_arrive(BAR(kBarP));
+
+            // dQ of this step (thread = query row), scaled, added into the fp32 accumulator.
+            if (!(ok = __all_sync(0xffffffffu, mbar_wait(BAR(kBarDQ), static_cast<uint32_t>(s) & 1u, abort_flag,
+                                                         p.status, kSiteBwd))))
+                break;
+            tc_fence_after_sync();
+            const bool valid = q0 + kr < p.Sq;
+            float *acc = p.dq_acc + ((static_cast<size_t>(b) * p.Hq + h) * p.Sq + (valid ? q0 + kr : 0)) * kD + 64 * grp;
+#pragma unroll 1
+            for (int c = 0; c < 2; ++c) {
+                uint32_t v[32];
+                tmem_ld32_wait(tQ + c * 32, v);
+                if (valid) {
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4)
+                        red_add_v4(acc + c * 32 + i, __uint_as_float(v[i]) * p.scale, __uint_as_float(v[i + 1]) * p.scale,
+                                   __uint_as_float(v[i + 2]) * p.scale, __uint_as_float(v[i + 3]) * p.scale);
+                }
+                __syncwarp();
+            }
+            tc_fence_before_sync();
+            mbar_arrive(BAR(kBarDQFree));
         }
-        // Epilogue: dK (scaled) and dV rows of this key. The whole warp loads (tcgen05.ld is
-        // warp-collective); only the stores of keys past Skv are skipped.
+        // Epilogue: dims [64 grp, 64 grp + 64) of dK (scaled) and dV of this key. The whole warp
+        // loads (tcgen05.ld is warp-collective); only the stores of keys past Skv are skipped.
         const bool okf = __all_sync(0xffffffffu, ok && mbar_wait(BAR(kBarFinal), 0, abort_flag, p.status, kSiteBwd));
         const bool key_store = key < p.Skv;
         if (okf) {
             tc_fence_after_sync();
             const size_t row = static_cast<size_t>(bh_kv) * p.Skv + (key_store ? key : 0);
-            __nv_bfloat16 *dk_row = p.dk + row * kD;
-            __nv_bfloat16 *dv_row = p.dv + row * kD;
+            __nv_bfloat16 *dk_row = p.dk + row * kD + 64 * grp;
+            __nv_bfloat16 *dv_row = p.dv + row * kD + 64 * grp;
 #pragma unroll 1
-            for (int c = 0; c < kD / 32; ++c) {
+            for (int c = 0; c < 2; ++c) {
                 uint32_t kv[32], vv[32];
                 if (n_steps > 0) {
-                    tmem_ld32_wait(tmem + lane_base + kColDK + c * 32, kv);
-                    tmem_ld32_wait(tmem + lane_base + kColDV + c * 32, vv);
+                    tmem_ld32_wait(tmem + lane_base + kColDK + 64u * grp + c * 32, kv);
+                    tmem_ld32_wait(tmem + lane_base + kColDV + 64u * grp + c * 32, vv);
                 } else {
 #pragma unroll
                     for (int i = 0; i < 32; ++i)
@@ -417,35 +454,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 __syncwarp();
             }
-        }
-    } else if (warp < 8) {
-        // ---------------------------------------------------------------- dQ warps: thread = query row
-        // (warps 4-7 only: warps 10 and 11 have no role and go straight to the final barrier)
-        const int qr = threadIdx.x - 128;  // row within the query tile == TMEM lane
-        const uint32_t lane_base = static_cast<uint32_t>((warp - 4) * 32) << 16;
-        const uint32_t tQ = tmem + lane_base + kColS;
-        for (int s = 0; s < n_steps; ++s) {
-            if (!__all_sync(0xffffffffu, mbar_wait(BAR(kBarDQ), static_cast<uint32_t>(s) & 1u, abort_flag, p.status,
-                                                   kSiteBwd)))
-                break;
-            tc_fence_after_sync();
-            const int h = step_head(s), q0 = step_q0(s);
-            const bool valid = q0 + qr < p.Sq;
-            float *acc = p.dq_acc + ((static_cast<size_t>(b) * p.Hq + h) * p.Sq + (valid ? q0 + qr : 0)) * kD;
-#pragma unroll 1
-            for (int c = 0; c < kD / 32; ++c) {
-                uint32_t v[32];
-                tmem_ld32_wait(tQ + c * 32, v);
-                if (valid) {
-#pragma unroll
-                    for (int i = 0; i < 32; i += 4)
-                        red_add_v4(acc + c * 32 + i, __uint_as_float(v[i]) * p.scale, __uint_as_float(v[i + 1]) * p.scale,
-                                   __uint_as_float(v[i + 2]) * p.scale, __uint_as_float(v[i + 3]) * p.scale);
-                }
-                __syncwarp();
-            }
-            tc_fence_before_sync();
-            mbar_arrive(BAR(kBarDQFree));
         }
     }
 

@@ -21,6 +21,11 @@
  *                     memory as P^T (16 x 128, K-major, 128-byte swizzle);
  *   O^T += V_c^T P^T  tcgen05.mma, M = 128 dims (A = V_c read MN-major), N = 16 heads, K = 128 keys.
  *
+ * With the e4m3 cache the softmax takes two chunks (256 keys) per round: both chunks' S^T are
+ * committed together and both chunks' PV products issued together, so the round's fixed chain is
+ * paid once per 32 KB of codes; after the first round of a segment the warps exchange their maxima
+ * only when some key passes the rescale threshold (a counting barrier decides).
+ *
  * The tensor core takes the dot products, so each key costs the CUDA cores a handful of
  * instructions per head and the kernel streams K/V at memory speed. S^T is double-buffered in
  * TMEM and P^T in shared memory: S^T of chunk c+1 is computed while the softmax of chunk c runs.
@@ -81,22 +86,24 @@ enum TcBar : int {
 };
 
 // Shared-memory layout of one variant. bf16 cache: K and V chunks of 32 KB (two 64-dim box
-// columns each), three in flight, Q^T and P^T in bf16; one CTA per SM. e4m3 cache: chunks of 16 KB
-// (one 128-byte box column), two in flight, Q^T and P^T each as three e4m3 parts (hi, mid, lo) of
-// 16 x 128 bytes; about 100 KB, so two CTAs share an SM. The e4m3 decode streams half the bytes of
-// the bf16 one per key but pays the same per-chunk softmax chain, which then takes longer than the
-// chunk's memory time: a second resident CTA runs its chain in the gaps of the first.
+// columns each), three in flight, Q^T and P^T in bf16. e4m3 cache: chunks of 16 KB (one 128-byte
+// box column), five in flight, Q^T and P^T each as three e4m3 parts (hi, mid, lo) of 16 x 128 bytes.
+// One CTA per SM either way (two smaller CTAs per SM measured slower for the e4m3 cache: pairs then
+// have to be split between CTAs and merged).
 template <bool kFp8>
 struct Lay {
-    static constexpr int kStages = kFp8 ? 2 : 3;
+    static constexpr int kStages = kFp8 ? 5 : 3;
     static constexpr int kBoxCols = kFp8 ? 1 : 2;          // 128-byte box columns per K or V row
     static constexpr int kTileBytes = kBoxCols * kHalfBytes;  // one K or V chunk
     static constexpr int kStageBytes = 2 * kTileBytes;        // K chunk, then V chunk
-    static constexpr int kSmallBytes = kFp8 ? 3 * kSmallHalf : 2 * kSmallHalf;  // one Q^T slot or P^T buffer
+    static constexpr int kSmallBytes = kFp8 ? 3 * kSmallHalf : 2 * kSmallHalf;  // one Q^T slot, one chunk's P^T
+    // Chunks per softmax round: the e4m3 decode scores two chunks (256 keys) per round, so that the
+    // round's fixed chain (TMEM load, barrier, P^T hand-off, PV issue) is paid once per 32 KB of codes.
+    static constexpr int kRound = kFp8 ? 2 : 1;
     static constexpr int kOffRing = 0;
     static constexpr int kOffQ = kOffRing + kStages * kStageBytes;  // two Q^T slots (one per segment parity)
-    static constexpr int kOffP = kOffQ + 2 * kSmallBytes;           // two P^T buffers (one per chunk parity)
-    static constexpr int kOffQScale = kOffP + 2 * kSmallBytes;      // [segment parity][head] score scales
+    static constexpr int kOffP = kOffQ + 2 * kSmallBytes;           // two P^T buffers (one per round parity)
+    static constexpr int kOffQScale = kOffP + 2 * kRound * kSmallBytes;  // [segment parity][head] score scales
     static constexpr int kOffRedMax = kOffQScale + 2 * kN * 4;      // [chunk parity][warp][head] chunk maxima
     static constexpr int kOffRedSum = kOffRedMax + 2 * 4 * kN * 4;  // [warp][head][2] running sums
     static constexpr int kOffBar = kOffRedSum + 4 * kN * 2 * 4;
@@ -110,6 +117,8 @@ struct Lay {
     static_assert(kOffQ % 1024 == 0 && kOffP % 1024 == 0 && kSmallBytes % 1024 == 0,
                   "swizzled tiles sit on 1024-byte boundaries");
     static_assert(kStages <= kMaxStages, "barrier arrays");
+    // The MMA issuer holds a round's chunks until the next round's S^T is issued: two rounds in the ring.
+    static_assert(kStages >= 2 * kRound, "ring deep enough for two rounds");
     // The reference max moves when a chunk's max exceeds it by more than this (log2 units). With the
     // e4m3 cache the weights are scaled by 16 before they are split, and 16 * 2^4 = 256 stays below
     // the e4m3 maximum of 448.
@@ -117,8 +126,17 @@ struct Lay {
     static constexpr float kPScale = kFp8 ? 16.0f : 1.0f;
 };
 static_assert(Lay<false>::kStageBytes == 65536 && Lay<false>::kSmallBytes == 4096, "bf16 layout");
-constexpr uint32_t kTmemCols = 64;  // S^T [0,16) and [16,32), O^T [32,48)
-constexpr uint32_t kColO = 32;
+// TMEM: S^T of a round's chunks [round parity][slot] in 16-column groups from column 0, then O^T.
+template <bool kFp8>
+struct TmemLay {
+    static constexpr int kRound = kFp8 ? 2 : 1;
+    static constexpr uint32_t kColO = 32u * kRound;                // bf16: 32; e4m3: 64
+    static constexpr uint32_t kCols = kFp8 ? 128u : 64u;           // a power of two >= kColO + 16
+    __host__ __device__ static constexpr uint32_t col_s(int parity, int slot)
+    {
+        return 16u * static_cast<uint32_t>(kRound * parity + slot);
+    }
+};
 
 struct TcParams {
     __nv_bfloat16 *o;
@@ -226,6 +244,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 {
     static_assert(G >= 1 && G <= kN, "one pair's heads fit the MMA's N");
     using L = Lay<kFp8>;
+    using TL = TmemLay<kFp8>;
+    constexpr int kRound = L::kRound;
+    constexpr uint32_t kColO = TL::kColO;
+    static_assert(TL::kRound == L::kRound, "one round size");
     constexpr int kStages = L::kStages, kStageBytes = L::kStageBytes, kTileBytes = L::kTileBytes;
     constexpr int kSmallBytes = L::kSmallBytes, kOffRing = L::kOffRing, kOffQ = L::kOffQ, kOffP = L::kOffP;
     constexpr int kOffRedMax = L::kOffRedMax, kOffRedSum = L::kOffRedSum, kOffBar = L::kOffBar;
@@ -277,7 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // producer: keep them zero. Q^T and P^T are adjacent.
     {
         constexpr int kZeroFrom = kFp8 ? kOffQ : kOffP;
-        for (int i = threadIdx.x; i < (kOffP + 2 * kSmallBytes - kZeroFrom) / 16; i += kThreads)
+        for (int i = threadIdx.x; i < (kOffP + 2 * L::kRound * kSmallBytes - kZeroFrom) / 16; i += kThreads)
             reinterpret_cast<uint4 *>(smem + kZeroFrom)[i] = make_uint4(0u, 0u, 0u, 0u);
     }
     fence_proxy_async_smem();
@@ -287,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(&tm_v);
     }
     if (warp == kWarpMma) {
-        tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+        tmem_alloc(smem_u32(tmem_slot), TmemLay<kFp8>::kCols);
         tmem_relinquish();
     }
     if constexpr (kPaged) {
@@ -526,7 +548,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (leader)
                 tc_commit(BAR(bar));
         };
-        auto issue_s = [&](int c, int qs) {
+        // S^T of chunk c (ring stage c % kStages) against the segment's Q^T slot qs, into TMEM column dcol.
+        auto issue_s = [&](int c, int qs, uint32_t dcol) {
             const uint64_t dk = desc_k0 + static_cast<uint64_t>((c % kStages) * (kStageBytes >> 4));
             const uint64_t dq = desc_q0 + static_cast<uint64_t>(qs * (kSmallBytes >> 4));
             if constexpr (kFp8) {
@@ -536,7 +559,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int t = 0; t < 3; ++t)
 #pragma unroll
                         for (int kk = 0; kk < kD / 32; ++kk)
-                            tc_mma_f8_ss(tmem + 16u * static_cast<uint32_t>(c & 1), dk + static_cast<uint64_t>((kk * 32) >> 4),
+                            tc_mma_f8_ss(tmem + dcol, dk + static_cast<uint64_t>((kk * 32) >> 4),
                                          dq + static_cast<uint64_t>((t * kSmallHalf + kk * 32) >> 4), kIdS,
                                          (t > 0 || kk > 0) ? 1u : 0u);
                 }
@@ -547,13 +570,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int kk = 0; kk < kD / 16; ++kk) {
                     const uint64_t oa = static_cast<uint64_t>(((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4);
                     const uint64_t ob = static_cast<uint64_t>(((kk >> 2) * kSmallHalf + (kk & 3) * 32) >> 4);
-                    tc_mma_ss(tmem + 16u * static_cast<uint32_t>(c & 1), dk + oa, dq + ob, kIdS, kk > 0 ? 1u : 0u);
+                    tc_mma_ss(tmem + dcol, dk + oa, dq + ob, kIdS, kk > 0 ? 1u : 0u);
                 }
             }
         };
-        auto issue_o = [&](int c, bool accumulate) {
+        // O^T += V_c^T P^T with P^T from buffer (round parity rp, slot).
+        auto issue_o = [&](int c, int rp, int slot, bool accumulate) {
             const uint64_t dv = desc_v0 + static_cast<uint64_t>((c % kStages) * (kStageBytes >> 4));
-            const uint64_t dp = desc_p0 + static_cast<uint64_t>((c & 1) * (kSmallBytes >> 4));
+            const uint64_t dp = desc_p0 + static_cast<uint64_t>((rp * kRound + slot) * (kSmallBytes >> 4));
             if constexpr (kFp8) {
                 // O^T += V^T (P^T_hi + P^T_mid + P^T_lo): per part four K steps of 32 keys (32 rows of
                 // 128 bytes of the MN-major V chunk; 32 bytes of a P^T row).
@@ -577,26 +601,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         };
-        // O^T += V_c^T P^T once chunk c's weights are written; a segment's first chunk overwrites
-        // O^T, after the previous segment's O^T has been read out.
-        auto finish_o = [&](int c, bool first, int sg) -> bool {
+        // The PV products of round rnd (chunks c0 .. c0 + nk - 1) once its weights are written; a
+        // segment's first round overwrites O^T, after the previous segment's O^T has been read out.
+        auto finish_round = [&](int rnd, int c0, int nk, bool first, int sg) -> bool {
             if (first && sg > 0 &&
                 !mbar_wait(BAR(kBarOFree), static_cast<uint32_t>(sg - 1) & 1u, abort_flag, p.status, kSiteDecodeConsumer))
                 return false;
-            if (!mbar_wait(BAR(kBarPFull0 + (c & 1)), static_cast<uint32_t>(c >> 1) & 1u, abort_flag, p.status,
+            if (!mbar_wait(BAR(kBarPFull0 + (rnd & 1)), static_cast<uint32_t>(rnd >> 1) & 1u, abort_flag, p.status,
                            kSiteDecodeConsumer))
                 return false;
             tc_fence_after_sync();
-            issue_o(c, !first);
-            commit(kBarODone0 + (c & 1));
-            commit(kBarEmpty0 + c % kStages);
+            for (int k = 0; k < nk; ++k)
+                issue_o(c0 + k, rnd & 1, k, !first || k > 0);
+            commit(kBarODone0 + (rnd & 1));
+            for (int k = 0; k < nk; ++k)
+                commit(kBarEmpty0 + (c0 + k) % kStages);
             return true;
         };
 
+        // Rounds of up to kRound chunks, never across a segment boundary: all of a round's S^T are
+        // committed together, then the previous round's PV products are issued.
         bool ok = true;
-        int c = 0, seg = -1;
-        bool have_prev = false, prev_first = false;
-        int prev_seg = 0;
+        int c = 0, seg = -1, rnd = -1, slot = 0, cur_c0 = 0;
+        bool cur_first = false, have_prev = false, prev_first = false;
+        int prev_seg = 0, prev_rnd = 0, prev_c0 = 0, prev_nk = 0;
         UnitPos pos = locate(g_begin);
         int local = pos.local, cpp = pos.cpp;
         for (long long g = g_begin; ok && g < g_end; ++g) {
@@ -604,24 +632,38 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool last = (g + 1 == g_end) || (local + 1 == cpp);
             if (first) {
                 ++seg;
+                slot = 0;
                 if (!(ok = mbar_wait(BAR(kBarQFull0 + (seg & 1)), static_cast<uint32_t>(seg >> 1) & 1u, abort_flag,
                                      p.status, kSiteDecodeConsumer)))
                     break;
+            }
+            if (slot == 0) {
+                ++rnd;
+                cur_c0 = c;
+                cur_first = first;
             }
             if (!(ok = mbar_wait(BAR(kBarFull0 + c % kStages), static_cast<uint32_t>(c / kStages) & 1u, abort_flag,
                                  p.status, kSiteDecodeConsumer)))
                 break;
             tc_fence_after_sync();
-            issue_s(c, seg & 1);
-            commit(kBarSFull0 + (c & 1));
-            if (last)
-                commit(kBarQEmpty0 + (seg & 1));
-            // S^T(c) is queued behind O^T(c-1)'s predecessor; now the PV product of the previous chunk.
-            if (have_prev && !(ok = finish_o(c - 1, prev_first, prev_seg)))
-                break;
-            have_prev = true;
-            prev_first = first;
-            prev_seg = seg;
+            issue_s(c, seg & 1, TL::col_s(rnd & 1, slot));
+            if (slot == kRound - 1 || last) {
+                commit(kBarSFull0 + (rnd & 1));
+                if (last)
+                    commit(kBarQEmpty0 + (seg & 1));
+                // This round's S^T is queued; now the PV products of the previous round.
+                if (have_prev && !(ok = finish_round(prev_rnd, prev_c0, prev_nk, prev_first, prev_seg)))
+                    break;
+                have_prev = true;
+                prev_rnd = rnd;
+                prev_c0 = cur_c0;
+                prev_nk = c - cur_c0 + 1;
+                prev_first = cur_first;
+                prev_seg = seg;
+                slot = 0;
+            } else {
+                ++slot;
+            }
             ++c;
             if (++local == cpp && g + 1 < g_end) {
                 pos = locate(g + 1);
@@ -630,7 +672,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         if (ok && have_prev)
-            ok = finish_o(c - 1, prev_first, prev_seg);
+            ok = finish_round(prev_rnd, prev_c0, prev_nk, prev_first, prev_seg);
         commit(kBarDrain);
         if (!wait_drain(BAR(kBarDrain), 0, kWaitLimitNs) && leader) {
             *abort_flag = 1;
@@ -658,7 +700,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         bool ok = true;
-        int c = 0, n_deferred = 0, sg = 0;
+        int c = 0, n_deferred = 0, sg = 0, rnd = 0;  // chunks, deferred pairs, segments, rounds so far
         for (long long g = g_begin; g < g_end;) {
             const UnitPos pos = locate(g);
             const long long pair = pos.pair;
@@ -700,45 +742,80 @@ __global__ void __launch_bounds__(kThreads, 1)
                 l[h] = 0.f;
                 lpv[h] = 0.f;
             }
-            for (int j = 0; j < n_chunks; ++j, ++c) {
-                // Agreed by the warp: it gates the warp-collective TMEM load.
-                const bool okw = __all_sync(0xffffffffu, mbar_wait(BAR(kBarSFull0 + (c & 1)), static_cast<uint32_t>(c >> 1) & 1u,
+            const int n_rounds = (n_chunks + kRound - 1) / kRound;
+            for (int jr = 0; jr < n_rounds; ++jr) {
+                const int nk = min(kRound, n_chunks - jr * kRound);  // chunks in this round
+                const int rp = rnd & 1;
+                // Agreed by the warp: it gates the warp-collective TMEM loads.
+                const bool okw = __all_sync(0xffffffffu, mbar_wait(BAR(kBarSFull0 + rp), static_cast<uint32_t>(rnd >> 1) & 1u,
                                                                    abort_flag, p.status, kSiteDecodeConsumer));
-                float x[G];
-                if (okw) {
-                    tc_fence_after_sync();
-                    uint32_t r[16];
-                    tmem_ld16_wait(tS + 16u * static_cast<uint32_t>(c & 1), r);
-                    const bool valid = (local0 + j) * kCK + i < seq_len;
+                float x[kRound][G];
 #pragma unroll
-                    for (int h = 0; h < G; ++h) {
-                        x[h] = valid ? __uint_as_float(r[h]) * sl2[h] : -INFINITY;
-                        float v = x[h];
-#pragma unroll
-                        for (int o = 16; o > 0; o >>= 1)
-                            v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-                        if (lane == 0)
-                            red_max[((c & 1) * 4 + warp) * kN + h] = v;
-                    }
-                }
-                // One barrier per chunk both exchanges the warps' maxima and agrees on carrying on.
-                if (!(ok = bar_and(kBarSoftmax, kSoftmaxThreads, okw && ok)))
-                    break;
-                const float *rm = red_max + (c & 1) * 4 * kN;
-                bool rescale = false;
-                float cmax[G];
-#pragma unroll
-                for (int h = 0; h < G; ++h) {
-                    cmax[h] = fmaxf(fmaxf(rm[h], rm[kN + h]), fmaxf(rm[2 * kN + h], rm[3 * kN + h]));
-                    rescale = rescale || (cmax[h] > m[h] + L::kRescaleThreshold);
-                }
-                if (j == 0) {
+                for (int sl = 0; sl < kRound; ++sl)
 #pragma unroll
                     for (int h = 0; h < G; ++h)
-                        m[h] = cmax[h];  // the chunk holds at least one key, so this is finite
+                        x[sl][h] = -INFINITY;
+                if (okw) {
+                    tc_fence_after_sync();
+#pragma unroll
+                    for (int sl = 0; sl < kRound; ++sl) {
+                        if (sl < nk) {
+                            uint32_t r[16];
+                            tmem_ld16_wait(tS + TL::col_s(rp, sl), r);
+                            const bool valid = (local0 + jr * kRound + sl) * kCK + i < seq_len;
+#pragma unroll
+                            for (int h = 0; h < G; ++h)
+                                x[sl][h] = valid ? __uint_as_float(r[h]) * sl2[h] : -INFINITY;
+                        }
+                    }
+                }
+                // After the first round the exact round max is only needed when some key exceeds the
+                // reference max by the threshold: one counting barrier decides (and also catches a
+                // wait that ran out); only then do the warps exchange their maxima.
+                bool full = (jr == 0);
+                if (!full) {
+                    bool need = !(okw && ok);
+#pragma unroll
+                    for (int sl = 0; sl < kRound; ++sl)
+#pragma unroll
+                        for (int h = 0; h < G; ++h)
+                            need = need || (x[sl][h] > m[h] + L::kRescaleThreshold);
+                    full = bar_popc(kBarSoftmax, kSoftmaxThreads, need) != 0;
+                }
+                bool rescale = false;
+                float cmax[G];
+                if (full) {
+                    if (okw) {
+#pragma unroll
+                        for (int h = 0; h < G; ++h) {
+                            float v = x[0][h];
+#pragma unroll
+                            for (int sl = 1; sl < kRound; ++sl)
+                                v = fmaxf(v, x[sl][h]);
+#pragma unroll
+                            for (int o = 16; o > 0; o >>= 1)
+                                v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+                            if (lane == 0)
+                                red_max[(rp * 4 + warp) * kN + h] = v;
+                        }
+                    }
+                    // This barrier both exchanges the warps' maxima and agrees on carrying on.
+                    if (!(ok = bar_and(kBarSoftmax, kSoftmaxThreads, okw && ok)))
+                        break;
+                    const float *rm = red_max + rp * 4 * kN;
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        cmax[h] = fmaxf(fmaxf(rm[h], rm[kN + h]), fmaxf(rm[2 * kN + h], rm[3 * kN + h]));
+                        rescale = rescale || (cmax[h] > m[h] + L::kRescaleThreshold);
+                    }
+                }
+                if (jr == 0) {
+#pragma unroll
+                    for (int h = 0; h < G; ++h)
+                        m[h] = cmax[h];  // the round holds at least one key, so this is finite
                 } else if (rescale) {
-                    // The same values in every thread, so every thread takes this branch. O^T(c-1)
-                    // must be complete before it is scaled.
+                    // The same values in every thread, so every thread takes this branch. O^T of the
+                    // previous round must be complete before it is scaled.
                     float alpha[G];
 #pragma unroll
                     for (int h = 0; h < G; ++h) {
@@ -748,8 +825,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         l[h] *= alpha[h];
                         lpv[h] *= alpha[h];
                     }
-                    if (__all_sync(0xffffffffu, mbar_wait(BAR(kBarODone0 + ((c - 1) & 1)),
-                                                          static_cast<uint32_t>((c - 1) >> 1) & 1u, abort_flag,
+                    if (__all_sync(0xffffffffu, mbar_wait(BAR(kBarODone0 + ((rnd - 1) & 1)),
+                                                          static_cast<uint32_t>((rnd - 1) >> 1) & 1u, abort_flag,
                                                           p.status, kSiteDecodeConsumer))) {
                         tc_fence_after_sync();
                         uint32_t ov[16];
@@ -762,69 +839,76 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                     }
                 }
-                // Weights, both running sums, and P^T (row h, column i) for the PV product. P^T is
-                // K-major with the 128-byte swizzle: key i sits in half i / 64 of row h, in 16-byte
-                // unit ((i % 64) / 8) XOR (h % 8).
-                if constexpr (kFp8) {
-                    // e4m3 cache: the weight times 16 as three e4m3 parts, each in its own 16 x 128-byte
-                    // tile: key i is byte (i % 16) of 16-byte unit (i / 16) XOR (h % 8) in row h. lpv sums
-                    // what the PV product uses (in units of 1/16, like O^T).
-                    uint8_t *pbuf = smem + kOffP + (c & 1) * kSmallBytes;
-                    auto off_of = [&](int h) { return (h >> 3) * 1024 + (h & 7) * 128 + ((((i >> 4) ^ (h & 7)) << 4) | (i & 15)); };
+                // Weights, both running sums, and P^T (row h, column i) of each chunk of the round for
+                // its PV product. P^T is K-major with the 128-byte swizzle: key i sits in half i / 64
+                // of row h, in 16-byte unit ((i % 64) / 8) XOR (h % 8).
 #pragma unroll
-                    for (int h = 0; h < G; h += 2) {  // two heads per conversion
-                        constexpr bool kPair = G > 1;
-                        const float pa = ex2(x[h] - m[h]);
-                        const float pb = kPair ? ex2(x[h + (kPair ? 1 : 0)] - m[h + (kPair ? 1 : 0)]) : 0.f;
-                        float wa = pa * L::kPScale, wb = pb * L::kPScale;
-                        const float ua = wa, ub = wb;
+                for (int sl = 0; sl < kRound; ++sl) {
+                    if (sl >= nk)
+                        break;
+                    if constexpr (kFp8) {
+                        // e4m3 cache: the weight times 16 as three e4m3 parts, each in its own 16 x 128-byte
+                        // tile: key i is byte (i % 16) of 16-byte unit (i / 16) XOR (h % 8) in row h. lpv sums
+                        // what the PV product uses (in units of 1/16, like O^T).
+                        uint8_t *pbuf = smem + kOffP + (rp * kRound + sl) * kSmallBytes;
+                        auto off_of = [&](int h) { return (h >> 3) * 1024 + (h & 7) * 128 + ((((i >> 4) ^ (h & 7)) << 4) | (i & 15)); };
 #pragma unroll
-                        for (int t = 0; t < 3; ++t) {
-                            const uint32_t cd = e4m3x2(wa, wb);
-                            const float2 v = e4m3x2_value(cd);
-                            wa -= v.x;
-                            wb -= v.y;
-                            pbuf[t * kSmallHalf + off_of(h)] = static_cast<uint8_t>(cd & 0xffu);
-                            if (kPair)
-                                pbuf[t * kSmallHalf + off_of(h + 1)] = static_cast<uint8_t>((cd >> 8) & 0xffu);
+                        for (int h = 0; h < G; h += 2) {  // two heads per conversion
+                            constexpr bool kPair = G > 1;
+                            const float pa = ex2(x[sl][h] - m[h]);
+                            const float pb = kPair ? ex2(x[sl][h + (kPair ? 1 : 0)] - m[h + (kPair ? 1 : 0)]) : 0.f;
+                            float wa = pa * L::kPScale, wb = pb * L::kPScale;
+                            const float ua = wa, ub = wb;
+#pragma unroll
+                            for (int t = 0; t < 3; ++t) {
+                                const uint32_t cd = e4m3x2(wa, wb);
+                                const float2 v = e4m3x2_value(cd);
+                                wa -= v.x;
+                                wb -= v.y;
+                                pbuf[t * kSmallHalf + off_of(h)] = static_cast<uint8_t>(cd & 0xffu);
+                                if (kPair)
+                                    pbuf[t * kSmallHalf + off_of(h + 1)] = static_cast<uint8_t>((cd >> 8) & 0xffu);
+                            }
+                            // The parts' sum is the weight minus what is left over (exact: it needs ~12 bits).
+                            l[h] += pa;
+                            lpv[h] += ua - wa;
+                            if (kPair) {
+                                l[h + (kPair ? 1 : 0)] += pb;
+                                lpv[h + (kPair ? 1 : 0)] += ub - wb;
+                            }
                         }
-                        // The parts' sum is the weight minus what is left over (exact: it needs ~12 bits).
-                        l[h] += pa;
-                        lpv[h] += ua - wa;
-                        if (kPair) {
-                            l[h + (kPair ? 1 : 0)] += pb;
-                            lpv[h + (kPair ? 1 : 0)] += ub - wb;
+                    } else {
+                        uint8_t *pbuf = smem + kOffP + (rp * kRound + sl) * kSmallBytes + (i >> 6) * kSmallHalf;
+                        const int kk = i & 63;
+#pragma unroll
+                        for (int h = 0; h < G; ++h) {
+                            const float pe = ex2(x[sl][h] - m[h]);
+                            l[h] += pe;
+                            const __nv_bfloat16 pb = __float2bfloat16_rn(pe);
+                            lpv[h] += __bfloat162float(pb);
+                            const int off = (h >> 3) * 1024 + (h & 7) * 128 + ((((kk >> 3) ^ (h & 7)) << 4) | ((kk & 7) << 1));
+                            *reinterpret_cast<__nv_bfloat16 *>(pbuf + off) = pb;
                         }
                     }
-                } else {
-                    uint8_t *pbuf = smem + kOffP + (c & 1) * kSmallBytes + (i >> 6) * kSmallHalf;
-                    const int kk = i & 63;
+                    if constexpr (kPaged) {
+                        // Rows past the sequence's length in its last page hold whatever the cache holds
+                        // there; their weights are 0, but 0 * NaN is not, so zero them before the PV product.
+                        if ((local0 + jr * kRound + sl) * kCK + i >= seq_len) {
+                            uint4 *vrow = reinterpret_cast<uint4 *>(smem + kOffRing + ((c + sl) % kStages) * kStageBytes +
+                                                                    kTileBytes + i * 128);
 #pragma unroll
-                    for (int h = 0; h < G; ++h) {
-                        const float pe = ex2(x[h] - m[h]);
-                        l[h] += pe;
-                        const __nv_bfloat16 pb = __float2bfloat16_rn(pe);
-                        lpv[h] += __bfloat162float(pb);
-                        const int off = (h >> 3) * 1024 + (h & 7) * 128 + ((((kk >> 3) ^ (h & 7)) << 4) | ((kk & 7) << 1));
-                        *reinterpret_cast<__nv_bfloat16 *>(pbuf + off) = pb;
-                    }
-                }
-                if constexpr (kPaged) {
-                    // Rows past the sequence's length in its last page hold whatever the cache holds
-                    // there; their weights are 0, but 0 * NaN is not, so zero them before the PV product.
-                    if ((local0 + j) * kCK + i >= seq_len) {
-                        uint4 *vrow = reinterpret_cast<uint4 *>(smem + kOffRing + (c % kStages) * kStageBytes + kTileBytes +
-                                                                i * 128);
+                            for (int hf = 0; hf < L::kBoxCols; ++hf)
 #pragma unroll
-                        for (int hf = 0; hf < L::kBoxCols; ++hf)
-#pragma unroll
-                            for (int u = 0; u < 8; ++u)
-                                vrow[hf * (kHalfBytes / 16) + u] = make_uint4(0u, 0u, 0u, 0u);
+                                for (int u = 0; u < 8; ++u)
+                                    vrow[hf * (kHalfBytes / 16) + u] = make_uint4(0u, 0u, 0u, 0u);
+                        }
                     }
                 }
                 fence_proxy_async_smem();
                 tc_fence_before_sync();
-                mbar_arrive(BAR(kBarPFull0 + (c & 1)));
+                mbar_arrive(BAR(kBarPFull0 + rp));
+                c += nk;
+                ++rnd;
             }
             if (!ok)
                 break;
@@ -843,7 +927,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     red_sum[(warp * kN + h) * 2 + 1] = q;
                 }
             }
-            const bool okw = mbar_wait(BAR(kBarODone0 + ((c - 1) & 1)), static_cast<uint32_t>((c - 1) >> 1) & 1u,
+            const bool okw = mbar_wait(BAR(kBarODone0 + ((rnd - 1) & 1)), static_cast<uint32_t>((rnd - 1) >> 1) & 1u,
                                        abort_flag, p.status, kSiteDecodeConsumer);
             if (!(ok = bar_and(kBarSoftmax, kSoftmaxThreads, okw && ok)))
                 break;
@@ -966,7 +1050,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     if (warp == kWarpMma) {
         tc_fence_after_sync();
-        tmem_dealloc(tmem, kTmemCols);
+        tmem_dealloc(tmem, TmemLay<kFp8>::kCols);
     }
 #undef BAR
 }

@@ -457,4 +457,16 @@ __device__ __forceinline__ bool bar_and(int id, int nthreads, bool pred)
     return out != 0;
 }
 
+// Named barrier `id` over `nthreads` threads that also counts the participants passing true.
+__device__ __forceinline__ uint32_t bar_popc(int id, int nthreads, bool pred)
+{
+    uint32_t out;
+    asm volatile("{\n\t.reg .pred pi;\n\tsetp.ne.u32 pi, %1, 0;\n\t"
+                 "barrier.red.popc.u32 %0, %2, %3, pi;\n\t}"
+                 : "=r"(out)
+                 : "r"(pred ? 1u : 0u), "r"(id), "r"(nthreads)
+                 : "memory");
+    return out;
+}
+
 }  // namespace attn_b200

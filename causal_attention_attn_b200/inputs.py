@@ -139,3 +139,56 @@ def sample_rows(w: Workload, every: int = 64, seed: int = 7) -> torch.Tensor:
             picks = set(range(0, w.Sq, every)) | {0, w.Sq - 1, min(max(w.offset, 0), w.Sq - 1)}
             rows.extend(base + i for i in sorted(picks))
     return torch.tensor(rows, dtype=torch.int64)
+
+
+def paged_cache(k: torch.Tensor, v: torch.Tensor, lens, page_size: int, seed: int):
+    """Scatter each sequence's first lens[b] rows of a dense cache k, v [B, Hkv, cap, D] into pages
+    of `page_size` slots in a seeded random order: ``(k_pages, v_pages, block_table)`` with pages
+    [num_pages, Hkv, page_size, D] (unused slots zero) and an int32 table [B, ceil(cap / page_size)]
+    whose unused entries point past the last page. Layout preparation for a paged cache only."""
+    B, Hkv, cap, D = k.shape
+    per_seq = -(-cap // page_size)
+    num_pages = B * per_seq
+    perm = torch.randperm(num_pages, generator=torch.Generator().manual_seed(seed))
+    table = torch.full((B, per_seq), num_pages, dtype=torch.int32)
+    kp = torch.zeros((num_pages, Hkv, page_size, D), dtype=k.dtype)
+    vp = torch.zeros_like(kp)
+    nxt = 0
+    for b in range(B):
+        for n in range(-(-min(int(lens[b]), cap) // page_size)):
+            pg = int(perm[nxt])
+            nxt += 1
+            table[b, n] = pg
+            lo, hi = n * page_size, min((n + 1) * page_size, int(lens[b]))
+            kp[pg, :, :hi - lo] = k[b, :, lo:hi]
+            vp[pg, :, :hi - lo] = v[b, :, lo:hi]
+    return kp, vp, table
+
+
+# Chunked prefill over a paged cache with per-sequence lengths: the chunked-prefill shape (8
+# sequences, 256 new tokens each, 32 query / 8 kv heads, D 128) with cache lengths drawn uniformly
+# from [256, 1024] (seed 1005), in pages of 64 keys.
+PAGED_CHUNKED = Workload("paged_chunked_prefill_b8_hq32_hkv8_sq256_skv256to1024_page64", 8, 32, 8, 256, 1024, 128,
+                         True, 1005)
+PAGED_CHUNKED_PAGE = 64
+
+
+def paged_chunked_lengths():
+    g = torch.Generator().manual_seed(PAGED_CHUNKED.seed)
+    return [int(x) for x in torch.randint(256, 1025, (PAGED_CHUNKED.B,), generator=g)]
+
+
+def paged_visible_pairs(Sq: int, lens, causal: bool = True) -> int:
+    """Visible (query, key) pairs per head summed over sequences: Sq new queries over len_b keys."""
+    total = 0
+    for L in lens:
+        if not causal:
+            total += Sq * L
+            continue
+        off = L - Sq
+        if off >= 0:
+            total += Sq * off + Sq * (Sq + 1) // 2
+        else:  # rows i < -off see no key
+            n = L
+            total += n * (n + 1) // 2
+    return total
