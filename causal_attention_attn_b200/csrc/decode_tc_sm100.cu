@@ -21,10 +21,10 @@
  *                     memory as P^T (16 x 128, K-major, 128-byte swizzle);
  *   O^T += V_c^T P^T  tcgen05.mma, M = 128 dims (A = V_c read MN-major), N = 16 heads, K = 128 keys.
  *
- * With the e4m3 cache the softmax takes two chunks (256 keys) per round: both chunks' S^T are
- * committed together and both chunks' PV products issued together, so the round's fixed chain is
- * paid once per 32 KB of codes; after the first round of a segment the warps exchange their maxima
- * only when some key passes the rescale threshold (a counting barrier decides).
+ * The softmax works in rounds of kRound chunks (one; the loop is written for more): a round's S^T
+ * are committed together and its PV products issued together. After the first round of a segment
+ * the warps exchange their maxima only when some key passes the rescale threshold (a counting
+ * barrier decides).
  *
  * The tensor core takes the dot products, so each key costs the CUDA cores a handful of
  * instructions per head and the kernel streams K/V at memory speed. S^T is double-buffered in
@@ -97,9 +97,10 @@ struct Lay {
     static constexpr int kTileBytes = kBoxCols * kHalfBytes;  // one K or V chunk
     static constexpr int kStageBytes = 2 * kTileBytes;        // K chunk, then V chunk
     static constexpr int kSmallBytes = kFp8 ? 3 * kSmallHalf : 2 * kSmallHalf;  // one Q^T slot, one chunk's P^T
-    // Chunks per softmax round: the e4m3 decode scores two chunks (256 keys) per round, so that the
-    // round's fixed chain (TMEM load, barrier, P^T hand-off, PV issue) is paid once per 32 KB of codes.
-    static constexpr int kRound = kFp8 ? 2 : 1;
+    // Chunks per softmax round (the S^T of a round's chunks is committed together and their PV
+    // products issued together). One for both caches: two-chunk rounds measured slower for the e4m3
+    // cache (41.0 -> 45.1 us), the issuer then holding four of the five ring stages.
+    static constexpr int kRound = 1;
     static constexpr int kOffRing = 0;
     static constexpr int kOffQ = kOffRing + kStages * kStageBytes;  // two Q^T slots (one per segment parity)
     static constexpr int kOffP = kOffQ + 2 * kSmallBytes;           // two P^T buffers (one per round parity)
@@ -129,9 +130,9 @@ static_assert(Lay<false>::kStageBytes == 65536 && Lay<false>::kSmallBytes == 409
 // TMEM: S^T of a round's chunks [round parity][slot] in 16-column groups from column 0, then O^T.
 template <bool kFp8>
 struct TmemLay {
-    static constexpr int kRound = kFp8 ? 2 : 1;
-    static constexpr uint32_t kColO = 32u * kRound;                // bf16: 32; e4m3: 64
-    static constexpr uint32_t kCols = kFp8 ? 128u : 64u;           // a power of two >= kColO + 16
+    static constexpr int kRound = Lay<kFp8>::kRound;
+    static constexpr uint32_t kColO = 32u * kRound;                // after the double-buffered S^T of the rounds
+    static constexpr uint32_t kCols = kRound == 1 ? 64u : 128u;    // a power of two >= kColO + 16
     __host__ __device__ static constexpr uint32_t col_s(int parity, int slot)
     {
         return 16u * static_cast<uint32_t>(kRound * parity + slot);
