@@ -128,14 +128,18 @@ struct Lay {
 };
 static_assert(Lay<false>::kStageBytes == 65536 && Lay<false>::kSmallBytes == 4096, "bf16 layout");
 // TMEM: S^T of a round's chunks [round parity][slot] in 16-column groups from column 0, then O^T.
+// With the e4m3 cache every product is a sum over three e4m3 parts (of Q^T or of P^T); each part
+// accumulates in its own 16 columns, so that the tensor core's chain of dependent accumulations is
+// four instructions long instead of twelve, and the readers add the parts.
 template <bool kFp8>
 struct TmemLay {
     static constexpr int kRound = Lay<kFp8>::kRound;
-    static constexpr uint32_t kColO = 32u * kRound;                // after the double-buffered S^T of the rounds
-    static constexpr uint32_t kCols = kRound == 1 ? 64u : 128u;    // a power of two >= kColO + 16
+    static constexpr int kParts = kFp8 ? 3 : 1;
+    static constexpr uint32_t kColO = 32u * kRound * kParts;       // after the double-buffered S^T of the rounds
+    static constexpr uint32_t kCols = (kColO + 16u * kParts <= 64u) ? 64u : (kColO + 16u * kParts <= 128u) ? 128u : 256u;
     __host__ __device__ static constexpr uint32_t col_s(int parity, int slot)
     {
-        return 16u * static_cast<uint32_t>(kRound * parity + slot);
+        return 16u * static_cast<uint32_t>((kRound * parity + slot) * kParts);
     }
 };
 
@@ -554,15 +558,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t dk = desc_k0 + static_cast<uint64_t>((c % kStages) * (kStageBytes >> 4));
             const uint64_t dq = desc_q0 + static_cast<uint64_t>(qs * (kSmallBytes >> 4));
             if constexpr (kFp8) {
-                // S^T = K (Q^T_hi + Q^T_mid + Q^T_lo): per part four K steps of 32 dims (32 bytes).
+                // S^T = K Q^T_hi + K Q^T_mid + K Q^T_lo, each part in its own accumulator: per part four
+                // K steps of 32 dims (32 bytes).
                 if (leader) {
 #pragma unroll
                     for (int t = 0; t < 3; ++t)
 #pragma unroll
                         for (int kk = 0; kk < kD / 32; ++kk)
-                            tc_mma_f8_ss(tmem + dcol, dk + static_cast<uint64_t>((kk * 32) >> 4),
+                            tc_mma_f8_ss(tmem + dcol + 16u * t, dk + static_cast<uint64_t>((kk * 32) >> 4),
                                          dq + static_cast<uint64_t>((t * kSmallHalf + kk * 32) >> 4), kIdS,
-                                         (t > 0 || kk > 0) ? 1u : 0u);
+                                         kk > 0 ? 1u : 0u);
                 }
                 return;
             }
@@ -580,16 +585,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t dv = desc_v0 + static_cast<uint64_t>((c % kStages) * (kStageBytes >> 4));
             const uint64_t dp = desc_p0 + static_cast<uint64_t>((rp * kRound + slot) * (kSmallBytes >> 4));
             if constexpr (kFp8) {
-                // O^T += V^T (P^T_hi + P^T_mid + P^T_lo): per part four K steps of 32 keys (32 rows of
-                // 128 bytes of the MN-major V chunk; 32 bytes of a P^T row).
+                // O^T_t += V^T P^T_t for the parts t = hi, mid, lo, each in its own accumulator: per part
+                // four K steps of 32 keys (32 rows of 128 bytes of the MN-major V chunk; 32 bytes of a
+                // P^T row).
                 if (leader) {
 #pragma unroll
                     for (int t = 0; t < 3; ++t)
 #pragma unroll
                         for (int kk = 0; kk < kCK / 32; ++kk)
-                            tc_mma_f8_ss(tmem + kColO, dv + static_cast<uint64_t>((kk * 32 * 128) >> 4),
+                            tc_mma_f8_ss(tmem + kColO + 16u * t, dv + static_cast<uint64_t>((kk * 32 * 128) >> 4),
                                          dp + static_cast<uint64_t>((t * kSmallHalf + kk * 32) >> 4), kIdO,
-                                         (accumulate || t > 0 || kk > 0) ? 1u : 0u);
+                                         (accumulate || kk > 0) ? 1u : 0u);
                 }
                 return;
             }
@@ -763,6 +769,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (sl < nk) {
                             uint32_t r[16];
                             tmem_ld16_wait(tS + TL::col_s(rp, sl), r);
+                            if constexpr (kFp8) {
+#pragma unroll
+                                for (int t = 1; t < TL::kParts; ++t) {
+                                    uint32_t rt[16];
+                                    tmem_ld16_wait(tS + TL::col_s(rp, sl) + 16u * t, rt);
+#pragma unroll
+                                    for (int h = 0; h < G; ++h)
+                                        r[h] = __float_as_uint(__uint_as_float(r[h]) + __uint_as_float(rt[h]));
+                                }
+                            }
                             const bool valid = (local0 + jr * kRound + sl) * kCK + i < seq_len;
 #pragma unroll
                             for (int h = 0; h < G; ++h)
@@ -830,12 +846,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                           static_cast<uint32_t>((rnd - 1) >> 1) & 1u, abort_flag,
                                                           p.status, kSiteDecodeConsumer))) {
                         tc_fence_after_sync();
-                        uint32_t ov[16];
-                        tmem_ld16_wait(tO, ov);
 #pragma unroll
-                        for (int h = 0; h < G; ++h)
-                            ov[h] = __float_as_uint(__uint_as_float(ov[h]) * alpha[h]);
-                        tmem_st16_wait(tO, ov);
+                        for (int t = 0; t < TL::kParts; ++t) {
+                            uint32_t ov[16];
+                            tmem_ld16_wait(tO + 16u * t, ov);
+#pragma unroll
+                            for (int h = 0; h < G; ++h)
+                                ov[h] = __float_as_uint(__uint_as_float(ov[h]) * alpha[h]);
+                            tmem_st16_wait(tO + 16u * t, ov);
+                        }
                     } else {
                         ok = false;
                     }
@@ -935,6 +954,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after_sync();
             uint32_t ov[16];
             tmem_ld16_wait(tO, ov);
+#pragma unroll
+            for (int t = 1; t < TL::kParts; ++t) {
+                uint32_t ot[16];
+                tmem_ld16_wait(tO + 16u * t, ot);
+#pragma unroll
+                for (int h = 0; h < G; ++h)
+                    ov[h] = __float_as_uint(__uint_as_float(ov[h]) + __uint_as_float(ot[h]));
+            }
             tc_fence_before_sync();
             mbar_arrive(BAR(kBarOFree));  // the next segment may overwrite O^T
 
