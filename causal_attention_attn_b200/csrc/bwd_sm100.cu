@@ -21,10 +21,14 @@
  *                      dK  += dS^T Q     (A = dS^T from TMEM, B = Q read MN-major)
  *                      dQ   = dS K       (A = dS from shared memory, B = K read MN-major)
  *                    the same warps (thread = query row, warpgroup g: dQ columns [64 g, 64 g + 64))
- *                    then drain dQ with fp32 vector reductions into the workspace; dK and dV stay in
- *                    TMEM until the last step. Splitting each step's columns over two warpgroups
- *                    halves the serial softmax and drain time of a step (a single warp per SM
- *                    sub-partition left them latency-bound);
+ *                    then copy dQ x scale out of TMEM into the step's Q/dO stage (free once the
+ *                    products are done), and warp 10 adds it into the fp32 workspace with TMA
+ *                    reduce-adds while the next step runs; dK and dV stay in TMEM until the last
+ *                    step. Splitting each step's columns over two warpgroups halves the serial
+ *                    softmax time of a step (a single warp per SM sub-partition left it
+ *                    latency-bound), and the asynchronous reduction takes the 64 KB of dQ per step
+ *                    off the chain (written by the warps themselves, it took a third of the step:
+ *                    the SM's store bandwidth to L2, not the reductions, bounded it);
  *   bwd_dq_kernel    dQ (fp32 workspace) -> bf16.
  *
  * TMEM (512 columns): [0,128) S^T, then P^T (bf16: queries 0-63 in [0,32), 64-127 in [64,96)), then
@@ -43,6 +47,7 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <type_traits>
 
 #include "kernels.h"
 #include "sm100_ptx.cuh"
@@ -57,6 +62,7 @@ constexpr int kBQ = 128;  // query rows per step
 constexpr int kThreads = 384;
 constexpr int kWarpTma = 8;
 constexpr int kWarpMma = 9;
+constexpr int kWarpRed = 10;  // issues the dQ reduce-adds
 constexpr float kLog2e = 1.4426950408889634f;
 
 constexpr int kHalf = 128 * 128;      // 128 rows x 64 dims (or 64 keys) of bf16, 128-byte swizzle
@@ -66,19 +72,20 @@ constexpr int kOffV = kOffK + kTile;
 constexpr int kOffStage = kOffV + kTile;  // two stages of Q_i, dO_i
 constexpr int kStageBytes = 2 * kTile;
 constexpr int kOffDS = kOffStage + 2 * kStageBytes;  // dS (queries x keys), A operand of dQ
+constexpr int kDqBox = 128 * 128;                   // 128 rows x 32 fp32 of dQ, 128-byte swizzle
 constexpr int kOffVec = kOffDS + kTile;              // two stages of [lse2 | D] (128 floats each)
 constexpr int kVecBytes = 2 * kBQ * 4;
 constexpr int kOffBar = kOffVec + 2 * kVecBytes;
 enum BwdBar : int {
     kBarKV = 0,
     kBarStageFull0 = 1,   // [2]
-    kBarStageEmpty0 = 3,  // [2]
+    kBarStageEmpty0 = 3,  // [2]: the products are done with Q, dO, and the stage's dQ has been reduced
     kBarSD = 5,           // S^T and dP^T ready
-    kBarP = 6,            // P^T, dS^T, dS written (128 arrivals)
+    kBarP = 6,            // P^T, dS^T, dS written (256 arrivals)
     kBarDQ = 7,           // dQ ready
-    kBarDQFree = 8,       // dQ drained (128 arrivals)
-    kBarFinal = 9,        // every MMA done
-    kNumBwdBars = 10,
+    kBarDQFree0 = 8,      // [2], by stage: dQ out of TMEM and staged in shared memory (256 arrivals)
+    kBarFinal = 10,       // every MMA done
+    kNumBwdBars = 11,
 };
 constexpr int kOffMisc = kOffBar + kNumBwdBars * 8;
 constexpr int kSmem = kOffMisc + 64;  // the dynamic window starts 1024-aligned (no static smem)
@@ -87,7 +94,6 @@ constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 384;
 
 struct BwdParams {
     __nv_bfloat16 *dk, *dv;
-    float *dq_acc;       // [B*Hq*Sq][D] fp32, zeroed before the launch
     const float *vec;    // [2][B*Hq][Sq_pad]: lse2 then D
     int *status;
     int B, Hq, Hkv, Sq, Skv, Sq_pad, group, offset, causal, n_ktiles;
@@ -105,13 +111,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);
-}
-
-// acc[0..3] += (a, b, c, d): one vector reduction into global memory (16-byte aligned).
-__device__ __forceinline__ void red_add_v4(float *acc, float a, float b, float c, float d)
-{
-    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(acc), "f"(a), "f"(b), "f"(c), "f"(d)
-                 : "memory");
 }
 
 __device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity, uint64_t limit_ns)
@@ -171,7 +170,7 @@ __global__ void __launch_bounds__(256) bwd_dq_kernel(const float4 *acc, uint2 *d
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-               const BwdParams p)
+               const __grid_constant__ CUtensorMap tm_dq, const BwdParams p)
 {
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t s_base = smem_u32(smem);
@@ -210,12 +209,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(BAR(kBarKV), 1);
         for (int s = 0; s < 2; ++s) {
             mbar_init(BAR(kBarStageFull0 + s), 1);
-            mbar_init(BAR(kBarStageEmpty0 + s), 1);
+            mbar_init(BAR(kBarStageEmpty0 + s), 2);  // the MMA commit and the reducer
+            mbar_init(BAR(kBarDQFree0 + s), 256);
         }
         mbar_init(BAR(kBarSD), 1);
         mbar_init(BAR(kBarP), 256);
         mbar_init(BAR(kBarDQ), 1);
-        mbar_init(BAR(kBarDQFree), 256);
         mbar_init(BAR(kBarFinal), 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -289,9 +288,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!(ok = mbar_wait(BAR(kBarStageFull0 + st), static_cast<uint32_t>(s >> 1) & 1u, abort_flag, p.status,
                                  kSiteBwd)))
                 break;
-            // S^T goes where the previous step's dQ was: wait until it is drained.
-            if (s > 0 && !(ok = mbar_wait(BAR(kBarDQFree), static_cast<uint32_t>(s - 1) & 1u, abort_flag, p.status,
-                                          kSiteBwd)))
+            // S^T goes where the previous step's dQ was: wait until it is out of TMEM.
+            if (s > 0 && !(ok = mbar_wait(BAR(kBarDQFree0 + ((s - 1) & 1)), static_cast<uint32_t>((s - 1) >> 1) & 1u,
+                                          abort_flag, p.status, kSiteBwd)))
                 break;
             tc_fence_after_sync();
             if (leader) {
@@ -326,6 +325,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             atomicExch(p.status, kSiteBwd);
         }
         __syncwarp();
+    } else if (warp == kWarpRed) {
+        // ---------------------------------------------------------------- dQ reducer
+        // One barrier per stage: a step's staged dQ cannot be followed by the same stage's next
+        // staging before this warp has reduced it (the stage is reloaded only after the arrival
+        // below), so a wait never misses a phase.
+        if (lane == 0 && n_steps > 0) {
+            for (int s = 0; s < n_steps; ++s) {
+                const int st = s & 1;
+                if (!mbar_wait(BAR(kBarDQFree0 + st), static_cast<uint32_t>(s >> 1) & 1u, abort_flag, p.status, kSiteBwd))
+                    break;
+                const int h = step_head(s), q0 = step_q0(s);
+                const uint32_t src = sStage + st * kStageBytes;
+                for (int c = 0; c < 4; ++c)
+                    tma_reduce_add_3d(&tm_dq, src + c * kDqBox, 32 * c, q0, b * p.Hq + h);
+                bulk_commit_group();
+                bulk_wait_group_read0();  // the producer may load the stage again
+                mbar_arrive(BAR(kBarStageEmpty0 + st));
+            }
+            bulk_wait_group0();  // every reduction has been performed before the CTA exits
+        }
     } else if (warp < 8) {
         // ---------------------------------------------------------------- softmax and dQ warps
         // Warps w and w + 4 share TMEM lanes 32 (w % 4) .. + 31 and split the 128 columns of a step:
@@ -361,35 +380,49 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int c = 0; c < 2; ++c) {
                 const int cq = (2 * grp + c) * 32;  // first query column of this chunk
                 uint32_t sr[32], dr[32];
-                tmem_ld32_wait(tS + c * 32, sr);
-                tmem_ld32_wait(tDP + c * 32, dr);
-                uint32_t pk[16], dk[16];
+                tmem_ld32x2_wait(tS + c * 32, tDP + c * 32, sr, dr);
+                float nl[32], dv[32];
 #pragma unroll
-                for (int i = 0; i < 32; i += 2) {
-                    float pe[2], ds[2];
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int q = cq + i + u;
-                        const bool vis = key_ok && q >= first_q && q <= last_q;
-                        // Masked entries are exact zeros (lse2 and D of padding rows are never read).
-                        const float w = vis ? ex2(__uint_as_float(sr[i + u]) * p.scale_log2 - lse2[q]) : 0.f;
-                        pe[u] = w;
-                        ds[u] = vis ? w * (__uint_as_float(dr[i + u]) - dvec[q]) : 0.f;
-                    }
-                    pk[i >> 1] = pack_bf16x2(pe[0], pe[1]);
-                    dk[i >> 1] = pack_bf16x2(ds[0], ds[1]);
-                    // dS (row q, column key) for the dQ product: K-major, 128-byte swizzle.
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int q = cq + i + u;
-                        const __nv_bfloat16 v = __float2bfloat16_rn(ds[u]);
-                        *reinterpret_cast<__nv_bfloat16 *>(dsrow_base + q * 128 +
-                                                           ((((kk >> 3) ^ (q & 7)) << 4) | ((kk & 7) << 1))) = v;
-                    }
+                for (int i = 0; i < 8; ++i) {
+                    const float4 x = reinterpret_cast<const float4 *>(lse2 + cq)[i];
+                    const float4 y = reinterpret_cast<const float4 *>(dvec + cq)[i];
+                    nl[4 * i] = -x.x; nl[4 * i + 1] = -x.y; nl[4 * i + 2] = -x.z; nl[4 * i + 3] = -x.w;
+                    dv[4 * i] = y.x; dv[4 * i + 1] = y.y; dv[4 * i + 2] = y.z; dv[4 * i + 3] = y.w;
                 }
-                // P^T and dS^T over the columns this warp has already read (in-place packing).
-                tmem_st16_wait(tS + c * 16, pk);
-                tmem_st16_wait(tDP + c * 16, dk);
+                uint32_t pk[16], dk[16];
+                auto body = [&](auto masked) {
+#pragma unroll
+                    for (int i = 0; i < 32; i += 2) {
+                        float pe[2], ds[2];
+#pragma unroll
+                        for (int u = 0; u < 2; ++u) {
+                            const int q = cq + i + u;
+                            const float w = ex2(fmaf(__uint_as_float(sr[i + u]), p.scale_log2, nl[i + u]));
+                            const float g = w * (__uint_as_float(dr[i + u]) - dv[i + u]);
+                            if constexpr (decltype(masked)::value) {
+                                const bool vis = key_ok && q >= first_q && q <= last_q;
+                                pe[u] = vis ? w : 0.f;
+                                ds[u] = vis ? g : 0.f;
+                            } else {
+                                pe[u] = w;
+                                ds[u] = g;
+                            }
+                        }
+                        pk[i >> 1] = pack_bf16x2(pe[0], pe[1]);
+                        dk[i >> 1] = pack_bf16x2(ds[0], ds[1]);
+#pragma unroll
+                        for (int u = 0; u < 2; ++u) {
+                            const int q = cq + i + u;
+                            *reinterpret_cast<uint16_t *>(dsrow_base + q * 128 + ((((kk >> 3) ^ (q & 7)) << 4) | ((kk & 7) << 1))) =
+                                static_cast<uint16_t>(u ? (dk[i >> 1] >> 16) : (dk[i >> 1] & 0xffffu));
+                        }
+                    }
+                };
+                if (key_ok && first_q <= cq && cq + 31 <= last_q)
+                    body(std::false_type{});
+                else
+                    body(std::true_type{});
+                tmem_st16x2_wait(tS + c * 16, pk, tDP + c * 16, dk);
             }
             fence_proxy_async_smem();
             tc_fence_before_sync();
@@ -400,22 +433,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                          p.status, kSiteBwd))))
                 break;
             tc_fence_after_sync();
-            const bool valid = q0 + kr < p.Sq;
-            float *acc = p.dq_acc + ((static_cast<size_t>(b) * p.Hq + h) * p.Sq + (valid ? q0 + kr : 0)) * kD + 64 * grp;
+            {
+                // dQ x scale into this step's Q/dO stage, which the products have finished with (the
+                // dQ commit covers every earlier product): four boxes of 128 rows x 32 fp32 in the
+                // 128-byte swizzle; the reducer warp adds them into the fp32 accumulator by TMA while
+                // the next step runs.
+                uint8_t *stage = smem + kOffStage + st * kStageBytes;
 #pragma unroll 1
-            for (int c = 0; c < 2; ++c) {
-                uint32_t v[32];
-                tmem_ld32_wait(tQ + c * 32, v);
-                if (valid) {
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t v[32];
+                    tmem_ld32_wait(tQ + c * 32, v);
+                    uint8_t *row = stage + (2 * grp + c) * kDqBox + kr * 128;
 #pragma unroll
-                    for (int i = 0; i < 32; i += 4)
-                        red_add_v4(acc + c * 32 + i, __uint_as_float(v[i]) * p.scale, __uint_as_float(v[i + 1]) * p.scale,
-                                   __uint_as_float(v[i + 2]) * p.scale, __uint_as_float(v[i + 3]) * p.scale);
+                    for (int u = 0; u < 8; ++u)
+                        *reinterpret_cast<float4 *>(row + ((u ^ (kr & 7)) << 4)) =
+                            make_float4(__uint_as_float(v[4 * u]) * p.scale, __uint_as_float(v[4 * u + 1]) * p.scale,
+                                        __uint_as_float(v[4 * u + 2]) * p.scale, __uint_as_float(v[4 * u + 3]) * p.scale);
                 }
-                __syncwarp();
             }
+            fence_proxy_async_smem();
             tc_fence_before_sync();
-            mbar_arrive(BAR(kBarDQFree));
+            mbar_arrive(BAR(kBarDQFree0 + st));
         }
         // Epilogue: dims [64 grp, 64 grp + 64) of dK (scaled) and dV of this key. The whole warp
         // loads (tcgen05.ld is warp-collective); only the stores of keys past Skv are skipped.
@@ -493,7 +531,7 @@ cudaError_t launch_bwd(const BwdArgs &a, cudaStream_t stream, int *encode_error)
         *encode_error = -1;
         return cudaErrorInitializationError;
     }
-    CUtensorMap tq, tk, tv, tdo;
+    CUtensorMap tq, tk, tv, tdo, tdq;
     if (!make_map(encode, &tq, a.q, kD, a.Sq, a.B * a.Hq, 64, kBQ, CU_TENSOR_MAP_SWIZZLE_128B, encode_error) ||
         !make_map(encode, &tdo, a.dout, kD, a.Sq, a.B * a.Hq, 64, kBQ, CU_TENSOR_MAP_SWIZZLE_128B, encode_error) ||
         !make_map(encode, &tk, a.k, kD, a.Skv, a.B * a.Hkv, 64, kBK, CU_TENSOR_MAP_SWIZZLE_128B, encode_error) ||
@@ -504,6 +542,8 @@ cudaError_t launch_bwd(const BwdArgs &a, cudaStream_t stream, int *encode_error)
     const size_t rows = static_cast<size_t>(a.B) * a.Hq * a.Sq;
     float *dq_acc = static_cast<float *>(a.ws);
     float *vec = dq_acc + rows * kD;
+    if (!make_map_f32(encode, &tdq, dq_acc, kD, a.Sq, a.B * a.Hq, 32, kBQ, CU_TENSOR_MAP_SWIZZLE_128B, encode_error))
+        return cudaErrorInvalidValue;
     cudaError_t e = cudaMemsetAsync(dq_acc, 0, rows * kD * sizeof(float), stream);
     if (e != cudaSuccess)
         return e;
@@ -518,7 +558,6 @@ cudaError_t launch_bwd(const BwdArgs &a, cudaStream_t stream, int *encode_error)
     BwdParams p;
     p.dk = static_cast<__nv_bfloat16 *>(a.dk);
     p.dv = static_cast<__nv_bfloat16 *>(a.dv);
-    p.dq_acc = dq_acc;
     p.vec = vec;
     p.status = a.status;
     p.B = a.B;
@@ -534,7 +573,7 @@ cudaError_t launch_bwd(const BwdArgs &a, cudaStream_t stream, int *encode_error)
     p.scale = a.scale;
     p.scale_log2 = a.scale * kLog2e;
     const long long grid = static_cast<long long>(p.n_ktiles) * a.B * a.Hkv;
-    bwd_kernel<<<static_cast<unsigned>(grid), kThreads, kSmem, stream>>>(tq, tk, tv, tdo, p);
+    bwd_kernel<<<static_cast<unsigned>(grid), kThreads, kSmem, stream>>>(tq, tk, tv, tdo, tdq, p);
     if ((e = cudaGetLastError()) != cudaSuccess)
         return e;
     const long long n4 = static_cast<long long>(rows) * kD / 4;

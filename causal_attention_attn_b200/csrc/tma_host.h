@@ -50,6 +50,24 @@ inline bool make_map(PFN_cuTensorMapEncodeTiled_v12000 encode, CUtensorMap *map,
     return true;
 }
 
+// As make_map for a contiguous fp32 tensor [BH][S][D] (the target of tiled reduce-adds).
+inline bool make_map_f32(PFN_cuTensorMapEncodeTiled_v12000 encode, CUtensorMap *map, void *base, int D, int S, int BH,
+                         int box_inner, int box_rows, CUtensorMapSwizzle swizzle, int *err)
+{
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(S), static_cast<cuuint64_t>(BH)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 4, static_cast<cuuint64_t>(S) * D * 4};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_rows), 1u};
+    cuuint32_t estr[3] = {1u, 1u, 1u};
+    CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        *err = static_cast<int>(r);
+        return false;
+    }
+    return true;
+}
+
 // As make_map for a contiguous tensor of 8-bit elements [BH][S][D] (D bytes per row), with a box
 // of (box_inner bytes, box_rows rows, 1).
 inline bool make_map_u8(PFN_cuTensorMapEncodeTiled_v12000 encode, CUtensorMap *map, const void *base, int D, int S,
