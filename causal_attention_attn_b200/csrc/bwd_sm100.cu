@@ -31,10 +31,11 @@
  *                    the SM's store bandwidth to L2, not the reductions, bounded it);
  *   bwd_dq_kernel    dQ (fp32 workspace) -> bf16.
  *
- * TMEM (512 columns): [0,128) S^T, then P^T (bf16: queries 0-63 in [0,32), 64-127 in [64,96)), then
- * dQ; [128,256) dP^T, then dS^T (likewise in [128,160) and [192,224)); [256,384) dV; [384,512) dK.
- * The MMAs of one thread run in issue order, so dV's read of P^T is done before dQ overwrites those
- * columns, and dK's read of dS^T before the next dP^T.
+ * TMEM (512 columns): [0,128) S^T, then P^T (bf16: queries 0-63 in [0,32), 64-127 in [64,96));
+ * [128,256) dP^T, then dS^T (likewise in [128,160) and [192,224)), then dQ; [256,384) dV; [384,512)
+ * dK. The MMAs of one thread run in issue order, so dK's read of dS^T is done before dQ overwrites
+ * those columns, and dV's read of P^T before the next S^T. The next step's S^T product needs only
+ * that order; its dP^T product waits until dQ is out of TMEM, so S^T overlaps the dQ drain.
  *
  * Sources (page title, section): the backward pass recomputes the weights from the LSE the forward
  * saved instead of storing them — "AI Infra 入门：RMSNorm、Softmax、Causal Mask、Sampling 的数学与底层
@@ -288,15 +289,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!(ok = mbar_wait(BAR(kBarStageFull0 + st), static_cast<uint32_t>(s >> 1) & 1u, abort_flag, p.status,
                                  kSiteBwd)))
                 break;
-            // S^T goes where the previous step's dQ was: wait until it is out of TMEM.
-            if (s > 0 && !(ok = mbar_wait(BAR(kBarDQFree0 + ((s - 1) & 1)), static_cast<uint32_t>((s - 1) >> 1) & 1u,
-                                          abort_flag, p.status, kSiteBwd)))
-                break;
             tc_fence_after_sync();
             if (leader) {
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk)
                     tc_mma_ss(tmem + kColS, kmaj(sK, kk), kmaj(sQ, kk), kIdSS, kk > 0 ? 1u : 0u);
+            }
+            // dP^T goes where the previous step's dQ is: wait until that is out of TMEM (S^T above
+            // runs meanwhile).
+            if (s > 0 && !(ok = mbar_wait(BAR(kBarDQFree0 + ((s - 1) & 1)), static_cast<uint32_t>((s - 1) >> 1) & 1u,
+                                          abort_flag, p.status, kSiteBwd)))
+                break;
+            tc_fence_after_sync();
+            if (leader) {
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk)
                     tc_mma_ss(tmem + kColDP, kmaj(sV, kk), kmaj(sDO, kk), kIdSS, kk > 0 ? 1u : 0u);
@@ -307,14 +312,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after_sync();
             if (leader) {
 #pragma unroll
-                for (int kk = 0; kk < kBQ / 16; ++kk)  // dV += P^T dO
-                    tc_mma_ts(tmem + kColDV, tmem + kColS + pcol(kk), mnmaj(sDO, kk), kIdTS, (s > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
                 for (int kk = 0; kk < kBQ / 16; ++kk)  // dK += dS^T Q
                     tc_mma_ts(tmem + kColDK, tmem + kColDP + pcol(kk), mnmaj(sQ, kk), kIdTS, (s > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
-                for (int kk = 0; kk < kBK / 16; ++kk)  // dQ = dS K (queries in TMEM lanes)
-                    tc_mma_ss(tmem + kColS, kmaj(sDS, kk), mnmaj(sK, kk), kIdQ, kk > 0 ? 1u : 0u);
+                for (int kk = 0; kk < kBQ / 16; ++kk)  // dV += P^T dO
+                    tc_mma_ts(tmem + kColDV, tmem + kColS + pcol(kk), mnmaj(sDO, kk), kIdTS, (s > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+                for (int kk = 0; kk < kBK / 16; ++kk)  // dQ = dS K (queries in TMEM lanes), over dS^T
+                    tc_mma_ss(tmem + kColDP, kmaj(sDS, kk), mnmaj(sK, kk), kIdQ, kk > 0 ? 1u : 0u);
             }
             commit(kBarDQ);
             commit(kBarStageEmpty0 + st);
@@ -356,7 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int key = k0 + kr;
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const uint32_t tS = tmem + lane_base + kColS + 64u * grp, tDP = tmem + lane_base + kColDP + 64u * grp;
-        const uint32_t tQ = tmem + lane_base + kColS + 64u * grp;
+        const uint32_t tQ = tmem + lane_base + kColDP + 64u * grp;
         bool ok = true;
         for (int s = 0; s < n_steps; ++s) {
             const int st = s & 1;
