@@ -82,11 +82,12 @@ enum BwdBar : int {
     kBarStageFull0 = 1,   // [2]
     kBarStageEmpty0 = 3,  // [2]: the products are done with Q, dO, and the stage's dQ has been reduced
     kBarSD = 5,           // S^T and dP^T ready
-    kBarP = 6,            // P^T, dS^T, dS written (256 arrivals)
-    kBarDQ = 7,           // dQ ready
-    kBarDQFree0 = 8,      // [2], by stage: dQ out of TMEM and staged in shared memory (256 arrivals)
-    kBarFinal = 10,       // every MMA done
-    kNumBwdBars = 11,
+    kBarP0 = 6,           // P^T, dS^T of each warp's first 32 query columns in TMEM (256 arrivals)
+    kBarP1 = 7,           // ... of all 64, and dS in shared memory (256 arrivals)
+    kBarDQ = 8,           // dQ ready
+    kBarDQFree0 = 9,      // [2], by stage: dQ out of TMEM and staged in shared memory (256 arrivals)
+    kBarFinal = 11,       // every MMA done
+    kNumBwdBars = 12,
 };
 constexpr int kOffMisc = kOffBar + kNumBwdBars * 8;
 constexpr int kSmem = kOffMisc + 64;  // the dynamic window starts 1024-aligned (no static smem)
@@ -214,7 +215,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(BAR(kBarDQFree0 + s), 256);
         }
         mbar_init(BAR(kBarSD), 1);
-        mbar_init(BAR(kBarP), 256);
+        mbar_init(BAR(kBarP0), 256);
+        mbar_init(BAR(kBarP1), 256);
         mbar_init(BAR(kBarDQ), 1);
         mbar_init(BAR(kBarFinal), 1);
         *abort_flag = 0;
@@ -307,16 +309,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_mma_ss(tmem + kColDP, kmaj(sV, kk), kmaj(sDO, kk), kIdSS, kk > 0 ? 1u : 0u);
             }
             commit(kBarSD);
-            if (!(ok = mbar_wait(BAR(kBarP), static_cast<uint32_t>(s) & 1u, abort_flag, p.status, kSiteBwd)))
+            // dK and dV over the query columns each softmax warp has finished first (16-query steps
+            // 0, 1, 4, 5), then over the rest once the softmax is done.
+            for (int half = 0; half < 2; ++half) {
+                if (!(ok = mbar_wait(BAR(kBarP0 + half), static_cast<uint32_t>(s) & 1u, abort_flag, p.status, kSiteBwd)))
+                    break;
+                tc_fence_after_sync();
+                if (leader) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {  // dK += dS^T Q
+                        const int kk = (i >> 1) * 4 + half * 2 + (i & 1);
+                        tc_mma_ts(tmem + kColDK, tmem + kColDP + pcol(kk), mnmaj(sQ, kk), kIdTS, (s > 0 || kk > 0) ? 1u : 0u);
+                    }
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {  // dV += P^T dO
+                        const int kk = (i >> 1) * 4 + half * 2 + (i & 1);
+                        tc_mma_ts(tmem + kColDV, tmem + kColS + pcol(kk), mnmaj(sDO, kk), kIdTS, (s > 0 || kk > 0) ? 1u : 0u);
+                    }
+                }
+            }
+            if (!ok)
                 break;
-            tc_fence_after_sync();
             if (leader) {
-#pragma unroll
-                for (int kk = 0; kk < kBQ / 16; ++kk)  // dK += dS^T Q
-                    tc_mma_ts(tmem + kColDK, tmem + kColDP + pcol(kk), mnmaj(sQ, kk), kIdTS, (s > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-                for (int kk = 0; kk < kBQ / 16; ++kk)  // dV += P^T dO
-                    tc_mma_ts(tmem + kColDV, tmem + kColS + pcol(kk), mnmaj(sDO, kk), kIdTS, (s > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
                 for (int kk = 0; kk < kBK / 16; ++kk)  // dQ = dS K (queries in TMEM lanes), over dS^T
                     tc_mma_ss(tmem + kColDP, kmaj(sDS, kk), mnmaj(sK, kk), kIdQ, kk > 0 ? 1u : 0u);
@@ -428,10 +442,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 else
                     body(std::true_type{});
                 tmem_st16x2_wait(tS + c * 16, pk, tDP + c * 16, dk);
+                if (c == 1)
+                    fence_proxy_async_smem();  // dS, for the dQ product
+                tc_fence_before_sync();
+                mbar_arrive(BAR(kBarP0 + c));
             }
-            fence_proxy_async_smem();
-            tc_fence_before_sync();
-            mbar_arrive(BAR(kBarP));
 
             // dQ of this step (thread = query row), scaled, added into the fp32 accumulator.
             if (!(ok = __all_sync(0xffffffffu, mbar_wait(BAR(kBarDQ), static_cast<uint32_t>(s) & 1u, abort_flag,
