@@ -129,8 +129,8 @@ struct Lay {
 static_assert(Lay<false>::kStageBytes == 65536 && Lay<false>::kSmallBytes == 4096, "bf16 layout");
 // TMEM: S^T of a round's chunks [round parity][slot] in 16-column groups from column 0, then O^T.
 // With the e4m3 cache every product is a sum over three e4m3 parts (of Q^T or of P^T); each part
-// accumulates in its own 16 columns, so that the tensor core's chain of dependent accumulations is
-// four instructions long instead of twelve, and the readers add the parts.
+// accumulates in its own 16 columns (one N = 48 instruction per K step computes all three), and
+// the readers add the parts.
 template <bool kFp8>
 struct TmemLay {
     static constexpr int kRound = Lay<kFp8>::kRound;
@@ -540,8 +540,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == kWarpMma) {
         // ---------------------------------------------------------------- MMA issuer
         // A = K chunk, B = Q^T; then A = V chunk read MN-major, B = P^T. e4m3 cache: both operands e4m3.
-        constexpr uint32_t kIdS = kFp8 ? idesc_e4m3_f32_ab(kCK, kN, false, false) : idesc_bf16_f32_ab(kCK, kN, false, false);
-        constexpr uint32_t kIdO = kFp8 ? idesc_e4m3_f32_ab(kD, kN, true, false) : idesc_bf16_f32_ab(kD, kN, true, false);
+        // e4m3: the three parts of Q^T (or of P^T) sit one after another (16 rows each, 8-row groups
+        // 1024 bytes apart), so one instruction of N = 48 takes all three, each part's product
+        // landing in its own 16 accumulator columns.
+        constexpr int kNP = kFp8 ? 3 * kN : kN;
+        constexpr uint32_t kIdS = kFp8 ? idesc_e4m3_f32_ab(kCK, kNP, false, false) : idesc_bf16_f32_ab(kCK, kN, false, false);
+        constexpr uint32_t kIdO = kFp8 ? idesc_e4m3_f32_ab(kD, kNP, true, false) : idesc_bf16_f32_ab(kD, kN, true, false);
         const bool leader = elect_one();
         // A K step moves the start address, the low field of a descriptor (address >> 4): every
         // address here is below 2^18, so the field never overflows.
@@ -558,16 +562,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t dk = desc_k0 + static_cast<uint64_t>((c % kStages) * (kStageBytes >> 4));
             const uint64_t dq = desc_q0 + static_cast<uint64_t>(qs * (kSmallBytes >> 4));
             if constexpr (kFp8) {
-                // S^T = K Q^T_hi + K Q^T_mid + K Q^T_lo, each part in its own accumulator: per part four
-                // K steps of 32 dims (32 bytes).
+                // [K Q^T_hi | K Q^T_mid | K Q^T_lo]: four K steps of 32 dims (32 bytes).
                 if (leader) {
 #pragma unroll
-                    for (int t = 0; t < 3; ++t)
-#pragma unroll
-                        for (int kk = 0; kk < kD / 32; ++kk)
-                            tc_mma_f8_ss(tmem + dcol + 16u * t, dk + static_cast<uint64_t>((kk * 32) >> 4),
-                                         dq + static_cast<uint64_t>((t * kSmallHalf + kk * 32) >> 4), kIdS,
-                                         kk > 0 ? 1u : 0u);
+                    for (int kk = 0; kk < kD / 32; ++kk)
+                        tc_mma_f8_ss(tmem + dcol, dk + static_cast<uint64_t>((kk * 32) >> 4),
+                                     dq + static_cast<uint64_t>((kk * 32) >> 4), kIdS, kk > 0 ? 1u : 0u);
                 }
                 return;
             }
@@ -585,17 +585,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t dv = desc_v0 + static_cast<uint64_t>((c % kStages) * (kStageBytes >> 4));
             const uint64_t dp = desc_p0 + static_cast<uint64_t>((rp * kRound + slot) * (kSmallBytes >> 4));
             if constexpr (kFp8) {
-                // O^T_t += V^T P^T_t for the parts t = hi, mid, lo, each in its own accumulator: per part
-                // four K steps of 32 keys (32 rows of 128 bytes of the MN-major V chunk; 32 bytes of a
-                // P^T row).
+                // [O^T_hi | O^T_mid | O^T_lo] += V^T [P^T_hi | P^T_mid | P^T_lo]: four K steps of 32
+                // keys (32 rows of 128 bytes of the MN-major V chunk; 32 bytes of a P^T row).
                 if (leader) {
 #pragma unroll
-                    for (int t = 0; t < 3; ++t)
-#pragma unroll
-                        for (int kk = 0; kk < kCK / 32; ++kk)
-                            tc_mma_f8_ss(tmem + kColO + 16u * t, dv + static_cast<uint64_t>((kk * 32 * 128) >> 4),
-                                         dp + static_cast<uint64_t>((t * kSmallHalf + kk * 32) >> 4), kIdO,
-                                         (accumulate || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < kCK / 32; ++kk)
+                        tc_mma_f8_ss(tmem + kColO, dv + static_cast<uint64_t>((kk * 32 * 128) >> 4),
+                                     dp + static_cast<uint64_t>((kk * 32) >> 4), kIdO, (accumulate || kk > 0) ? 1u : 0u);
                 }
                 return;
             }
