@@ -13,27 +13,26 @@
  *                    head of the kv head's group and every 128-row query tile that sees any of its
  *                    keys. Per step (one query tile), with keys in TMEM lanes:
  *                      S^T  = K Q^T      and  dP^T = V dO^T     (tcgen05.mma, both operands TMA tiles)
- *                      P^T, dS^T         warps 0-7 (thread = key; warpgroup g takes query columns
- *                                        [64 g, 64 g + 64)) recompute the weights from the LSE,
+ *                      P^T, dS^T         warps 0-15 (thread = key; warpgroup g takes query columns
+ *                                        [32 g, 32 g + 32)) recompute the weights from the LSE,
  *                                        apply the causal mask, form dS, and write P^T and dS^T back
- *                                        into TMEM as bf16 and dS into shared memory;
- *                      dV  += P^T dO     (A = P^T from TMEM, B = dO read MN-major)
+ *                                        into TMEM as bf16 and dS into shared memory, in two chunks
+ *                                        of 16 columns;
  *                      dK  += dS^T Q     (A = dS^T from TMEM, B = Q read MN-major)
+ *                      dV  += P^T dO     (A = P^T from TMEM, B = dO read MN-major); both start on
+ *                                        every warp's first chunk while the second is computed
  *                      dQ   = dS K       (A = dS from shared memory, B = K read MN-major)
- *                    the same warps (thread = query row, warpgroup g: dQ columns [64 g, 64 g + 64))
+ *                    the same warps (thread = query row, warpgroup g: dQ dims [32 g, 32 g + 32))
  *                    then copy dQ x scale out of TMEM into the step's Q/dO stage (free once the
- *                    products are done), and warp 10 adds it into the fp32 workspace with TMA
+ *                    products are done), and warp 18 adds it into the fp32 workspace with TMA
  *                    reduce-adds while the next step runs; dK and dV stay in TMEM until the last
- *                    step. Splitting each step's columns over two warpgroups halves the serial
- *                    softmax time of a step (a single warp per SM sub-partition left it
- *                    latency-bound), and the asynchronous reduction takes the 64 KB of dQ per step
- *                    off the chain (written by the warps themselves, it took a third of the step:
- *                    the SM's store bandwidth to L2, not the reductions, bounded it);
+ *                    step. The asynchronous reduction takes the 64 KB of dQ per step off the chain
+ *                    (written by the warps themselves, it took a third of the step: the SM's store
+ *                    bandwidth to L2, not the reductions, bounded it);
  *   bwd_dq_kernel    dQ (fp32 workspace) -> bf16.
  *
- * TMEM (512 columns): [0,128) S^T, then P^T (bf16: queries 0-63 in [0,32), 64-127 in [64,96));
- * [128,256) dP^T, then dS^T (likewise in [128,160) and [192,224)), then dQ; [256,384) dV; [384,512)
- * dK. The MMAs of one thread run in issue order, so dK's read of dS^T is done before dQ overwrites
+ * TMEM (512 columns): [0,128) S^T, then P^T (bf16: warpgroup g's queries in [32 g, 32 g + 16));
+ * [128,256) dP^T, then dS^T (likewise from column 128), then dQ; [256,384) dV; [384,512) dK. The MMAs of one thread run in issue order, so dK's read of dS^T is done before dQ overwrites
  * those columns, and dV's read of P^T before the next S^T. The next step's S^T product needs only
  * that order; its dP^T product waits until dQ is out of TMEM, so S^T overlaps the dQ drain.
  *
@@ -60,10 +59,12 @@ namespace {
 constexpr int kD = 128;
 constexpr int kBK = 128;  // keys per CTA tile (TMEM lanes of S^T, dP^T, dV, dK)
 constexpr int kBQ = 128;  // query rows per step
-constexpr int kThreads = 384;
-constexpr int kWarpTma = 8;
-constexpr int kWarpMma = 9;
-constexpr int kWarpRed = 10;  // issues the dQ reduce-adds
+constexpr int kSoftWarps = 16;     // four warpgroups: warp w serves TMEM lanes 32 (w % 4) .. + 31
+constexpr int kGroupCols = 32;     // query columns (and dQ, dK, dV dims) per warpgroup
+constexpr int kThreads = 640;
+constexpr int kWarpTma = 16;
+constexpr int kWarpMma = 17;
+constexpr int kWarpRed = 18;  // issues the dQ reduce-adds
 constexpr float kLog2e = 1.4426950408889634f;
 
 constexpr int kHalf = 128 * 128;      // 128 rows x 64 dims (or 64 keys) of bf16, 128-byte swizzle
@@ -212,11 +213,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < 2; ++s) {
             mbar_init(BAR(kBarStageFull0 + s), 1);
             mbar_init(BAR(kBarStageEmpty0 + s), 2);  // the MMA commit and the reducer
-            mbar_init(BAR(kBarDQFree0 + s), 256);
+            mbar_init(BAR(kBarDQFree0 + s), 32 * kSoftWarps);
         }
         mbar_init(BAR(kBarSD), 1);
-        mbar_init(BAR(kBarP0), 256);
-        mbar_init(BAR(kBarP1), 256);
+        mbar_init(BAR(kBarP0), 32 * kSoftWarps);
+        mbar_init(BAR(kBarP1), 32 * kSoftWarps);
         mbar_init(BAR(kBarDQ), 1);
         mbar_init(BAR(kBarFinal), 1);
         *abort_flag = 0;
@@ -274,9 +275,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         auto kmaj = [](uint32_t base, int kk) {  // K-major tile, K step kk (16 elements)
             return smem_desc(base + (kk >> 2) * kHalf + (kk & 3) * 32, 16, 1024, kSwizzle128B);
         };
-        // Packed P^T / dS^T of queries [16 kk, 16 kk + 16): each query half's bf16 pairs sit at the start
-        // of that half's own 64 fp32 columns (see the softmax warps).
-        auto pcol = [](int kk) { return static_cast<uint32_t>((kk >> 2) * 64 + (kk & 3) * 8); };
+        // Packed P^T / dS^T of queries [16 kk, 16 kk + 16): each warpgroup's bf16 pairs sit at the
+        // start of its own 32 fp32 columns (see the softmax warps).
+        auto pcol = [](int kk) { return static_cast<uint32_t>((kk >> 1) * kGroupCols + (kk & 1) * 8); };
         auto mnmaj = [](uint32_t base, int kk) {  // MN-major tile, K step kk (16 rows of 128 bytes)
             return smem_desc(base + kk * 16 * 128, kHalf, 1024, kSwizzle128B);
         };
@@ -318,12 +319,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (leader) {
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {  // dK += dS^T Q
-                        const int kk = (i >> 1) * 4 + half * 2 + (i & 1);
+                        const int kk = 2 * i + half;
                         tc_mma_ts(tmem + kColDK, tmem + kColDP + pcol(kk), mnmaj(sQ, kk), kIdTS, (s > 0 || kk > 0) ? 1u : 0u);
                     }
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {  // dV += P^T dO
-                        const int kk = (i >> 1) * 4 + half * 2 + (i & 1);
+                        const int kk = 2 * i + half;
                         tc_mma_ts(tmem + kColDV, tmem + kColS + pcol(kk), mnmaj(sDO, kk), kIdTS, (s > 0 || kk > 0) ? 1u : 0u);
                     }
                 }
@@ -364,18 +365,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             bulk_wait_group0();  // every reduction has been performed before the CTA exits
         }
-    } else if (warp < 8) {
+    } else if (warp < kSoftWarps) {
         // ---------------------------------------------------------------- softmax and dQ warps
-        // Warps w and w + 4 share TMEM lanes 32 (w % 4) .. + 31 and split the 128 columns of a step:
-        // warpgroup g takes query columns [64 g, 64 g + 64) of S^T and dP^T (thread = key), then dQ
-        // columns [64 g, 64 g + 64) (thread = query row). Each half packs its P^T and dS^T (bf16) in
-        // place at the start of its own columns, so the halves never write what the other reads.
+        // Warps w, w + 4, w + 8, w + 12 share TMEM lanes 32 (w % 4) .. + 31 and split the 128 columns
+        // of a step: warpgroup g takes query columns [32 g, 32 g + 32) of S^T and dP^T (thread = key),
+        // then dQ dims [32 g, 32 g + 32) (thread = query row). Each group packs its P^T and dS^T (bf16) in
+        // place at the start of its own columns, so no group writes what another still reads.
         const int grp = warp >> 2;
         const int kr = threadIdx.x & 127;  // key (softmax) or query row (dQ) within the tile == TMEM lane
         const int key = k0 + kr;
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        const uint32_t tS = tmem + lane_base + kColS + 64u * grp, tDP = tmem + lane_base + kColDP + 64u * grp;
-        const uint32_t tQ = tmem + lane_base + kColDP + 64u * grp;
+        const uint32_t tS = tmem + lane_base + kColS + kGroupCols * grp, tDP = tmem + lane_base + kColDP + kGroupCols * grp;
+        const uint32_t tQ = tmem + lane_base + kColDP + kGroupCols * grp;
         bool ok = true;
         for (int s = 0; s < n_steps; ++s) {
             const int st = s & 1;
@@ -397,51 +398,50 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int kk = kr & 63;
 #pragma unroll 1
             for (int c = 0; c < 2; ++c) {
-                const int cq = (2 * grp + c) * 32;  // first query column of this chunk
-                uint32_t sr[32], dr[32];
-                tmem_ld32x2_wait(tS + c * 32, tDP + c * 32, sr, dr);
-                float nl[32], dv[32];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float4 x = reinterpret_cast<const float4 *>(lse2 + cq)[i];
-                    const float4 y = reinterpret_cast<const float4 *>(dvec + cq)[i];
-                    nl[4 * i] = -x.x; nl[4 * i + 1] = -x.y; nl[4 * i + 2] = -x.z; nl[4 * i + 3] = -x.w;
-                    dv[4 * i] = y.x; dv[4 * i + 1] = y.y; dv[4 * i + 2] = y.z; dv[4 * i + 3] = y.w;
-                }
-                uint32_t pk[16], dk[16];
+                const int cq = kGroupCols * grp + 16 * c;  // first query column of this chunk
+                uint32_t sr[16], dr[16];
+                tmem_ld16x2_wait(tS + c * 16, tDP + c * 16, sr, dr);
+                uint32_t pk[8], dk[8];
                 auto body = [&](auto masked) {
 #pragma unroll
-                    for (int i = 0; i < 32; i += 2) {
-                        float pe[2], ds[2];
+                    for (int i4 = 0; i4 < 16; i4 += 4) {
+                        const float4 x = *reinterpret_cast<const float4 *>(lse2 + cq + i4);
+                        const float4 y = *reinterpret_cast<const float4 *>(dvec + cq + i4);
+                        const float nl[4] = {-x.x, -x.y, -x.z, -x.w};
+                        const float dv[4] = {y.x, y.y, y.z, y.w};
 #pragma unroll
-                        for (int u = 0; u < 2; ++u) {
-                            const int q = cq + i + u;
-                            const float w = ex2(fmaf(__uint_as_float(sr[i + u]), p.scale_log2, nl[i + u]));
-                            const float g = w * (__uint_as_float(dr[i + u]) - dv[i + u]);
-                            if constexpr (decltype(masked)::value) {
-                                const bool vis = key_ok && q >= first_q && q <= last_q;
-                                pe[u] = vis ? w : 0.f;
-                                ds[u] = vis ? g : 0.f;
-                            } else {
-                                pe[u] = w;
-                                ds[u] = g;
+                        for (int i = i4; i < i4 + 4; i += 2) {
+                            float pe[2], ds[2];
+#pragma unroll
+                            for (int u = 0; u < 2; ++u) {
+                                const int q = cq + i + u;
+                                const float w = ex2(fmaf(__uint_as_float(sr[i + u]), p.scale_log2, nl[i - i4 + u]));
+                                const float g = w * (__uint_as_float(dr[i + u]) - dv[i - i4 + u]);
+                                if constexpr (decltype(masked)::value) {
+                                    const bool vis = key_ok && q >= first_q && q <= last_q;
+                                    pe[u] = vis ? w : 0.f;
+                                    ds[u] = vis ? g : 0.f;
+                                } else {
+                                    pe[u] = w;
+                                    ds[u] = g;
+                                }
                             }
-                        }
-                        pk[i >> 1] = pack_bf16x2(pe[0], pe[1]);
-                        dk[i >> 1] = pack_bf16x2(ds[0], ds[1]);
+                            pk[i >> 1] = pack_bf16x2(pe[0], pe[1]);
+                            dk[i >> 1] = pack_bf16x2(ds[0], ds[1]);
 #pragma unroll
-                        for (int u = 0; u < 2; ++u) {
-                            const int q = cq + i + u;
-                            *reinterpret_cast<uint16_t *>(dsrow_base + q * 128 + ((((kk >> 3) ^ (q & 7)) << 4) | ((kk & 7) << 1))) =
-                                static_cast<uint16_t>(u ? (dk[i >> 1] >> 16) : (dk[i >> 1] & 0xffffu));
+                            for (int u = 0; u < 2; ++u) {
+                                const int q = cq + i + u;
+                                *reinterpret_cast<uint16_t *>(dsrow_base + q * 128 + ((((kk >> 3) ^ (q & 7)) << 4) | ((kk & 7) << 1))) =
+                                    static_cast<uint16_t>(u ? (dk[i >> 1] >> 16) : (dk[i >> 1] & 0xffffu));
+                            }
                         }
                     }
                 };
-                if (key_ok && first_q <= cq && cq + 31 <= last_q)
+                if (key_ok && first_q <= cq && cq + 15 <= last_q)
                     body(std::false_type{});
                 else
                     body(std::true_type{});
-                tmem_st16x2_wait(tS + c * 16, pk, tDP + c * 16, dk);
+                tmem_st8x2_wait(tS + c * 8, pk, tDP + c * 8, dk);
                 if (c == 1)
                     fence_proxy_async_smem();  // dS, for the dQ product
                 tc_fence_before_sync();
@@ -459,58 +459,51 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // 128-byte swizzle; the reducer warp adds them into the fp32 accumulator by TMA while
                 // the next step runs.
                 uint8_t *stage = smem + kOffStage + st * kStageBytes;
-#pragma unroll 1
-                for (int c = 0; c < 2; ++c) {
-                    uint32_t v[32];
-                    tmem_ld32_wait(tQ + c * 32, v);
-                    uint8_t *row = stage + (2 * grp + c) * kDqBox + kr * 128;
+                uint32_t v[32];
+                tmem_ld32_wait(tQ, v);
+                uint8_t *row = stage + grp * kDqBox + kr * 128;
 #pragma unroll
-                    for (int u = 0; u < 8; ++u)
-                        *reinterpret_cast<float4 *>(row + ((u ^ (kr & 7)) << 4)) =
-                            make_float4(__uint_as_float(v[4 * u]) * p.scale, __uint_as_float(v[4 * u + 1]) * p.scale,
-                                        __uint_as_float(v[4 * u + 2]) * p.scale, __uint_as_float(v[4 * u + 3]) * p.scale);
-                }
+                for (int u = 0; u < 8; ++u)
+                    *reinterpret_cast<float4 *>(row + ((u ^ (kr & 7)) << 4)) =
+                        make_float4(__uint_as_float(v[4 * u]) * p.scale, __uint_as_float(v[4 * u + 1]) * p.scale,
+                                    __uint_as_float(v[4 * u + 2]) * p.scale, __uint_as_float(v[4 * u + 3]) * p.scale);
             }
             fence_proxy_async_smem();
             tc_fence_before_sync();
             mbar_arrive(BAR(kBarDQFree0 + st));
         }
-        // Epilogue: dims [64 grp, 64 grp + 64) of dK (scaled) and dV of this key. The whole warp
+        // Epilogue: dims [32 grp, 32 grp + 32) of dK (scaled) and dV of this key. The whole warp
         // loads (tcgen05.ld is warp-collective); only the stores of keys past Skv are skipped.
         const bool okf = __all_sync(0xffffffffu, ok && mbar_wait(BAR(kBarFinal), 0, abort_flag, p.status, kSiteBwd));
         const bool key_store = key < p.Skv;
         if (okf) {
             tc_fence_after_sync();
             const size_t row = static_cast<size_t>(bh_kv) * p.Skv + (key_store ? key : 0);
-            __nv_bfloat16 *dk_row = p.dk + row * kD + 64 * grp;
-            __nv_bfloat16 *dv_row = p.dv + row * kD + 64 * grp;
-#pragma unroll 1
-            for (int c = 0; c < 2; ++c) {
-                uint32_t kv[32], vv[32];
-                if (n_steps > 0) {
-                    tmem_ld32_wait(tmem + lane_base + kColDK + 64u * grp + c * 32, kv);
-                    tmem_ld32_wait(tmem + lane_base + kColDV + 64u * grp + c * 32, vv);
-                } else {
+            __nv_bfloat16 *dk_row = p.dk + row * kD + kGroupCols * grp;
+            __nv_bfloat16 *dv_row = p.dv + row * kD + kGroupCols * grp;
+            uint32_t kv[32], vv[32];
+            if (n_steps > 0) {
+                tmem_ld32x2_wait(tmem + lane_base + kColDK + kGroupCols * grp, tmem + lane_base + kColDV + kGroupCols * grp,
+                                 kv, vv);
+            } else {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        kv[i] = vv[i] = 0u;
-                }
-                uint32_t pkk[16], pkv[16];
+                for (int i = 0; i < 32; ++i)
+                    kv[i] = vv[i] = 0u;
+            }
+            if (key_store) {
+                uint4 *dkk = reinterpret_cast<uint4 *>(dk_row);
+                uint4 *dvv = reinterpret_cast<uint4 *>(dv_row);
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    pkk[i] = pack_bf16x2(__uint_as_float(kv[2 * i]) * p.scale, __uint_as_float(kv[2 * i + 1]) * p.scale);
-                    pkv[i] = pack_bf16x2(__uint_as_float(vv[2 * i]), __uint_as_float(vv[2 * i + 1]));
+                for (int i = 0; i < 4; ++i) {
+                    dkk[i] = make_uint4(pack_bf16x2(__uint_as_float(kv[8 * i]) * p.scale, __uint_as_float(kv[8 * i + 1]) * p.scale),
+                                        pack_bf16x2(__uint_as_float(kv[8 * i + 2]) * p.scale, __uint_as_float(kv[8 * i + 3]) * p.scale),
+                                        pack_bf16x2(__uint_as_float(kv[8 * i + 4]) * p.scale, __uint_as_float(kv[8 * i + 5]) * p.scale),
+                                        pack_bf16x2(__uint_as_float(kv[8 * i + 6]) * p.scale, __uint_as_float(kv[8 * i + 7]) * p.scale));
+                    dvv[i] = make_uint4(pack_bf16x2(__uint_as_float(vv[8 * i]), __uint_as_float(vv[8 * i + 1])),
+                                        pack_bf16x2(__uint_as_float(vv[8 * i + 2]), __uint_as_float(vv[8 * i + 3])),
+                                        pack_bf16x2(__uint_as_float(vv[8 * i + 4]), __uint_as_float(vv[8 * i + 5])),
+                                        pack_bf16x2(__uint_as_float(vv[8 * i + 6]), __uint_as_float(vv[8 * i + 7])));
                 }
-                if (key_store) {
-                    uint4 *dkk = reinterpret_cast<uint4 *>(dk_row + c * 32);
-                    uint4 *dvv = reinterpret_cast<uint4 *>(dv_row + c * 32);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        dkk[i] = make_uint4(pkk[4 * i], pkk[4 * i + 1], pkk[4 * i + 2], pkk[4 * i + 3]);
-                        dvv[i] = make_uint4(pkv[4 * i], pkv[4 * i + 1], pkv[4 * i + 2], pkv[4 * i + 3]);
-                    }
-                }
-                __syncwarp();
             }
         }
     }
