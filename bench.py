@@ -341,8 +341,8 @@ def run_ours(args):
     tensor_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
 
-    # End to end through the public call on HOST buffers: pinned H2D of q, k, v, the kernel, D2H of
-    # o and lse, for the headline workload.
+    # End to end through the public call on HOST buffers (attn_fwd_host: the H2D copies of q, k, v,
+    # the attention and the D2H copies of o and lse, pipelined slice by slice), headline workload.
     hq, hk, hv = (t.pin_memory() for t in host[HEADLINE.name])
     ho = torch.empty(hq.shape, dtype=torch.bfloat16, pin_memory=True)
     hl = torch.empty(hq.shape[:3], dtype=torch.float32, pin_memory=True)
@@ -443,7 +443,7 @@ def run_ours(args):
             "timed_region_ms": region_ms,
             "e2e": {"value": e2e_tflops, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": e2e_steps,
-                    "what": "32K prefill through attn_fwd on pinned host buffers, copies included"},
+                    "what": "32K prefill through attn_fwd_host on pinned host buffers: copies in and out pipelined against the attention in eight slices, all inside the timed region"},
             "gpu_launches": n_w * args.steps,
             "device_status": status,
             "clocks": clk,

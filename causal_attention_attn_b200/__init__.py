@@ -5,7 +5,7 @@ The compute lives in ``libattn_b200.so`` (hand-written CUDA, C ABI declared in `
 load the library, so the seeded-input module can be used on machines without the build.
 """
 
-__version__ = "0.5.0"
+__version__ = "0.6.0"
 
 
 def __getattr__(name):

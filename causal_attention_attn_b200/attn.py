@@ -24,7 +24,7 @@ STATUS_NAMES = {
     -9: "ATTN_ERR_LAUNCH", -10: "ATTN_ERR_DEVICE_TIMEOUT", -11: "ATTN_ERR_SCALE", -12: "ATTN_ERR_CUDA",
     -13: "ATTN_ERR_SCRATCH_LIMIT",
 }
-EXPORTED = ("attn_fwd", "attn_fwd_ex", "attn_fwd_strided", "attn_decode_ctas", "attn_status_string", "attn_version",
+EXPORTED = ("attn_fwd", "attn_fwd_ex", "attn_fwd_host", "attn_fwd_strided", "attn_decode_ctas", "attn_status_string", "attn_version",
             "attn_device_status", "attn_decode_noalloc", "attn_decode_paged", "attn_prefill_paged", "attn_bwd", "attn_decode_fp8",
             "attn_decode_paged_fp8", "attn_lse_merge")
 
@@ -54,6 +54,8 @@ def load_library(path: str | None = None):
         lib.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp]
         lib.attn_fwd_ex.restype = i
         lib.attn_fwd_ex.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, vp]
+        lib.attn_fwd_host.restype = i
+        lib.attn_fwd_host.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp]
         ll3 = ctypes.POINTER(ctypes.c_longlong)
         lib.attn_fwd_strided.restype = i
         lib.attn_fwd_strided.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, ll3, ll3, ll3, ll3, f, i, vp]
@@ -191,31 +193,46 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: float | N
 
 def attn_fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: float | None = None,
                   causal: bool = True, device="cuda", stream=None, out_host=None, lse_host=None, dev_bufs=None):
-    """End-to-end call on HOST tensors: copy q, k, v to the device, run attn_fwd, copy o and lse back.
+    """End-to-end call on HOST tensors through ``attn_fwd_host``: the library copies q, k, v in,
+    runs the attention and copies o and lse out, slice by slice, with the copies of one slice
+    overlapping the attention of the next (so pinned inputs and outputs matter: pageable memory
+    works but does not overlap).
 
-    Inputs should be pinned for asynchronous copies. ``dev_bufs`` optionally supplies reusable
-    device tensors (q, k, v, o, lse) so that a loop of calls does not allocate. Returns host
-    (o, lse); the call synchronises on the stream before returning.
+    ``dev_bufs`` optionally supplies the device staging tensors (q, k, v, o, lse) so that a loop of
+    calls does not allocate. Returns host (o, lse); the call synchronises on the stream before
+    returning.
     """
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not isinstance(t, torch.Tensor) or t.device.type != "cpu" or t.dtype != torch.bfloat16:
+            raise ValueError(f"{name} must be a bf16 host tensor")
+        if t.dim() != 4 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous [batch, head, row, dim] tensor")
+    B, Hq, Sq, D = q.shape
+    Hkv, Skv = k.shape[1], k.shape[2]
+    if tuple(k.shape) != (B, Hkv, Skv, D) or tuple(v.shape) != tuple(k.shape):
+        raise ValueError(f"k {tuple(k.shape)} / v {tuple(v.shape)} do not match q {tuple(q.shape)}")
+    if scale is None:
+        scale = D ** -0.5
     stream = stream or torch.cuda.current_stream(device)
-    with torch.cuda.stream(stream):
-        if dev_bufs is None:
-            qd = q.to(device, non_blocking=True)
-            kd = k.to(device, non_blocking=True)
-            vd = v.to(device, non_blocking=True)
-            od, ld = None, None
-        else:
-            qd, kd, vd, od, ld = dev_bufs
-            qd.copy_(q, non_blocking=True)
-            kd.copy_(k, non_blocking=True)
-            vd.copy_(v, non_blocking=True)
-        od, ld = attn_fwd(qd, kd, vd, scale=scale, causal=causal, out=od, lse=ld, stream=stream)
-        if out_host is None:
-            out_host = torch.empty(od.shape, dtype=od.dtype, pin_memory=True)
-        if lse_host is None:
-            lse_host = torch.empty(ld.shape, dtype=ld.dtype, pin_memory=True)
-        out_host.copy_(od, non_blocking=True)
-        lse_host.copy_(ld, non_blocking=True)
+    if dev_bufs is None:
+        dev_bufs = (torch.empty(q.shape, dtype=torch.bfloat16, device=device),
+                    torch.empty(k.shape, dtype=torch.bfloat16, device=device),
+                    torch.empty(v.shape, dtype=torch.bfloat16, device=device),
+                    torch.empty(q.shape, dtype=torch.bfloat16, device=device),
+                    torch.empty((B, Hq, Sq), dtype=torch.float32, device=device))
+    qd, kd, vd, od, ld = dev_bufs
+    if out_host is None:
+        out_host = torch.empty(q.shape, dtype=torch.bfloat16, pin_memory=True)
+    if lse_host is None:
+        lse_host = torch.empty((B, Hq, Sq), dtype=torch.float32, pin_memory=True)
+    for name, t in (("out_host", out_host), ("lse_host", lse_host)):
+        if t.device.type != "cpu" or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous host tensor")
+    rc = load_library().attn_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), out_host.data_ptr(),
+                                      lse_host.data_ptr(), qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), od.data_ptr(),
+                                      ld.data_ptr(), B, Hq, Hkv, Sq, Skv, D, float(scale), int(bool(causal)),
+                                      _stream_handle(stream))
+    _check(rc)
     stream.synchronize()
     return out_host, lse_host
 

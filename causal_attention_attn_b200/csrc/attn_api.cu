@@ -16,7 +16,7 @@
 namespace attn_b200 {
 namespace {
 
-constexpr int kVersion = 500;  // 0.5.0: attn_fwd_strided, attn_prefill_paged, stream-ordered workspace growth
+constexpr int kVersion = 600;  // 0.6.0: attn_fwd_host (host buffers, copies pipelined against the kernels)
 
 struct DeviceState {
     bool probed = false;
@@ -31,6 +31,10 @@ struct DeviceState {
     size_t partial_floats = 0;
     void *bwd_block = nullptr;  // backward pass: dq accumulator and per-row vectors
     size_t bwd_bytes = 0;
+    // attn_fwd_host: a stream for the copies in, one for the copies out, and the events that order
+    // them against the caller's stream (created on first use, kept for the process).
+    cudaStream_t copy_in = nullptr, copy_out = nullptr;
+    cudaEvent_t ev_start = nullptr, ev_in = nullptr, ev_done = nullptr, ev_out = nullptr;
 };
 
 std::mutex g_mutex;
@@ -130,6 +134,29 @@ int ensure_workspace(DeviceState &s, size_t counters, size_t partials, cudaStrea
     s.counter_count = nc;
     s.partials = reinterpret_cast<float *>(static_cast<char *>(block) + head + cbytes);
     s.partial_floats = np;
+    return ATTN_OK;
+}
+
+// The copy streams and events of attn_fwd_host, created once per device (under g_mutex).
+int ensure_host_pipeline(DeviceState &s)
+{
+    if (s.ev_out)
+        return ATTN_OK;
+    if (!s.copy_in && cudaStreamCreateWithFlags(&s.copy_in, cudaStreamNonBlocking) != cudaSuccess)
+        s.copy_in = nullptr;
+    if (s.copy_in && !s.copy_out && cudaStreamCreateWithFlags(&s.copy_out, cudaStreamNonBlocking) != cudaSuccess)
+        s.copy_out = nullptr;
+    cudaEvent_t *evs[4] = {&s.ev_start, &s.ev_in, &s.ev_done, &s.ev_out};
+    bool ok = s.copy_in && s.copy_out;
+    for (cudaEvent_t *e : evs)
+        if (ok && !*e && cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) {
+            *e = nullptr;
+            ok = false;
+        }
+    if (!ok) {
+        cudaGetLastError();
+        return ATTN_ERR_CUDA;
+    }
     return ATTN_OK;
 }
 
@@ -251,6 +278,94 @@ extern "C" int attn_fwd_ex(const void *q, const void *k, const void *v, void *o,
 {
     return run(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, D, scale, causal, decode_ctas,
                contiguous_layouts(Hq, Hkv, Sq, Skv, D), stream);
+}
+
+extern "C" int attn_fwd_host(const void *q_host, const void *k_host, const void *v_host, void *o_host,
+                             float *lse_host, void *q_dev, void *k_dev, void *v_dev, void *o_dev, float *lse_dev,
+                             int B, int Hq, int Hkv, int Sq, int Skv, int D, float scale, int causal, void *stream_ptr)
+{
+    if (!q_host || !k_host || !v_host || !o_host || !lse_host)
+        return ATTN_ERR_NULL;
+    int rc = validate(q_dev, k_dev, v_dev, o_dev, lse_dev, B, Hq, Hkv, Sq, Skv, D, scale, causal);
+    if (rc != ATTN_OK)
+        return rc;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+    cudaStream_t s_in, s_out;
+    cudaEvent_t ev_start, ev_in, ev_done, ev_out;
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        int err = ATTN_OK;
+        DeviceState *s = device_state(&err);
+        if (!s)
+            return err;
+        if ((rc = ensure_host_pipeline(*s)) != ATTN_OK)
+            return rc;
+        s_in = s->copy_in;
+        s_out = s->copy_out;
+        ev_start = s->ev_start;
+        ev_in = s->ev_in;
+        ev_done = s->ev_done;
+        ev_out = s->ev_out;
+    }
+    // A unit is one (batch, kv head) with its group of query heads; its q, k, v, o and lse rows are
+    // contiguous, so a run of units is one copy per tensor and one attention call over B' = units,
+    // Hq' = group, Hkv' = 1. Slice boundaries fall on whole 16-byte blocks of lse.
+    const int group = Hq / Hkv;
+    const long long units = static_cast<long long>(B) * Hkv;
+    long long align = 1;
+    while ((static_cast<long long>(group) * Sq * align) % 4 != 0)
+        align *= 2;
+    constexpr long long kSlices = 8;
+    const size_t q_unit = static_cast<size_t>(group) * Sq * D * 2, kv_unit = static_cast<size_t>(Skv) * D * 2;
+    const size_t lse_unit = static_cast<size_t>(group) * Sq;
+    auto at = [](const void *p, size_t off) { return static_cast<const char *>(p) + off; };
+    auto atw = [](void *p, size_t off) { return static_cast<char *>(p) + off; };
+    // The copy streams start after the work already queued on `stream` (which may still use the
+    // device buffers), and `stream` continues after the last copy out.
+    if (cudaEventRecord(ev_start, stream) != cudaSuccess || cudaStreamWaitEvent(s_in, ev_start, 0) != cudaSuccess ||
+        cudaStreamWaitEvent(s_out, ev_start, 0) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_CUDA;
+    }
+    long long u0 = 0;
+    for (long long i = 1; i <= kSlices && u0 < units && rc == ATTN_OK; ++i) {
+        long long u1 = (i == kSlices) ? units : (units * i / kSlices) / align * align;
+        if (u1 <= u0)
+            continue;
+        const size_t n = static_cast<size_t>(u1 - u0);
+        const size_t qo = static_cast<size_t>(u0) * q_unit, ko = static_cast<size_t>(u0) * kv_unit;
+        const size_t lo = static_cast<size_t>(u0) * lse_unit;
+        if (cudaMemcpyAsync(atw(q_dev, qo), at(q_host, qo), n * q_unit, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
+            cudaMemcpyAsync(atw(k_dev, ko), at(k_host, ko), n * kv_unit, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
+            cudaMemcpyAsync(atw(v_dev, ko), at(v_host, ko), n * kv_unit, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
+            cudaEventRecord(ev_in, s_in) != cudaSuccess || cudaStreamWaitEvent(stream, ev_in, 0) != cudaSuccess) {
+            cudaGetLastError();
+            rc = ATTN_ERR_CUDA;
+            break;
+        }
+        rc = run(at(q_dev, qo), at(k_dev, ko), at(v_dev, ko), atw(o_dev, qo), lse_dev + lo, static_cast<int>(n), group, 1,
+                 Sq, Skv, D, scale, causal, 0, contiguous_layouts(group, 1, Sq, Skv, D), stream);
+        if (rc != ATTN_OK)
+            break;
+        if (cudaEventRecord(ev_done, stream) != cudaSuccess || cudaStreamWaitEvent(s_out, ev_done, 0) != cudaSuccess ||
+            cudaMemcpyAsync(atw(o_host, qo), at(o_dev, qo), n * q_unit, cudaMemcpyDeviceToHost, s_out) != cudaSuccess ||
+            cudaMemcpyAsync(lse_host + lo, lse_dev + lo, n * lse_unit * sizeof(float), cudaMemcpyDeviceToHost, s_out) !=
+                cudaSuccess) {
+            cudaGetLastError();
+            rc = ATTN_ERR_CUDA;
+            break;
+        }
+        u0 = u1;
+    }
+    // Join the copy streams back into `stream` on every path, so that later work on it (or a
+    // synchronisation of it) covers everything this call queued.
+    if (cudaEventRecord(ev_in, s_in) != cudaSuccess || cudaStreamWaitEvent(stream, ev_in, 0) != cudaSuccess ||
+        cudaEventRecord(ev_out, s_out) != cudaSuccess || cudaStreamWaitEvent(stream, ev_out, 0) != cudaSuccess) {
+        cudaGetLastError();
+        if (rc == ATTN_OK)
+            rc = ATTN_ERR_CUDA;
+    }
+    return rc;
 }
 
 namespace {

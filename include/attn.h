@@ -90,6 +90,33 @@ int attn_fwd_ex(const void *q, const void *k, const void *v, void *o, float *lse
                 float scale, int causal, int decode_ctas, void *stream);
 
 /*
+ * attn_fwd_host — attn_fwd from host memory to host memory, with the copies pipelined against the
+ * attention: the (batch, kv head) units are cut into up to eight slices, and while slice i is
+ * copied in, slice i-1 is computed and slice i-2 is copied out (two copy streams of the library's
+ * own, ordered against `stream` with events). Same operation and results as attn_fwd on the same
+ * values (each unit is computed the same way; the decode's split over CTAs may differ, within
+ * rounding) — "第11节：Attention 实现（Flash vs Fallback）", §3 for the mask, as attn_fwd.
+ *   q_host, k_host, v_host   host pointers, bf16, the contiguous layouts above. Page-locked
+ *                            (pinned) memory lets the copies overlap the kernels; pageable memory
+ *                            works but the copies then do not overlap.
+ *   o_host, lse_host         host pointers, bf16 [B, Hq, Sq, D] and fp32 [B, Hq, Sq].
+ *   q_dev .. lse_dev         device staging buffers of the same shapes, 16-byte aligned, owned by
+ *                            the caller and not used by other work until the call's work is done.
+ *   other arguments          as attn_fwd.
+ * Ordering: the copies start after the work already queued on `stream`, and work queued on
+ * `stream` after the call starts after the last copy back. The call returns once everything is
+ * queued: synchronise `stream` before reading o_host and lse_host, and keep every buffer alive
+ * until then. The first call on a device creates two streams and four events that live for the
+ * process; otherwise the call allocates only what attn_fwd does.
+ * Returns ATTN_OK or a negative attn_status: ATTN_ERR_NULL for a null host or device pointer, the
+ * attn_fwd errors for the shapes and the device buffers, ATTN_ERR_CUDA when a copy cannot be
+ * queued (the streams are joined back into `stream` on every path).
+ */
+int attn_fwd_host(const void *q_host, const void *k_host, const void *v_host, void *o_host, float *lse_host,
+                  void *q_dev, void *k_dev, void *v_dev, void *o_dev, float *lse_dev,
+                  int B, int Hq, int Hkv, int Sq, int Skv, int D, float scale, int causal, void *stream);
+
+/*
  * attn_fwd_strided — attn_fwd over tensors in any layout whose head dim is contiguous, e.g. the
  * token-major [B, S, H, D] that a projection writes, as well as the heads-major [B, H, S, D].
  *

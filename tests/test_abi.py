@@ -37,7 +37,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.attn_version() == 500
+    assert lib.attn_version() == 600
     for code, name in attn.STATUS_NAMES.items():
         s = attn.status_string(code)
         assert s and s != "unknown status", (code, name)
@@ -248,3 +248,33 @@ def _prefill_paged_call(lib, **kw):
 ])
 def test_prefill_paged_argument_errors(lib, name, override, expected):
     assert _prefill_paged_call(lib, **override) == expected, name
+
+
+# attn_fwd_host: host pointers are checked first, then the device buffers as attn_fwd checks its
+# arguments; every case below is rejected before any CUDA call.
+H = [0x110000, 0x120000, 0x130000, 0x140000, 0x150000]
+
+
+def _fwd_host_call(lib, host=None, dev=None, **kw):
+    a = dict(GOOD, **kw)
+    host = H if host is None else host
+    dev = A if dev is None else dev
+    return lib.attn_fwd_host(*host, *dev, a["B"], a["Hq"], a["Hkv"], a["Sq"], a["Skv"], a["D"], a["scale"],
+                             a["causal"], None)
+
+
+FWD_HOST_CASES = [
+    ("null q_host", dict(host=[0, H[1], H[2], H[3], H[4]]), -1),
+    ("null lse_host", dict(host=[H[0], H[1], H[2], H[3], 0]), -1),
+    ("null o_dev", dict(dev=[A[0], A[1], A[2], 0, A[4]]), -1),
+    ("misaligned k_dev", dict(dev=[A[0], A[1] + 8, A[2], A[3], A[4]]), -5),
+    ("group not integral", dict(Hq=3, Hkv=2), -3),
+    ("head dim 48", dict(D=48), -4),
+    ("causal with Sq > Skv", dict(Sq=9, Skv=8), -6),
+    ("zero scale", dict(scale=0.0), -11),
+]
+
+
+@pytest.mark.parametrize("name,override,expected", FWD_HOST_CASES, ids=[c[0] for c in FWD_HOST_CASES])
+def test_fwd_host_argument_errors(lib, name, override, expected):
+    assert _fwd_host_call(lib, **override) == expected, name

@@ -52,7 +52,9 @@ def test_backward_leg_reports_rate_and_roofline(monkeypatch):
     assert abs(out["us_per_launch"] - 1000.0) < 1e-9
     assert abs(out["value"] - flops / 1e-3 / 1e12) < 1e-6
     assert abs(out["roofline"]["frac"] - out["roofline"]["achieved"] / out["roofline"]["peak"]) < 1e-12
-    assert out["roofline"]["bound"] == "tensor" and out["roofline"]["traffic"] is None
+    assert out["roofline"]["bound"] == "tensor"
+    # traffic comes from the committed capture when its source hash matches the kernel's source
+    assert out["roofline"]["traffic"] == bench.read_traffic("bwd_kernel", w.name)
 
 
 def test_whole_job_rate_scales_with_ranks_for_the_backward_leg(monkeypatch):
