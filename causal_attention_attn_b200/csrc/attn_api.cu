@@ -39,6 +39,9 @@ struct DeviceState {
 
 std::mutex g_mutex;
 DeviceState g_dev[kMaxDevices];
+// attn_fwd_host: the copy streams and the events are shared by all calls on a device, so one call
+// queues its whole pipeline before the next starts (the events are re-recorded per slice).
+std::mutex g_host_mutex;
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -290,6 +293,7 @@ extern "C" int attn_fwd_host(const void *q_host, const void *k_host, const void 
     if (rc != ATTN_OK)
         return rc;
     cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+    std::lock_guard<std::mutex> host_lock(g_host_mutex);
     cudaStream_t s_in, s_out;
     cudaEvent_t ev_start, ev_in, ev_done, ev_out;
     {

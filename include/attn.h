@@ -107,7 +107,8 @@ int attn_fwd_ex(const void *q, const void *k, const void *v, void *o, float *lse
  * `stream` after the call starts after the last copy back. The call returns once everything is
  * queued: synchronise `stream` before reading o_host and lse_host, and keep every buffer alive
  * until then. The first call on a device creates two streams and four events that live for the
- * process; otherwise the call allocates only what attn_fwd does.
+ * process; otherwise the call allocates only what attn_fwd does. Calls from several host threads
+ * queue one after another (they share those streams and events).
  * Returns ATTN_OK or a negative attn_status: ATTN_ERR_NULL for a null host or device pointer, the
  * attn_fwd errors for the shapes and the device buffers, ATTN_ERR_CUDA when a copy cannot be
  * queued (the streams are joined back into `stream` on every path).
