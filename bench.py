@@ -397,6 +397,12 @@ def run_ours(args):
     except Exception as e:  # an extra leg that fails is reported in its object, not allowed to drop the line
         paged = {"metric": "paged chunked prefill TFLOP/s", "error": f"{type(e).__name__}: {e}"}
 
+    # The chunked prefill over an e4m3 cache of the same shape (attn_prefill_fp8), timed the same way.
+    try:
+        prefill_fp8 = prefill_fp8_leg(attn, args, ranks, dev, stream, clear_l2, world, peaks, peak_kind)
+    except Exception as e:
+        prefill_fp8 = {"metric": "chunked prefill TFLOP/s, e4m3 K/V cache", "error": f"{type(e).__name__}: {e}"}
+
     # The backward pass of the 8B prefill workload (dq, dk, dv from dout and the forward's o, lse),
     # timed the same way. Reported beside the step, not part of it.
     try:
@@ -440,6 +446,7 @@ def run_ours(args):
             },
             "backward": backward,
             "paged_prefill": paged,
+            "prefill_fp8": prefill_fp8,
             "timed_region_ms": region_ms,
             "e2e": {"value": e2e_tflops, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": e2e_steps,
@@ -464,6 +471,7 @@ KERNEL_SOURCES = {
     "bwd_kernel": ["bwd_sm100.cu", "sm100_ptx.cuh"],
     "decode_tc_kernel": ["decode_tc_sm100.cu", "sm100_ptx.cuh"],
     "decode_tc_kernel_fp8": ["decode_tc_sm100.cu", "sm100_ptx.cuh"],
+    "prefill_fp8_kernel": ["prefill_fp8_sm100.cu", "sm100_ptx.cuh"],
 }
 
 
@@ -580,6 +588,44 @@ def paged_prefill_leg(attn, args, ranks, dev, stream, clear_l2, world, peaks, pe
             "us_per_launch": launch_s * 1e6, "flops_per_launch": flops}
 
 
+def prefill_fp8_leg(attn, args, ranks, dev, stream, clear_l2, world, peaks, peak_kind):
+    """Time attn_prefill_fp8 on the chunked-prefill workload over its e4m3 cache: L2 flushed
+    before every launch, CUDA events around each, max over ranks. The roofline's peak is the e4m3
+    dense rate (twice the measured bf16 one, the nominal ratio); the kernel issues every product
+    three times (three e4m3 parts of q * k_scale and of the weights), which the algorithmic FLOPs do
+    not count."""
+    w = inputs.CHUNKED_PREFILL
+    q, k8, v8, ks, vs = (t.to(dev) for t in inputs.generate_fp8(w))
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+    call = lambda: attn.attn_prefill_fp8(q, k8, v8, ks, vs, scale=w.scale, causal=True, out=o, lse=lse, stream=stream)
+    for _ in range(args.warmup):
+        clear_l2()
+        call()
+    steps = max(3, min(args.steps, 100))
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+    ranks.barrier()
+    torch.cuda.synchronize(dev)
+    for s in range(steps):
+        clear_l2()
+        ev[s][0].record(stream)
+        call()
+        ev[s][1].record(stream)
+    torch.cuda.synchronize(dev)
+    ms = ranks.max([sum(a.elapsed_time(b) for a, b in ev)])[0]
+    launch_s = ms * 1e-3 / steps
+    e4m3_peak = 2.0 * float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    achieved = w.flops() / launch_s / 1e12
+    return {"metric": "chunked prefill TFLOP/s, e4m3 K/V cache", "value": whole_job_rate(world, w.flops(), launch_s) / 1e12,
+            "unit": "TFLOP/s", "config": dict(w.config(), kv_dtype="e4m3", scales="fp32 per (kv head, channel)"),
+            "steps": steps,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": e4m3_peak, "unit": "TFLOP/s",
+                         "frac": achieved / e4m3_peak, "traffic": read_traffic("prefill_fp8_kernel", w.name),
+                         "peak_kind": f"{peak_kind} bf16 dense (burst) x 2 (e4m3 nominal ratio)",
+                         "kernel": "prefill_fp8_kernel", "products_issued_per_algorithmic": 3},
+            "us_per_launch": launch_s * 1e6, "flops_per_launch": w.flops()}
+
+
 def fp8_decode_bytes(w) -> int:
     """Bytes the e4m3 decode must move once: K and V codes, q, o, lse and both coefficient tables."""
     kv = 2 * w.B * w.Hkv * w.Skv * w.D
@@ -621,6 +667,20 @@ def run_case(args):
         print(json.dumps({"case": w.name, "repeat": args.repeat, "us_per_launch": ms * 1e3,
                           "tflops": flops / (ms * 1e-3) / 1e12, "device_status": attn.device_status()}), flush=True)
         return 0
+    if args.case == "prefill_fp8":
+        w = inputs.CHUNKED_PREFILL
+        q, k8, v8, ks, vs = (t.cuda() for t in inputs.generate_fp8(w))
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        ev[0].record()
+        for _ in range(args.repeat):
+            attn.attn_prefill_fp8(q, k8, v8, ks, vs, scale=w.scale, causal=True)
+        ev[1].record()
+        torch.cuda.synchronize()
+        ms = ev[0].elapsed_time(ev[1]) / args.repeat
+        print(json.dumps({"case": w.name + "_e4m3", "repeat": args.repeat, "us_per_launch": ms * 1e3,
+                          "tflops": w.flops() / (ms * 1e-3) / 1e12, "device_status": attn.device_status()}),
+              flush=True)
+        return 0
     if args.case == "decode_fp8":
         w = inputs.DECODE_GQA
         q, k8, v8, ks, vs = (t.cuda() for t in inputs.generate_fp8(w))
@@ -660,7 +720,7 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--case", choices=sorted(inputs.SHORT_NAMES) + ["decode_fp8", "backward", "chunked_paged"],
+    ap.add_argument("--case", choices=sorted(inputs.SHORT_NAMES) + ["decode_fp8", "backward", "chunked_paged", "prefill_fp8"],
                     default=None,
                     help="only run this workload --repeat times (for profiling); prints no bench line")
     ap.add_argument("--repeat", type=int, default=3)

@@ -25,7 +25,7 @@ STATUS_NAMES = {
     -13: "ATTN_ERR_SCRATCH_LIMIT",
 }
 EXPORTED = ("attn_fwd", "attn_fwd_ex", "attn_fwd_host", "attn_fwd_strided", "attn_decode_ctas", "attn_status_string", "attn_version",
-            "attn_device_status", "attn_decode_noalloc", "attn_decode_paged", "attn_prefill_paged", "attn_bwd", "attn_decode_fp8",
+            "attn_device_status", "attn_decode_noalloc", "attn_decode_paged", "attn_prefill_paged", "attn_bwd", "attn_decode_fp8", "attn_prefill_fp8",
             "attn_decode_paged_fp8", "attn_lse_merge")
 
 _lock = threading.Lock()
@@ -76,6 +76,8 @@ def load_library(path: str | None = None):
         lib.attn_prefill_paged.restype = i
         lib.attn_prefill_paged.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, f, i, vp]
         lib.attn_decode_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
+        lib.attn_prefill_fp8.restype = i
+        lib.attn_prefill_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp]
         lib.attn_decode_paged_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, vp]
         lib.attn_lse_merge.restype = i
         lib.attn_lse_merge.argtypes = [vp, vp, vp, vp, vp, ctypes.c_longlong, i, vp]
@@ -369,6 +371,35 @@ def attn_decode_fp8(q: torch.Tensor, k8: torch.Tensor, v8: torch.Tensor, k_scale
         rc = load_library().attn_decode_fp8(q.data_ptr(), k8.data_ptr(), v8.data_ptr(), k_scale.data_ptr(),
                                             v_scale.data_ptr(), out.data_ptr(), lse.data_ptr(), B, Hq, Hkv, Skv, D,
                                             float(scale), int(decode_ctas), _stream_handle(stream))
+    _check(rc)
+    return out, lse
+
+
+def attn_prefill_fp8(q: torch.Tensor, k8: torch.Tensor, v8: torch.Tensor, k_scale: torch.Tensor,
+                     v_scale: torch.Tensor, scale: float | None = None, causal: bool = True,
+                     out: torch.Tensor | None = None, lse: torch.Tensor | None = None, stream=None):
+    """Attention of Sq queries over an e4m3 K/V cache through ``attn_prefill_fp8`` (the causal mask
+    aligned to the last Sq keys). q: [B, Hq, Sq, 128] bf16; k8, v8: [B, Hkv, Skv, 128] e4m3 codes
+    (uint8 or float8_e4m3fn); k_scale, v_scale: fp32 [Hkv, 128]. Returns (o, lse)."""
+    _check_tensor("q", q, torch.bfloat16, 4)
+    k8, v8 = _as_codes("k8", k8), _as_codes("v8", v8)
+    _check_tensor("k_scale", k_scale, torch.float32, 2)
+    _check_tensor("v_scale", v_scale, torch.float32, 2)
+    B, Hq, Sq, D = q.shape
+    Bk, Hkv, Skv, Dk = k8.shape
+    if tuple(v8.shape) != tuple(k8.shape) or Bk != B or Dk != D \
+            or tuple(k_scale.shape) != (Hkv, D) or tuple(v_scale.shape) != (Hkv, D):
+        raise ValueError("expected q [B,Hq,Sq,D], k8, v8 [B,Hkv,Skv,D] and scales [Hkv,D]")
+    if scale is None:
+        scale = D ** -0.5
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check_tensor("out", out, torch.bfloat16, 4)
+    _check_tensor("lse", lse, torch.float32, 3)
+    with torch.cuda.device(q.device):
+        rc = load_library().attn_prefill_fp8(q.data_ptr(), k8.data_ptr(), v8.data_ptr(), k_scale.data_ptr(),
+                                             v_scale.data_ptr(), out.data_ptr(), lse.data_ptr(), B, Hq, Hkv, Sq, Skv,
+                                             D, float(scale), int(bool(causal)), _stream_handle(stream))
     _check(rc)
     return out, lse
 

@@ -20,7 +20,8 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD_DIR = os.path.join(PKG, "_build")
 LIB_NAME = "libattn_b200.so"
 LIB_PATH = os.path.join(PKG, LIB_NAME)
-SOURCES = ["attn_api.cu", "prefill_sm100.cu", "decode_sm100.cu", "decode_tc_sm100.cu", "bwd_sm100.cu", "merge_sm100.cu", "attn_noalloc.cu"]
+SOURCES = ["attn_api.cu", "prefill_sm100.cu", "prefill_fp8_sm100.cu", "decode_sm100.cu", "decode_tc_sm100.cu", "bwd_sm100.cu",
+           "merge_sm100.cu", "attn_noalloc.cu"]
 HEADERS = ["kernels.h", "sm100_ptx.cuh", "tma_host.h"]
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr"]

@@ -16,7 +16,7 @@
 namespace attn_b200 {
 namespace {
 
-constexpr int kVersion = 600;  // 0.6.0: attn_fwd_host (host buffers, copies pipelined against the kernels)
+constexpr int kVersion = 700;  // 0.7.0: attn_prefill_fp8 (prefill over an e4m3 K/V cache); 0.6.0: attn_fwd_host
 
 struct DeviceState {
     bool probed = false;
@@ -662,6 +662,64 @@ extern "C" int attn_decode_paged_fp8(const void *q, const void *k_pages, const v
 {
     return decode_paged_impl(q, k_pages, v_pages, k_scale, v_scale, block_table, seq_lens, o, lse, B, Hq, Hkv,
                              num_pages, page_size, pages_per_seq, max_seq_len, scale, decode_ctas, stream_ptr, true);
+}
+
+extern "C" int attn_prefill_fp8(const void *q, const void *k8, const void *v8, const float *k_scale,
+                                const float *v_scale, void *o, float *lse, int B, int Hq, int Hkv, int Sq, int Skv,
+                                int D, float scale, int causal, void *stream_ptr)
+{
+    using namespace attn_b200;
+    if (!q || !k8 || !v8 || !k_scale || !v_scale || !o || !lse)
+        return ATTN_ERR_NULL;
+    if (B < 1 || Hq < 1 || Hkv < 1 || Sq < 1 || Skv < 1 || (causal != 0 && causal != 1))
+        return ATTN_ERR_SHAPE;
+    if (Hq % Hkv != 0)
+        return ATTN_ERR_GQA;
+    if (D != 128)
+        return ATTN_ERR_HEADDIM;
+    // Flat row indices and tensor-map coordinates must fit in 32 bits; so must the grid.
+    if (static_cast<long long>(B) * Hq * Sq > INT_MAX || static_cast<long long>(B) * Hkv * Skv > INT_MAX)
+        return ATTN_ERR_SHAPE;
+    if (causal && Sq > Skv)
+        return ATTN_ERR_CAUSAL_SQ_GT_SKV;
+    if (!aligned16(q) || !aligned16(k8) || !aligned16(v8) || !aligned16(k_scale) || !aligned16(v_scale) ||
+        !aligned16(o) || !aligned16(lse))
+        return ATTN_ERR_ALIGN;
+    if (!(scale > 0.f) || !std::isfinite(scale))
+        return ATTN_ERR_SCALE;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+    std::lock_guard<std::mutex> lock(g_mutex);
+    int err = ATTN_OK;
+    DeviceState *s = device_state(&err);
+    if (!s)
+        return err;
+    int rc = ensure_workspace(*s, 0, 0, stream);  // the status word
+    if (rc != ATTN_OK)
+        return rc;
+    PrefillFp8Args a;
+    a.q = q;
+    a.k8 = k8;
+    a.v8 = v8;
+    a.k_scale = k_scale;
+    a.v_scale = v_scale;
+    a.o = o;
+    a.lse = lse;
+    a.B = B;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.Sq = Sq;
+    a.Skv = Skv;
+    a.D = D;
+    a.scale = scale;
+    a.causal = causal;
+    a.status = s->status;
+    int encode_error = 0;
+    const cudaError_t e = launch_prefill_fp8(a, stream, &encode_error);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return encode_error != 0 ? ATTN_ERR_CUDA : ATTN_ERR_LAUNCH;
+    }
+    return ATTN_OK;
 }
 
 extern "C" int attn_decode_fp8(const void *q, const void *k8, const void *v8, const float *k_scale,

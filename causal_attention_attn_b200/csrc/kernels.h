@@ -39,6 +39,7 @@ enum WaitSite : int {
     kSiteDecodeProducer = 16,
     kSiteDecodeConsumer = 17,
     kSiteBwd = 24,
+    kSiteFp8Prefill = 32,
 };
 
 // Element strides of a [batch][head][row][dim] tensor with a contiguous dim (see tma_host.h).
@@ -107,6 +108,20 @@ struct DecodeArgs {
 
 // Returns a cudaError_t value (cudaSuccess on success); never synchronises.
 cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t stream, int *encode_error);
+
+// Prefill over an e4m3 K/V cache (head dim 128): k8, v8 [B][Hkv][Skv][D] codes, k_scale, v_scale
+// [Hkv][D] fp32 coefficients; q, o [B][Hq][Sq][D] bf16, lse [B][Hq][Sq]; contiguous.
+struct PrefillFp8Args {
+    const void *q, *k8, *v8;
+    const float *k_scale, *v_scale;
+    void *o;
+    float *lse;
+    int B, Hq, Hkv, Sq, Skv, D;
+    float scale;
+    int causal;
+    int *status;  // device status word
+};
+cudaError_t launch_prefill_fp8(const PrefillFp8Args &a, cudaStream_t stream, int *encode_error);
 
 // Backward pass (head dim 128): dq, dk, dv from q, k, v, o, dout and the forward's lse.
 struct BwdArgs {

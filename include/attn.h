@@ -294,6 +294,28 @@ int attn_decode_fp8(const void *q, const void *k8, const void *v8, const float *
                     void *stream);
 
 /*
+ * attn_prefill_fp8 — attn_fwd for any Sq (a prefill of Sq new tokens over a cached prefix, the
+ * causal mask aligned to the last Sq keys) over the e4m3 K/V cache of attn_decode_fp8: the result
+ * is attn_fwd over k~, v~ (the dequantised cache).
+ *
+ * Source (page title, section): "MLA 矩阵乘法吸收的数值稳定性治理", §五 (FP8 cache, higher-precision
+ * accumulation) and §二.1 (a coefficient per channel); "第11节：Attention 实现（Flash vs Fallback）",
+ * §3 (the mask aligned to the last Sq keys).
+ *
+ * Layout (device pointers owned by the caller, 16-byte aligned): q, o bf16 [B, Hq, Sq, 128];
+ * lse fp32 [B, Hq, Sq]; k8, v8 e4m3 codes [B, Hkv, Skv, 128]; k_scale, v_scale fp32 [Hkv, 128].
+ * The tensor core reads the codes as they are; q * k_scale (scaled per query row by a power of two
+ * into the top of the e4m3 range) and the softmax weights enter the products as sums of three e4m3
+ * parts (about 12 significant bits), with fp32 accumulation in tensor memory, so the result matches
+ * the dequantised cache to about the accuracy of the bf16 path. causal 0 or 1; with causal,
+ * Sq <= Skv. Head dim 128 only; Hq % Hkv == 0. Non-finite codes, coefficients or q values give
+ * undefined results. Returns ATTN_OK or a negative attn_status (argument errors before any launch).
+ */
+int attn_prefill_fp8(const void *q, const void *k8, const void *v8, const float *k_scale, const float *v_scale,
+                     void *o, float *lse, int B, int Hq, int Hkv, int Sq, int Skv, int D, float scale, int causal,
+                     void *stream);
+
+/*
  * attn_decode_paged_fp8 — attn_decode_paged over an e4m3 cache: k_pages, v_pages hold e4m3 codes
  * [num_pages, Hkv, page_size, 128] and k_scale, v_scale are as for attn_decode_fp8. Every other
  * argument, rule and return value is attn_decode_paged's.

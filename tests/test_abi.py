@@ -37,7 +37,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.attn_version() == 600
+    assert lib.attn_version() == 700
     for code, name in attn.STATUS_NAMES.items():
         s = attn.status_string(code)
         assert s and s != "unknown status", (code, name)
@@ -278,3 +278,31 @@ FWD_HOST_CASES = [
 @pytest.mark.parametrize("name,override,expected", FWD_HOST_CASES, ids=[c[0] for c in FWD_HOST_CASES])
 def test_fwd_host_argument_errors(lib, name, override, expected):
     assert _fwd_host_call(lib, **override) == expected, name
+
+
+# attn_prefill_fp8: (q, k8, v8, k_scale, v_scale, o, lse) pointers, then the sizes; every case below
+# is rejected before any CUDA call.
+F8 = [0x210000, 0x220000, 0x230000, 0x240000, 0x250000, 0x260000, 0x270000]
+
+
+def _prefill_fp8_call(lib, ptrs=None, B=1, Hq=4, Hkv=2, Sq=8, Skv=8, D=128, scale=0.125, causal=1):
+    ptrs = F8 if ptrs is None else ptrs
+    return lib.attn_prefill_fp8(*ptrs, B, Hq, Hkv, Sq, Skv, D, scale, causal, None)
+
+
+PREFILL_FP8_CASES = [
+    ("null k_scale", dict(ptrs=[F8[0], F8[1], F8[2], 0, F8[4], F8[5], F8[6]]), -1),
+    ("null lse", dict(ptrs=F8[:6] + [0]), -1),
+    ("zero query rows", dict(Sq=0), -2),
+    ("causal flag 2", dict(causal=2), -2),
+    ("group not integral", dict(Hq=3), -3),
+    ("head dim 64", dict(D=64), -4),
+    ("misaligned v8", dict(ptrs=[F8[0], F8[1], F8[2] + 4, F8[3], F8[4], F8[5], F8[6]]), -5),
+    ("causal with Sq > Skv", dict(Sq=9), -6),
+    ("negative scale", dict(scale=-1.0), -11),
+]
+
+
+@pytest.mark.parametrize("name,override,expected", PREFILL_FP8_CASES, ids=[c[0] for c in PREFILL_FP8_CASES])
+def test_prefill_fp8_argument_errors(lib, name, override, expected):
+    assert _prefill_fp8_call(lib, **override) == expected, name
