@@ -18,11 +18,13 @@
  *     S = [Q_1 | Q_2 | Q_3] [K | K | K]^T   12 instructions of M = N = 128, K = 32 into TMEM
  *     softmax  thread = row: S * 2^-e * scale * log2(e), causal mask, row max in two passes over
  *              the tile (the reference max moves only when it grows by more than 4, then O is
- *              rescaled), weights 2^(s - m) times 16 split into three e4m3 parts and written back
- *              into TMEM over the S columns already read (part t of keys 32c.. in columns
- *              24c + 8t: never a column the pass has not read yet);
- *     O += [P_1 | P_2 | P_3] [V; V; V]       12 instructions, A = the parts from TMEM, B = V read
- *              MN-major (one 128-byte atom spans the 128 dims);
+ *              rescaled), weights 2^(s - m) times 16 split into two e4m3 parts (about 8
+ *              significant bits, the precision the bf16 path gives P) and written back into TMEM
+ *              over the S columns already read (part t of keys 32c.. in columns 16c + 8t: never a
+ *              column the pass has not read yet);
+ *     O += [P_1 | P_2] [V; V]                8 instructions, A = the parts from TMEM, B = V read
+ *              MN-major (one 128-byte atom spans the 128 dims). Three parts for the weights
+ *              measured 12-15% slower for no accuracy the tolerance needs;
  *   epilogue O * v_scale / (sum of the parts' values), LSE from the sum of the exact weights.
  *
  * TMEM: 256 columns per CTA, S (then P) in [0, 128), O in [128, 256). The MMAs of one thread run
@@ -56,7 +58,8 @@ constexpr int kThreads = 192;
 constexpr int kWarpTma = 4;
 constexpr int kWarpMma = 5;
 constexpr int kStages = 2;
-constexpr int kParts = 3;
+constexpr int kParts = 3;   // e4m3 parts of q * k_scale (about 12 significant bits)
+constexpr int kPParts = 2;  // e4m3 parts of the weights (about 8 significant bits, as bf16 P)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kThreshold = 4.0f;  // log2 units; weights stay below 2^4 * 16 = 256 < 448
 constexpr float kPScale = 16.0f;
@@ -324,12 +327,12 @@ __global__ void __launch_bounds__(kThreads, 2)
                 break;
             tc_fence_after_sync();
             if (leader) {
-                // Part pt of keys 32 kk .. 32 kk + 31 sits in columns 24 kk + 8 pt.
+                // Part pt of keys 32 kk .. 32 kk + 31 sits in columns 16 kk + 8 pt.
 #pragma unroll
-                for (int pt = 0; pt < kParts; ++pt)
+                for (int pt = 0; pt < kPParts; ++pt)
 #pragma unroll
                     for (int kk = 0; kk < kBN / 32; ++kk)
-                        tc_mma_f8_ts(tmem + kColO, tmem + kColS + 24u * kk + 8u * pt,
+                        tc_mma_f8_ts(tmem + kColO, tmem + kColS + 8u * kPParts * kk + 8u * pt,
                                      smem_desc(sV + kk * 32 * 128, kTileBytes, 1024, kSwizzle128B), kIdO,
                                      (j > 0 || pt > 0 || kk > 0) ? 1u : 0u);
             }
@@ -398,12 +401,12 @@ __global__ void __launch_bounds__(kThreads, 2)
                 l *= alpha;
                 lpv *= alpha;
             }
-            // Pass 2: weights, their three e4m3 parts (x16) into TMEM over the columns already read.
+            // Pass 2: weights, their two e4m3 parts (x16) into TMEM over the columns already read.
 #pragma unroll 1
             for (int c = 0; c < kBN / 32; ++c) {
                 uint32_t sr[32];
                 tmem_ld32_wait(tS + c * 32, sr);
-                uint32_t pw[kParts][8];
+                uint32_t pw[kPParts][8];
 #pragma unroll
                 for (int g = 0; g < 8; ++g) {
                     float x4[4], u4[4];
@@ -415,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                         x4[u] = u4[u] = w * kPScale;
                     }
 #pragma unroll
-                    for (int pt = 0; pt < kParts; ++pt)
+                    for (int pt = 0; pt < kPParts; ++pt)
                         pw[pt][g] = split4(x4);
                     // What the PV product uses: the parts' sum, the weight minus the remainder.
 #pragma unroll
@@ -423,8 +426,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                         lpv += u4[u] - x4[u];
                 }
 #pragma unroll
-                for (int pt = 0; pt < kParts; ++pt)
-                    tmem_st8(tS + 24u * c + 8u * pt, pw[pt]);
+                for (int pt = 0; pt < kPParts; ++pt)
+                    tmem_st8(tS + 8u * kPParts * c + 8u * pt, pw[pt]);
             }
             tmem_wait_st();
             tc_fence_before_sync();

@@ -305,9 +305,10 @@ int attn_decode_fp8(const void *q, const void *k8, const void *v8, const float *
  * Layout (device pointers owned by the caller, 16-byte aligned): q, o bf16 [B, Hq, Sq, 128];
  * lse fp32 [B, Hq, Sq]; k8, v8 e4m3 codes [B, Hkv, Skv, 128]; k_scale, v_scale fp32 [Hkv, 128].
  * The tensor core reads the codes as they are; q * k_scale (scaled per query row by a power of two
- * into the top of the e4m3 range) and the softmax weights enter the products as sums of three e4m3
- * parts (about 12 significant bits), with fp32 accumulation in tensor memory, so the result matches
- * the dequantised cache to about the accuracy of the bf16 path. causal 0 or 1; with causal,
+ * into the top of the e4m3 range) enters the score product as a sum of three e4m3 parts (about 12
+ * significant bits) and the softmax weights the PV product as a sum of two (about 8, as the bf16
+ * path rounds them), with fp32 accumulation in tensor memory, so the result matches the
+ * dequantised cache to about the accuracy of the bf16 path. causal 0 or 1; with causal,
  * Sq <= Skv. Head dim 128 only; Hq % Hkv == 0. Non-finite codes, coefficients or q values give
  * undefined results. Returns ATTN_OK or a negative attn_status (argument errors before any launch).
  */
