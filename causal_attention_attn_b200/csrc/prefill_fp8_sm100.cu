@@ -19,7 +19,8 @@
  *     softmax  thread = row: S * 2^-e * scale * log2(e), causal mask, row max in two passes over
  *              the tile (the reference max moves only when it grows by more than 4, then O is
  *              rescaled), weights 2^(s - m) times 16 split into two e4m3 parts (about 8
- *              significant bits, the precision the bf16 path gives P) and written back into TMEM
+ *              significant bits, the precision the bf16 path gives P; the split runs in f16x2
+ *              arithmetic, two weights per instruction) and written back into TMEM
  *              over the S columns already read (part t of keys 32c.. in columns 16c + 8t: never a
  *              column the pass has not read yet);
  *     O += [P_1 | P_2] [V; V]                8 instructions, A = the parts from TMEM, B = V read
@@ -409,21 +410,30 @@ __global__ void __launch_bounds__(kThreads, 2)
                 uint32_t pw[kPParts][8];
 #pragma unroll
                 for (int g = 0; g < 8; ++g) {
-                    float x4[4], u4[4];
+                    float w4[4];
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
                         const int key = k0 + c * 32 + 4 * g + u;
-                        const float w = (key <= key_limit) ? ex2(__uint_as_float(sr[4 * g + u]) * row_factor - m_ref) : 0.f;
-                        l += w;
-                        x4[u] = u4[u] = w * kPScale;
+                        w4[u] = (key <= key_limit) ? ex2(__uint_as_float(sr[4 * g + u]) * row_factor - m_ref) : 0.f;
+                        l += w4[u];
                     }
+                    // Two keys at a time in f16x2 (11 bits, above the parts' 8): x = hi + lo + rest.
+                    uint32_t hi = 0u, lo = 0u;
 #pragma unroll
-                    for (int pt = 0; pt < kPParts; ++pt)
-                        pw[pt][g] = split4(x4);
-                    // What the PV product uses: the parts' sum, the weight minus the remainder.
-#pragma unroll
-                    for (int u = 0; u < 4; ++u)
-                        lpv += u4[u] - x4[u];
+                    for (int pr = 0; pr < 2; ++pr) {
+                        const __half2 x = __floats2half2_rn(w4[2 * pr] * kPScale, w4[2 * pr + 1] * kPScale);
+                        const uint32_t ch = __nv_cvt_halfraw2_to_fp8x2(__half2_raw(x), __NV_SATFINITE, __NV_E4M3);
+                        const __half2 vh = __half2(__nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(ch), __NV_E4M3));
+                        const uint32_t cl = __nv_cvt_halfraw2_to_fp8x2(__half2_raw(__hsub2(x, vh)), __NV_SATFINITE, __NV_E4M3);
+                        const __half2 vl = __half2(__nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(cl), __NV_E4M3));
+                        // What the PV product uses: the parts' sum (exact in f16).
+                        const float2 used = __half22float2(__hadd2(vh, vl));
+                        lpv += used.x + used.y;
+                        hi |= (ch & 0xffffu) << (16 * pr);
+                        lo |= (cl & 0xffffu) << (16 * pr);
+                    }
+                    pw[0][g] = hi;
+                    pw[1][g] = lo;
                 }
 #pragma unroll
                 for (int pt = 0; pt < kPParts; ++pt)
