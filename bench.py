@@ -44,6 +44,7 @@ STEP_WORKLOADS = (inputs.TINY_PREFILL, inputs.PREFILL_8B, inputs.DECODE_GQA, inp
 SHORT = {w.name: n for n, w in inputs.SHORT_NAMES.items()}
 L2_FLUSH_BYTES = 256 * 1024 * 1024
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+DATASHEET_BF16_TFLOPS = 2250.0  # B200 dense bf16, nominal
 
 
 def load_peaks():
@@ -249,8 +250,11 @@ def config_entry(w, launch_s, world, peaks, peak_kind, baseline=None):
         value, unit = whole_job_rate(world, w.io_bytes(), launch_s) / 1e9, "GB/s"
     else:
         achieved = w.flops() / launch_s / 1e12
+        sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
         roof = {"bound": "tensor", "achieved": achieved, "peak": tensor_peak, "unit": "TFLOP/s",
                 "frac": achieved / tensor_peak, "peak_kind": f"{peak_kind} bf16 dense (burst)",
+                "frac_of_sustained": achieved / sustained,  # the measured peak under the power cap
+                "frac_of_datasheet": achieved / DATASHEET_BF16_TFLOPS,  # nominal dense bf16
                 "flops_per_launch": w.flops()}
         value, unit = whole_job_rate(world, w.flops(), launch_s) / 1e12, "TFLOP/s"
     roof["traffic"] = read_traffic(kernel, w.name)

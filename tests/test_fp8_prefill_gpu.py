@@ -46,6 +46,8 @@ SHAPES = [
     (1, 8, 8, 64, 1000, False),    # non-causal, one query tile, eight KV tiles
     (3, 4, 2, 1, 257, True),       # a single query row per head
     (1, 32, 8, 384, 384, True),    # 8B-layer head structure
+    (2, 4, 4, 300, 100, False),    # non-causal with more queries than keys, one partial KV tile
+    (1, 2, 2, 17, 17, True),       # tiny: one partial query tile and one partial KV tile
 ]
 
 
