@@ -91,3 +91,36 @@ def test_copies_wait_for_earlier_work_on_the_stream_and_stay_in_bounds():
     assert torch.equal(o, o_ref.cpu()) and torch.equal(lse, l_ref.cpu())
     assert (obuf[:pad] == 7.0).all() and (obuf[pad + q.numel():] == 7.0).all()
     assert (lbuf[:pad] == 7.0).all() and (lbuf[pad + q.numel() // q.shape[3]:] == 7.0).all()
+
+
+def test_concurrent_host_calls_from_two_threads():
+    """Two host threads calling at once on their own streams (the library's copy streams and events
+    are shared, so the calls queue one after another): each gets its own, correct result."""
+    import threading
+
+    shapes = [inputs.custom(2, 8, 2, 200, 333, 128, True, seed=101), inputs.custom(1, 4, 4, 130, 600, 64, True, seed=102)]
+    data = [tuple(t.pin_memory() for t in inputs.generate(w)) for w in shapes]
+    refs = [attn.attn_fwd(*(t.cuda() for t in d), scale=w.scale, causal=True) for w, d in zip(shapes, data)]
+    torch.cuda.synchronize()
+    results, errors = [None, None], []
+
+    def worker(i):
+        try:
+            torch.cuda.set_device(0)
+            stream = torch.cuda.Stream()
+            outs = []
+            for _ in range(5):
+                outs.append(attn.attn_fwd_host(*data[i], scale=shapes[i].scale, causal=True, stream=stream))
+            results[i] = outs
+        except Exception as e:  # reported below
+            errors.append(e)
+
+    threads = [threading.Thread(target=worker, args=(i,)) for i in range(2)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join()
+    assert not errors, errors
+    for i in range(2):
+        for o, lse in results[i]:
+            assert torch.equal(o, refs[i][0].cpu()) and torch.equal(lse, refs[i][1].cpu()), i
