@@ -8,7 +8,8 @@
  *
  * Kernels:
  *   bwd_pre_kernel   D_i = dO_i . O_i and lse_i in log2 units, per row, into the workspace (rows
- *                    padded to whole 128-row tiles per (batch, head));
+ *                    padded to whole 128-row tiles per (batch, head)), and the row's fp32 dq
+ *                    accumulator cleared (no separate memset);
  *   bwd_kernel       one CTA per (128-key tile of K and V, batch, kv head); it walks every query
  *                    head of the kv head's group and every 128-row query tile that sees any of its
  *                    keys. Per step (one query tile), with keys in TMEM lanes:
@@ -135,24 +136,38 @@ __device__ __forceinline__ int first_qtile(const BwdParams &p, int k0)
     return q_min <= 0 ? 0 : q_min / kBQ;
 }
 
-// One warp per query row (grid-stride, 64-bit row indices): D_i = dO_i . O_i and lse_i in log2 units.
+// Half a warp per query row, two rows per warp and step (grid-stride, 64-bit row indices): each lane
+// reads 16 bytes of O and of dO, D_i = dO_i . O_i is summed over the half-warp, and lse_i goes to
+// log2 units; the same lanes clear the row's fp32 dq accumulator (512 bytes) that the main kernel
+// adds into.
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16 *o, const __nv_bfloat16 *dout,
-                                                     const float *lse, float *vec, long long rows, int Sq, int Sq_pad,
-                                                     size_t total_pad)
+                                                     const float *lse, float *vec, float *dq_acc, long long rows,
+                                                     int Sq, int Sq_pad, size_t total_pad)
 {
     const int lane = threadIdx.x & 31;
-    const long long n_warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
-    for (long long row = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; row < rows;
-         row += n_warps) {
-        const uint2 a = reinterpret_cast<const uint2 *>(o + static_cast<size_t>(row) * kD)[lane];
-        const uint2 b = reinterpret_cast<const uint2 *>(dout + static_cast<size_t>(row) * kD)[lane];
-        auto lo = [](uint32_t w) { return __uint_as_float(w << 16); };
-        auto hi = [](uint32_t w) { return __uint_as_float(w & 0xffff0000u); };
-        float d = lo(a.x) * lo(b.x) + hi(a.x) * hi(b.x) + lo(a.y) * lo(b.y) + hi(a.y) * hi(b.y);
+    const int hl = lane & 15;  // lane within the row's half-warp
+    const long long n_pairs = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
+    for (long long pr = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; 2 * pr < rows;
+         pr += n_pairs) {
+        const long long row = 2 * pr + (lane >> 4);
+        const bool valid = row < rows;
+        float d = 0.f;
+        if (valid) {
+            const uint4 a = reinterpret_cast<const uint4 *>(o + static_cast<size_t>(row) * kD)[hl];
+            const uint4 b = reinterpret_cast<const uint4 *>(dout + static_cast<size_t>(row) * kD)[hl];
+            const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1)
+            for (int u = 0; u < 4; ++u)
+                d += __uint_as_float(aw[u] << 16) * __uint_as_float(bw[u] << 16) +
+                     __uint_as_float(aw[u] & 0xffff0000u) * __uint_as_float(bw[u] & 0xffff0000u);
+            float4 *acc = reinterpret_cast<float4 *>(dq_acc + static_cast<size_t>(row) * kD) + 2 * hl;
+            acc[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+            acc[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int off = 8; off > 0; off >>= 1)
             d += __shfl_xor_sync(0xffffffffu, d, off);
-        if (lane == 0) {
+        if (valid && hl == 0) {
             const long long bh = row / Sq, i = row % Sq;
             const size_t idx = static_cast<size_t>(bh) * Sq_pad + static_cast<size_t>(i);
             vec[idx] = lse[row] * kLog2e;
@@ -161,12 +176,17 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16 *o, co
     }
 }
 
+// dQ (fp32 accumulator) -> bf16, two 16-byte loads in flight per thread and step.
 __global__ void __launch_bounds__(256) bwd_dq_kernel(const float4 *acc, uint2 *dq, long long n4)
 {
-    for (long long t = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; t < n4;
-         t += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+    for (long long t = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; t < n4; t += 2 * stride) {
+        const bool second = t + stride < n4;
         const float4 a = acc[t];
+        const float4 c = second ? acc[t + stride] : make_float4(0.f, 0.f, 0.f, 0.f);
         dq[t] = make_uint2(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w));
+        if (second)
+            dq[t + stride] = make_uint2(pack_bf16x2(c.x, c.y), pack_bf16x2(c.z, c.w));
     }
 }
 
@@ -557,15 +577,13 @@ cudaError_t launch_bwd(const BwdArgs &a, cudaStream_t stream, int *encode_error)
     float *vec = dq_acc + rows * kD;
     if (!make_map_f32(encode, &tdq, dq_acc, kD, a.Sq, a.B * a.Hq, 32, kBQ, CU_TENSOR_MAP_SWIZZLE_128B, encode_error))
         return cudaErrorInvalidValue;
-    cudaError_t e = cudaMemsetAsync(dq_acc, 0, rows * kD * sizeof(float), stream);
-    if (e != cudaSuccess)
-        return e;
     const size_t total_pad = static_cast<size_t>(a.B) * a.Hq * Sq_pad;
-    const size_t pre_blocks = (rows + 7) / 8;  // eight warps (rows) per block, at most 64K blocks (grid-stride)
+    const size_t pre_blocks = (rows + 15) / 16;  // eight warps of two rows per block, at most 64K blocks (grid-stride)
     bwd_pre_kernel<<<static_cast<unsigned>(pre_blocks < 65536 ? pre_blocks : 65536), 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16 *>(a.o), static_cast<const __nv_bfloat16 *>(a.dout), a.lse, vec,
+        static_cast<const __nv_bfloat16 *>(a.o), static_cast<const __nv_bfloat16 *>(a.dout), a.lse, vec, dq_acc,
         static_cast<long long>(rows), a.Sq, Sq_pad, total_pad);
-    if ((e = cudaGetLastError()) != cudaSuccess)
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess)
         return e;
 
     BwdParams p;
@@ -590,7 +608,9 @@ cudaError_t launch_bwd(const BwdArgs &a, cudaStream_t stream, int *encode_error)
     if ((e = cudaGetLastError()) != cudaSuccess)
         return e;
     const long long n4 = static_cast<long long>(rows) * kD / 4;
-    bwd_dq_kernel<<<296, 256, 0, stream>>>(reinterpret_cast<const float4 *>(dq_acc), static_cast<uint2 *>(a.dq), n4);
+    const long long dq_blocks = (n4 + 2 * 256 - 1) / (2 * 256);  // two float4 per thread, at most 64K blocks
+    bwd_dq_kernel<<<static_cast<unsigned>(dq_blocks < 65536 ? dq_blocks : 65536), 256, 0, stream>>>(
+        reinterpret_cast<const float4 *>(dq_acc), static_cast<uint2 *>(a.dq), n4);
     return cudaGetLastError();
 }
 
