@@ -871,6 +871,7 @@ extern "C" int attn_bwd(const void *q, const void *k, const void *v, const void 
     a.causal = causal;
     a.ws = s->bwd_block;
     a.status = s->status;
+    a.sm_count = s->sm_count;
     int encode_error = 0;
     if (launch_bwd(a, stream, &encode_error) != cudaSuccess) {
         cudaGetLastError();

@@ -29,7 +29,12 @@
  *                    reduce-adds while the next step runs; dK and dV stay in TMEM until the last
  *                    step. The asynchronous reduction takes the 64 KB of dQ per step off the chain
  *                    (written by the warps themselves, it took a third of the step: the SM's store
- *                    bandwidth to L2, not the reductions, bounded it);
+ *                    bandwidth to L2, not the reductions, bounded it).
+ *                    When the key tiles are fewer than the SMs and the group splits evenly, each
+ *                    key tile is a cluster of two CTAs that walk half of the query heads each; at
+ *                    the end CTA 1 stages its partial dK, dV (fp32) in its shared memory and CTA 0
+ *                    reads them through the cluster's distributed shared memory, adds them to its
+ *                    own and stores the sums;
  *   bwd_dq_kernel    dQ (fp32 workspace) -> bf16.
  *
  * TMEM (512 columns): [0,128) S^T, then P^T (bf16: warpgroup g's queries in [32 g, 32 g + 16));
@@ -89,7 +94,9 @@ enum BwdBar : int {
     kBarDQ = 8,           // dQ ready
     kBarDQFree0 = 9,      // [2], by stage: dQ out of TMEM and staged in shared memory (256 arrivals)
     kBarFinal = 11,       // every MMA done
-    kNumBwdBars = 12,
+    kBarPeerReady = 12,   // cluster of two, CTA 0: CTA 1's partial dK (phase 0), dV (phase 1) staged (512 arrivals)
+    kBarPeerDone = 13,    // CTA 1: CTA 0 has read the staged dK (512 arrivals)
+    kNumBwdBars = 14,
 };
 constexpr int kOffMisc = kOffBar + kNumBwdBars * 8;
 constexpr int kSmem = kOffMisc + 64;  // the dynamic window starts 1024-aligned (no static smem)
@@ -101,8 +108,58 @@ struct BwdParams {
     const float *vec;    // [2][B*Hq][Sq_pad]: lse2 then D
     int *status;
     int B, Hq, Hkv, Sq, Skv, Sq_pad, group, offset, causal, n_ktiles;
+    int n_split;  // CTAs per key tile (1, or 2 as a cluster), each with group / n_split of the query heads
     float scale, scale_log2;
 };
+
+// ---- a 2-CTA cluster's exchange through distributed shared memory ----------------------------
+__device__ __forceinline__ uint32_t cluster_rank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// The address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t peer_addr(uint32_t addr, uint32_t rank)
+{
+    uint32_t out;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(addr), "r"(rank));
+    return out;
+}
+__device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr)
+{
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr)
+                 : "memory");
+    return v;
+}
+// Arrival (release at cluster scope) on an mbarrier of the peer CTA, given its cluster address.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_bar)
+{
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+}
+// Bounded wait (acquire at cluster scope: the peer's writes before its arrival are visible after).
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, uint64_t limit_ns)
+{
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+        uint32_t done;
+        asm volatile("{\n\t.reg .pred q;\n\tmbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 q, [%1], %2;\n\t"
+                     "selp.u32 %0, 1, 0, q;\n\t}"
+                     : "=r"(done)
+                     : "r"(bar), "r"(parity)
+                     : "memory");
+        if (done)
+            return true;
+        if (global_timer_ns() - t0 > limit_ns)
+            return false;
+    }
+}
+// Every thread of both CTAs: the cluster barrier (release / acquire).
+__device__ __forceinline__ void cluster_sync()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
 
 __device__ __forceinline__ float ex2(float x)
 {
@@ -213,8 +270,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         return;
     }
 
-    // Work decode: kv heads fastest, then batch, then key tiles from the first (the most rows see them).
+    // Work decode: the head split fastest (a cluster's two CTAs), then kv heads, then batch, then key
+    // tiles from the first (the most rows see them).
     int t = blockIdx.x;
+    const int sp = t % p.n_split;
+    t /= p.n_split;
     const int g = t % p.Hkv;
     t /= p.Hkv;
     const int b = t % p.B;
@@ -224,8 +284,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int n_qtiles = (p.Sq + kBQ - 1) / kBQ;
     const int qt0 = first_qtile(p, k0);
     const int steps_per_head = (qt0 < n_qtiles) ? n_qtiles - qt0 : 0;
-    const int n_steps = steps_per_head * p.group;
-    auto step_head = [&](int s) { return g * p.group + s / steps_per_head; };
+    const int heads = p.group / p.n_split;  // query heads of this CTA
+    const int n_steps = steps_per_head * heads;
+    auto step_head = [&](int s) { return g * p.group + sp * heads + s / steps_per_head; };
     auto step_q0 = [&](int s) { return (qt0 + s % steps_per_head) * kBQ; };
 
     if (threadIdx.x == 0) {
@@ -240,6 +301,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(BAR(kBarP1), 32 * kSoftWarps);
         mbar_init(BAR(kBarDQ), 1);
         mbar_init(BAR(kBarFinal), 1);
+        mbar_init(BAR(kBarPeerReady), 32 * kSoftWarps);
+        mbar_init(BAR(kBarPeerDone), 32 * kSoftWarps);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -250,6 +313,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
+    if (p.n_split > 1)
+        cluster_sync();  // both CTAs' barriers are initialised before any remote arrival
     const uint32_t tmem = *tmem_slot;
 
     if (warp == kWarpTma) {
@@ -496,12 +561,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // loads (tcgen05.ld is warp-collective); only the stores of keys past Skv are skipped.
         const bool okf = __all_sync(0xffffffffu, ok && mbar_wait(BAR(kBarFinal), 0, abort_flag, p.status, kSiteBwd));
         const bool key_store = key < p.Skv;
+        uint32_t kv[32], vv[32];
         if (okf) {
             tc_fence_after_sync();
-            const size_t row = static_cast<size_t>(bh_kv) * p.Skv + (key_store ? key : 0);
-            __nv_bfloat16 *dk_row = p.dk + row * kD + kGroupCols * grp;
-            __nv_bfloat16 *dv_row = p.dv + row * kD + kGroupCols * grp;
-            uint32_t kv[32], vv[32];
             if (n_steps > 0) {
                 tmem_ld32x2_wait(tmem + lane_base + kColDK + kGroupCols * grp, tmem + lane_base + kColDV + kGroupCols * grp,
                                  kv, vv);
@@ -510,6 +572,52 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int i = 0; i < 32; ++i)
                     kv[i] = vv[i] = 0u;
             }
+        }
+        bool store_ok = okf;
+        if (p.n_split > 1) {
+            // The cluster's CTA 1 stages its partial dK, then dV (fp32, [key][dim] with the 16-byte
+            // unit index XOR key % 32, in the K/V tiles, which no product reads any more); CTA 0
+            // adds them to its own and stores the sums. Waits are bounded; the cluster barrier at
+            // the end keeps both CTAs' shared memory alive until every access is done.
+            const uint32_t rank = cluster_rank();
+            const uint32_t buf = s_base + kOffK;
+            auto unit = [&](int c) { return static_cast<uint32_t>(kr * 512 + (((grp * 8 + c) ^ (kr & 31)) << 4)); };
+            for (int round = 0; round < 2; ++round) {
+                uint32_t(&val)[32] = round ? vv : kv;
+                if (rank == 1) {
+                    if (okf) {
+#pragma unroll
+                        for (int c = 0; c < 8; ++c)
+                            *reinterpret_cast<uint4 *>(smem + kOffK + unit(c)) =
+                                make_uint4(val[4 * c], val[4 * c + 1], val[4 * c + 2], val[4 * c + 3]);
+                        mbar_arrive_remote(peer_addr(BAR(kBarPeerReady), 0));
+                    }
+                    if (round == 0 && okf && !mbar_wait_cluster(BAR(kBarPeerDone), 0, kWaitLimitNs))
+                        atomicExch(p.status, kSiteBwd);
+                } else {
+                    store_ok = store_ok && mbar_wait_cluster(BAR(kBarPeerReady), static_cast<uint32_t>(round), kWaitLimitNs);
+                    if (store_ok) {
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {
+                            const float4 x = ld_cluster_f4(peer_addr(buf + unit(c), 1));
+                            val[4 * c] = __float_as_uint(__uint_as_float(val[4 * c]) + x.x);
+                            val[4 * c + 1] = __float_as_uint(__uint_as_float(val[4 * c + 1]) + x.y);
+                            val[4 * c + 2] = __float_as_uint(__uint_as_float(val[4 * c + 2]) + x.z);
+                            val[4 * c + 3] = __float_as_uint(__uint_as_float(val[4 * c + 3]) + x.w);
+                        }
+                    } else if (okf) {
+                        atomicExch(p.status, kSiteBwd);
+                    }
+                    if (round == 0)
+                        mbar_arrive_remote(peer_addr(BAR(kBarPeerDone), 1));
+                }
+            }
+            store_ok = store_ok && rank == 0;
+        }
+        if (store_ok) {
+            const size_t row = static_cast<size_t>(bh_kv) * p.Skv + (key_store ? key : 0);
+            __nv_bfloat16 *dk_row = p.dk + row * kD + kGroupCols * grp;
+            __nv_bfloat16 *dv_row = p.dv + row * kD + kGroupCols * grp;
             if (key_store) {
                 uint4 *dkk = reinterpret_cast<uint4 *>(dk_row);
                 uint4 *dvv = reinterpret_cast<uint4 *>(dv_row);
@@ -530,6 +638,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     tc_fence_before_sync();
     __syncthreads();
+    if (p.n_split > 1)
+        cluster_sync();  // neither CTA leaves while the other may still touch its shared memory
     if (warp == kWarpMma) {
         tc_fence_after_sync();
         tmem_dealloc(tmem, 512);
@@ -601,10 +711,32 @@ cudaError_t launch_bwd(const BwdArgs &a, cudaStream_t stream, int *encode_error)
     p.offset = a.Skv - a.Sq;
     p.causal = a.causal;
     p.n_ktiles = (a.Skv + kBK - 1) / kBK;
+    // A grid of fewer key tiles than SMs leaves SMs idle: then each key tile's query heads are split
+    // over a cluster of two CTAs (when the group splits evenly). Larger grids keep one CTA per key
+    // tile, where the split's second set-up and exchange cost more than the balance gains.
+    const long long tiles = static_cast<long long>(p.n_ktiles) * a.B * a.Hkv;
+    p.n_split = ((a.Hq / a.Hkv) % 2 == 0 && tiles < a.sm_count) ? 2 : 1;
     p.scale = a.scale;
     p.scale_log2 = a.scale * kLog2e;
-    const long long grid = static_cast<long long>(p.n_ktiles) * a.B * a.Hkv;
-    bwd_kernel<<<static_cast<unsigned>(grid), kThreads, kSmem, stream>>>(tq, tk, tv, tdo, tdq, p);
+    const long long grid = static_cast<long long>(p.n_ktiles) * a.B * a.Hkv * p.n_split;
+    if (p.n_split > 1) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(grid));
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = kSmem;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if ((e = cudaLaunchKernelEx(&cfg, bwd_kernel, tq, tk, tv, tdo, tdq, p)) != cudaSuccess)
+            return e;
+    } else {
+        bwd_kernel<<<static_cast<unsigned>(grid), kThreads, kSmem, stream>>>(tq, tk, tv, tdo, tdq, p);
+    }
     if ((e = cudaGetLastError()) != cudaSuccess)
         return e;
     const long long n4 = static_cast<long long>(rows) * kD / 4;

@@ -131,8 +131,9 @@ struct BwdArgs {
     int B, Hq, Hkv, Sq, Skv, D;
     float scale;
     int causal;
-    void *ws;     // bwd_workspace_bytes(B, Hq, Sq, D) bytes, 256-byte aligned
-    int *status;  // device status word
+    void *ws;      // bwd_workspace_bytes(B, Hq, Sq, D) bytes, 256-byte aligned
+    int *status;   // device status word
+    int sm_count;  // SMs of the device (chooses the head split)
 };
 size_t bwd_workspace_bytes(int B, int Hq, int Sq, int D);
 cudaError_t launch_bwd(const BwdArgs &a, cudaStream_t stream, int *encode_error);

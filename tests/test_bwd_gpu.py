@@ -30,6 +30,9 @@ def gpu():
     assert attn.device_status() == 0, "a kernel-side wait ran out during the backward tests"
 
 
+# Shapes with fewer key tiles than SMs and an even group run each key tile as a cluster of two CTAs
+# (half of the query heads each, partial dK and dV summed through distributed shared memory); the
+# others one CTA per key tile.
 SHAPES = [
     # B, Hq, Hkv, Sq, Skv, causal
     (1, 2, 1, 128, 128, True),    # one tile, GQA 2
@@ -38,6 +41,7 @@ SHAPES = [
     (1, 2, 1, 200, 130, False),   # non-causal, more queries than keys
     (1, 8, 2, 512, 512, True),    # several tiles each way, GQA 4
     (1, 1, 1, 64, 1000, True),    # a short chunk over a long cache: many key tiles no row sees early
+    (19, 2, 1, 1000, 1000, True),  # 152 key tiles (not fewer than the SMs): no head split, one CTA per key tile
 ]
 
 
