@@ -13,7 +13,9 @@
  *   O_X += P_X V_j     P_X rounded to bf16 and written back into TMEM over the first half of
  *                      S_X's columns, then tcgen05.mma with A = P_X read from TMEM and B = V_j read
  *                      MN-major from shared memory;
- *   epilogue           O_X / l_X to bf16, LSE = (m + log2 l) * ln 2.
+ *   epilogue           O_X / l_X to bf16, LSE = (m + log2 l) * ln 2; for D = 128, O leaves through
+ *                      TMA tensor stores from a staging box per warp, so the warps start the next
+ *                      item without waiting for their stores to drain.
  *
  * The two tiles ping-pong: while the softmax warps of A work on S_A(j), the tensor core runs
  * S_B(j) and the PV product and next S of B, and the other way round. Because the MMAs of one
@@ -92,7 +94,12 @@ struct Cfg {
     static constexpr int kTileBytes = 128 * D * 2;
     static constexpr int kOffQ = 0;  // Q_A, then Q_B
     static constexpr int kOffRing = kOffQ + 2 * kTileBytes;
-    static constexpr int kOffBar = kOffRing + kRing * kTileBytes;
+    // D = 128: O leaves through TMA stores, each softmax warp staging its 32 rows x 64 dims (4 KB,
+    // 128-byte swizzle) at a time.
+    static constexpr bool kTmaStore = (D == 128);
+    static constexpr int kWarpStageBytes = 32 * 128;
+    static constexpr int kOffStage = kOffRing + kRing * kTileBytes;
+    static constexpr int kOffBar = kOffStage + (kTmaStore ? 8 * kWarpStageBytes : 0);
     static constexpr int kUsed = kOffBar + 256;
     // >= 118 KB so that two CTAs never share an SM: each one allocates all 512 TMEM columns.
     static constexpr int kSmem = (kUsed + 1024 > 118 * 1024) ? kUsed + 1024 : 118 * 1024;
@@ -263,7 +270,7 @@ __device__ __forceinline__ int next_active(const Params &p, int r)
 template <int D, bool kPaged>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, const Params p)
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o, const Params p)
 {
     using C = Cfg<D>;
     extern __shared__ uint8_t smem_raw[];
@@ -300,6 +307,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
+        if constexpr (C::kTmaStore)
+            tma_prefetch_desc(&tm_o);
     }
     if (warp == kWarpMma) {
         tmem_alloc(smem_u32(tmem_slot), kTmemCols);
@@ -760,25 +769,66 @@ __global__ void __launch_bounds__(kThreads, 1)
             const Item it = decode_item<kPaged>(p, w);
             const int hq = x ? it.hq[1] : it.hq[0];
             const size_t bh_q = static_cast<size_t>(it.b) * p.Hq + hq;
-            __nv_bfloat16 *orow = p.o + it.b * p.o_sb + hq * p.o_sh + (store ? row : 0) * p.o_ss;
+            if constexpr (C::kTmaStore) {
+                // The warp's 32 rows, 64 dims at a time: TMEM -> bf16 -> the warp's staging box (rows of
+                // 128 bytes, 16-byte units XOR row % 8: the 128-byte swizzle) -> one TMA store by lane 0.
+                // The staging box is reused once the previous store has read it; rows past Sq are
+                // clipped by the store.
+                const uint32_t wstage = s_base + C::kOffStage + static_cast<uint32_t>(warp) * C::kWarpStageBytes;
+                uint8_t *wrow = smem + C::kOffStage + warp * C::kWarpStageBytes + lane * 128;
+                const int row0 = q0 + 32 * (warp & 3);
 #pragma unroll 1
-            for (int cc = 0; cc < D / 32; ++cc) {
-                uint32_t ov[32];
-                tmem_ld32_wait(tO + cc * 32, ov);
-                uint32_t pkd[16];
+                for (int h = 0; h < D / 64; ++h) {
+                    uint32_t oa[32], ob[32];
+                    tmem_ld32x2_wait(tO + h * 64, tO + h * 64 + 32, oa, ob);
+                    uint32_t pkd[32];
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    pkd[i] = pack_bf16x2(__uint_as_float(ov[2 * i]) * inv_l, __uint_as_float(ov[2 * i + 1]) * inv_l);
-                if (store) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(orow + cc * 32);
+                    for (int i = 0; i < 16; ++i) {
+                        pkd[i] = pack_bf16x2(__uint_as_float(oa[2 * i]) * inv_l, __uint_as_float(oa[2 * i + 1]) * inv_l);
+                        pkd[16 + i] = pack_bf16x2(__uint_as_float(ob[2 * i]) * inv_l, __uint_as_float(ob[2 * i + 1]) * inv_l);
+                    }
+                    if (lane == 0)
+                        bulk_wait_group_read0();
+                    __syncwarp();
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        dst[i] = make_uint4(pkd[4 * i], pkd[4 * i + 1], pkd[4 * i + 2], pkd[4 * i + 3]);
+                    for (int u = 0; u < 8; ++u)
+                        *reinterpret_cast<uint4 *>(wrow + ((u ^ (lane & 7)) << 4)) =
+                            make_uint4(pkd[4 * u], pkd[4 * u + 1], pkd[4 * u + 2], pkd[4 * u + 3]);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0 && row0 < p.Sq) {
+                        tma_store_4d(&tm_o, wstage, h * 64, row0, hq, it.b);
+                        bulk_commit_group();
+                    }
+                }
+            } else {
+                __nv_bfloat16 *orow = p.o + it.b * p.o_sb + hq * p.o_sh + (store ? row : 0) * p.o_ss;
+    #pragma unroll 1
+                for (int cc = 0; cc < D / 32; ++cc) {
+                    uint32_t ov[32];
+                    tmem_ld32_wait(tO + cc * 32, ov);
+                    uint32_t pkd[16];
+    #pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        pkd[i] = pack_bf16x2(__uint_as_float(ov[2 * i]) * inv_l, __uint_as_float(ov[2 * i + 1]) * inv_l);
+                    if (store) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(orow + cc * 32);
+    #pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            dst[i] = make_uint4(pkd[4 * i], pkd[4 * i + 1], pkd[4 * i + 2], pkd[4 * i + 3]);
+                    }
                 }
             }
             if (store)
                 p.lse[bh_q * p.Sq + row] = (m + log2f(l)) * kLn2;
             tc_fence_before_sync();
+        }
+        if constexpr (C::kTmaStore) {
+            // Every store issued by this warp has completed (its staging is read and O is written)
+            // before the CTA can exit.
+            if (lane == 0)
+                bulk_wait_group0();
+            __syncwarp();
         }
     }
 
@@ -802,10 +852,17 @@ cudaError_t launch(const PrefillArgs &a, cudaStream_t stream, int *encode_error)
     }
     const CUtensorMapSwizzle swz =
         (C::kSwizzleBytes == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, to;
     auto st = [](const TensorStrides &t) { return Strides{t.b, t.h, t.s}; };
     if (!make_map4(encode, &tq, a.q, 2, D, a.Sq, a.Hq, a.B, st(a.qs), C::kChunkElems, 128, swz, encode_error))
         return cudaErrorInvalidValue;
+    // O as (dim, row, head, batch), stored in boxes of 64 dims x 32 rows (one warp's rows); unused
+    // (a copy of Q's map) without TMA stores.
+    to = tq;
+    if constexpr (C::kTmaStore)
+        if (!make_map4(encode, &to, a.o, 2, D, a.Sq, a.Hq, a.B, st(a.os), 64, 32, CU_TENSOR_MAP_SWIZZLE_128B,
+                       encode_error))
+            return cudaErrorInvalidValue;
     if constexpr (kPaged) {
         // Pages [num_pages][Hkv][page_size][D] as (dim, slot, kv head, page), boxes of
         // min(page_size, 128) slots; the page index num_pages lies past the end: zeros.
@@ -876,7 +933,7 @@ cudaError_t launch(const PrefillArgs &a, cudaStream_t stream, int *encode_error)
     p.n_work = static_cast<int>(n_work);
     // Persistent: one CTA per SM (each holds all 512 TMEM columns), never more than the items.
     const int grid = static_cast<int>(n_work < a.sm_count ? n_work : a.sm_count);
-    prefill_kernel<D, kPaged><<<static_cast<unsigned>(grid), kThreads, C::kSmem, stream>>>(tq, tk, tv, p);
+    prefill_kernel<D, kPaged><<<static_cast<unsigned>(grid), kThreads, C::kSmem, stream>>>(tq, tk, tv, to, p);
     return cudaGetLastError();
 }
 
