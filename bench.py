@@ -394,6 +394,18 @@ def run_ours(args):
     fp8_ms = ranks.max([sum(a.elapsed_time(b) for a, b in fev)])[0]
     fp8_launch_s = fp8_ms * 1e-3 / fp8_steps
 
+    # The floor of this timing method: an empty kernel (torch.cuda._sleep(0), one block) launched
+    # and event-timed exactly like the kernels above. A launch's event-timed duration is its body
+    # plus about this much; short kernels (the decodes) feel it most.
+    floor_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(25)]
+    for a, b in floor_ev:
+        clear_l2()
+        a.record(stream)
+        torch.cuda._sleep(0)
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    launch_floor_us = statistics.median(a.elapsed_time(b) * 1e3 for a, b in floor_ev[5:])
+
     # Chunked prefill over a paged cache with per-sequence lengths (attn_prefill_paged), timed the
     # same way: inputs resident, L2 flushed before every launch.
     try:
@@ -436,7 +448,8 @@ def run_ours(args):
             "configs": configs,
             "decode": {"metric": "decode KV-read GB/s", "value": dec["value"], "unit": "GB/s",
                        "config": DECODE.config(), "roofline": dec["roofline"], "us_per_launch": dec["us_per_launch"],
-                       "ctas": attn.decode_ctas(DECODE.B, DECODE.Hq, DECODE.Hkv, DECODE.Skv, DECODE.D)},
+                       "ctas": attn.decode_ctas(DECODE.B, DECODE.Hq, DECODE.Hkv, DECODE.Skv, DECODE.D),
+                       "launch_floor_us": launch_floor_us},
             "decode_fp8": {
                 "metric": "decode KV-read GB/s, e4m3 K/V cache", "value": whole_job_rate(world, fp8_bytes, fp8_launch_s) / 1e9,
                 "unit": "GB/s", "config": dict(DECODE.config(), kv_dtype="e4m3", scales="fp32 per (kv head, channel)"),
@@ -447,7 +460,10 @@ def run_ours(args):
                              "peak_kind": f"{peak_kind} HBM copy", "kernel": "decode_tc_kernel<4, e4m3>"},
                 "us_per_launch": fp8_launch_s * 1e6,
                 "bytes_per_launch": fp8_bytes,
+                "launch_floor_us": launch_floor_us,
             },
+            "launch_floor_us": launch_floor_us,
+            "launch_floor_what": "median event-timed duration of an empty kernel (torch.cuda._sleep(0)) launched like the timed kernels, L2 flushed before each; every us_per_launch includes about this much besides the kernel's body",
             "backward": backward,
             "paged_prefill": paged,
             "prefill_fp8": prefill_fp8,

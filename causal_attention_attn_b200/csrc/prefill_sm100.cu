@@ -139,6 +139,15 @@ struct Params {
     int num_pages = 0, page_size = 0, pages_per_seq = 0, cap = 0;
 };
 
+// Tiled bulk store of a shared-memory box into global memory (4-D map), tracked by the issuing
+// thread's bulk async-group. Elements outside the tensor are not written.
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap *map, uint32_t src, int c0, int c1, int c2, int c3)
+{
+    asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];"
+                 ::"l"(reinterpret_cast<uint64_t>(map)), "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+                 : "memory");
+}
+
 // Reference max of a row that has seen no key yet (paged variant): finite, so that the weights of
 // masked scores are 2^(-inf) = 0 rather than NaN, and far below any real score.
 constexpr float kNoKeyMax = -1e30f;

@@ -138,15 +138,6 @@ __device__ __forceinline__ void tma_load_4d_hint(uint32_t dst, const CUtensorMap
                  : "memory");
 }
 
-// Tiled bulk store of a shared-memory box into global memory (4-D map), tracked by the issuing
-// thread's bulk async-group. Elements outside the tensor are not written.
-__device__ __forceinline__ void tma_store_4d(const CUtensorMap *map, uint32_t src, int c0, int c1, int c2, int c3)
-{
-    asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];"
-                 ::"l"(reinterpret_cast<uint64_t>(map)), "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
-                 : "memory");
-}
-
 // Tiled bulk reduce-add of a shared-memory box into global memory (3-D map, element type of the
 // map), tracked by the issuing thread's bulk async-group. Elements outside the tensor are skipped.
 __device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap *map, uint32_t src, int c0, int c1, int c2)
