@@ -629,31 +629,42 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t phases = 0;  // bit 0: phase of SFull_X (one per S_X tile); bit 1: of OFinal_X (one per item)
         bool ok = true;
 
-        for (int k = 0; ok; ++k) {
-            const int w = work_index(p, k);
-            if (w < 0)
-                break;
-            int n, q0, skv, off;
-            {
-                const Item it = decode_item<kPaged>(p, w);
-                n = x ? it.n[1] : it.n[0];
-                q0 = x ? it.q0[1] : it.q0[0];
-                skv = it.skv;
-                off = it.off;
-            }
+        // This tile's part of a work item. The next item's is decoded while the epilogue waits for
+        // the last PV product (the integer divisions of a decode cost ~0.5 us of issue here), so the
+        // next item's softmax starts right after the epilogue.
+        struct Tile {
+            int n = 0, q0 = 0, skv = 0, off = 0, hq = 0, b = 0;
+        };
+        auto tile_of = [&](int w) {
+            const Item it = decode_item<kPaged>(p, w);
+            Tile t;
+            t.n = x ? it.n[1] : it.n[0];
+            t.q0 = x ? it.q0[1] : it.q0[0];
+            t.skv = it.skv;
+            t.off = it.off;
+            t.hq = x ? it.hq[1] : it.hq[0];
+            t.b = it.b;
+            return t;
+        };
+        int w = work_index(p, 0);
+        Tile cur = (w >= 0) ? tile_of(w) : Tile{};
+        Tile nxt{};
+        int w_next = -1;
+        for (int k = 0; ok && w >= 0; ++k, w = w_next, cur = nxt) {
+            w_next = work_index(p, k + 1);
+            const int n = cur.n, q0 = cur.q0, skv = cur.skv, off = cur.off;
             const int row = q0 + r;
             if (kPaged && n == 0 && q0 < p.Sq) {
                 // Paged: a tile none of whose rows sees a key (the sequence holds fewer keys than
                 // the rows before it): O = 0 and LSE = -inf, with no product to wait for.
                 if (row < p.Sq) {
-                    const Item it = decode_item<kPaged>(p, w);
-                    const int hq = x ? it.hq[1] : it.hq[0];
-                    uint4 *dst = reinterpret_cast<uint4 *>(p.o + it.b * p.o_sb + hq * p.o_sh + row * p.o_ss);
+                    uint4 *dst = reinterpret_cast<uint4 *>(p.o + cur.b * p.o_sb + cur.hq * p.o_sh + row * p.o_ss);
 #pragma unroll
                     for (int i = 0; i < D / 8; ++i)
                         dst[i] = make_uint4(0u, 0u, 0u, 0u);
-                    p.lse[(static_cast<size_t>(it.b) * p.Hq + hq) * p.Sq + row] = -INFINITY;
+                    p.lse[(static_cast<size_t>(cur.b) * p.Hq + cur.hq) * p.Sq + row] = -INFINITY;
                 }
+                nxt = (w_next >= 0) ? tile_of(w_next) : Tile{};
                 continue;
             }
             float m = -INFINITY;  // reference max, log2-scaled units
@@ -760,6 +771,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 l = l * alpha + (s01.x + s01.y);
                 l_pv = l_pv * alpha + q01;
             }
+            nxt = (w_next >= 0) ? tile_of(w_next) : Tile{};
             if (!ok || n == 0)
                 continue;
 
@@ -775,9 +787,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             // Paged: a row that saw no key has l = 0: O = 0 and LSE = m + log2(0) = -inf.
             const float inv_l = (kPaged && !(l_pv > 0.f)) ? 0.f : 1.f / l_pv;
             const bool store = row < p.Sq;
-            const Item it = decode_item<kPaged>(p, w);
-            const int hq = x ? it.hq[1] : it.hq[0];
-            const size_t bh_q = static_cast<size_t>(it.b) * p.Hq + hq;
+            const int hq = cur.hq;
+            const size_t bh_q = static_cast<size_t>(cur.b) * p.Hq + hq;
             if constexpr (C::kTmaStore) {
                 // The warp's 32 rows, 64 dims at a time: TMEM -> bf16 -> the warp's staging box (rows of
                 // 128 bytes, 16-byte units XOR row % 8: the 128-byte swizzle) -> one TMA store by lane 0.
@@ -806,12 +817,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0 && row0 < p.Sq) {
-                        tma_store_4d(&tm_o, wstage, h * 64, row0, hq, it.b);
+                        tma_store_4d(&tm_o, wstage, h * 64, row0, hq, cur.b);
                         bulk_commit_group();
                     }
                 }
             } else {
-                __nv_bfloat16 *orow = p.o + it.b * p.o_sb + hq * p.o_sh + (store ? row : 0) * p.o_ss;
+                __nv_bfloat16 *orow = p.o + cur.b * p.o_sb + hq * p.o_sh + (store ? row : 0) * p.o_ss;
     #pragma unroll 1
                 for (int cc = 0; cc < D / 32; ++cc) {
                     uint32_t ov[32];
