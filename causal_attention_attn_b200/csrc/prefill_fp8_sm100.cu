@@ -170,6 +170,14 @@ __device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity, uint64
     return true;
 }
 
+// Three-input maximum (one instruction on sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 __global__ void __launch_bounds__(kThreads, 2)
     prefill_fp8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                        const Fp8PrefillParams p)
@@ -363,18 +371,39 @@ __global__ void __launch_bounds__(kThreads, 2)
                 break;
             tc_fence_after_sync();
             const int k0 = j * kBN;
-            // Pass 1: the row max of the tile (masked keys excluded).
-            float mx = -INFINITY;
-#pragma unroll 1
-            for (int c = 0; c < kBN / 32; ++c) {
-                uint32_t sr[32];
-                tmem_ld32_wait(tS + c * 32, sr);
+            // Every key of the tile visible to this row: no per-key mask below.
+            const bool full = k0 + kBN - 1 <= key_limit;
+            // Pass 1: the row max of the tile (masked keys excluded), on the raw part sums (the
+            // factor to score units is positive), in eight independent chains.
+            float mx8[8];
 #pragma unroll
-                for (int u = 0; u < 32; ++u) {
-                    const float s = __uint_as_float(sr[u]) * row_factor;
-                    mx = (k0 + c * 32 + u <= key_limit) ? fmaxf(mx, s) : mx;
+            for (int i = 0; i < 8; ++i)
+                mx8[i] = -INFINITY;
+#pragma unroll 1
+            for (int c2 = 0; c2 < kBN / 64; ++c2) {
+                uint32_t sra[32], srb[32];
+                tmem_ld32x2_wait(tS + c2 * 64, tS + c2 * 64 + 32, sra, srb);
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    const int c = 2 * c2 + hf;
+                    uint32_t(&sr)[32] = hf ? srb : sra;
+                    if (full) {
+#pragma unroll
+                        for (int u = 0; u < 32; u += 4) {
+                            float &m8 = mx8[u / 4];
+                            m8 = fmax3(m8, __uint_as_float(sr[u]), __uint_as_float(sr[u + 1]));
+                            m8 = fmax3(m8, __uint_as_float(sr[u + 2]), __uint_as_float(sr[u + 3]));
+                        }
+                    } else {
+#pragma unroll
+                        for (int u = 0; u < 32; ++u)
+                            if (k0 + c * 32 + u <= key_limit)
+                                mx8[u & 7] = fmaxf(mx8[u & 7], __uint_as_float(sr[u]));
+                    }
                 }
             }
+            const float mx =
+                fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])) * row_factor;
             // The reference max: the first tile's max (finite: every row sees key 0), then moved
             // only when a tile's max exceeds it by more than the threshold; O is then rescaled once
             // the previous tile's PV product is done.
@@ -402,43 +431,54 @@ __global__ void __launch_bounds__(kThreads, 2)
                 l *= alpha;
                 lpv *= alpha;
             }
-            // Pass 2: weights, their two e4m3 parts (x16) into TMEM over the columns already read.
+            // Pass 2: weights, their two e4m3 parts (x16) into TMEM over the columns already read; the
+            // sums in four independent chains each.
+            float l4[4] = {0.f, 0.f, 0.f, 0.f}, lpv4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
-            for (int c = 0; c < kBN / 32; ++c) {
-                uint32_t sr[32];
-                tmem_ld32_wait(tS + c * 32, sr);
-                uint32_t pw[kPParts][8];
+            for (int c2 = 0; c2 < kBN / 64; ++c2) {
+                uint32_t sra[32], srb[32];
+                tmem_ld32x2_wait(tS + c2 * 64, tS + c2 * 64 + 32, sra, srb);
 #pragma unroll
-                for (int g = 0; g < 8; ++g) {
-                    float w4[4];
+                for (int hf = 0; hf < 2; ++hf) {
+                    const int c = 2 * c2 + hf;
+                    uint32_t(&sr)[32] = hf ? srb : sra;
+                    uint32_t pw[kPParts][8];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int key = k0 + c * 32 + 4 * g + u;
-                        w4[u] = (key <= key_limit) ? ex2(__uint_as_float(sr[4 * g + u]) * row_factor - m_ref) : 0.f;
-                        l += w4[u];
+                    for (int g = 0; g < 8; ++g) {
+                        float w4[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int key = k0 + c * 32 + 4 * g + u;
+                            const float wv = ex2(__uint_as_float(sr[4 * g + u]) * row_factor - m_ref);
+                            w4[u] = (full || key <= key_limit) ? wv : 0.f;
+                            l4[u] += w4[u];
+                        }
+                        // Two keys at a time in f16x2 (11 bits, above the parts' 8): x = hi + lo + rest.
+                        uint32_t hi = 0u, lo = 0u;
+#pragma unroll
+                        for (int pr = 0; pr < 2; ++pr) {
+                            const __half2 x = __floats2half2_rn(w4[2 * pr] * kPScale, w4[2 * pr + 1] * kPScale);
+                            const uint32_t ch = __nv_cvt_halfraw2_to_fp8x2(__half2_raw(x), __NV_SATFINITE, __NV_E4M3);
+                            const __half2 vh = __half2(__nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(ch), __NV_E4M3));
+                            const uint32_t cl = __nv_cvt_halfraw2_to_fp8x2(__half2_raw(__hsub2(x, vh)), __NV_SATFINITE, __NV_E4M3);
+                            const __half2 vl = __half2(__nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(cl), __NV_E4M3));
+                            // What the PV product uses: the parts' sum (exact in f16).
+                            const float2 used = __half22float2(__hadd2(vh, vl));
+                            lpv4[2 * pr] += used.x;
+                            lpv4[2 * pr + 1] += used.y;
+                            hi |= (ch & 0xffffu) << (16 * pr);
+                            lo |= (cl & 0xffffu) << (16 * pr);
+                        }
+                        pw[0][g] = hi;
+                        pw[1][g] = lo;
                     }
-                    // Two keys at a time in f16x2 (11 bits, above the parts' 8): x = hi + lo + rest.
-                    uint32_t hi = 0u, lo = 0u;
 #pragma unroll
-                    for (int pr = 0; pr < 2; ++pr) {
-                        const __half2 x = __floats2half2_rn(w4[2 * pr] * kPScale, w4[2 * pr + 1] * kPScale);
-                        const uint32_t ch = __nv_cvt_halfraw2_to_fp8x2(__half2_raw(x), __NV_SATFINITE, __NV_E4M3);
-                        const __half2 vh = __half2(__nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(ch), __NV_E4M3));
-                        const uint32_t cl = __nv_cvt_halfraw2_to_fp8x2(__half2_raw(__hsub2(x, vh)), __NV_SATFINITE, __NV_E4M3);
-                        const __half2 vl = __half2(__nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(cl), __NV_E4M3));
-                        // What the PV product uses: the parts' sum (exact in f16).
-                        const float2 used = __half22float2(__hadd2(vh, vl));
-                        lpv += used.x + used.y;
-                        hi |= (ch & 0xffffu) << (16 * pr);
-                        lo |= (cl & 0xffffu) << (16 * pr);
-                    }
-                    pw[0][g] = hi;
-                    pw[1][g] = lo;
+                    for (int pt = 0; pt < kPParts; ++pt)
+                        tmem_st8(tS + 8u * kPParts * c + 8u * pt, pw[pt]);
                 }
-#pragma unroll
-                for (int pt = 0; pt < kPParts; ++pt)
-                    tmem_st8(tS + 8u * kPParts * c + 8u * pt, pw[pt]);
             }
+            l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+            lpv += (lpv4[0] + lpv4[1]) + (lpv4[2] + lpv4[3]);
             tmem_wait_st();
             tc_fence_before_sync();
             mbar_arrive(BAR(kBarPFull));
