@@ -215,24 +215,32 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int qi = q0 + r;
         const bool valid = qi < p.Sq;
         const __nv_bfloat16 *qrow = p.q + ((static_cast<size_t>(b) * p.Hq + h) * p.Sq + (valid ? qi : 0)) * kD;
-        const float *ks = p.k_scale + static_cast<size_t>(kvh) * kD;
-        // x = q * k_scale, 16 dims at a time (two passes over the row keep few registers live).
+        const float4 *ks4 = reinterpret_cast<const float4 *>(p.k_scale + static_cast<size_t>(kvh) * kD);
+        // The row (256 bytes) is loaded once, all sixteen 16-byte loads in flight together; x = q *
+        // k_scale is then formed 16 dims at a time from it (two passes over the row).
+        uint4 qr[kD / 8];
+        {
+            const uint4 *src = reinterpret_cast<const uint4 *>(qrow);
+#pragma unroll
+            for (int t = 0; t < kD / 8; ++t)
+                qr[t] = valid ? src[t] : make_uint4(0u, 0u, 0u, 0u);
+        }
         auto load16 = [&](int c, float (&x)[16]) {
-            const uint4 *src = reinterpret_cast<const uint4 *>(qrow) + 2 * c;
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
-                const uint4 raw = valid ? src[hf] : make_uint4(0u, 0u, 0u, 0u);
+                const uint4 raw = qr[2 * c + hf];
                 const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+                const float4 sa = ks4[4 * c + 2 * hf], sb = ks4[4 * c + 2 * hf + 1];
+                const float sc[8] = {sa.x, sa.y, sa.z, sa.w, sb.x, sb.y, sb.z, sb.w};
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    const int d = 16 * c + 8 * hf + 2 * u;
-                    x[8 * hf + 2 * u] = __uint_as_float(w[u] << 16) * ks[d];
-                    x[8 * hf + 2 * u + 1] = __uint_as_float(w[u] & 0xffff0000u) * ks[d + 1];
+                    x[8 * hf + 2 * u] = __uint_as_float(w[u] << 16) * sc[2 * u];
+                    x[8 * hf + 2 * u + 1] = __uint_as_float(w[u] & 0xffff0000u) * sc[2 * u + 1];
                 }
             }
         };
         float mx = 0.f;
-#pragma unroll 1
+#pragma unroll
         for (int c = 0; c < kD / 16; ++c) {
             float x[16];
             load16(c, x);
@@ -245,7 +253,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         row_factor = p.scale_log2 * exp2_int(-e);
         // Part pt of row r: 128 bytes, 16-byte unit c (dims 16c .. 16c + 15) at ((c ^ (r % 8)) << 4)
         // (K-major, 128-byte swizzle).
-#pragma unroll 1
+#pragma unroll
         for (int c = 0; c < kD / 16; ++c) {
             float x[16];
             load16(c, x);
