@@ -320,8 +320,44 @@ extern "C" int attn_fwd_host(const void *q_host, const void *k_host, const void 
     while ((static_cast<long long>(group) * Sq * align) % 4 != 0)
         align *= 2;
     constexpr long long kSlices = 8;
-    const size_t q_unit = static_cast<size_t>(group) * Sq * D * 2, kv_unit = static_cast<size_t>(Skv) * D * 2;
-    const size_t lse_unit = static_cast<size_t>(group) * Sq;
+    const size_t q_head = static_cast<size_t>(Sq) * D * 2, kv_unit = static_cast<size_t>(Skv) * D * 2;
+    // A slice: the query heads [a, b) of the flat (unit, head) order, which cover the units
+    // [a / group, (b - 1) / group]; either whole units or one half of one unit.
+    struct Slice {
+        long long a, b;
+    };
+    Slice slices[kSlices + 2];
+    int n_slices = 0;
+    // The pipeline's fill (the first slice's copy in) and drain (the last slice's attention and copy
+    // out) are not overlapped: with few units the first and the last unit go in halves (of its query
+    // heads; the first half also brings the unit's K and V), which shortens both.
+    // (Half a group of Sq rows is then a whole number of 16-byte blocks of lse, and so is every unit.)
+    const bool halves = units >= 2 && group % 2 == 0 && (static_cast<long long>(group / 2) * Sq) % 4 == 0;
+    if (halves) {
+        const long long g = group, h = group / 2;
+        slices[n_slices++] = {0, h};
+        slices[n_slices++] = {h, g};
+        const long long mid = units - 2;  // whole units 1 .. units - 2, in up to kSlices - 2 slices
+        long long m0 = 0;
+        for (long long i = 1; i <= kSlices - 2 && m0 < mid; ++i) {
+            const long long m1 = mid * i / (kSlices - 2);
+            if (m1 <= m0)
+                continue;
+            slices[n_slices++] = {(1 + m0) * g, (1 + m1) * g};
+            m0 = m1;
+        }
+        slices[n_slices++] = {(units - 1) * g, (units - 1) * g + h};
+        slices[n_slices++] = {(units - 1) * g + h, units * g};
+    } else {
+        long long u0 = 0;
+        for (long long i = 1; i <= kSlices && u0 < units; ++i) {
+            const long long u1 = (i == kSlices) ? units : (units * i / kSlices) / align * align;
+            if (u1 <= u0)
+                continue;
+            slices[n_slices++] = {u0 * group, u1 * group};
+            u0 = u1;
+        }
+    }
     auto at = [](const void *p, size_t off) { return static_cast<const char *>(p) + off; };
     auto atw = [](void *p, size_t off) { return static_cast<char *>(p) + off; };
     // The copy streams start after the work already queued on `stream` (which may still use the
@@ -331,35 +367,47 @@ extern "C" int attn_fwd_host(const void *q_host, const void *k_host, const void 
         cudaGetLastError();
         return ATTN_ERR_CUDA;
     }
-    long long u0 = 0;
-    for (long long i = 1; i <= kSlices && u0 < units && rc == ATTN_OK; ++i) {
-        long long u1 = (i == kSlices) ? units : (units * i / kSlices) / align * align;
-        if (u1 <= u0)
-            continue;
-        const size_t n = static_cast<size_t>(u1 - u0);
-        const size_t qo = static_cast<size_t>(u0) * q_unit, ko = static_cast<size_t>(u0) * kv_unit;
-        const size_t lo = static_cast<size_t>(u0) * lse_unit;
-        if (cudaMemcpyAsync(atw(q_dev, qo), at(q_host, qo), n * q_unit, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
-            cudaMemcpyAsync(atw(k_dev, ko), at(k_host, ko), n * kv_unit, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
-            cudaMemcpyAsync(atw(v_dev, ko), at(v_host, ko), n * kv_unit, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
-            cudaEventRecord(ev_in, s_in) != cudaSuccess || cudaStreamWaitEvent(stream, ev_in, 0) != cudaSuccess) {
+    long long kv_done = 0;  // units whose K and V have been queued for copying in
+    for (int i = 0; i < n_slices && rc == ATTN_OK; ++i) {
+        const long long a = slices[i].a, b = slices[i].b;
+        const long long u0 = a / group, u1 = (b - 1) / group + 1;
+        const bool whole = a % group == 0 && b % group == 0;
+        const size_t qo = static_cast<size_t>(a) * q_head, qn = static_cast<size_t>(b - a) * q_head;
+        const size_t lo = static_cast<size_t>(a) * Sq, ln = static_cast<size_t>(b - a) * Sq;
+        if (cudaMemcpyAsync(atw(q_dev, qo), at(q_host, qo), qn, cudaMemcpyHostToDevice, s_in) != cudaSuccess) {
             cudaGetLastError();
             rc = ATTN_ERR_CUDA;
             break;
         }
-        rc = run(at(q_dev, qo), at(k_dev, ko), at(v_dev, ko), atw(o_dev, qo), lse_dev + lo, static_cast<int>(n), group, 1,
-                 Sq, Skv, D, scale, causal, 0, contiguous_layouts(group, 1, Sq, Skv, D), stream);
+        if (kv_done < u1) {
+            const size_t ko = static_cast<size_t>(kv_done) * kv_unit, kn = static_cast<size_t>(u1 - kv_done) * kv_unit;
+            if (cudaMemcpyAsync(atw(k_dev, ko), at(k_host, ko), kn, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
+                cudaMemcpyAsync(atw(v_dev, ko), at(v_host, ko), kn, cudaMemcpyHostToDevice, s_in) != cudaSuccess) {
+                cudaGetLastError();
+                rc = ATTN_ERR_CUDA;
+                break;
+            }
+            kv_done = u1;
+        }
+        if (cudaEventRecord(ev_in, s_in) != cudaSuccess || cudaStreamWaitEvent(stream, ev_in, 0) != cudaSuccess) {
+            cudaGetLastError();
+            rc = ATTN_ERR_CUDA;
+            break;
+        }
+        const size_t ku = static_cast<size_t>(u0) * kv_unit;
+        const int nb = whole ? static_cast<int>(u1 - u0) : 1, nh = whole ? group : static_cast<int>(b - a);
+        rc = run(at(q_dev, qo), at(k_dev, ku), at(v_dev, ku), atw(o_dev, qo), lse_dev + lo, nb, nh, 1, Sq, Skv, D, scale,
+                 causal, 0, contiguous_layouts(nh, 1, Sq, Skv, D), stream);
         if (rc != ATTN_OK)
             break;
         if (cudaEventRecord(ev_done, stream) != cudaSuccess || cudaStreamWaitEvent(s_out, ev_done, 0) != cudaSuccess ||
-            cudaMemcpyAsync(atw(o_host, qo), at(o_dev, qo), n * q_unit, cudaMemcpyDeviceToHost, s_out) != cudaSuccess ||
-            cudaMemcpyAsync(lse_host + lo, lse_dev + lo, n * lse_unit * sizeof(float), cudaMemcpyDeviceToHost, s_out) !=
+            cudaMemcpyAsync(atw(o_host, qo), at(o_dev, qo), qn, cudaMemcpyDeviceToHost, s_out) != cudaSuccess ||
+            cudaMemcpyAsync(lse_host + lo, lse_dev + lo, ln * sizeof(float), cudaMemcpyDeviceToHost, s_out) !=
                 cudaSuccess) {
             cudaGetLastError();
             rc = ATTN_ERR_CUDA;
             break;
         }
-        u0 = u1;
     }
     // Join the copy streams back into `stream` on every path, so that later work on it (or a
     // synchronisation of it) covers everything this call queued.

@@ -91,9 +91,11 @@ int attn_fwd_ex(const void *q, const void *k, const void *v, void *o, float *lse
 
 /*
  * attn_fwd_host — attn_fwd from host memory to host memory, with the copies pipelined against the
- * attention: the (batch, kv head) units are cut into up to eight slices, and while slice i is
+ * attention: the (batch, kv head) units are cut into up to ten slices, and while slice i is
  * copied in, slice i-1 is computed and slice i-2 is copied out (two copy streams of the library's
- * own, ordered against `stream` with events). Same operation and results as attn_fwd on the same
+ * own, ordered against `stream` with events). When the group splits evenly (and half a group of
+ * rows is a whole number of 16-byte blocks of lse), the first and the last unit go in two halves
+ * of their query heads, which shortens the unoverlapped first copy in and last copy out. Same operation and results as attn_fwd on the same
  * values (each unit is computed the same way; the decode's split over CTAs may differ, within
  * rounding) — "第11节：Attention 实现（Flash vs Fallback）", §3 for the mask, as attn_fwd.
  *   q_host, k_host, v_host   host pointers, bf16, the contiguous layouts above. Page-locked

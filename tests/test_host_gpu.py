@@ -29,11 +29,12 @@ def gpu():
 
 SHAPES = [
     # B, Hq, Hkv, Sq, Skv, D, causal
-    (1, 32, 8, 1024, 1024, 128, True),   # eight units: one per slice
+    (1, 32, 8, 1024, 1024, 128, True),   # eight units: halves of the first and last, one per slice between
     (3, 6, 3, 130, 400, 128, True),      # nine units over eight slices; group * Sq even
     (2, 5, 5, 67, 67, 64, True),         # ten units; group * Sq odd: slices fall on whole lse blocks
     (1, 4, 1, 257, 300, 32, False),      # one unit
-    (16, 32, 8, 200, 600, 128, True),    # 128 units
+    (16, 32, 8, 200, 600, 128, True),    # 128 units; the first and last in halves of their heads
+    (2, 4, 2, 256, 300, 128, True),      # four units; halves of one head each at both ends
 ]
 
 
