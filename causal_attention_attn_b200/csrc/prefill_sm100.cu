@@ -137,7 +137,15 @@ struct Params {
     const int *seq_lens = nullptr;
     const int *block_table = nullptr;
     int num_pages = 0, page_size = 0, pages_per_seq = 0, cap = 0;
+    // Paged: 1 when the (batch, query-tile) pairs are few enough (<= kMaxSorted) to be put in order of
+    // their KV-tile count at the start of the kernel (the lengths are known on the device only).
+    int sorted = 0;
 };
+
+// The sorted order of (batch, query-tile) pairs (e = b + B * item) and their KV-tile counts.
+constexpr int kMaxSorted = 64;
+__shared__ uint16_t s_pair_order[kMaxSorted];
+__shared__ int s_pair_tiles[kMaxSorted];
 
 // Tiled bulk store of a shared-memory box into global memory (4-D map), tracked by the issuing
 // thread's bulk async-group. Elements outside the tensor are not written.
@@ -240,9 +248,15 @@ __device__ __forceinline__ Item decode_item(const Params &p, int w)
     int t = w;
     const int hu = t % hpu;
     t /= hpu;
-    const int b = t % p.B;
-    t /= p.B;
-    const int item = p.n_items - 1 - t;
+    int b, item;
+    if (kPaged && p.sorted) {
+        const int e = s_pair_order[t];
+        b = e % p.B;
+        item = e / p.B;
+    } else {
+        b = t % p.B;
+        item = p.n_items - 1 - t / p.B;
+    }
     const int h_a = hu * heads_per_item;
     Item it;
     it.q0[0] = p.pair_heads ? item * kBM : item * 2 * kBM;
@@ -311,6 +325,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(BAR(kBarDrain), 1);
         *abort_flag = 0;
         fence_mbar_init();
+    }
+    if (kPaged && p.sorted && warp == 10) {
+        // Heaviest first by the pairs' real KV-tile counts (ties: lower e first), ranked by one warp.
+        const int n = p.B * p.n_items;
+        for (int e = lane; e < n; e += 32) {
+            const int b = e % p.B, item = e / p.B;
+            const int skv = min(max(__ldg(p.seq_lens + b), 0), p.cap), off = skv - p.Sq;
+            const int q0a = p.pair_heads ? item * kBM : item * 2 * kBM;
+            const int q0b = p.pair_heads ? q0a : q0a + kBM;
+            s_pair_tiles[e] = max(kv_tiles_for(p, q0a, skv, off), kv_tiles_for(p, q0b, skv, off));
+        }
+        __syncwarp();
+        for (int e = lane; e < n; e += 32) {
+            const int c = s_pair_tiles[e];
+            int rank = 0;
+            for (int f = 0; f < n; ++f) {
+                const int cf = s_pair_tiles[f];
+                rank += (cf > c || (cf == c && f < e)) ? 1 : 0;
+            }
+            s_pair_order[rank] = static_cast<uint16_t>(e);
+        }
     }
     if (warp == kWarpTma && lane == 0) {
         tma_prefetch_desc(&tm_q);
@@ -946,6 +981,7 @@ cudaError_t launch(const PrefillArgs &a, cudaStream_t stream, int *encode_error)
     const int n_qtiles = (a.Sq + kBM - 1) / kBM;
     p.pair_heads = (p.group % 2 == 0) ? 1 : 0;
     p.n_items = p.pair_heads ? n_qtiles : (n_qtiles + 1) / 2;
+    p.sorted = (kPaged && static_cast<long long>(p.n_items) * a.B <= kMaxSorted) ? 1 : 0;
     p.scale_log2 = a.scale * kLog2e;
     const long long n_work = static_cast<long long>(p.n_items) * a.B * (a.Hq / (p.pair_heads ? 2 : 1));
     if (n_work > INT_MAX)
