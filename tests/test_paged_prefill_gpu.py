@@ -99,6 +99,9 @@ CASES = [
     (4, 6, 2, 130, 512, 64, [512, 129, 0, 200], True),                              # odd group, len < Sq, empty
     (2, 4, 4, 64, 700, 256, [700, 65], False),                                      # non-causal, 256-key pages
     (2, 16, 2, 300, 2048, 32, [2048, 1000], True),                                  # long, 32-key pages
+    # 72 (batch, query-tile) pairs: more than the kernel puts in order of their real KV-tile counts,
+    # so the work list keeps the equal-length order
+    (9, 4, 2, 1024, 1100, 64, [1100, 1024, 1050, 1080, 1024, 1099, 1070, 1030, 1060], True),
 ]
 
 
