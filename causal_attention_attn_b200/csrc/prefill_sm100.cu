@@ -858,17 +858,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             } else {
                 __nv_bfloat16 *orow = p.o + cur.b * p.o_sb + hq * p.o_sh + (store ? row : 0) * p.o_ss;
-    #pragma unroll 1
+#pragma unroll 1
                 for (int cc = 0; cc < D / 32; ++cc) {
                     uint32_t ov[32];
                     tmem_ld32_wait(tO + cc * 32, ov);
                     uint32_t pkd[16];
-    #pragma unroll
+#pragma unroll
                     for (int i = 0; i < 16; ++i)
                         pkd[i] = pack_bf16x2(__uint_as_float(ov[2 * i]) * inv_l, __uint_as_float(ov[2 * i + 1]) * inv_l);
                     if (store) {
                         uint4 *dst = reinterpret_cast<uint4 *>(orow + cc * 32);
-    #pragma unroll
+#pragma unroll
                         for (int i = 0; i < 4; ++i)
                             dst[i] = make_uint4(pkd[4 * i], pkd[4 * i + 1], pkd[4 * i + 2], pkd[4 * i + 3]);
                     }
