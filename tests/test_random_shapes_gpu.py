@@ -75,3 +75,49 @@ def test_random_shape(shape):
         o2, l2 = attn.attn_fwd(qt, kt, vt, scale=scale, causal=causal, out=ot)
         torch.cuda.synchronize()
         assert torch.equal(o2.cpu(), o.cpu()) and torch.equal(l2.cpu(), lse.cpu())
+
+
+def draw_backward_shapes(n, seed=4048, max_pairs=1_500_000):
+    rng = np.random.default_rng(seed)
+    shapes = []
+    while len(shapes) < n:
+        B = int(rng.integers(1, 4))
+        Hkv = int(rng.choice([1, 2, 4]))
+        group = int(rng.choice([1, 2, 3, 4]))
+        causal = bool(rng.integers(0, 2))
+        Sq = int(rng.integers(2, 600))
+        Skv = int(rng.integers(1, 1200))
+        if causal and Skv < Sq:
+            Skv = Sq + int(rng.integers(0, 300))
+        scale = float(np.float32(rng.uniform(0.03, 0.3)))
+        if B * Hkv * group * Sq * Skv > max_pairs:
+            continue
+        shapes.append((B, Hkv * group, Hkv, Sq, Skv, causal, scale))
+    return shapes
+
+
+BWD_SHAPES = draw_backward_shapes(6)
+
+
+@pytest.mark.parametrize("shape", BWD_SHAPES, ids=lambda s: "b{}_hq{}_hkv{}_sq{}_skv{}_{}_s{:.3f}".format(
+    *s[:5], "c" if s[5] else "nc", s[6]))
+def test_random_backward_shape(shape):
+    """attn_bwd (head dim 128) against the oracle's gradients, with the backward tests' bound: max
+    |err| <= 1e-2 and mean |err| <= 1e-3 of each gradient's largest magnitude. Even groups on grids
+    of fewer key tiles than SMs take the two-CTA head split."""
+    B, Hq, Hkv, Sq, Skv, causal, scale = shape
+    w = inputs.custom(B, Hq, Hkv, Sq, Skv, 128, causal, seed=int(sum(shape[:5])))
+    q, k, v = inputs.generate(w)
+    dout = torch.randn(q.shape, generator=torch.Generator().manual_seed(17)).to(torch.bfloat16)
+    qg, kg, vg, dg = q.cuda(), k.cuda(), v.cuda(), dout.cuda()
+    o, lse = attn.attn_fwd(qg, kg, vg, scale=scale, causal=causal)
+    dq, dk, dv = attn.attn_bwd(qg, kg, vg, o, lse, dg, scale=scale, causal=causal)
+    torch.cuda.synchronize()
+    ref = oracle.attention_bwd(q, k, v, dout, scale, causal)
+    for name, got, want in (("dq", dq, ref[0]), ("dk", dk, ref[1]), ("dv", dv, ref[2])):
+        g = got.cpu().double().numpy()
+        err = np.abs(g - want)
+        top = np.abs(want).max()
+        assert np.isfinite(g).all(), name
+        assert err.max() <= 1e-2 * top and err.mean() <= 1e-3 * top, (
+            f"{name}: max|err| {err.max():.3e} mean|err| {err.mean():.3e} vs max|ref| {top:.3e}")
