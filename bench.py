@@ -10,7 +10,10 @@ events. Each launch is timed with CUDA events on the launching stream.
 
 The line's ``value`` is the prefill TFLOP/s of the largest single-GPU workload (the 32K prefill);
 ``configs`` holds every workload's own throughput, roofline fraction, DRAM traffic and oracle
-baseline, and ``decode`` repeats the GQA decode's.
+baseline, and ``decode`` repeats the GQA decode's. After the timed steps come the end-to-end leg
+(``e2e``: the 32K prefill from pinned host buffers through ``attn_fwd_host``), the e4m3 decode,
+the event-timing floor of an empty launch (``launch_floor_us``), the paged chunked prefill, the
+e4m3 chunked prefill and the backward pass of the 8B layer, each timed the same way.
 
 ``python bench.py --gpus N --steps K --warmup W`` prints one JSON line (rank 0). For N > 1 it is
 launched with torchrun, one rank per GPU; every rank processes its own copy of the workloads (the
