@@ -241,7 +241,13 @@ def run_reference(args):
     return 0
 
 
-def config_entry(w, launch_s, world, peaks, peak_kind, baseline=None):
+# A timed region at least this long runs the step's kernels back to back under the power cap: the
+# prefills are then "timed inside a long step" and their roofline peak is the measured sustained
+# bf16 figure (a seconds-long loop of cuBLAS under the same cap); shorter runs use the burst one.
+SUSTAINED_REGION_MS = 1000.0
+
+
+def config_entry(w, launch_s, world, peaks, peak_kind, baseline=None, sustained_regime=False):
     """The JSON object of one workload: throughput, roofline of its kernel, oracle baseline."""
     tensor_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
@@ -254,8 +260,12 @@ def config_entry(w, launch_s, world, peaks, peak_kind, baseline=None):
     else:
         achieved = w.flops() / launch_s / 1e12
         sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
-        roof = {"bound": "tensor", "achieved": achieved, "peak": tensor_peak, "unit": "TFLOP/s",
-                "frac": achieved / tensor_peak, "peak_kind": f"{peak_kind} bf16 dense (burst)",
+        peak = sustained if sustained_regime else tensor_peak
+        kind = ("sustained: the timed region ran the step back to back for at least "
+                f"{SUSTAINED_REGION_MS / 1000:.0f} s under the power cap") if sustained_regime else "burst"
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "peak_kind": f"{peak_kind} bf16 dense ({kind})",
+                "frac_of_burst": achieved / tensor_peak,  # the measured peak of a short run
                 "frac_of_sustained": achieved / sustained,  # the measured peak under the power cap
                 "frac_of_datasheet": achieved / DATASHEET_BF16_TFLOPS,  # nominal dense bf16
                 "flops_per_launch": w.flops()}
@@ -432,7 +442,9 @@ def run_ours(args):
 
     if rank == 0:
         baselines = {w.name: workload_baseline(w, host[w.name]) for w in STEP_WORKLOADS} if world == 1 else {}
-        configs = {SHORT[w.name]: config_entry(w, launch_s[w.name], world, peaks, peak_kind, baselines.get(w.name))
+        sustained_regime = region_ms >= SUSTAINED_REGION_MS
+        configs = {SHORT[w.name]: config_entry(w, launch_s[w.name], world, peaks, peak_kind, baselines.get(w.name),
+                                               sustained_regime)
                    for w in STEP_WORKLOADS}
         head = configs[SHORT[HEADLINE.name]]
         dec = configs[SHORT[DECODE.name]]
