@@ -170,6 +170,17 @@ __device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity, uint64
     return true;
 }
 
+// acc + lo + hi for the two f16 values packed in w, each added with fp32 accumulation (mixed-
+// precision adds: no separate widening of the f16 halves).
+__device__ __forceinline__ float add_f16x2(float acc, uint32_t w)
+{
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\t"
+        "add.rn.f32.f16 %0, lo, %0;\n\tadd.rn.f32.f16 %0, hi, %0;\n\t}"
+        : "+f"(acc)
+        : "r"(w));
+    return acc;
+}
+
 // Three-input maximum (one instruction on sm_100).
 __device__ __forceinline__ float fmax3(float a, float b, float c)
 {
@@ -441,7 +452,10 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
             // Pass 2: weights, their two e4m3 parts (x16) into TMEM over the columns already read; the
             // sums in four independent chains each.
-            float l4[4] = {0.f, 0.f, 0.f, 0.f}, lpv4[4] = {0.f, 0.f, 0.f, 0.f};
+            // The weights come out times 16 (kPScale) straight from the exponent; l is kept in those
+            // units within the tile and scaled back (exactly) when it joins the running sum.
+            const float m16 = m_ref - 4.0f;  // 2^4 = kPScale
+            float l4[4] = {0.f, 0.f, 0.f, 0.f}, lpv4[2] = {0.f, 0.f};
 #pragma unroll 1
             for (int c2 = 0; c2 < kBN / 64; ++c2) {
                 uint32_t sra[32], srb[32];
@@ -457,7 +471,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
                         for (int u = 0; u < 4; ++u) {
                             const int key = k0 + c * 32 + 4 * g + u;
-                            const float wv = ex2(__uint_as_float(sr[4 * g + u]) * row_factor - m_ref);
+                            const float wv = ex2(__uint_as_float(sr[4 * g + u]) * row_factor - m16);
                             w4[u] = (full || key <= key_limit) ? wv : 0.f;
                             l4[u] += w4[u];
                         }
@@ -465,15 +479,14 @@ __global__ void __launch_bounds__(kThreads, 2)
                         uint32_t hi = 0u, lo = 0u;
 #pragma unroll
                         for (int pr = 0; pr < 2; ++pr) {
-                            const __half2 x = __floats2half2_rn(w4[2 * pr] * kPScale, w4[2 * pr + 1] * kPScale);
+                            const __half2 x = __floats2half2_rn(w4[2 * pr], w4[2 * pr + 1]);
                             const uint32_t ch = __nv_cvt_halfraw2_to_fp8x2(__half2_raw(x), __NV_SATFINITE, __NV_E4M3);
                             const __half2 vh = __half2(__nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(ch), __NV_E4M3));
                             const uint32_t cl = __nv_cvt_halfraw2_to_fp8x2(__half2_raw(__hsub2(x, vh)), __NV_SATFINITE, __NV_E4M3);
                             const __half2 vl = __half2(__nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(cl), __NV_E4M3));
                             // What the PV product uses: the parts' sum (exact in f16).
-                            const float2 used = __half22float2(__hadd2(vh, vl));
-                            lpv4[2 * pr] += used.x;
-                            lpv4[2 * pr + 1] += used.y;
+                            const __half2 used = __hadd2(vh, vl);
+                            lpv4[pr] = add_f16x2(lpv4[pr], *reinterpret_cast<const uint32_t *>(&used));
                             hi |= (ch & 0xffffu) << (16 * pr);
                             lo |= (cl & 0xffffu) << (16 * pr);
                         }
@@ -485,8 +498,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                         tmem_st8(tS + 8u * kPParts * c + 8u * pt, pw[pt]);
                 }
             }
-            l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
-            lpv += (lpv4[0] + lpv4[1]) + (lpv4[2] + lpv4[3]);
+            l += ((l4[0] + l4[1]) + (l4[2] + l4[3])) * (1.0f / kPScale);
+            lpv += lpv4[0] + lpv4[1];
             tmem_wait_st();
             tc_fence_before_sync();
             mbar_arrive(BAR(kBarPFull));
