@@ -440,6 +440,13 @@ def run_ours(args):
     except Exception as e:  # an extra leg that fails is reported in its object, not allowed to drop the line
         backward = {"metric": "backward TFLOP/s (dq, dk, dv)", "error": f"{type(e).__name__}: {e}"}
 
+    # The ring's per-rank compute at eight ranks, emulated here (blocks and merges, no exchange).
+    try:
+        lq, lk, lv, _, _ = bufs[HEADLINE.name]
+        ring = ring_compute_leg(attn, args, ranks, dev, stream, clear_l2, lq, lk, lv, launch_s[HEADLINE.name])
+    except Exception as e:
+        ring = {"metric": "ring attention compute per rank (no exchange), ms", "error": f"{type(e).__name__}: {e}"}
+
     if rank == 0:
         baselines = {w.name: workload_baseline(w, host[w.name]) for w in STEP_WORKLOADS} if world == 1 else {}
         sustained_regime = region_ms >= SUSTAINED_REGION_MS
@@ -480,6 +487,7 @@ def run_ours(args):
             "launch_floor_us": launch_floor_us,
             "launch_floor_what": "median event-timed duration of an empty kernel (torch.cuda._sleep(0)) launched like the timed kernels, L2 flushed before each; every us_per_launch includes about this much besides the kernel's body",
             "backward": backward,
+            "ring_compute": ring,
             "paged_prefill": paged,
             "prefill_fp8": prefill_fp8,
             "timed_region_ms": region_ms,
@@ -541,6 +549,63 @@ def read_traffic(kernel: str, workload: str):
         return entry.get("dram_bytes_per_launch")
     except (OSError, ValueError, AttributeError):
         return None
+
+
+def ring_compute_leg(attn, args, ranks, dev, stream, clear_l2, q, k, v, head_launch_s, world_ring=8):
+    """The compute of ring attention on the 32K workload at world_ring ranks, emulated on this GPU
+    with no exchange: every virtual rank runs its zigzag schedule's blocks (attn_fwd) and LSE merges
+    (attn_lse_merge) over K/V shards already resident, L2 flushed before each rank. The slowest
+    rank's time is compared with a world_ring-th of the single 32K launch: the cost of cutting the
+    sequence into blocks (more launches, each with its ramp and tail) and merging them. The
+    exchange over NVLink is not part of it (it needs several GPUs)."""
+    from causal_attention_attn_b200.ring import DIAG, ring_schedule, zigzag_shard
+
+    w = HEADLINE
+    S = w.Sq // world_ring  # tokens per rank: two chunks
+    c = S // 2
+
+    def halves(x):
+        return x[:, :, :c].contiguous(), x[:, :, c:].contiguous()
+
+    shards = [(halves(zigzag_shard(q, r, world_ring)), halves(zigzag_shard(k, r, world_ring)),
+               halves(zigzag_shard(v, r, world_ring))) for r in range(world_ring)]
+
+    def run_rank(rank):
+        qs = shards[rank][0]
+        o_acc = [torch.zeros(x.shape, dtype=torch.float32, device=dev) for x in qs]
+        lse_acc = [torch.full(x.shape[:-1], float("-inf"), dtype=torch.float32, device=dev) for x in qs]
+        out = [torch.empty(x.shape, dtype=torch.bfloat16, device=dev) for x in qs]
+        sched = ring_schedule(rank, world_ring, True)
+        last = {qh: (t, b) for t, _, blocks in sched for b, (qh, _, _) in enumerate(blocks)}
+        launches = 0
+        clear_l2()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for t, j, blocks in sched:
+            ks, vs = shards[j][1], shards[j][2]
+            for b, (qh, kh, mode) in enumerate(blocks):
+                o_p, l_p = attn.attn_fwd(qs[qh], ks[kh], vs[kh], scale=w.scale, causal=(mode == DIAG), stream=stream)
+                attn.attn_lse_merge(o_acc[qh], lse_acc[qh], o_p, l_p, out=out[qh] if last[qh] == (t, b) else None,
+                                    stream=stream)
+                launches += 2
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1), launches
+
+    for r in range(world_ring):  # warm-up
+        run_rank(r)
+    reps = 3
+    per_rank = [min(run_rank(r)[0] for _ in range(reps)) for r in range(world_ring)]
+    launches = run_rank(0)[1]
+    slowest = ranks.max([max(per_rank)])[0]
+    share = head_launch_s * 1e3 / world_ring
+    return {"metric": "ring attention compute per rank (no exchange), ms", "world": world_ring,
+            "config": dict(w.config(), tokens_per_rank=S, chunk=c, order="zigzag"),
+            "slowest_rank_ms": slowest, "fastest_rank_ms": min(per_rank),
+            "single_launch_share_ms": share, "overhead_vs_share": slowest / share,
+            "launches_per_rank": launches,
+            "what": "every virtual rank's blocks and LSE merges on K/V shards already in HBM, L2 flushed "
+                    "before each rank, best of 3; the exchange between GPUs is not part of it"}
 
 
 def backward_leg(attn, args, ranks, dev, stream, clear_l2, q, k, v, o, lse, world):
